@@ -1,0 +1,181 @@
+"""fp64 CPU oracle for the sparse MoE feed-forward layer (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's ``cpu_baseline`` / reference leg are the only callers.  The
+product library never imports, links or runs anything here, and this package
+imports nothing from the product package.
+
+Every function mirrors one in ``moe_oracle.c``; the C file's header says
+which passage of the pages each one follows.  Parity status: route, layout,
+expert FFN and forward are pinned by the ``-m "not gpu"`` tests against the
+walkthrough's worked example (yeyulingfeng.com/587419.html section 4), the
+closed form of the same section, brute-force top-k and counting sort, a dense
+"run every expert then mask" evaluation (llama-cpp-visual-guide lesson 35,
+ggml_mul_mat_id section), the E=1/k=1 plain gated MLP, and torch's own SiLU
+and tanh-GELU in float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain C, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or \
+            os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE",
+                               "-fPIC", "-shared", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int
+        lib.oracle_num_threads.restype = i32
+        lib.oracle_act.argtypes = [i32, i64, P, P]
+        lib.oracle_route.argtypes = [i64, i32, i32, P, P, P, P, P]
+        lib.oracle_layout_capacity.argtypes = [i64, i32, i32, i32, i32]
+        lib.oracle_layout_capacity.restype = i64
+        lib.oracle_layout.argtypes = [i64, i32, i32, i32, i32, P, P, P, i64, P]
+        lib.oracle_expert_rows.argtypes = [i32, i32, i32, P, P, P, i64, P, P,
+                                           i32, i32, P]
+        lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, i32, i32,
+                                       P, P, P, P, P, P, P, P, i64, i32, i32,
+                                       P, P, P]
+        for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
+                  lib.oracle_expert_rows, lib.oracle_forward):
+            f.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    """bf16 torch tensor or uint16 ndarray -> contiguous uint16 ndarray."""
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return np.ascontiguousarray(a, dtype=np.uint16)
+    import torch
+    t = a.detach().to("cpu").contiguous()
+    assert t.dtype == torch.bfloat16, t.dtype
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _f32(a) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    if not isinstance(a, np.ndarray):
+        a = a.detach().to("cpu").numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def act(kind: int, v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty_like(v)
+    _check(_load().oracle_act(kind, v.size, _ptr(v), _ptr(out)), "act")
+    return out
+
+
+def route(logits, k: int, scale=None, want_probs: bool = False):
+    """-> ids [T,k] int32, w [T,k] float64 (and probs [T,E] if asked)."""
+    z = _f32(logits)
+    T, E = z.shape
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    probs = np.empty((T, E), np.float64) if want_probs else None
+    sc = _f32(scale)
+    _check(_load().oracle_route(T, E, k, _ptr(z), _ptr(sc), _ptr(ids), _ptr(w),
+                                _ptr(probs)), "route")
+    return (ids, w, probs) if want_probs else (ids, w)
+
+
+def layout_capacity(T: int, E: int, k: int, S: int = 0, P: int = 128) -> int:
+    return int(_load().oracle_layout_capacity(T, E, k, S, P))
+
+
+def layout(ids, E: int, S: int = 0, P: int = 128, cap: Optional[int] = None):
+    """-> offsets [E+S+1], sorted_slots [cap], slot_row [T,k+S] (int32)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    if cap is None:
+        cap = layout_capacity(T, E, k, S, P)
+    offsets = np.empty(E + S + 1, np.int32)
+    sorted_slots = np.empty(cap, np.int32)
+    slot_row = np.empty((T, k + S), np.int32)
+    _check(_load().oracle_layout(T, E, k, S, P, _ptr(ids), _ptr(offsets),
+                                 _ptr(sorted_slots), cap, _ptr(slot_row)),
+           "layout")
+    return offsets, sorted_slots, slot_row
+
+
+def expert_rows(x, w13, w2, tok, exp_id, act_kind: int, round_h: bool = False,
+                nthreads: int = 0) -> np.ndarray:
+    """Unweighted FFN outputs y[n,H] of (token, expert) pairs."""
+    xu, w13u, w2u = _u16(x), _u16(w13), _u16(w2)
+    H = xu.shape[-1]
+    I = w2u.shape[-1]
+    tok = np.ascontiguousarray(tok, dtype=np.int64)
+    exp_id = np.ascontiguousarray(exp_id, dtype=np.int32)
+    n = tok.size
+    y = np.empty((n, H), np.float64)
+    _check(_load().oracle_expert_rows(H, I, act_kind, _ptr(xu), _ptr(w13u),
+                                      _ptr(w2u), n, _ptr(tok), _ptr(exp_id),
+                                      int(round_h), nthreads, _ptr(y)),
+           "expert_rows")
+    return y
+
+
+def forward(x, logits, w13, w2, k: int, act_kind: int, scale=None,
+            w13_sh=None, w2_sh=None, tokens=None, round_h: bool = False,
+            nthreads: int = 0):
+    """Whole layer in fp64 -> (out [n,H] float64, ids [T,k], w [T,k])."""
+    xu, w13u, w2u = _u16(x), _u16(w13), _u16(w2)
+    z = _f32(logits)
+    T, H = xu.shape
+    E = z.shape[1]
+    I = w2u.shape[-1]
+    sh13, sh2 = _u16(w13_sh), _u16(w2_sh)
+    S = 0 if sh13 is None else sh13.shape[0]
+    Is = 0 if sh2 is None else sh2.shape[-1]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, np.int64)
+    n = T if tok is None else tok.size
+    out = np.empty((n, H), np.float64)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    sc = _f32(scale)
+    _check(_load().oracle_forward(T, H, E, k, I, act_kind, S, Is, _ptr(xu),
+                                  _ptr(z), _ptr(sc), _ptr(w13u), _ptr(w2u),
+                                  _ptr(sh13), _ptr(sh2), _ptr(tok), n,
+                                  int(round_h), nthreads, _ptr(out),
+                                  _ptr(ids), _ptr(w)), "forward")
+    return out, ids, w

@@ -1,0 +1,408 @@
+/*
+ * moe_oracle.c -- plain, slow, fp64 CPU oracle for the sparse MoE
+ * feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header, table or helper with the CUDA
+ * library; the two meet only in the seeded input generators.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *   route   -- yeyulingfeng.com/587419.html, section 4 (routing math): top-k
+ *              on the raw fp32 router logits, softmax over ALL E logits, a
+ *              0/1 indicator mask of the chosen k, renormalisation of the
+ *              masked probabilities with the guard "sum > 0 ? sum : 1", and a
+ *              gather to [T,k].  Section 5 (per-expert scale) and the
+ *              Gemma4MoE routing_function on the vLLM API page
+ *              (vllm.model_executor.models.gemma4) then multiply each weight
+ *              by per_expert_scale[id] after the renormalisation.
+ *   layout  -- section 7 (tensor flow) of the same walkthrough: "token picks
+ *              k experts" is reordered into "expert receives a token list".
+ *              The pages leave the permutation unspecified; this oracle
+ *              fixes it as a stable counting sort of the flat slot t*k+j by
+ *              expert, every expert segment padded to a multiple of P rows
+ *              with -1, shared-expert segments after the routed ones.
+ *   expert  -- gated FFN of the "MOE Inference" blog (gaohongy.github.io,
+ *              "门控(Gated) FFN"): y = (Act(x.w1) (*) (x.w3)) . w2, with the
+ *              packed [w1, w3] = w13 (gate rows first, up rows second, as in
+ *              section 6 of the walkthrough and load_weights on the vLLM
+ *              page).  Act is SiLU, v/(1+e^-v), or the tanh GELU,
+ *              0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))) (walkthrough
+ *              section 6).
+ *   combine -- walkthrough section 7 step 4: the k expert outputs of a token
+ *              are summed weighted by its (scale-folded) gate weights; shared
+ *              experts (llama-cpp-visual-guide lesson 35, "shared expert")
+ *              are added with weight 1.
+ *
+ * All floating point is double; bf16 inputs convert to double exactly.
+ * Nothing is blocked, fused or reordered beyond the definitions above.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define OK 0
+#define EINVAL_ARG (-1)
+#define ENOMEM_ARG (-2)
+
+/* ---------------------------------------------------------------- helpers */
+
+static double bf16_to_double(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Round a double to the nearest bf16 value (8 significant bits, ties to
+ * even), returned as a double.  Used only by the diagnostic "round h" flag. */
+static double round_to_bf16(double v) {
+  if (v == 0.0 || !isfinite(v)) return v;
+  int e;
+  double m = frexp(v, &e);          /* v = m * 2^e, 0.5 <= |m| < 1 */
+  double r = nearbyint(ldexp(m, 8)); /* default rounding mode: ties to even */
+  return ldexp(r, e - 8);
+}
+
+int oracle_num_threads(void) {
+  long n = sysconf(_SC_NPROCESSORS_ONLN);
+  return n > 0 ? (int)n : 1;
+}
+
+typedef void (*range_fn)(void* ctx, int64_t begin, int64_t end);
+typedef struct {
+  range_fn fn;
+  void* ctx;
+  int64_t begin, end;
+} range_job;
+
+static void* range_thread(void* p) {
+  range_job* j = (range_job*)p;
+  j->fn(j->ctx, j->begin, j->end);
+  return NULL;
+}
+
+/* Run fn over [0,n) split into contiguous chunks, one per thread. */
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
+  if (nthreads <= 0) nthreads = oracle_num_threads();
+  if (nthreads > n) nthreads = (int)(n > 0 ? n : 1);
+  if (nthreads <= 1) {
+    fn(ctx, 0, n);
+    return;
+  }
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
+  range_job* jobs = (range_job*)malloc(sizeof(range_job) * nthreads);
+  int64_t chunk = (n + nthreads - 1) / nthreads;
+  int started = 0;
+  for (int i = 0; i < nthreads; ++i) {
+    int64_t b = i * chunk, e = b + chunk < n ? b + chunk : n;
+    if (b >= e) break;
+    jobs[i].fn = fn;
+    jobs[i].ctx = ctx;
+    jobs[i].begin = b;
+    jobs[i].end = e;
+    if (pthread_create(&th[i], NULL, range_thread, &jobs[i]) != 0) {
+      fn(ctx, b, e); /* could not start a thread: do the chunk inline */
+      jobs[i].fn = NULL;
+    }
+    started = i + 1;
+  }
+  for (int i = 0; i < started; ++i)
+    if (jobs[i].fn) pthread_join(th[i], NULL);
+  free(th);
+  free(jobs);
+}
+
+/* ------------------------------------------------------------ activation */
+
+/* Act(v): 0 = SiLU v/(1+exp(-v)); 1 = tanh GELU
+ * 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))). */
+static double act_fn(int act, double v) {
+  if (act == 0) return v / (1.0 + exp(-v));
+  const double c = sqrt(2.0 / M_PI);
+  return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+int oracle_act(int act, int64_t n, const double* v, double* out) {
+  if (act != 0 && act != 1) return EINVAL_ARG;
+  for (int64_t i = 0; i < n; ++i) out[i] = act_fn(act, v[i]);
+  return OK;
+}
+
+/* ----------------------------------------------------------------- route */
+
+typedef struct {
+  float v;
+  int id;
+} logit_id;
+
+/* Descending logit; equal logits go to the lower expert id first. */
+static int cmp_logit_desc(const void* a, const void* b) {
+  const logit_id* x = (const logit_id*)a;
+  const logit_id* y = (const logit_id*)b;
+  if (x->v > y->v) return -1;
+  if (x->v < y->v) return 1;
+  return (x->id > y->id) - (x->id < y->id);
+}
+
+/*
+ * Routing of every token (walkthrough section 4 steps 1-5, section 5 fold).
+ *   logits [T,E] fp32, scale [E] fp32 or NULL (= all ones)
+ *   ids    [T,k] int32 out, ordered by descending logit, ties to lower id
+ *   w      [T,k] double out (renormalised, then times scale[id])
+ *   probs  [T,E] double out or NULL: the softmax over all E (step 2)
+ * Returns -1 on a bad size or a non-finite logit.
+ */
+int oracle_route(int64_t T, int E, int k, const float* logits,
+                 const float* scale, int32_t* ids, double* w, double* probs) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return EINVAL_ARG;
+  logit_id* pairs = (logit_id*)malloc(sizeof(logit_id) * E);
+  double* p = (double*)malloc(sizeof(double) * E);
+  double* gate = (double*)malloc(sizeof(double) * E);
+  if (!pairs || !p || !gate) {
+    free(pairs); free(p); free(gate);
+    return ENOMEM_ARG;
+  }
+  int rc = OK;
+  for (int64_t t = 0; t < T && rc == OK; ++t) {
+    const float* z = logits + t * E;
+    for (int e = 0; e < E; ++e) {
+      if (!isfinite(z[e])) { rc = EINVAL_ARG; break; }
+      pairs[e].v = z[e];
+      pairs[e].id = e;
+    }
+    if (rc != OK) break;
+    /* step 1: top-k on the raw logits */
+    qsort(pairs, (size_t)E, sizeof(logit_id), cmp_logit_desc);
+    /* step 2: softmax over all E (shifted by the max, same value) */
+    double zmax = (double)pairs[0].v, den = 0.0;
+    for (int e = 0; e < E; ++e) {
+      p[e] = exp((double)z[e] - zmax);
+      den += p[e];
+    }
+    for (int e = 0; e < E; ++e) p[e] /= den;
+    if (probs) memcpy(probs + t * E, p, sizeof(double) * E);
+    /* steps 3-4: indicator of the chosen k times the probabilities */
+    for (int e = 0; e < E; ++e) gate[e] = 0.0;
+    for (int j = 0; j < k; ++j) gate[pairs[j].id] = p[pairs[j].id];
+    /* step 5: renormalise with the guard sum > 0 ? sum : 1 */
+    double renorm = 0.0;
+    for (int e = 0; e < E; ++e) renorm += gate[e];
+    if (!(renorm > 0.0)) renorm = 1.0;
+    /* gather to [T,k], then fold per_expert_scale (section 5) */
+    for (int j = 0; j < k; ++j) {
+      int id = pairs[j].id;
+      ids[t * k + j] = id;
+      double wt = gate[id] / renorm;
+      if (scale) wt *= (double)scale[id];
+      w[t * k + j] = wt;
+    }
+  }
+  free(pairs);
+  free(p);
+  free(gate);
+  return rc;
+}
+
+/* ---------------------------------------------------------------- layout */
+
+/* Rows the permuted buffers need in the worst case:
+ * T*k + T*S + (E+S)*(P-1). */
+int64_t oracle_layout_capacity(int64_t T, int E, int k, int S, int P) {
+  return T * k + T * S + (int64_t)(E + S) * (P - 1);
+}
+
+/*
+ * Stable counting sort of the flat slots s = t*k + j by expert.
+ *   offsets      [E+S+1]  start row of each segment, each a multiple of P;
+ *                         offsets[E+S] = rows in use
+ *   sorted_slots [cap]    slot held by each permuted row, -1 on padding;
+ *                         shared expert s holds tokens 0..T-1 as the slots
+ *                         T*k + s*T + t
+ *   slot_row     [T,k+S]  permuted row of (token t, choice j) and of
+ *                         (token t, shared expert s) at column k+s
+ */
+int oracle_layout(int64_t T, int E, int k, int S, int P, const int32_t* ids,
+                  int32_t* offsets, int32_t* sorted_slots, int64_t cap,
+                  int32_t* slot_row) {
+  if (T < 0 || E < 1 || k < 1 || k > E || S < 0 || P < 1) return EINVAL_ARG;
+  int G = E + S;
+  int64_t* count = (int64_t*)calloc((size_t)G, sizeof(int64_t));
+  int64_t* cursor = (int64_t*)malloc(sizeof(int64_t) * G);
+  if (!count || !cursor) {
+    free(count); free(cursor);
+    return ENOMEM_ARG;
+  }
+  for (int64_t s = 0; s < T * k; ++s) {
+    int e = ids[s];
+    if (e < 0 || e >= E) { free(count); free(cursor); return EINVAL_ARG; }
+    count[e]++;
+  }
+  for (int s = 0; s < S; ++s) count[E + s] = T;
+  int64_t off = 0;
+  for (int g = 0; g < G; ++g) {
+    offsets[g] = (int32_t)off;
+    cursor[g] = off;
+    off += (count[g] + P - 1) / P * P;
+  }
+  offsets[G] = (int32_t)off;
+  if (off > cap) { free(count); free(cursor); return EINVAL_ARG; }
+  for (int64_t r = 0; r < cap; ++r) sorted_slots[r] = -1;
+  for (int64_t s = 0; s < T * k; ++s) {
+    int64_t t = s / k, j = s % k;
+    int64_t row = cursor[ids[s]]++;
+    sorted_slots[row] = (int32_t)s;
+    slot_row[t * (k + S) + j] = (int32_t)row;
+  }
+  for (int s = 0; s < S; ++s)
+    for (int64_t t = 0; t < T; ++t) {
+      int64_t row = cursor[E + s]++;
+      sorted_slots[row] = (int32_t)(T * k + s * T + t);
+      slot_row[t * (k + S) + k + s] = (int32_t)row;
+    }
+  free(count);
+  free(cursor);
+  return OK;
+}
+
+/* ------------------------------------------------------------ expert FFN */
+
+/* y[H] += weight * W2 (Act(W1 x) (*) W3 x) for one token row, where
+ * w13e = [W1; W3] is [2I,H] and w2e is [H,I]. */
+static void ffn_row(int H, int I, int act, const uint16_t* x,
+                    const uint16_t* w13e, const uint16_t* w2e, int round_h,
+                    double weight, double* xd, double* a, double* y) {
+  for (int h = 0; h < H; ++h) xd[h] = bf16_to_double(x[h]);
+  for (int i = 0; i < I; ++i) {
+    const uint16_t* r1 = w13e + (int64_t)i * H;        /* gate row */
+    const uint16_t* r3 = w13e + (int64_t)(I + i) * H;  /* up row */
+    double g = 0.0, u = 0.0;
+    for (int h = 0; h < H; ++h) {
+      g += xd[h] * bf16_to_double(r1[h]);
+      u += xd[h] * bf16_to_double(r3[h]);
+    }
+    double v = act_fn(act, g) * u;
+    a[i] = round_h ? round_to_bf16(v) : v;
+  }
+  for (int h = 0; h < H; ++h) {
+    const uint16_t* r2 = w2e + (int64_t)h * I;
+    double acc = 0.0;
+    for (int i = 0; i < I; ++i) acc += a[i] * bf16_to_double(r2[i]);
+    y[h] += weight * acc;
+  }
+}
+
+typedef struct {
+  int H, I, act, round_h;
+  const uint16_t* x;
+  const uint16_t* w13;
+  const uint16_t* w2;
+  const int64_t* tok;
+  const int32_t* exp_id;
+  double* y;
+} rows_ctx;
+
+static void rows_worker(void* p, int64_t b, int64_t e) {
+  rows_ctx* c = (rows_ctx*)p;
+  double* xd = (double*)malloc(sizeof(double) * c->H);
+  double* a = (double*)malloc(sizeof(double) * c->I);
+  for (int64_t r = b; r < e; ++r) {
+    double* y = c->y + r * c->H;
+    for (int h = 0; h < c->H; ++h) y[h] = 0.0;
+    int64_t ex = c->exp_id[r];
+    ffn_row(c->H, c->I, c->act, c->x + c->tok[r] * c->H,
+            c->w13 + ex * 2 * (int64_t)c->I * c->H,
+            c->w2 + ex * (int64_t)c->H * c->I, c->round_h, 1.0, xd, a, y);
+  }
+  free(xd);
+  free(a);
+}
+
+/*
+ * Unweighted expert outputs of n (token, expert) pairs:
+ *   y[r,:] = W2_e (Act(W1_e x_t) (*) W3_e x_t),  t = tok[r], e = exp_id[r],
+ * with w13 [*,2I,H] and w2 [*,H,I] the packed weights of that expert set.
+ */
+int oracle_expert_rows(int H, int I, int act, const uint16_t* x,
+                       const uint16_t* w13, const uint16_t* w2, int64_t n,
+                       const int64_t* tok, const int32_t* exp_id, int round_h,
+                       int nthreads, double* y) {
+  if (H < 1 || I < 1 || (act != 0 && act != 1) || n < 0) return EINVAL_ARG;
+  rows_ctx c = {H, I, act, round_h, x, w13, w2, tok, exp_id, y};
+  parallel_for(n, nthreads, rows_worker, &c);
+  return OK;
+}
+
+/* --------------------------------------------------------------- forward */
+
+typedef struct {
+  int64_t T;
+  int H, E, k, I, act, S, Is, round_h;
+  const uint16_t *x, *w13, *w2, *w13_sh, *w2_sh;
+  const int32_t* ids;
+  const double* w;
+  const int64_t* tokens;
+  double* out;
+} fwd_ctx;
+
+static void fwd_worker(void* p, int64_t b, int64_t e) {
+  fwd_ctx* c = (fwd_ctx*)p;
+  int Imax = c->I > c->Is ? c->I : c->Is;
+  double* xd = (double*)malloc(sizeof(double) * c->H);
+  double* a = (double*)malloc(sizeof(double) * Imax);
+  for (int64_t r = b; r < e; ++r) {
+    int64_t t = c->tokens ? c->tokens[r] : r;
+    double* y = c->out + r * c->H;
+    for (int h = 0; h < c->H; ++h) y[h] = 0.0;
+    const uint16_t* xt = c->x + t * c->H;
+    for (int j = 0; j < c->k; ++j) {
+      int64_t ex = c->ids[t * c->k + j];
+      ffn_row(c->H, c->I, c->act, xt, c->w13 + ex * 2 * (int64_t)c->I * c->H,
+              c->w2 + ex * (int64_t)c->H * c->I, c->round_h,
+              c->w[t * c->k + j], xd, a, y);
+    }
+    for (int s = 0; s < c->S; ++s)
+      ffn_row(c->H, c->Is, c->act, xt,
+              c->w13_sh + (int64_t)s * 2 * c->Is * c->H,
+              c->w2_sh + (int64_t)s * c->H * c->Is, c->round_h, 1.0, xd, a, y);
+  }
+  free(xd);
+  free(a);
+}
+
+/*
+ * The whole layer for the tokens listed in ``tokens`` (NULL = all T):
+ *   out[r,:] = sum_j w[t,j] * FFN_{ids[t,j]}(x_t) + sum_s FFN_shared_s(x_t)
+ * Routing is done for all T tokens; ids_out/w_out (NULL ok) receive it.
+ */
+int oracle_forward(int64_t T, int H, int E, int k, int I, int act, int S,
+                   int Is, const uint16_t* x, const float* logits,
+                   const float* scale, const uint16_t* w13,
+                   const uint16_t* w2, const uint16_t* w13_sh,
+                   const uint16_t* w2_sh, const int64_t* tokens,
+                   int64_t n_tokens, int round_h, int nthreads, double* out,
+                   int32_t* ids_out, double* w_out) {
+  if (T < 0 || H < 1 || I < 1 || S < 0 || (S > 0 && (Is < 1 || !w13_sh || !w2_sh)))
+    return EINVAL_ARG;
+  int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (T * k + 1));
+  double* w = w_out ? w_out : (double*)malloc(sizeof(double) * (T * k + 1));
+  if (!ids || !w) return ENOMEM_ARG;
+  int rc = oracle_route(T, E, k, logits, scale, ids, w, NULL);
+  if (rc == OK) {
+    if (!tokens) n_tokens = T;
+    for (int64_t r = 0; tokens && r < n_tokens; ++r)
+      if (tokens[r] < 0 || tokens[r] >= T) rc = EINVAL_ARG;
+  }
+  if (rc == OK) {
+    fwd_ctx c = {T, H, E, k, I, act, S, Is, round_h, x, w13, w2, w13_sh,
+                 w2_sh, ids, w, tokens, out};
+    parallel_for(n_tokens, nthreads, fwd_worker, &c);
+  }
+  if (!ids_out) free(ids);
+  if (!w_out) free(w);
+  return rc;
+}

@@ -1,0 +1,277 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: the worked
+example printed in section 4 of the Gemma 4 MoE walkthrough
+(yeyulingfeng.com/587419.html), the closed form derived in the same section,
+brute-force sorting, a dense "run every expert, then discard" evaluation
+(llama-cpp-visual-guide lesson 35, the ggml_mul_mat_id section), the E=1/k=1
+plain gated MLP (walkthrough section 6, Gemma4MLP) evaluated by torch in
+float64, and torch's own SiLU / tanh-GELU in float64.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from mixture_experts_ffn_06_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_to_f64(t: torch.Tensor) -> torch.Tensor:
+    return t.to(torch.float64)
+
+
+# ----------------------------------------------------------------- routing
+
+def test_worked_example_from_the_page():
+    with open(os.path.join(GOLDEN, "route_worked_example.json")) as f:
+        g = json.load(f)
+    z = np.array([g["logits"]], np.float32)
+    ids, w, probs = oracle.route(z, g["k"], want_probs=True)
+    half4 = 0.5 * 10 ** -g["softmax_all_decimals"]
+    assert np.all(np.abs(probs[0] - g["softmax_all"]) <= half4 + 1e-12)
+    assert ids[0].tolist() == g["topk_ids"]
+    half3 = 0.5 * 10 ** -g["weights_decimals"]
+    assert np.all(np.abs(w[0] - g["topk_weights"]) <= half3 + 1e-12)
+    renorm = probs[0][ids[0]].sum()
+    assert abs(renorm - g["renorm_factor"]) <= 0.5 * 10 ** -g["renorm_factor_decimals"]
+    disp = np.zeros(4)
+    disp[ids[0]] = w[0]
+    assert np.all(np.abs(disp - g["dispatch_weights"]) <= half3 + 1e-12)
+    # the exact values the printed ones round from
+    assert w[0][0] == pytest.approx(1 / (1 + math.exp(-1)), rel=1e-15)
+
+
+def _brute_topk(row, k):
+    return sorted(range(len(row)), key=lambda e: (-float(row[e]), e))[:k]
+
+
+@pytest.mark.parametrize("E,k", [(4, 2), (8, 2), (64, 6), (128, 8), (16, 16)])
+def test_topk_matches_brute_force_and_closed_form(E, k):
+    gen = torch.Generator().manual_seed(E * 31 + k)
+    z = inputs.router_logits(50, E, k, gen, "cpu").numpy()
+    ids, w = oracle.route(z, k)
+    for t in range(z.shape[0]):
+        sel = _brute_topk(z[t], k)
+        assert ids[t].tolist() == sel
+        # walkthrough section 4: softmax-all + mask + renorm equals a softmax
+        # over the k selected logits alone
+        ex = [math.exp(float(z[t][e]) - float(z[t][sel[0]])) for e in sel]
+        den = math.fsum(ex)
+        np.testing.assert_allclose(w[t], [v / den for v in ex], rtol=1e-13,
+                                   atol=0)
+        assert math.fsum(w[t]) == pytest.approx(1.0, abs=1e-14)
+
+
+def test_topk_ties_go_to_the_lower_id():
+    z = np.array([[0.5, 0.9, 0.9, 0.1, 0.9],
+                  [1.0, 1.0, 1.0, 1.0, 1.0]], np.float32)
+    ids, w = oracle.route(z, 3)
+    assert ids[0].tolist() == [1, 2, 4]
+    assert ids[1].tolist() == [0, 1, 2]
+    np.testing.assert_allclose(w[1], [1 / 3] * 3, rtol=1e-15)
+
+
+def test_non_finite_logits_are_rejected():
+    z = np.array([[0.0, float("nan"), 1.0]], np.float32)
+    with pytest.raises(ValueError):
+        oracle.route(z, 1)
+
+
+def test_scale_fold():
+    gen = torch.Generator().manual_seed(7)
+    E, k = 16, 4
+    z = inputs.router_logits(40, E, k, gen, "cpu").numpy()
+    ids0, w0 = oracle.route(z, k)
+    ids1, w1 = oracle.route(z, k, scale=np.ones(E, np.float32))
+    assert (ids0 == ids1).all() and (w0 == w1).all()  # scale = 1 is identity
+    sc = (0.5 + np.arange(E) / E).astype(np.float32)
+    ids2, w2 = oracle.route(z, k, scale=sc)
+    assert (ids2 == ids0).all()
+    np.testing.assert_allclose(w2, w0 * sc[ids0].astype(np.float64),
+                               rtol=1e-15)
+
+
+# ------------------------------------------------------------------ layout
+
+def _brute_layout(ids, E, S, P):
+    T, k = ids.shape
+    segs = []
+    for e in range(E):
+        segs.append([t * k + j for t in range(T) for j in range(k)
+                     if ids[t, j] == e])
+    for s in range(S):
+        segs.append([T * k + s * T + t for t in range(T)])
+    offsets, rows = [0], []
+    for seg in segs:
+        padded = (len(seg) + P - 1) // P * P
+        rows += seg + [-1] * (padded - len(seg))
+        offsets.append(offsets[-1] + padded)
+    return offsets, rows
+
+
+@pytest.mark.parametrize("T,E,k,S,P", [(1, 8, 2, 0, 128), (37, 8, 2, 0, 16),
+                                       (64, 128, 8, 0, 128), (50, 64, 6, 2, 8),
+                                       (5, 4, 4, 1, 1), (0, 8, 2, 0, 128)])
+def test_layout_matches_brute_force(T, E, k, S, P):
+    gen = torch.Generator().manual_seed(T + E)
+    z = inputs.router_logits(T, E, k, gen, "cpu").numpy()
+    ids, _ = oracle.route(z, k) if T else (np.zeros((0, k), np.int32), None)
+    cap = oracle.layout_capacity(T, E, k, S, P)
+    assert cap == T * k + T * S + (E + S) * (P - 1)
+    offsets, sorted_slots, slot_row = oracle.layout(ids, E, S, P)
+    want_off, want_rows = _brute_layout(ids, E, S, P)
+    assert offsets.tolist() == want_off
+    n = want_off[-1]
+    assert sorted_slots[:n].tolist() == want_rows
+    assert (sorted_slots[n:] == -1).all()
+    assert all(o % P == 0 for o in offsets)
+    # slot_row inverts sorted_slots
+    for t in range(T):
+        for j in range(k):
+            assert sorted_slots[slot_row[t, j]] == t * k + j
+        for s in range(S):
+            assert sorted_slots[slot_row[t, k + s]] == T * k + s * T + t
+    used = sorted_slots[sorted_slots >= 0]
+    assert sorted(used.tolist()) == list(range(T * k + T * S))
+
+
+# -------------------------------------------------------------- activation
+
+def test_activations_match_torch_float64():
+    v = np.concatenate([np.linspace(-30, 30, 2001),
+                        [0.0, 1e-300, -1e-300, 5e-8, -700.0, 700.0]])
+    vt = torch.from_numpy(v)
+    np.testing.assert_allclose(oracle.act(0, v), F.silu(vt).numpy(),
+                               rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(oracle.act(1, v),
+                               F.gelu(vt, approximate="tanh").numpy(),
+                               rtol=1e-14, atol=1e-15)
+    # tanh-GELU is not erf-GELU: the pages insist on the tanh form
+    gap = np.abs(oracle.act(1, v) - F.gelu(vt).numpy()).max()
+    assert gap > 1e-5
+
+
+# ---------------------------------------------------------------- FFN/layer
+
+def _ffn_dense_torch(x, w13_e, w2_e, act_kind):
+    """Plain gated MLP in torch float64 with the gate rows first."""
+    I = w2_e.shape[-1]
+    w1, w3 = _bf16_to_f64(w13_e[:I]), _bf16_to_f64(w13_e[I:])
+    g = F.linear(x, w1)
+    u = F.linear(x, w3)
+    a = F.silu(g) if act_kind == 0 else F.gelu(g, approximate="tanh")
+    return F.linear(a * u, _bf16_to_f64(w2_e))
+
+
+@pytest.mark.parametrize("act_kind", [0, 1])
+def test_single_expert_is_a_plain_gated_mlp(act_kind):
+    shp = inputs.Shape(T=9, H=24, E=1, k=1, I=40, act=act_kind)
+    inp = inputs.make_inputs(shp, seed=3)
+    out, ids, w = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 1,
+                                 act_kind, scale=inp.scale)
+    assert (ids == 0).all() and (w == 1.0).all()
+    want = _ffn_dense_torch(_bf16_to_f64(inp.x), inp.w13[0], inp.w2[0],
+                            act_kind).numpy()
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-14)
+    # swapping the gate and up halves changes the answer (order is pinned)
+    swapped = torch.cat([inp.w13[0][40:], inp.w13[0][:40]])[None]
+    out_sw, _, _ = oracle.forward(inp.x, inp.logits, swapped, inp.w2, 1,
+                                  act_kind)
+    assert np.abs(out_sw - out).max() > 1e-3 * np.abs(out).max()
+
+
+@pytest.mark.parametrize("S", [0, 2])
+def test_sparse_equals_dense_compute_all_then_mask(S):
+    shp = inputs.Shape(T=7, H=16, E=6, k=3, I=12, act=1, n_shared=S,
+                       I_shared=20 if S else 0)
+    inp = inputs.make_inputs(shp, seed=11, scale="uniform")
+    out, ids, w = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, shp.k,
+                                 shp.act, scale=inp.scale, w13_sh=inp.w13_sh,
+                                 w2_sh=inp.w2_sh)
+    x = _bf16_to_f64(inp.x)
+    D = np.zeros((shp.T, shp.E))
+    for t in range(shp.T):
+        D[t, ids[t]] = w[t]
+    dense = np.zeros((shp.T, shp.H))
+    for e in range(shp.E):  # every expert on every token
+        ye = _ffn_dense_torch(x, inp.w13[e], inp.w2[e], shp.act).numpy()
+        dense += D[:, e:e + 1] * ye
+    for s in range(S):
+        dense += _ffn_dense_torch(x, inp.w13_sh[s], inp.w2_sh[s],
+                                  shp.act).numpy()
+    np.testing.assert_allclose(out, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_unselected_experts_are_never_read():
+    shp = inputs.Shape(T=5, H=16, E=8, k=2, I=8)
+    inp = inputs.make_inputs(shp, seed=5)
+    out, ids, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0)
+    unused = sorted(set(range(8)) - set(ids.ravel().tolist()))
+    assert unused
+    w13 = inp.w13.clone()
+    w2 = inp.w2.clone()
+    w13[unused] = float("nan")
+    w2[unused] = float("nan")
+    out2, _, _ = oracle.forward(inp.x, inp.logits, w13, w2, 2, 0)
+    assert (out2 == out).all()
+
+
+def test_scale_constant_scales_the_output():
+    shp = inputs.Shape(T=6, H=16, E=8, k=2, I=8)
+    inp = inputs.make_inputs(shp, seed=9)
+    base, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0)
+    c = np.full(8, 1.75, np.float32)
+    scaled, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0,
+                                  scale=c)
+    np.testing.assert_allclose(scaled, 1.75 * base, rtol=1e-14, atol=1e-300)
+
+
+def test_expert_rows_recombine_to_forward():
+    shp = inputs.Shape(T=8, H=32, E=4, k=2, I=16, act=1)
+    inp = inputs.make_inputs(shp, seed=2, scale="uniform")
+    out, ids, w = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 1,
+                                 scale=inp.scale, tokens=[3, 0, 7])
+    tok = np.repeat(np.arange(8), 2)
+    y = oracle.expert_rows(inp.x, inp.w13, inp.w2, tok, ids.ravel(), 1)
+    comb = (y.reshape(8, 2, 32) * w[:, :, None]).sum(1)
+    np.testing.assert_allclose(out, comb[[3, 0, 7]], rtol=1e-13, atol=1e-15)
+
+
+def test_round_h_is_a_small_perturbation():
+    shp = inputs.Shape(T=4, H=64, E=4, k=2, I=64)
+    inp = inputs.make_inputs(shp, seed=4)
+    a, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0)
+    b, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0,
+                             round_h=True)
+    rms = np.sqrt((a ** 2).mean())
+    assert 0 < np.abs(a - b).max() < 2e-2 * rms
+
+
+def test_threads_do_not_change_the_answer():
+    shp = inputs.Shape(T=16, H=32, E=8, k=2, I=16)
+    inp = inputs.make_inputs(shp, seed=6)
+    a, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0,
+                             nthreads=1)
+    b, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, 2, 0,
+                             nthreads=5)
+    assert (a == b).all()
+
+
+def test_parameter_counts_from_the_page():
+    # walkthrough section 2: one Gemma-4 expert has 3*2816*704 ~ 5.95M
+    # parameters, 128 of them ~ 761M, and the dense MLP 3*2816*2112 ~ 17.8M
+    shp = inputs.shape_of("decode_t1")
+    per_expert = 3 * shp.H * shp.I
+    assert round(per_expert / 1e6, 2) == 5.95
+    assert round(per_expert * shp.E / 1e6) == 761
+    assert round(3 * shp.H * 2112 / 1e6, 1) == 17.8
+    # lesson 35: top-2 of 8 computes a quarter of the equal-capacity dense
+    mix = inputs.shape_of("mixtral_prefill")
+    assert mix.flops() / (6.0 * mix.H * mix.I * mix.T * mix.E) == 0.25
