@@ -1,0 +1,414 @@
+"""Benchmark of the sparse MoE feed-forward layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config mixtral_prefill]
+
+One step is one whole layer (route, permute, expert FFN, combine) over one
+batch of synthetic tokens, through the C ABI call ``moe_forward``.  The
+default workload is the Mixtral-shaped prefill (T=4096, H=4096, E=8, k=2,
+I=14336, SiLU).  Inputs are resident in HBM when the timed region starts; the
+expert weights (2.8 GB) are far larger than L2, so every step streams them
+from HBM.  ``e2e`` repeats the measurement with the token inputs copied from
+pinned host memory and the output copied back inside the timed region.
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own replica of
+the layer on its own batch: the layer has no cross-GPU exchange, so there is
+no collective on the data path (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
+bounded token sample per step) and prints the same line with
+``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("MoE layer tokens/s on 1 B200 + % of roofline "
+          "(bf16 TFLOPS prefill / HBM GB/s decode)")
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", default="mixtral_prefill")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_name(cfg_name, shp):
+    act = "SiLU" if shp.act == 0 else "tanh-GELU"
+    s = (f"{cfg_name}: T={shp.T} H={shp.H} E={shp.E} k={shp.k} I={shp.I} "
+         f"{act}")
+    if shp.n_shared:
+        s += f" + {shp.n_shared} shared (I={shp.I_shared})"
+    return s
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,"
+             "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_for(kernel_src: str):
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel source still matches the one the counters were taken on."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "mixture_experts_ffn_06_b200", "csrc", kernel_src)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    ent = d.get(kernel_src)
+    if not ent or ent.get("source_sha256_16") != sha:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------- CPU baseline
+
+def cpu_oracle_rate(inp, budget_s: float = 12.0, max_rounds: int = 64):
+    """Time the oracle as it stands on the host cores, on rounds of
+    ``cores`` tokens until ``budget_s`` has passed.  Returns
+    (tokens/s, cores used, tokens, seconds)."""
+    import numpy as np
+    import oracle
+    cores = oracle.num_threads()
+    T = inp.shape.T
+    host = {k: (None if v is None else v.cpu()) for k, v in
+            dict(x=inp.x, logits=inp.logits, w13=inp.w13, w2=inp.w2,
+                 scale=inp.scale, w13_sh=inp.w13_sh, w2_sh=inp.w2_sh).items()}
+    xu = oracle._u16(host["x"])
+    w13u, w2u = oracle._u16(host["w13"]), oracle._u16(host["w2"])
+    sh13, sh2 = oracle._u16(host["w13_sh"]), oracle._u16(host["w2_sh"])
+    rng = np.random.default_rng(1)
+    per_round = min(cores, T)
+    done, elapsed, rounds = 0, 0.0, 0
+    while rounds < max_rounds and (elapsed < budget_s or rounds == 0):
+        tok = rng.choice(T, per_round, replace=False)
+        t0 = time.perf_counter()
+        oracle.forward(xu, host["logits"], w13u, w2u, inp.shape.k,
+                       inp.shape.act, scale=host["scale"], w13_sh=sh13,
+                       w2_sh=sh2, tokens=tok, nthreads=per_round)
+        elapsed += time.perf_counter() - t0
+        done += per_round
+        rounds += 1
+    return done / elapsed, per_round, done, elapsed
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_ffn_06_b200 import api, inputs
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    inp = inputs.make_inputs(args.config, seed=args.seed + rank, device=dev)
+    shp = inp.shape
+    s = api.shape_from(shp)
+    ws = api.alloc_workspace(s, dev)
+    out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        if events is None:
+            api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                            inp.w13_sh, inp.w2_sh, out, ws)
+        else:
+            api.moe_forward_staged(s, inp.x, inp.logits, inp.w13, inp.w2,
+                                   inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
+                                   events)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    status = api.moe_read_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device error during warm-up: {status}")
+
+    # ---- device-resident timed region (per-stage events on the stream)
+    nst = api.NUM_STAGES
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+                for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start before the timed work
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(stage_ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_per_step = ms_total / args.steps
+    stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev)
+                for j in range(nst)]
+    status = api.moe_read_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device error in the timed region: {status}")
+
+    # ---- end to end: pinned host inputs in, host output back, every step
+    x_h = inp.x.cpu().pin_memory()
+    z_h = inp.logits.cpu().pin_memory()
+    out_h = torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(inp.x)
+    z_d = torch.empty_like(inp.logits)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        z_d.copy_(z_h, non_blocking=True)
+        api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                        inp.w2_sh, out, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        value = world * shp.T / (ms_per_step / 1e3)
+        # dominant kernel: the w13 grouped GEMM with the fused activation
+        # (2/3 of the layer's FLOPs); algorithmic FLOPs count real rows only
+        w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) \
+            * shp.H * 2
+        w13_ms = stage_ms[3]
+        achieved = w13_flops / (w13_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        traffic = traffic_for("gemm_tc.cu")
+        layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
+        launches_per_step = 9  # route, layout x4, gather, 2 GEMMs, combine
+        cpu = None
+        if world == 1:
+            rate, cores, ntok, secs = cpu_oracle_rate(inp)
+            cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": f"{ntok} tokens drawn from the same {shp.T}-token "
+                             f"batch in rounds of {cores}, full layer per token "
+                             f"(fp64), {secs:.1f} s"}
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) tokens, N(0,0.02) bf16 random-init "
+                    "expert weights, fp32 router logits with a 1e-3 top-k margin",
+            "config": {"workload": workload_name(args.config, shp),
+                       "global_batch": world * shp.T, "seq_len": shp.T,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs larger than L2: expert weights "
+                             f"{(inp.w13.numel() + inp.w2.numel()) * 2 / 1e9:.2f} GB "
+                             "streamed every step"},
+            "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<0> "
+                         "(w13 + activation)",
+                         "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "traffic": traffic},
+            "layer_tflops": layer_tflops,
+            "stage_ms": dict(zip(api.STAGE_NAMES, stage_ms)),
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * shp.T / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+    import oracle
+    from mixture_experts_ffn_06_b200 import inputs
+
+    inp = inputs.make_inputs(args.config, seed=args.seed, device="cpu")
+    shp = inp.shape
+    cores = oracle.num_threads()
+    per_step = min(cores, shp.T)
+    xu, w13u, w2u = oracle._u16(inp.x), oracle._u16(inp.w13), oracle._u16(inp.w2)
+    sh13, sh2 = oracle._u16(inp.w13_sh), oracle._u16(inp.w2_sh)
+    rng = np.random.default_rng(1)
+
+    def step():
+        tok = rng.choice(shp.T, per_step, replace=False)
+        oracle.forward(xu, inp.logits, w13u, w2u, shp.k, shp.act,
+                       scale=inp.scale, w13_sh=sh13, w2_sh=sh2, tokens=tok,
+                       nthreads=per_step)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    secs = time.perf_counter() - t0
+    value = per_step * args.steps / secs
+    sample = (f"{per_step} tokens per step drawn from the {shp.T}-token batch, "
+              f"full layer per token in fp64")
+    result = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same recipe and seed as the CUDA arm)",
+        "config": {"workload": workload_name(args.config, shp),
+                   "global_batch": shp.T, "seq_len": shp.T,
+                   "parallelism": "single"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per_step,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+    return result
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

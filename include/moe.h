@@ -1,0 +1,203 @@
+/*
+ * moe.h -- C ABI of the sparse mixture-of-experts feed-forward layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (Gemma 4 MoE walkthrough, yeyulingfeng.com/587419.html,
+ * sections 4-7; vLLM API page vllm.model_executor.models.gemma4, class
+ * Gemma4MoE; llama-cpp-visual-guide lesson 35):
+ *
+ *   route    per token: top-k of the fp32 router logits, softmax over all E,
+ *            mask to the chosen k, renormalise, times per_expert_scale[id];
+ *   permute  reorder (token, choice) slots into expert-contiguous rows;
+ *   expert   per row: h = Act(x W1^T) (*) (x W3^T), y = h W2^T, where
+ *            W13 = [W1; W3] packs the gate rows first, then the up rows;
+ *   combine  out[t] = sum_j w[t,j] y[t,j] + sum_s y_shared[t,s]  (bf16 out).
+ *
+ * Conventions (every entry point):
+ *   - All pointers are DEVICE pointers unless a parameter says otherwise.
+ *     The caller owns every buffer.  The library never allocates, frees or
+ *     synchronises (except moe_read_error, which says so).
+ *   - Buffers are dense, row-major and 16-byte aligned.
+ *   - bf16 data is passed as uint16_t bit patterns (moe_bf16).
+ *   - Work is enqueued on ``stream`` and runs asynchronously.
+ *   - Argument and shape errors are returned before anything is launched.
+ *     A launch failure returns MOE_ERR_CUDA.  A device-side wait that runs
+ *     past its time limit records MOE_ERR_TIMEOUT in the workspace error
+ *     word (its first 4 bytes), which moe_read_error returns and clears.
+ *     Zero the first 256 bytes of a workspace once before its first use;
+ *     the workspace must be 256-byte aligned.
+ *   - Router logits must be finite.  With NaN or infinite logits the ids are
+ *     still valid expert indices but their choice is unspecified.
+ *   - Limits: 1 <= k <= min(E, 32), E <= 512, H % 8 == 0, I % 8 == 0,
+ *     n_shared <= 8 and I_shared == I when n_shared > 0, pad == 128 (or 0
+ *     for the default 128), T < 2^24.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* cudaStream_t;
+
+typedef uint16_t moe_bf16;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad pointer, size or shape */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but outside the limits above */
+  MOE_ERR_WORKSPACE = 3,   /* workspace smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  MOE_ERR_TIMEOUT = 5      /* a device-side wait gave up (see moe_read_error) */
+} moe_status;
+
+typedef enum {
+  MOE_ACT_SILU = 0,      /* v / (1 + e^-v) */
+  MOE_ACT_GELU_TANH = 1  /* 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))) */
+} moe_act;
+
+typedef struct {
+  int64_t T;        /* tokens */
+  int32_t H;        /* hidden size */
+  int32_t E;        /* routed experts */
+  int32_t k;        /* experts chosen per token */
+  int32_t I;        /* routed expert intermediate size */
+  int32_t n_shared; /* always-active shared experts S (weight 1) */
+  int32_t I_shared; /* shared expert intermediate size (== I when S > 0) */
+  int32_t act;      /* moe_act */
+  int32_t pad;      /* segment padding P in rows: 128, or 0 for 128 */
+} moe_shape;
+
+/* Rows of the permuted buffers: T*k + T*S + (E+S)*(P-1).  0 on a bad shape. */
+MOE_API int64_t moe_layout_capacity(const moe_shape* shape);
+
+/* Bytes of scratch every entry point below may use (one size for all). */
+MOE_API size_t moe_workspace_size(const moe_shape* shape);
+
+/*
+ * moe_route -- routing of every token (walkthrough section 4 steps 1-5 and
+ * section 5; Gemma4MoE.routing_function on the vLLM page).
+ *   logits [T,E] fp32, scale [E] fp32 or NULL (all ones)
+ *   ids    [T,k] int32 out: the k largest logits, in descending order, equal
+ *          logits to the lower id first (bit-exact with the oracle)
+ *   w      [T,k] fp32 out: exp(z_id - z_max) / sum over the chosen k, times
+ *          scale[id]; computed in fp64 and rounded once to fp32
+ */
+MOE_API moe_status moe_route(const moe_shape* shape, const float* logits,
+                     const float* scale, int32_t* ids, float* w,
+                     cudaStream_t stream);
+
+/*
+ * moe_permute -- the dispatch permutation (walkthrough sections 6-7: the
+ * "permutation map" turning token picks into per-expert token lists).
+ *   ids          [T,k] int32 in (each in [0,E))
+ *   offsets      [E+S+1] int32 out: first row of each expert segment; every
+ *                segment is padded to a multiple of P rows; offsets[E+S] is
+ *                the number of rows in use
+ *   sorted_slots [cap] int32 out, cap = moe_layout_capacity: the slot held by
+ *                each row, -1 on padding and past offsets[E+S].  Routed slot
+ *                t*k+j; shared expert s holds slot T*k + s*T + t.  Within a
+ *                segment slots ascend (a stable sort).
+ *   slot_row     [T,k+S] int32 out: the row of (t, j), and of (t, shared s)
+ *                at column k+s
+ *   ws           workspace of ws_bytes >= moe_workspace_size bytes
+ */
+MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
+                       int32_t* offsets, int32_t* sorted_slots,
+                       int32_t* slot_row, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/*
+ * moe_expert_ffn -- the gated expert FFN on every permuted row (walkthrough
+ * section 6; "MOE Inference" blog, gated FFN: [y1,y3] = x [w1,w3]).
+ *   x         [T,H] bf16
+ *   offsets, sorted_slots  from moe_permute
+ *   w13       [E,2I,H] bf16: rows [0,I) gate (w1), rows [I,2I) up (w3)
+ *   w2        [E,H,I] bf16
+ *   w13_sh    [S,2I,H] bf16 or NULL when S == 0;  w2_sh [S,H,I] likewise
+ *   y_perm    [cap,H] bf16 out: unweighted expert output of every row in use;
+ *             padding rows get 0, rows past offsets[E+S] are not written
+ * h = Act(g) (*) u is rounded to bf16 (the second GEMM's operand); every
+ * product accumulates in fp32 on the tensor cores.
+ */
+MOE_API moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
+                          const int32_t* offsets, const int32_t* sorted_slots,
+                          const moe_bf16* w13, const moe_bf16* w2,
+                          const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                          moe_bf16* y_perm, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/*
+ * moe_combine -- weighted combine (walkthrough section 7 step 4; the weighted
+ * sum after ggml_mul_mat_id in lesson 35), with shared experts at weight 1.
+ *   y_perm [cap,H] bf16, slot_row [T,k+S] int32, w [T,k] fp32
+ *   out    [T,H] bf16 out, summed in fp32 and rounded once
+ */
+MOE_API moe_status moe_combine(const moe_shape* shape, const moe_bf16* y_perm,
+                       const int32_t* slot_row, const float* w, moe_bf16* out,
+                       cudaStream_t stream);
+
+/*
+ * moe_forward -- the whole layer: route, permute, expert FFN and combine on
+ * one stream, with every intermediate in the workspace (vLLM FusedMoE as the
+ * walkthrough's section 6 describes it).  ids_out [T,k] and w_out [T,k] may
+ * be NULL; when given they receive the routing.
+ */
+MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
+                       const float* logits, const moe_bf16* w13,
+                       const moe_bf16* w2, const float* scale,
+                       const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                       moe_bf16* out, int32_t* ids_out, float* w_out,
+                       void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * moe_forward_staged -- moe_forward that also records CUDA events between its
+ * stages, for per-kernel timing on the launch stream.  stage_events is NULL
+ * or an array of MOE_NUM_STAGES + 1 cudaEvent_t created by the caller; event
+ * i is recorded before stage i and event MOE_NUM_STAGES after the last one.
+ * Stages: 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
+ * 4 w2 GEMM, 5 combine.
+ */
+#define MOE_NUM_STAGES 6
+MOE_API moe_status moe_forward_staged(
+    const moe_shape* shape, const moe_bf16* x, const float* logits,
+    const moe_bf16* w13, const moe_bf16* w2, const float* scale,
+    const moe_bf16* w13_sh, const moe_bf16* w2_sh, moe_bf16* out,
+    int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes,
+    void* const* stage_events, cudaStream_t stream);
+
+/*
+ * moe_read_error -- SYNCHRONISES ``stream``, then returns the status recorded
+ * in the workspace error word by earlier calls on it (MOE_OK if none) and
+ * clears the word.  ws is the device workspace used by those calls.
+ */
+MOE_API moe_status moe_read_error(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * moe_selftest_wait_timeout -- exercises the device-side wait limit: launches
+ * one block that waits on a flag nothing ever sets, for at most timeout_us
+ * microseconds, then records MOE_ERR_TIMEOUT in the workspace error word and
+ * returns.  No GPU fault, trap or hang is involved.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes,
+                                     uint32_t timeout_us, cudaStream_t stream);
+
+/* A static, human-readable name for a status. */
+MOE_API const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

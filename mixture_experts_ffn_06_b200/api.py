@@ -1,0 +1,189 @@
+"""Python binding of the C ABI in ``include/moe.h`` (argument marshalling only).
+
+Every function has the name of the C entry point it calls and forwards torch
+CUDA tensors as raw device pointers on the current torch stream.  Nothing is
+computed here: there is no CPU or PyTorch fallback, and importing this module
+without the built ``libmoe_b200.so`` raises.  Build it with
+``python -m mixture_experts_ffn_06_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+NUM_STAGES = 6
+STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act", "w2_gemm",
+               "combine")
+EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_route",
+           "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+           "moe_forward_staged",
+           "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} returned {STATUS_NAMES.get(status, status)}")
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("I_shared", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("pad", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m mixture_experts_ffn_06_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S = ctypes.c_void_p, ctypes.POINTER(moe_shape)
+    st = ctypes.c_int
+    lib.moe_layout_capacity.argtypes = [S]
+    lib.moe_layout_capacity.restype = ctypes.c_int64
+    lib.moe_workspace_size.argtypes = [S]
+    lib.moe_workspace_size.restype = ctypes.c_size_t
+    lib.moe_route.argtypes = [S, P, P, P, P, P]
+    lib.moe_permute.argtypes = [S, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.moe_expert_ffn.argtypes = [S, P, P, P, P, P, P, P, P, P,
+                                   ctypes.c_size_t, P]
+    lib.moe_combine.argtypes = [S, P, P, P, P, P]
+    lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P,
+                                ctypes.c_size_t, P]
+    lib.moe_forward_staged.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P,
+                                       ctypes.c_size_t, P, P]
+    lib.moe_read_error.argtypes = [P, ctypes.c_size_t, P]
+    lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t,
+                                              ctypes.c_uint32, P]
+    lib.moe_status_string.argtypes = [st]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+                 "moe_forward", "moe_forward_staged", "moe_read_error", "moe_selftest_wait_timeout"):
+        getattr(lib, name).restype = st
+    return lib
+
+
+lib = _load()
+
+
+def make_shape(T: int, H: int, E: int, k: int, I: int, act: int = 0,
+               n_shared: int = 0, I_shared: int = 0, pad: int = 0) -> moe_shape:
+    return moe_shape(T, H, E, k, I, n_shared, I_shared, act, pad)
+
+
+def shape_from(s) -> moe_shape:
+    """From an ``inputs.Shape`` (or anything with the same attributes)."""
+    return make_shape(s.T, s.H, s.E, s.k, s.I, s.act, s.n_shared, s.I_shared)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def moe_status_string(status: int) -> str:
+    return lib.moe_status_string(status).decode()
+
+
+def moe_layout_capacity(shape: moe_shape) -> int:
+    return int(lib.moe_layout_capacity(ctypes.byref(shape)))
+
+
+def moe_workspace_size(shape: moe_shape) -> int:
+    return int(lib.moe_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: moe_shape, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace (torch allocation), error word zeroed."""
+    n = moe_workspace_size(shape)
+    if n == 0:
+        raise MoEError(1, "moe_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def moe_route(shape, logits, scale, ids, w, stream=None):
+    _check(lib.moe_route(ctypes.byref(shape), _p(logits), _p(scale), _p(ids),
+                         _p(w), _stream(stream)), "moe_route")
+
+
+def moe_permute(shape, ids, offsets, sorted_slots, slot_row, ws, stream=None):
+    _check(lib.moe_permute(ctypes.byref(shape), _p(ids), _p(offsets),
+                           _p(sorted_slots), _p(slot_row), _p(ws), ws.numel(),
+                           _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(shape, x, offsets, sorted_slots, w13, w2, w13_sh, w2_sh,
+                   y_perm, ws, stream=None):
+    _check(lib.moe_expert_ffn(ctypes.byref(shape), _p(x), _p(offsets),
+                              _p(sorted_slots), _p(w13), _p(w2), _p(w13_sh),
+                              _p(w2_sh), _p(y_perm), _p(ws), ws.numel(),
+                              _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(shape, y_perm, slot_row, w, out, stream=None):
+    _check(lib.moe_combine(ctypes.byref(shape), _p(y_perm), _p(slot_row), _p(w),
+                           _p(out), _stream(stream)), "moe_combine")
+
+
+def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
+                ids_out=None, w_out=None, stream=None):
+    _check(lib.moe_forward(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
+                           _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
+                           _p(ids_out), _p(w_out), _p(ws), ws.numel(),
+                           _stream(stream)), "moe_forward")
+
+
+def moe_forward_staged(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
+                       ws, events, ids_out=None, w_out=None, stream=None):
+    """moe_forward recording ``events`` (NUM_STAGES + 1 torch.cuda.Event,
+    created with enable_timing=True) around its stages."""
+    if len(events) != NUM_STAGES + 1:
+        raise ValueError("need NUM_STAGES + 1 events")
+    arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
+        *[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib.moe_forward_staged(ctypes.byref(shape), _p(x), _p(logits),
+                                  _p(w13), _p(w2), _p(scale), _p(w13_sh),
+                                  _p(w2_sh), _p(out), _p(ids_out), _p(w_out),
+                                  _p(ws), ws.numel(), arr, _stream(stream)),
+           "moe_forward_staged")
+
+
+def moe_read_error(ws, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the workspace error word."""
+    return int(lib.moe_read_error(_p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_selftest_wait_timeout(ws, timeout_us: int, stream=None):
+    _check(lib.moe_selftest_wait_timeout(_p(ws), ws.numel(), timeout_us,
+                                         _stream(stream)),
+           "moe_selftest_wait_timeout")

@@ -1,0 +1,427 @@
+// gemm_tc.cu -- grouped expert GEMMs on the sm_100a tensor cores.
+//
+// The expert FFN of the Gemma 4 MoE walkthrough (yeyulingfeng.com/587419.html
+// section 6; "MOE Inference" blog, gated FFN) is two grouped GEMMs over the
+// expert-contiguous rows built by layout.cu:
+//   mode 0 (w13): h[r, n] = Act(x_r . W1_e[n]) * (x_r . W3_e[n]),  n < I
+//   mode 1 (w2):  y[r, n] = h_r . W2_e[n],                         n < H
+// The pages batch these as FusedMoE's grouped GEMM (walkthrough section 7
+// step 3) and ggml_mul_mat_id (llama-cpp-visual-guide lesson 35); their
+// Triton / ggml kernels are prior art only.  This kernel is written for
+// B200:
+//
+//   * persistent: one 192-thread CTA per SM walks the tile list
+//     (expert-major, then n-tile, then m-tile, so the CTAs running at once
+//     share weight tiles through L2);
+//   * warp 0 lane 0 is the TMA producer: 128x64 A tiles and 256x64 B tiles
+//     (mode 0: 128 gate rows + the matching 128 up rows) into a 4-stage ring
+//     of 128-byte-swizzled shared memory;
+//   * warp 1 lane 0 issues tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32)
+//     into one of two 256-column TMEM accumulators and releases ring slots
+//     and accumulators with tcgen05.commit;
+//   * warps 2-5 are the epilogue: tcgen05.ld of their 32 TMEM lanes, the
+//     gate activation fused in mode 0 (so g and u never reach HBM), bf16
+//     stores.  Two accumulators let the epilogue of tile i overlap the MMAs
+//     of tile i+1.
+// Every wait is bounded (tc_ptx.cuh: mbar_wait); on a timeout the block
+// records MOE_ERR_TIMEOUT, drains what it issued and frees its TMEM.
+#include <mutex>
+
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN_ACC = 256;
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;       // 16 KiB
+constexpr int B_STAGE = BN_ACC * BK * 2;   // 32 KiB
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN_ACC;
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+struct KParams {
+  const int32_t* offsets;
+  int G, E, N, K, NT, KB;
+  int32_t b_rows_per_group;  // rows of one expert in the B tensor
+  int32_t up_off;            // mode 0: row offset of the up half (= N)
+  __nv_bfloat16* out;
+  int act;
+  uint32_t* err;
+  uint64_t timeout_ns;
+};
+
+struct Tile {
+  int g;
+  int64_t row0;
+  int n0;
+};
+
+template <int MODE>
+__device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs, int G,
+                                         int NT) {
+  constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
+  int lo = 0, hi = G - 1;  // last g with (offs[g]/BM)*NT <= i
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)(offs[mid] / BM) * NT <= i) lo = mid; else hi = mid - 1;
+  }
+  const int64_t mt0 = offs[lo] / BM;
+  const int64_t mtg = (offs[lo + 1] - offs[lo]) / BM;
+  const int64_t local = i - mt0 * NT;
+  const int64_t nt = local / mtg;
+  const int64_t mt = local - nt * mtg;
+  return Tile{lo, (mt0 + mt) * BM, (int)nt * BN_OUT};
+}
+
+__device__ __forceinline__ float act_apply(int act, float g) {
+  if (act == MOE_ACT_SILU) return g / (1.0f + expf(-g));
+  const float c = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * g * (1.0f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmBs, const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sA = base;
+  const uint32_t sB = base + STAGES * A_STAGE;
+  Ctl* ctl = reinterpret_cast<Ctl*>(gbase + STAGES * (A_STAGE + B_STAGE));
+  int32_t* offs = reinterpret_cast<int32_t*>(ctl + 1);
+  volatile int32_t* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p.G; i += THREADS) offs[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&ctl->tmem_full[a]), 1);
+      mbar_init(smem_u32(&ctl->tmem_empty[a]), 128);
+    }
+    mbar_init(smem_u32(&ctl->drain), 1);
+    ctl->abort_flag = 0;
+    mbar_init_fence();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBs);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int64_t total = (int64_t)(offs[p.G] / BM) * p.NT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int32_t last_fill[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_fill[s] = -1;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const Tile tl = map_tile<MODE>(t, offs, p.G, p.NT);
+        const bool routed = tl.g < p.E;
+        const CUtensorMap* mb = routed ? &tmB : &tmBs;
+        const int32_t gl = routed ? tl.g : tl.g - p.E;
+        const int32_t brow = gl * p.b_rows_per_group + tl.n0;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          const uint32_t fb = smem_u32(&ctl->full[stage]);
+          if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
+                         p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(fb, A_STAGE + B_STAGE);
+          tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0, fb);
+          if (MODE == 0) {
+            tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+            tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * BK,
+                        brow + p.up_off, fb);
+          } else {
+            tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+          }
+          last_fill[stage] = (int32_t)phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the block exits
+        int32_t none = 0;
+        volatile int32_t* never = &none;
+        for (int s = 0; s < STAGES; ++s)
+          if (last_fill[s] >= 0)
+            mbar_wait(smem_u32(&ctl->full[s]), (uint32_t)last_fill[s], never,
+                      p.timeout_ns, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN_ACC);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        if (!mbar_wait(smem_u32(&ctl->tmem_empty[acc]), acc_phase ^ 1u, abort_flag,
+                       p.timeout_ns, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN_ACC;
+        for (int kb = 0; kb < p.KB; ++kb) {
+          if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, abort_flag,
+                         p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_kmajor_desc(sA + stage * A_STAGE);
+          const uint64_t bd = sw128_kmajor_desc(sB + stage * B_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(d, ad + 2u * kk, bd + 2u * kk, idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(smem_u32(&ctl->empty[stage]));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&ctl->tmem_full[acc]));
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok || *abort_flag) {
+        // wait for the MMAs already issued before TMEM is released
+        int32_t none = 0;
+        volatile int32_t* never = &none;
+        umma_commit(smem_u32(&ctl->drain));
+        mbar_wait(smem_u32(&ctl->drain), 0, never, p.timeout_ns, p.err);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
+    uint32_t acc = 0, acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+      const Tile tl = map_tile<MODE>(t, offs, p.G, p.NT);
+      const bool got = mbar_wait(smem_u32(&ctl->tmem_full[acc]), acc_phase,
+                                 abort_flag, p.timeout_ns, p.err);
+      // warp-uniform decision; also reconverges the warp for tcgen05.ld
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
+      const int64_t row = tl.row0 + q * 32 + lane;
+      __nv_bfloat16* orow = p.out + row * (int64_t)p.N;
+      if (MODE == 0) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = tl.n0 + c * 32;
+          if (col0 >= p.N) break;
+          uint32_t g[32], u[32];
+          tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            if (col0 + v * 8 < p.N) {
+              uint4 o;
+              uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i0 = v * 8 + 2 * e;
+                const float h0 = act_apply(p.act, __uint_as_float(g[i0])) *
+                                 __uint_as_float(u[i0]);
+                const float h1 = act_apply(p.act, __uint_as_float(g[i0 + 1])) *
+                                 __uint_as_float(u[i0 + 1]);
+                op[e] = pack_bf16x2(h0, h1);
+              }
+              *reinterpret_cast<uint4*>(orow + col0 + v * 8) = o;
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = tl.n0 + c * 32;
+          if (col0 >= p.N) break;
+          uint32_t y[32];
+          tmem_ld32(tb + c * 32, y);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            if (col0 + v * 8 < p.N) {
+              uint4 o;
+              uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                op[e] = pack_bf16x2(__uint_as_float(y[v * 8 + 2 * e]),
+                                    __uint_as_float(y[v * 8 + 2 * e + 1]));
+              *reinterpret_cast<uint4*>(orow + col0 + v * 8) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [outer, inner] row-major bf16 tensor, box {64, box_rows}, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* ptr, uint64_t inner,
+                     uint64_t outer, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
+  constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
+  CUtensorMap mA, mB, mBs;
+  cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM);
+  if (e != cudaSuccess) return e;
+  const uint64_t rows_per_group = MODE == 0 ? 2ull * a.N : (uint64_t)a.N;
+  const uint32_t box_rows = MODE == 0 ? BN_ACC / 2 : BN_ACC;
+  e = make_map(&mB, a.B, (uint64_t)a.K, rows_per_group * (uint64_t)a.E, box_rows);
+  if (e != cudaSuccess) return e;
+  if (a.B_sh && a.G > a.E) {
+    e = make_map(&mBs, a.B_sh, (uint64_t)a.K,
+                 rows_per_group * (uint64_t)(a.G - a.E), box_rows);
+    if (e != cudaSuccess) return e;
+  } else {
+    mBs = mB;
+  }
+  KParams p;
+  p.offsets = a.offsets;
+  p.G = a.G;
+  p.E = a.E;
+  p.N = a.N;
+  p.K = a.K;
+  p.NT = (a.N + BN_OUT - 1) / BN_OUT;
+  p.KB = (a.K + BK - 1) / BK;
+  p.b_rows_per_group = (int32_t)rows_per_group;
+  p.up_off = MODE == 0 ? a.N : 0;
+  p.out = a.out;
+  p.act = a.act;
+  p.err = a.err;
+  p.timeout_ns = kTimeoutNs;
+
+  const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + sizeof(Ctl) +
+                      sizeof(int32_t) * (size_t)(a.G + 1);
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t max_tiles = (a.cap / BM) * p.NT;
+  int grid = num_sms();
+  if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
+  grouped_gemm_kernel<MODE><<<grid, THREADS, smem, st>>>(mA, mB, mBs, p);
+  return cudaGetLastError();
+}
+
+__global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    mbar_init_fence();
+  }
+  __syncthreads();
+  // nothing ever arrives on ``bar``: the bounded wait must give up
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns, err);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
+  return a.mode == 0 ? launch_mode<0>(a, st) : launch_mode<1>(a, st);
+}
+
+cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
+                                 cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(err, (uint64_t)timeout_us * 1000ull);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,101 @@
+// internal.cuh -- shared declarations of the MoE library's translation units:
+// the workspace map, launch wrappers, and the device-side wait helpers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kSegPad = 128;       // rows per expert-segment granule (GEMM M tile)
+constexpr int kLayoutTile = 1024;  // slots per layout block
+constexpr int kMaxExperts = 512;
+constexpr int kMaxShared = 8;
+constexpr int kMaxTopK = 32;
+
+// Device error word values are moe_status codes.
+constexpr uint32_t kErrTimeout = MOE_ERR_TIMEOUT;
+
+// Byte offsets of everything that lives in the caller's workspace.
+struct WsMap {
+  size_t err;          // uint32 error word (+ padding)
+  size_t ids, w;       // [T,k] int32 / fp32 (moe_forward)
+  size_t offsets;      // [G+1] int32
+  size_t sorted_slots; // [cap] int32
+  size_t slot_row;     // [T,k+S] int32
+  size_t lt_count;     // [n_lt, E] int32 per-layout-block histograms
+  size_t lt_base;      // [n_lt, E] int32 per-layout-block exclusive bases
+  size_t lt_rank;      // [T*k] int32 stable rank inside the layout block
+  size_t x_perm;       // [cap,H] bf16 gathered activations
+  size_t h;            // [cap,I] bf16 gated intermediate
+  size_t y_perm;       // [cap,H] bf16 expert outputs (moe_forward)
+  size_t total;
+  int64_t cap;
+  int64_t n_lt;
+};
+
+WsMap workspace_map(const moe_shape& s);
+
+// ---- launch wrappers (return cudaGetLastError of the launch) ----
+cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
+                         int E, int k, int32_t* ids, float* w, cudaStream_t st);
+
+cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
+                          int32_t* offsets, int32_t* sorted_slots,
+                          int32_t* slot_row, int64_t cap, int32_t* lt_count,
+                          int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
+                          cudaStream_t st);
+
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
+                          const int32_t* offsets, int G, int64_t T, int k,
+                          int H, int64_t cap, __nv_bfloat16* x_perm,
+                          cudaStream_t st);
+
+cudaError_t launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row,
+                           const float* w, int64_t T, int k, int S, int H,
+                           __nv_bfloat16* out, cudaStream_t st);
+
+// Grouped GEMMs on tcgen05.  mode 0: h = Act(A W1^T) (*) (A W3^T) with B the
+// packed [G][2N][K] gate/up rows; mode 1: y = A W^T with B = [G][N][K].
+struct GroupedGemmArgs {
+  int mode;
+  const __nv_bfloat16* A;       // [cap, K]
+  const __nv_bfloat16* B;       // routed experts' weights
+  const __nv_bfloat16* B_sh;    // shared experts' weights (or nullptr)
+  const int32_t* offsets;       // [G+1]
+  int G, E;                     // groups, routed groups
+  int N, K;                     // output columns, reduction length
+  int64_t cap;                  // rows of A / out
+  __nv_bfloat16* out;           // [cap, N]
+  int act;
+  uint32_t* err;
+};
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
+
+cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
+                                 cudaStream_t st);
+
+// ---------------------------------------------------------------- device
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
+  if (err) atomicCAS(err, 0u, code);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace moe

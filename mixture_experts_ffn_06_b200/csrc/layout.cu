@@ -1,0 +1,236 @@
+// layout.cu -- the dispatch permutation and the activation gather.
+//
+// The Gemma 4 MoE walkthrough (yeyulingfeng.com/587419.html, sections 6-7)
+// describes FusedMoE's dispatch as a "permutation map" that turns
+// "each token picked k experts" into "each expert received a token list",
+// without moving tokens; the pages leave the map itself open.  Here it is a
+// stable counting sort of the flat slots s = t*k + j by expert, each expert
+// segment padded to a multiple of 128 rows (the GEMM M tile), with the
+// always-active shared experts (llama-cpp-visual-guide lesson 35) appended
+// as segments that hold every token.
+//
+// Three launches, all integer work, coalesced:
+//   layout_count   one block per 1024 slots: stable rank of every slot among
+//                  the equal-expert slots of its block (warp match + per-warp
+//                  counts) and the block histogram;
+//   layout_scan    one block: per-expert exclusive scan over blocks, padded
+//                  segment sizes and their exclusive scan -> offsets;
+//   layout_scatter every slot writes sorted_slots[row] and slot_row;
+//   layout_pad     padding rows and rows past the last segment get -1.
+// gather_rows then copies x[token] into x_perm[row] (zeros on padding) with
+// 16-byte vector loads, one warp per row.
+#include "internal.cuh"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(kLayoutTile)
+layout_count(const int32_t* __restrict__ ids, int64_t R, int E,
+             int32_t* __restrict__ lt_count, int32_t* __restrict__ lt_rank) {
+  extern __shared__ int32_t wc[];  // [32 warps][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 32 * E; i += blockDim.x) wc[i] = 0;
+  __syncthreads();
+
+  const int64_t s = (int64_t)blockIdx.x * kLayoutTile + tid;
+  const int e = (s < R) ? __ldg(ids + s) : -1;
+  const bool valid = (e >= 0 && e < E);
+  const int key = valid ? e : -1;
+  const uint32_t peers = __match_any_sync(0xffffffffu, key);
+  const uint32_t lower = peers & ((1u << lane) - 1u);
+  const int rank_in_warp = __popc(lower);
+  if (valid && lower == 0) wc[warp * E + e] = __popc(peers);
+  __syncthreads();
+
+  if (valid) {
+    int base = 0;
+    for (int w2 = 0; w2 < warp; ++w2) base += wc[w2 * E + e];
+    lt_rank[s] = base + rank_in_warp;
+  }
+  for (int x = tid; x < E; x += blockDim.x) {
+    int c = 0;
+    for (int w2 = 0; w2 < 32; ++w2) c += wc[w2 * E + x];
+    lt_count[(int64_t)blockIdx.x * E + x] = c;
+  }
+}
+
+__global__ void __launch_bounds__(1024)
+layout_scan(const int32_t* __restrict__ lt_count, int64_t n_lt, int E, int S,
+            int64_t T, int P, int32_t* __restrict__ lt_base,
+            int32_t* __restrict__ offsets) {
+  __shared__ int32_t seg[kMaxExperts + kMaxShared + 1];
+  __shared__ int32_t warp_sum[32];
+  const int tid = threadIdx.x;
+  const int G = E + S;
+  // per-expert running sum over layout blocks
+  for (int e = tid; e < G; e += blockDim.x) {
+    int64_t total = 0;
+    if (e < E) {
+      for (int64_t b = 0; b < n_lt; ++b) {
+        lt_base[b * E + e] = (int32_t)total;
+        total += lt_count[b * E + e];
+      }
+    } else {
+      total = T;
+    }
+    seg[e] = (int32_t)((total + P - 1) / P * P);
+  }
+  __syncthreads();
+  // exclusive scan of seg[0..G) (G <= 520 < 1024: one element per thread)
+  const int lane = tid & 31, warp = tid >> 5;
+  int v = (tid < G) ? seg[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sum[lane];
+    int wincl = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wincl, off);
+      if (lane >= off) wincl += n;
+    }
+    warp_sum[lane] = wincl - ws;  // exclusive
+  }
+  __syncthreads();
+  const int excl = incl - v + warp_sum[warp];
+  if (tid < G) offsets[tid] = excl;
+  if (tid == G - 1) offsets[G] = excl + v;
+}
+
+// Index space: [0,R) routed slots, then [R, R+T*S) shared-expert slots.
+__global__ void __launch_bounds__(256)
+layout_scatter(const int32_t* __restrict__ ids, int64_t T, int k, int E, int S,
+               const int32_t* __restrict__ offsets,
+               const int32_t* __restrict__ lt_base,
+               const int32_t* __restrict__ lt_rank,
+               int32_t* __restrict__ sorted_slots,
+               int32_t* __restrict__ slot_row) {
+  const int64_t R = T * k, RS = T * S;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < R + RS;
+       i += stride) {
+    if (i < R) {
+      const int e = ids[i];
+      const int64_t b = i / kLayoutTile;
+      const int64_t row = (int64_t)offsets[e] + lt_base[b * E + e] + lt_rank[i];
+      sorted_slots[row] = (int32_t)i;
+      const int64_t t = i / k, j = i - t * k;
+      slot_row[t * (k + S) + j] = (int32_t)row;
+    } else {
+      const int64_t q = i - R, s = q / T, t = q - s * T;
+      const int64_t row = (int64_t)offsets[E + s] + t;
+      sorted_slots[row] = (int32_t)(R + q);
+      slot_row[t * (k + S) + k + s] = (int32_t)row;
+    }
+  }
+}
+
+// Padding rows: block g < G clears segment g's tail (its slots fill rows
+// [offsets[g], offsets[g] + count_g); the rest up to offsets[g+1] get -1);
+// the blocks past G clear the rows from offsets[G] to cap.
+__global__ void __launch_bounds__(256)
+layout_pad(const int32_t* __restrict__ offsets, const int32_t* __restrict__ lt_base,
+           const int32_t* __restrict__ lt_count, int64_t n_lt, int E, int S,
+           int64_t T, int P, int64_t cap, int32_t* __restrict__ sorted_slots) {
+  const int G = E + S;
+  const int g = blockIdx.x;
+  if (g < G) {
+    int64_t count;
+    if (g < E) {
+      count = (n_lt > 0) ? (int64_t)lt_base[(n_lt - 1) * E + g] +
+                               lt_count[(n_lt - 1) * E + g]
+                         : 0;
+    } else {
+      count = T;
+    }
+    const int64_t beg = offsets[g] + count, end = offsets[g + 1];
+    for (int64_t r = beg + threadIdx.x; r < end; r += blockDim.x)
+      sorted_slots[r] = -1;
+  } else {
+    // rows past offsets[G]
+    const int64_t used = offsets[G];
+    const int64_t stride = (int64_t)(gridDim.x - G) * blockDim.x;
+    for (int64_t r = used + (int64_t)(g - G) * blockDim.x + threadIdx.x; r < cap;
+         r += stride)
+      sorted_slots[r] = -1;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slots,
+            const int32_t* __restrict__ offsets, int G, int64_t T, int k,
+            int H, uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t rows = offsets[G];
+  const int chunks = H >> 3;  // 8 bf16 per 16-byte chunk
+  const int64_t R = T * k;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < rows; r += warps) {
+    const int s = sorted_slots[r];
+    uint4* dst = x_perm + r * chunks;
+    if (s < 0) {
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      for (int c = lane; c < chunks; c += 32) dst[c] = z;
+      continue;
+    }
+    const int64_t t = (s < R) ? (int64_t)s / k : ((int64_t)s - R) % T;
+    const uint4* src = x + t * chunks;
+    for (int c = lane; c < chunks; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
+                          int32_t* offsets, int32_t* sorted_slots,
+                          int32_t* slot_row, int64_t cap, int32_t* lt_count,
+                          int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
+                          cudaStream_t st) {
+  const int64_t R = s.T * s.k;
+  const int E = s.E, S = s.n_shared, G = E + S;
+  const int P = s.pad ? s.pad : kSegPad;
+  if (R > 0) {
+    const size_t smem = sizeof(int32_t) * 32 * (size_t)E;
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(
+          layout_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    layout_count<<<(unsigned)n_lt, kLayoutTile, smem, st>>>(ids, R, E, lt_count,
+                                                           lt_rank);
+  }
+  layout_scan<<<1, 1024, 0, st>>>(lt_count, R > 0 ? n_lt : 0, E, S, s.T, P,
+                                  lt_base, offsets);
+  const int64_t work = R + s.T * S;
+  if (work > 0) {
+    const int64_t blocks = (work + 255) / 256;
+    layout_scatter<<<(unsigned)(blocks < 65535 * 16 ? blocks : 65535 * 16), 256,
+                     0, st>>>(ids, s.T, s.k, E, S, offsets, lt_base, lt_rank,
+                              sorted_slots, slot_row);
+  }
+  layout_pad<<<(unsigned)(G + 148), 256, 0, st>>>(
+      offsets, lt_base, lt_count, R > 0 ? n_lt : 0, E, S, s.T, P, cap,
+      sorted_slots);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
+                          const int32_t* offsets, int G, int64_t T, int k,
+                          int H, int64_t cap, __nv_bfloat16* x_perm,
+                          cudaStream_t st) {
+  const int64_t want = (cap + 7) / 8;
+  const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+  gather_rows<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(x), sorted_slots, offsets, G, T, k, H,
+      reinterpret_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

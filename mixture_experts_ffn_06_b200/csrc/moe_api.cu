@@ -1,0 +1,301 @@
+// moe_api.cu -- the C entry points declared in include/moe.h: argument
+// checks, the workspace map, and the launch sequence of each call.  Every
+// argument error is returned before anything is enqueued; nothing here
+// allocates, frees or synchronises (moe_read_error excepted, as documented).
+#include "internal.cuh"
+
+namespace moe {
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static int seg_pad(const moe_shape& s) { return s.pad ? s.pad : kSegPad; }
+
+WsMap workspace_map(const moe_shape& s) {
+  WsMap m{};
+  const int64_t T = s.T, k = s.k, S = s.n_shared, G = s.E + s.n_shared;
+  const int P = seg_pad(s);
+  m.cap = T * k + T * S + G * (P - 1);
+  m.n_lt = (T * k + kLayoutTile - 1) / kLayoutTile;
+  if (m.n_lt < 1) m.n_lt = 1;
+  const int64_t Imax = s.I > s.I_shared ? s.I : s.I_shared;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  m.err = take(256);
+  m.ids = take(sizeof(int32_t) * T * k);
+  m.w = take(sizeof(float) * T * k);
+  m.offsets = take(sizeof(int32_t) * (G + 1));
+  m.sorted_slots = take(sizeof(int32_t) * m.cap);
+  m.slot_row = take(sizeof(int32_t) * T * (k + S));
+  m.lt_count = take(sizeof(int32_t) * m.n_lt * s.E);
+  m.lt_base = take(sizeof(int32_t) * m.n_lt * s.E);
+  m.lt_rank = take(sizeof(int32_t) * T * k);
+  m.x_perm = take(2ull * m.cap * s.H);
+  m.h = take(2ull * m.cap * Imax);
+  m.y_perm = take(2ull * m.cap * s.H);
+  m.total = o;
+  return m;
+}
+
+static moe_status check_shape(const moe_shape* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->E <= 0 || s->k <= 0 || s->I <= 0 ||
+      s->n_shared < 0 || s->pad < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->act != MOE_ACT_SILU && s->act != MOE_ACT_GELU_TANH)
+    return MOE_ERR_INVALID_ARG;
+  if (s->E > kMaxExperts || s->k > kMaxTopK || s->n_shared > kMaxShared)
+    return MOE_ERR_UNSUPPORTED;
+  if (s->H % 8 != 0 || s->I % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (s->n_shared > 0 && s->I_shared != s->I) return MOE_ERR_UNSUPPORTED;
+  if (s->pad != 0 && s->pad != kSegPad) return MOE_ERR_UNSUPPORTED;
+  if (s->T >= (int64_t(1) << 24)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+static moe_status from_cuda(cudaError_t e) {
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static moe_status check_ws(const moe_shape& s, const void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_map(s).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <class P>
+static uint8_t* at(P* base, size_t off) {
+  return reinterpret_cast<uint8_t*>(const_cast<void*>(static_cast<const void*>(base))) + off;
+}
+
+// Record stage event i (if the caller asked for stage events).
+static bool mark(void* const* ev, int i, cudaStream_t st) {
+  if (!ev) return true;
+  return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+}
+
+static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
+                                 const int32_t* offsets,
+                                 const int32_t* sorted_slots,
+                                 const __nv_bfloat16* w13, const __nv_bfloat16* w2,
+                                 const __nv_bfloat16* w13_sh,
+                                 const __nv_bfloat16* w2_sh, __nv_bfloat16* y_perm,
+                                 void* ws, cudaStream_t st,
+                                 void* const* ev = nullptr) {
+  const WsMap m = workspace_map(s);
+  const int G = s.E + s.n_shared;
+  auto* x_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.x_perm));
+  auto* h = reinterpret_cast<__nv_bfloat16*>(at(ws, m.h));
+  auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
+  if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
+  cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
+                                x_perm, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(ev, 3, st)) return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.mode = 0;
+  a.A = x_perm;
+  a.B = w13;
+  a.B_sh = w13_sh;
+  a.offsets = offsets;
+  a.G = G;
+  a.E = s.E;
+  a.N = s.I;
+  a.K = s.H;
+  a.cap = m.cap;
+  a.out = h;
+  a.act = s.act;
+  a.err = err;
+  e = launch_grouped_gemm(a, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
+  a.mode = 1;
+  a.A = h;
+  a.B = w2;
+  a.B_sh = w2_sh;
+  a.N = s.H;
+  a.K = s.I;
+  a.out = y_perm;
+  return from_cuda(launch_grouped_gemm(a, st));
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_layout_capacity(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return workspace_map(*shape).cap;
+}
+
+size_t moe_workspace_size(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return workspace_map(*shape).total;
+}
+
+moe_status moe_route(const moe_shape* shape, const float* logits,
+                     const float* scale, int32_t* ids, float* w,
+                     cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  if (!logits || !ids || !w) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_route(logits, scale, shape->T, shape->E, shape->k, ids,
+                                w, stream));
+}
+
+moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
+                       int32_t* offsets, int32_t* sorted_slots,
+                       int32_t* slot_row, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!offsets || !sorted_slots || (shape->T > 0 && (!ids || !slot_row)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsMap m = workspace_map(*shape);
+  return from_cuda(launch_layout(
+      *shape, ids, offsets, sorted_slots, slot_row, m.cap,
+      reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
+      reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
+      reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt, stream));
+}
+
+moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
+                          const int32_t* offsets, const int32_t* sorted_slots,
+                          const moe_bf16* w13, const moe_bf16* w2,
+                          const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                          moe_bf16* y_perm, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!offsets || !sorted_slots || !w13 || !w2 || !y_perm ||
+      (shape->T > 0 && !x))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  return run_expert_ffn(*shape, reinterpret_cast<const __nv_bfloat16*>(x), offsets,
+                        sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
+                        reinterpret_cast<const __nv_bfloat16*>(w2),
+                        reinterpret_cast<const __nv_bfloat16*>(w13_sh),
+                        reinterpret_cast<const __nv_bfloat16*>(w2_sh),
+                        reinterpret_cast<__nv_bfloat16*>(y_perm), ws, stream);
+}
+
+moe_status moe_combine(const moe_shape* shape, const moe_bf16* y_perm,
+                       const int32_t* slot_row, const float* w, moe_bf16* out,
+                       cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  if (!y_perm || !slot_row || !w || !out) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_combine(reinterpret_cast<const __nv_bfloat16*>(y_perm),
+                                  slot_row, w, shape->T, shape->k,
+                                  shape->n_shared, shape->H,
+                                  reinterpret_cast<__nv_bfloat16*>(out), stream));
+}
+
+moe_status moe_forward_staged(const moe_shape* shape, const moe_bf16* x,
+                              const float* logits, const moe_bf16* w13,
+                              const moe_bf16* w2, const float* scale,
+                              const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                              moe_bf16* out, int32_t* ids_out, float* w_out,
+                              void* ws, size_t ws_bytes, void* const* ev,
+                              cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!w13 || !w2 || (shape->T > 0 && (!x || !logits || !out)))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (ev)
+    for (int i = 0; i <= MOE_NUM_STAGES; ++i)
+      if (!ev[i]) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) {
+    for (int i = 0; i <= MOE_NUM_STAGES; ++i)
+      if (!mark(ev, i, stream)) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const moe_shape& s = *shape;
+  const WsMap m = workspace_map(s);
+  int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(at(ws, m.ids));
+  float* w = w_out ? w_out : reinterpret_cast<float*>(at(ws, m.w));
+  auto* offsets = reinterpret_cast<int32_t*>(at(ws, m.offsets));
+  auto* sorted_slots = reinterpret_cast<int32_t*>(at(ws, m.sorted_slots));
+  auto* slot_row = reinterpret_cast<int32_t*>(at(ws, m.slot_row));
+  auto* y_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.y_perm));
+  if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
+  if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (!mark(ev, 1, stream)) return MOE_ERR_CUDA;
+  if (launch_layout(s, ids, offsets, sorted_slots, slot_row, m.cap,
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt,
+                    stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = run_expert_ffn(s, reinterpret_cast<const __nv_bfloat16*>(x), offsets,
+                      sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
+                      reinterpret_cast<const __nv_bfloat16*>(w2),
+                      reinterpret_cast<const __nv_bfloat16*>(w13_sh),
+                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), y_perm, ws,
+                      stream, ev);
+  if (st != MOE_OK) return st;
+  if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
+  if (launch_combine(y_perm, slot_row, w, s.T, s.k, s.n_shared, s.H,
+                     reinterpret_cast<__nv_bfloat16*>(out), stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
+                       const float* logits, const moe_bf16* w13,
+                       const moe_bf16* w2, const float* scale,
+                       const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                       moe_bf16* out, int32_t* ids_out, float* w_out, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  return moe_forward_staged(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
+                            ids_out, w_out, ws, ws_bytes, nullptr, stream);
+}
+
+moe_status moe_read_error(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!ws || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof word) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word == 0) return MOE_OK;
+  if (word >= 1 && word <= MOE_ERR_TIMEOUT) return static_cast<moe_status>(word);
+  return MOE_ERR_CUDA;
+}
+
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes,
+                                     uint32_t timeout_us, cudaStream_t stream) {
+  if (!ws || ws_bytes < 256 || timeout_us == 0 || timeout_us > 10000000u)
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_wait_selftest(reinterpret_cast<uint32_t*>(ws), timeout_us, stream));
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+}  // extern "C"

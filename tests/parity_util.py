@@ -1,0 +1,58 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+and compare it with the fp64 oracle on the same seeded inputs."""
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_ffn_06_b200 import inputs
+
+OUT_TOL = 2e-2      # max |err| <= OUT_TOL * RMS(oracle output)
+WEIGHT_RTOL = 1e-6  # gate weights, relative
+
+
+def to_device(inp: inputs.MoEInputs, device="cuda") -> inputs.MoEInputs:
+    def mv(t):
+        return None if t is None else t.to(device).contiguous()
+    return inputs.MoEInputs(shape=inp.shape, x=mv(inp.x), logits=mv(inp.logits),
+                            scale=mv(inp.scale), w13=mv(inp.w13), w2=mv(inp.w2),
+                            w13_sh=mv(inp.w13_sh), w2_sh=mv(inp.w2_sh),
+                            bias=mv(inp.bias))
+
+
+def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True):
+    s = api.shape_from(inp.shape)
+    T, H, k = inp.shape.T, inp.shape.H, inp.shape.k
+    dev = inp.x.device
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev) if with_routing else None
+    w = torch.empty(T, k, dtype=torch.float32, device=dev) if with_routing else None
+    ws = api.alloc_workspace(s, dev)
+    api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                    inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w)
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    return out, ids, w
+
+
+def oracle_forward(inp: inputs.MoEInputs, tokens=None):
+    return oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, inp.shape.k,
+                          inp.shape.act, scale=inp.scale, w13_sh=inp.w13_sh,
+                          w2_sh=inp.w2_sh, tokens=tokens)
+
+
+def assert_out_close(got_bf16: torch.Tensor, want: np.ndarray, what=""):
+    got = got_bf16.float().cpu().numpy().astype(np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    err = float(np.abs(got - want).max())
+    assert err <= OUT_TOL * rms, f"{what}: max|err| {err:.3e} > {OUT_TOL} x RMS {rms:.3e}"
+    return err / rms
+
+
+def assert_routing_exact(ids_gpu, w_gpu, ids_ref, w_ref):
+    ids = ids_gpu.cpu().numpy()
+    assert (ids == ids_ref).all(), "top-k ids differ"
+    w = w_gpu.cpu().numpy().astype(np.float64)
+    rel = np.abs(w - w_ref) / np.abs(w_ref)
+    assert rel.max() <= WEIGHT_RTOL, f"gate weights rel err {rel.max():.3e}"

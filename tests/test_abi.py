@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every function ``include/moe.h`` declares, and
+reject bad arguments before it touches the GPU.  Only calls that return
+before any CUDA call are made here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def api():
+    from mixture_experts_ffn_06_b200 import build
+    build.build()
+    from mixture_experts_ffn_06_b200 import api as a
+    return a
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[\w\s\*]+?\b(moe_\w+)\s*\(", text,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+                 "moe_forward", "moe_workspace_size", "moe_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(api):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(api.lib, n), n
+    assert set(api.EXPORTS) <= set(names)
+
+
+def test_nvcc_targets_sm100a():
+    from mixture_experts_ffn_06_b200 import build
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+
+
+def _shape(api, **kw):
+    base = dict(T=64, H=256, E=8, k=2, I=512, act=0, n_shared=0, I_shared=0,
+                pad=0)
+    base.update(kw)
+    return api.make_shape(**base)
+
+
+def test_capacity_and_workspace_size(api):
+    s = _shape(api)
+    assert api.moe_layout_capacity(s) == 64 * 2 + 8 * 127
+    ws = api.moe_workspace_size(s)
+    cap = 64 * 2 + 8 * 127
+    assert ws >= cap * 256 * 2 * 2 + cap * 512 * 2  # x_perm, y_perm, h
+    sh = _shape(api, n_shared=2, I_shared=512)
+    assert api.moe_layout_capacity(sh) == 64 * 2 + 64 * 2 + 10 * 127
+    assert api.moe_workspace_size(sh) > ws
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=9), 1),            # k > E
+    (dict(k=0), 1),
+    (dict(T=-1), 1),
+    (dict(act=7), 1),
+    (dict(E=513, k=2), 2),     # above the supported expert count
+    (dict(E=64, k=33), 2),
+    (dict(H=260), 2),          # rows must be 16-byte multiples
+    (dict(I=500), 2),
+    (dict(n_shared=1, I_shared=256), 2),
+    (dict(pad=64), 2),
+    (dict(T=1 << 24), 2),
+])
+def test_bad_shapes_are_rejected_before_launch(api, kw, status):
+    s = _shape(api, **kw)
+    assert api.moe_layout_capacity(s) == 0
+    assert api.moe_workspace_size(s) == 0
+    null = ctypes.c_void_p(0)
+    rc = api.lib.moe_route(ctypes.byref(s), null, null, null, null, null)
+    assert rc == status
+    rc = api.lib.moe_forward(ctypes.byref(s), null, null, null, null, null,
+                             null, null, null, null, null, null, 0, null)
+    assert rc == status
+
+
+def test_null_pointers_and_small_workspace(api):
+    s = _shape(api)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: checks come first
+    assert api.lib.moe_route(ctypes.byref(s), null, null, null, null, null) == 1
+    need = api.moe_workspace_size(s)
+    rc = api.lib.moe_permute(ctypes.byref(s), fake, fake, fake, fake, fake,
+                             need - 1, null)
+    assert rc == 3  # MOE_ERR_WORKSPACE
+    rc = api.lib.moe_permute(ctypes.byref(s), fake, fake, fake, fake, null,
+                             need, null)
+    assert rc == 1
+    unaligned = ctypes.c_void_p((1 << 20) + 16)
+    rc = api.lib.moe_permute(ctypes.byref(s), fake, fake, fake, fake,
+                             unaligned, need, null)
+    assert rc == 1
+    sh = _shape(api, n_shared=1, I_shared=512)
+    rc = api.lib.moe_expert_ffn(ctypes.byref(sh), fake, fake, fake, fake, fake,
+                                null, null, fake, fake,
+                                api.moe_workspace_size(sh), null)
+    assert rc == 1  # shared weights missing
+
+
+def test_empty_batch_is_a_no_op(api):
+    s = _shape(api, T=0)
+    null = ctypes.c_void_p(0)
+    assert api.lib.moe_route(ctypes.byref(s), null, null, null, null, null) == 0
+    assert api.lib.moe_combine(ctypes.byref(s), null, null, null, null,
+                               null) == 0
+
+
+def test_status_strings(api):
+    assert api.moe_status_string(0) == "MOE_OK"
+    assert api.moe_status_string(5) == "MOE_ERR_TIMEOUT"
+    assert api.moe_status_string(99) == "MOE_ERR_UNKNOWN"

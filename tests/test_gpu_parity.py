@@ -1,0 +1,240 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Bars: top-k ids, the permutation and the slot maps bit-exact; gate weights
+within 1e-6 relative; layer outputs within max|err| <= 2e-2 x RMS(oracle).
+Small shapes are compared on every output element; the full-size workloads
+on every routing decision and on a token sample that covers every expert.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_ffn_06_b200 import inputs
+from parity_util import (assert_out_close, assert_routing_exact, gpu_forward,
+                         oracle_forward, to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixture_experts_ffn_06_b200 import api as a
+    return a
+
+
+SMALL = {
+    "tiny": (inputs.shape_of("tiny"), "zero", "ones"),
+    "ragged": (inputs.Shape(T=37, H=200, E=5, k=3, I=104, act=1), "zero", "uniform"),
+    "tail704": (inputs.Shape(T=50, H=256, E=16, k=4, I=704, act=1), "zero", "uniform"),
+    "shared": (inputs.Shape(T=40, H=128, E=6, k=2, I=96, n_shared=2, I_shared=96),
+               "zero", "ones"),
+    "single_expert": (inputs.Shape(T=19, H=64, E=1, k=1, I=64), "zero", "uniform"),
+    "k_equals_E": (inputs.Shape(T=33, H=64, E=4, k=4, I=32, act=1), "zero", "uniform"),
+    "one_token": (inputs.Shape(T=1, H=128, E=8, k=2, I=128), "zero", "uniform"),
+    "gemma_shapes_T130": (inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),
+                          "zero", "uniform"),
+    "wide_tiles": (inputs.Shape(T=300, H=520, E=3, k=2, I=392), "normal0.5", "uniform"),
+}
+
+
+def _small(name, seed=0):
+    shp, bias, scale = SMALL[name]
+    return inputs.make_inputs(shp, seed=seed, bias=bias, scale=scale)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small_every_element(api, name):
+    inp = _small(name)
+    want, ids_ref, w_ref = oracle_forward(inp)
+    out, ids, w = gpu_forward(api, to_device(inp))
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out, want, name)
+
+
+def test_all_tokens_on_one_expert(api):
+    # one expert takes every token: a segment of several M tiles, others empty
+    shp = inputs.Shape(T=300, H=128, E=8, k=1, I=256)
+    inp = inputs.make_inputs(shp, seed=1)
+    inp.logits[:, 5] += 50.0
+    want, ids_ref, w_ref = oracle_forward(inp)
+    assert (ids_ref == 5).all()
+    out, ids, w = gpu_forward(api, to_device(inp))
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out, want, "one hot expert")
+
+
+def _layout_gpu(api, s, ids_dev, E, S):
+    cap = api.moe_layout_capacity(s)
+    T, k = ids_dev.shape
+    offsets = torch.full((E + S + 1,), -7, dtype=torch.int32, device="cuda")
+    sorted_slots = torch.full((cap,), -7, dtype=torch.int32, device="cuda")
+    slot_row = torch.full((T, k + S), -7, dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(s)
+    api.moe_permute(s, ids_dev, offsets, sorted_slots, slot_row, ws)
+    torch.cuda.synchronize()
+    return offsets.cpu().numpy(), sorted_slots.cpu().numpy(), slot_row.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "gemma_shapes_T130",
+                                  "one_token", "k_equals_E"])
+def test_permute_bit_exact(api, name):
+    inp = _small(name)
+    shp = inp.shape
+    s = api.shape_from(shp)
+    ids_ref, _ = oracle.route(inp.logits, shp.k, scale=inp.scale)
+    got = _layout_gpu(api, s, torch.from_numpy(ids_ref).cuda(), shp.E, shp.n_shared)
+    want = oracle.layout(ids_ref, shp.E, shp.n_shared, 128)
+    for g, w_, what in zip(got, want, ("offsets", "sorted_slots", "slot_row")):
+        assert (g == w_).all(), what
+
+
+def test_permute_large_random_ids(api):
+    # many layout blocks (T*k > 1024) and skewed counts
+    T, E, k, S = 5000, 64, 6, 2
+    gen = torch.Generator().manual_seed(3)
+    z = inputs.router_logits(T, E, k, gen, "cpu",
+                             bias=(-1.1 * torch.log(torch.arange(E) + 1.0)).float())
+    ids_ref, _ = oracle.route(z, k)
+    s = api.make_shape(T=T, H=64, E=E, k=k, I=64, n_shared=S, I_shared=64)
+    got = _layout_gpu(api, s, torch.from_numpy(ids_ref).cuda(), E, S)
+    want = oracle.layout(ids_ref, E, S, 128)
+    for g, w_, what in zip(got, want, ("offsets", "sorted_slots", "slot_row")):
+        assert (g == w_).all(), what
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "tail704"])
+def test_four_call_chain_matches_fused_and_oracle_rows(api, name):
+    inp = _small(name)
+    shp = inp.shape
+    d = to_device(inp)
+    s = api.shape_from(shp)
+    T, k, S, H = shp.T, shp.k, shp.n_shared, shp.H
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    api.moe_route(s, d.logits, d.scale, ids, w)
+    cap = api.moe_layout_capacity(s)
+    offsets = torch.empty(shp.E + S + 1, dtype=torch.int32, device="cuda")
+    sorted_slots = torch.empty(cap, dtype=torch.int32, device="cuda")
+    slot_row = torch.empty(T, k + S, dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(s)
+    api.moe_permute(s, ids, offsets, sorted_slots, slot_row, ws)
+    y_perm = torch.empty(cap, H, dtype=torch.bfloat16, device="cuda")
+    api.moe_expert_ffn(s, d.x, offsets, sorted_slots, d.w13, d.w2, d.w13_sh,
+                       d.w2_sh, y_perm, ws)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    api.moe_combine(s, y_perm, slot_row, w, out)
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    fused, _, _ = gpu_forward(api, d)
+    assert torch.equal(out, fused)  # same kernels, same order: bit-exact
+
+    # unweighted expert rows against the oracle, every row in use
+    used = int(offsets[-1])
+    slots = sorted_slots[:used].cpu().numpy()
+    rows = np.nonzero(slots >= 0)[0]
+    sl = slots[rows]
+    R = T * k
+    routed = sl < R
+    ids_np = ids.cpu().numpy().ravel()
+    y = y_perm[:used].float().cpu().numpy()
+    if routed.any():
+        tok = sl[routed] // k
+        ex = ids_np[sl[routed]]
+        want = oracle.expert_rows(inp.x, inp.w13, inp.w2, tok, ex, shp.act)
+        got = y[rows[routed]].astype(np.float64)
+        rms = np.sqrt(np.mean(want ** 2))
+        assert np.abs(got - want).max() <= 2e-2 * rms
+    if S:
+        q = sl[~routed] - R
+        want = oracle.expert_rows(inp.x, inp.w13_sh, inp.w2_sh, q % T, q // T,
+                                  shp.act)
+        got = y[rows[~routed]].astype(np.float64)
+        rms = np.sqrt(np.mean(want ** 2))
+        assert np.abs(got - want).max() <= 2e-2 * rms
+    pad = np.nonzero(slots < 0)[0]
+    assert (y[pad] == 0).all()  # padding rows hold zeros
+
+
+def test_deterministic_across_calls(api):
+    inp = to_device(_small("gemma_shapes_T130"))
+    a, _, _ = gpu_forward(api, inp)
+    b, _, _ = gpu_forward(api, inp)
+    assert torch.equal(a, b)
+
+
+def test_device_wait_limit_reports_timeout(api):
+    s = api.make_shape(T=8, H=64, E=4, k=2, I=64)
+    ws = api.alloc_workspace(s)
+    api.moe_selftest_wait_timeout(ws, 2000)
+    assert api.moe_read_error(ws) == 5  # MOE_ERR_TIMEOUT, context still usable
+    assert api.moe_read_error(ws) == 0  # cleared
+    inp = to_device(inputs.make_inputs(inputs.Shape(T=8, H=64, E=4, k=2, I=64)))
+    out, _, _ = gpu_forward(api, inp)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_workspace_too_small_is_refused(api):
+    inp = to_device(_small("tiny"))
+    s = api.shape_from(inp.shape)
+    ws = torch.zeros(api.moe_workspace_size(s) - 256, dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(inp.shape.T, inp.shape.H, dtype=torch.bfloat16,
+                      device="cuda")
+    with pytest.raises(api.MoEError) as e:
+        api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                        None, None, out, ws)
+    assert e.value.status == 3
+
+
+# ----------------------------------------------------------- full workloads
+
+def _cover_tokens(ids: np.ndarray, E: int, extra: int, seed: int) -> np.ndarray:
+    """Token sample that routes to every expert that any token uses, plus a
+    few seeded random tokens and the first and last token."""
+    T = ids.shape[0]
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(T)
+    chosen, seen = [], set()
+    for t in order:
+        new = set(ids[t].tolist()) - seen
+        if new:
+            chosen.append(int(t))
+            seen |= new
+        if len(seen) == len(set(ids.ravel().tolist())):
+            break
+    chosen += [0, T - 1] + [int(t) for t in rng.choice(T, extra, replace=False)]
+    return np.array(sorted(set(chosen)), np.int64)
+
+
+@pytest.mark.parametrize("name", ["decode_t1", "decode_t4", "decode_t16",
+                                  "decode_t64", "decode_t256"])
+def test_decode_sweep_every_element(api, name):
+    inp = inputs.make_inputs(name, seed=0, device="cuda")
+    out, ids, w = gpu_forward(api, inp)
+    want, ids_ref, w_ref = oracle_forward(inp)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out, want, name)
+
+
+@pytest.mark.parametrize("name", ["mixtral_prefill", "many_small_prefill",
+                                  "skewed_shared_prefill"])
+def test_prefill_full_size(api, name):
+    inp = inputs.make_inputs(name, seed=0, device="cuda")
+    shp = inp.shape
+    out, ids, w = gpu_forward(api, inp)
+    # routing of every token, bit-exact ids
+    ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    # permutation of every slot
+    s = api.shape_from(shp)
+    got = _layout_gpu(api, s, ids, shp.E, shp.n_shared)
+    want = oracle.layout(ids_ref, shp.E, shp.n_shared, 128)
+    for g, w_, what in zip(got, want, ("offsets", "sorted_slots", "slot_row")):
+        assert (g == w_).all(), what
+    # outputs on a token sample covering every expert
+    tok = _cover_tokens(ids_ref, shp.E, extra=6, seed=1)
+    want_out, _, _ = oracle_forward(inp, tokens=tok)
+    assert_out_close(out[torch.from_numpy(tok).cuda()], want_out, name)
