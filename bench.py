@@ -216,9 +216,9 @@ def run_ours(args):
             api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                             inp.w13_sh, inp.w2_sh, out, ws)
         else:
-            api.moe_forward_staged(s, inp.x, inp.logits, inp.w13, inp.w2,
-                                   inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
-                                   events)
+            api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2,
+                               inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
+                               events=events)
 
     def barrier():
         if world > 1:
@@ -308,7 +308,7 @@ def run_ours(args):
         peak = float(peaks["bf16_tflops"])
         traffic = traffic_for("gemm_tc.cu")
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
-        launches_per_step = 9  # route, layout x4, gather, 2 GEMMs, combine
+        launches_per_step = 9  # route, layout x4, gather, 2 GEMMs, round
         cpu = None
         if world == 1:
             rate, cores, ntok, secs = cpu_oracle_rate(inp)

@@ -126,7 +126,7 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
  *   w13       [E,2I,H] bf16: rows [0,I) gate (w1), rows [I,2I) up (w3)
  *   w2        [E,H,I] bf16
  *   w13_sh    [S,2I,H] bf16 or NULL when S == 0;  w2_sh [S,H,I] likewise
- *   y_perm    [cap,H] bf16 out: unweighted expert output of every row in use;
+ *   y_perm    [cap,H] fp32 out: unweighted expert output of every row in use;
  *             padding rows get 0, rows past offsets[E+S] are not written
  * h = Act(g) (*) u is rounded to bf16 (the second GEMM's operand); every
  * product accumulates in fp32 on the tensor cores.
@@ -135,16 +135,17 @@ MOE_API moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
                           const int32_t* offsets, const int32_t* sorted_slots,
                           const moe_bf16* w13, const moe_bf16* w2,
                           const moe_bf16* w13_sh, const moe_bf16* w2_sh,
-                          moe_bf16* y_perm, void* ws, size_t ws_bytes,
+                          float* y_perm, void* ws, size_t ws_bytes,
                           cudaStream_t stream);
 
 /*
  * moe_combine -- weighted combine (walkthrough section 7 step 4; the weighted
  * sum after ggml_mul_mat_id in lesson 35), with shared experts at weight 1.
- *   y_perm [cap,H] bf16, slot_row [T,k+S] int32, w [T,k] fp32
- *   out    [T,H] bf16 out, summed in fp32 and rounded once
+ *   y_perm [cap,H] fp32, slot_row [T,k+S] int32, w [T,k] fp32
+ *   out    [T,H] bf16 out: sum over j in order 0..k-1, then the shared
+ *          experts, in fp32, rounded once to bf16 (deterministic)
  */
-MOE_API moe_status moe_combine(const moe_shape* shape, const moe_bf16* y_perm,
+MOE_API moe_status moe_combine(const moe_shape* shape, const float* y_perm,
                        const int32_t* slot_row, const float* w, moe_bf16* out,
                        cudaStream_t stream);
 
@@ -153,6 +154,12 @@ MOE_API moe_status moe_combine(const moe_shape* shape, const moe_bf16* y_perm,
  * one stream, with every intermediate in the workspace (vLLM FusedMoE as the
  * walkthrough's section 6 describes it).  ids_out [T,k] and w_out [T,k] may
  * be NULL; when given they receive the routing.
+ * Here the combine is fused into the w2 GEMM's epilogue: each expert row is
+ * multiplied by its gate weight and added into an fp32 [T,H] accumulator
+ * with atomic vector adds, which a last pass rounds to bf16.  The order of
+ * those fp32 additions is not fixed, so two calls may differ in the last bit
+ * of the fp32 sum (and rarely in one bf16 ulp); moe_combine is the
+ * deterministic alternative.
  */
 MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        const float* logits, const moe_bf16* w13,
@@ -162,20 +169,27 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
- * moe_forward_staged -- moe_forward that also records CUDA events between its
- * stages, for per-kernel timing on the launch stream.  stage_events is NULL
- * or an array of MOE_NUM_STAGES + 1 cudaEvent_t created by the caller; event
- * i is recorded before stage i and event MOE_NUM_STAGES after the last one.
- * Stages: 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
- * 4 w2 GEMM, 5 combine.
+ * moe_forward_ex -- moe_forward with options (opts may be NULL):
+ *   stage_events  NULL or MOE_NUM_STAGES + 1 cudaEvent_t created by the
+ *                 caller; event i is recorded before stage i and event
+ *                 MOE_NUM_STAGES after the last one, on ``stream``.  Stages:
+ *                 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
+ *                 4 w2 GEMM + weighted combine, 5 bf16 rounding.
+ *   out_f32       NULL or [T,H] fp32: receives the layer output before its
+ *                 rounding to bf16 (it is then used as the accumulator).
  */
 #define MOE_NUM_STAGES 6
-MOE_API moe_status moe_forward_staged(
+typedef struct {
+  void* const* stage_events;
+  float* out_f32;
+} moe_forward_opts;
+
+MOE_API moe_status moe_forward_ex(
     const moe_shape* shape, const moe_bf16* x, const float* logits,
     const moe_bf16* w13, const moe_bf16* w2, const float* scale,
     const moe_bf16* w13_sh, const moe_bf16* w2_sh, moe_bf16* out,
     int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes,
-    void* const* stage_events, cudaStream_t stream);
+    const moe_forward_opts* opts, cudaStream_t stream);
 
 /*
  * moe_read_error -- SYNCHRONISES ``stream``, then returns the status recorded

@@ -21,11 +21,11 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 NUM_STAGES = 6
-STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act", "w2_gemm",
-               "combine")
+STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act",
+               "w2_gemm_combine", "round_bf16")
 EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_route",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
-           "moe_forward_staged",
+           "moe_forward_ex",
            "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string")
 
 
@@ -33,6 +33,11 @@ class MoEError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where} returned {STATUS_NAMES.get(status, status)}")
+
+
+class moe_forward_opts(ctypes.Structure):
+    _fields_ = [("stage_events", ctypes.c_void_p),
+                ("out_f32", ctypes.c_void_p)]
 
 
 class moe_shape(ctypes.Structure):
@@ -62,15 +67,17 @@ def _load() -> ctypes.CDLL:
     lib.moe_combine.argtypes = [S, P, P, P, P, P]
     lib.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P,
                                 ctypes.c_size_t, P]
-    lib.moe_forward_staged.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P,
-                                       ctypes.c_size_t, P, P]
+    lib.moe_forward_ex.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P,
+                                   ctypes.c_size_t,
+                                   ctypes.POINTER(moe_forward_opts), P]
     lib.moe_read_error.argtypes = [P, ctypes.c_size_t, P]
     lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t,
                                               ctypes.c_uint32, P]
     lib.moe_status_string.argtypes = [st]
     lib.moe_status_string.restype = ctypes.c_char_p
     for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
-                 "moe_forward", "moe_forward_staged", "moe_read_error", "moe_selftest_wait_timeout"):
+                 "moe_forward", "moe_forward_ex", "moe_read_error",
+                 "moe_selftest_wait_timeout"):
         getattr(lib, name).restype = st
     return lib
 
@@ -163,19 +170,30 @@ def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                            _stream(stream)), "moe_forward")
 
 
-def moe_forward_staged(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
-                       ws, events, ids_out=None, w_out=None, stream=None):
-    """moe_forward recording ``events`` (NUM_STAGES + 1 torch.cuda.Event,
-    created with enable_timing=True) around its stages."""
-    if len(events) != NUM_STAGES + 1:
-        raise ValueError("need NUM_STAGES + 1 events")
-    arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
-        *[ctypes.c_void_p(e.cuda_event) for e in events])
-    _check(lib.moe_forward_staged(ctypes.byref(shape), _p(x), _p(logits),
-                                  _p(w13), _p(w2), _p(scale), _p(w13_sh),
-                                  _p(w2_sh), _p(out), _p(ids_out), _p(w_out),
-                                  _p(ws), ws.numel(), arr, _stream(stream)),
-           "moe_forward_staged")
+def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
+                   ids_out=None, w_out=None, events=None, out_f32=None,
+                   stream=None):
+    """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
+    created with enable_timing=True) recorded around the stages, and
+    ``out_f32`` ([T,H] fp32) receiving the output before its bf16 rounding."""
+    arr = None
+    if events is not None:
+        if len(events) != NUM_STAGES + 1:
+            raise ValueError("need NUM_STAGES + 1 events")
+        st = stream if stream is not None else torch.cuda.current_stream()
+        for e in events:
+            if not e.cuda_event:  # torch creates its events lazily
+                e.record(st)
+        arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
+            *[ctypes.c_void_p(e.cuda_event) for e in events])
+    opts = moe_forward_opts(
+        ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
+        _p(out_f32))
+    _check(lib.moe_forward_ex(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
+                              _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
+                              _p(ids_out), _p(w_out), _p(ws), ws.numel(),
+                              ctypes.byref(opts), _stream(stream)),
+           "moe_forward_ex")
 
 
 def moe_read_error(ws, stream=None) -> int:

@@ -6,33 +6,25 @@
 // lesson 35 adds always-active shared experts, which enter with weight 1.
 // The sum is kept in fp32 and rounded to bf16 once.
 //
-// One block per token (grid-stride over tokens); each thread owns 8 hidden
-// columns (one 16-byte vector) at a time and gathers the k+S rows of y_perm
-// that slot_row names.  HBM-bound: reads (k+S)*H*2 bytes, writes H*2.
+// combine_kernel (the unfused, deterministic path): one block per token
+// (grid-stride over tokens); each thread owns 4 hidden columns at a time and
+// sums the k+S fp32 rows of y_perm that slot_row names in a fixed order.
+// HBM-bound: reads (k+S)*H*4 bytes, writes H*2.
+// finalize_kernel (the fused path): the w2 epilogue has already added every
+// weighted expert row into an fp32 [T,H] accumulator; this pass rounds it.
 #include "internal.cuh"
 
 namespace moe {
 namespace {
 
-__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& v,
-                                           float wt) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(p[i]);
-    acc[2 * i] = fmaf(wt, f.x, acc[2 * i]);
-    acc[2 * i + 1] = fmaf(wt, f.y, acc[2 * i + 1]);
-  }
-}
-
 __global__ void __launch_bounds__(256)
-combine_kernel(const uint4* __restrict__ y_perm,
+combine_kernel(const float4* __restrict__ y_perm,
                const int32_t* __restrict__ slot_row,
                const float* __restrict__ w, int64_t T, int k, int S, int H,
-               uint4* __restrict__ out) {
+               uint2* __restrict__ out) {
   __shared__ int64_t rows[kMaxTopK + kMaxShared];
   __shared__ float wts[kMaxTopK + kMaxShared];
-  const int chunks = H >> 3;
+  const int chunks = H >> 2;  // 4 fp32 per 16-byte chunk
   const int ks = k + S;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
@@ -42,42 +34,71 @@ combine_kernel(const uint4* __restrict__ y_perm,
     }
     __syncthreads();
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      int j = 0;
-      for (; j + 4 <= ks; j += 4) {
-        const uint4 v0 = __ldg(y_perm + rows[j] + c);
-        const uint4 v1 = __ldg(y_perm + rows[j + 1] + c);
-        const uint4 v2 = __ldg(y_perm + rows[j + 2] + c);
-        const uint4 v3 = __ldg(y_perm + rows[j + 3] + c);
-        acc_bf16x8(acc, v0, wts[j]);
-        acc_bf16x8(acc, v1, wts[j + 1]);
-        acc_bf16x8(acc, v2, wts[j + 2]);
-        acc_bf16x8(acc, v3, wts[j + 3]);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      // fixed order: routed choices j = 0..k-1, then the shared experts
+      for (int j = 0; j < ks; ++j) {
+        const float4 v = __ldg(y_perm + rows[j] + c);
+        const float wt = wts[j];
+        a0 = fmaf(wt, v.x, a0);
+        a1 = fmaf(wt, v.y, a1);
+        a2 = fmaf(wt, v.z, a2);
+        a3 = fmaf(wt, v.w, a3);
       }
-      for (; j < ks; ++j) acc_bf16x8(acc, __ldg(y_perm + rows[j] + c), wts[j]);
-      uint4 o;
-      __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        op[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(a2, a3);
+      uint2 o;
+      o.x = *reinterpret_cast<const uint32_t*>(&lo);
+      o.y = *reinterpret_cast<const uint32_t*>(&hi);
       out[t * chunks + c] = o;
     }
   }
 }
 
+// bf16 rounding of the fp32 accumulator, 8 values per thread-iteration.
+__global__ void __launch_bounds__(256)
+finalize_kernel(const float4* __restrict__ acc, int64_t n8,
+                uint4* __restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += stride) {
+    const float4 a = __ldg(acc + 2 * i);
+    const float4 b = __ldg(acc + 2 * i + 1);
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
+    const __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&p0);
+    o.y = *reinterpret_cast<const uint32_t*>(&p1);
+    o.z = *reinterpret_cast<const uint32_t*>(&p2);
+    o.w = *reinterpret_cast<const uint32_t*>(&p3);
+    out[i] = o;
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row,
+cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,
                            __nv_bfloat16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const int64_t blocks = T < 148 * 64 ? T : 148 * 64;
-  const int threads = (H / 8) >= 256 ? 256 : (((H / 8) + 31) / 32) * 32;
+  const int chunks = H / 4;
+  const int threads = chunks >= 256 ? 256 : ((chunks + 31) / 32) * 32;
   combine_kernel<<<(unsigned)blocks, threads < 64 ? 64 : threads, 0, st>>>(
-      reinterpret_cast<const uint4*>(y_perm), slot_row, w, T, k, S, H,
-      reinterpret_cast<uint4*>(out));
+      reinterpret_cast<const float4*>(y_perm), slot_row, w, T, k, S, H,
+      reinterpret_cast<uint2*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
+                            cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  const int64_t want = (n8 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  finalize_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc), n8,
+                                          reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }
 

@@ -57,10 +57,14 @@ struct KParams {
   int G, E, N, K, NT, KB;
   int32_t b_rows_per_group;  // rows of one expert in the B tensor
   int32_t up_off;            // mode 0: row offset of the up half (= N)
-  __nv_bfloat16* out;
+  void* out;
   int act;
   uint32_t* err;
   uint64_t timeout_ns;
+  const int32_t* sorted_slots;  // mode 2
+  const float* w;               // mode 2
+  int64_t T;                    // mode 2
+  int k;                        // mode 2
 };
 
 struct Tile {
@@ -95,6 +99,14 @@ __device__ __forceinline__ float act_apply(int act, float g) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Vector fp32 reduction into global memory (16-byte aligned destination).
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c,
+                                           float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 template <int MODE>
@@ -236,8 +248,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
       const int64_t row = tl.row0 + q * 32 + lane;
-      __nv_bfloat16* orow = p.out + row * (int64_t)p.N;
       if (MODE == 0) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + row * (int64_t)p.N;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           const int col0 = tl.n0 + c * 32;
@@ -263,22 +275,47 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       } else {
+        // mode 1: plain fp32 rows; mode 2: weight and add into the token row
+        float* orow;
+        float wt = 1.0f;
+        bool live = true;
+        if (MODE == 1) {
+          orow = static_cast<float*>(p.out) + row * (int64_t)p.N;
+        } else {
+          const int32_t slot = p.sorted_slots[row];
+          live = slot >= 0;
+          const int64_t R = p.T * p.k;
+          int64_t tok = 0;
+          if (live) {
+            if (slot < R) {
+              tok = slot / p.k;
+              wt = __ldg(p.w + slot);
+            } else {
+              tok = (slot - R) % p.T;
+            }
+          }
+          orow = static_cast<float*>(p.out) + tok * (int64_t)p.N;
+        }
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           const int col0 = tl.n0 + c * 32;
           if (col0 >= p.N) break;
           uint32_t y[32];
-          tmem_ld32(tb + c * 32, y);
+          tmem_ld32(tb + c * 32, y);  // warp-collective: every lane loads
+          if (!live) continue;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (col0 + v * 8 < p.N) {
-              uint4 o;
-              uint32_t* op = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                op[e] = pack_bf16x2(__uint_as_float(y[v * 8 + 2 * e]),
-                                    __uint_as_float(y[v * 8 + 2 * e + 1]));
-              *reinterpret_cast<uint4*>(orow + col0 + v * 8) = o;
+          for (int v = 0; v < 8; ++v) {
+            if (col0 + v * 4 < p.N) {
+              float* dst = orow + col0 + v * 4;
+              const float a0 = __uint_as_float(y[v * 4 + 0]);
+              const float a1 = __uint_as_float(y[v * 4 + 1]);
+              const float a2 = __uint_as_float(y[v * 4 + 2]);
+              const float a3 = __uint_as_float(y[v * 4 + 3]);
+              if (MODE == 1) {
+                *reinterpret_cast<float4*>(dst) = make_float4(a0, a1, a2, a3);
+              } else {
+                red_add_v4(dst, wt * a0, wt * a1, wt * a2, wt * a3);
+              }
             }
           }
         }
@@ -381,6 +418,10 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
   p.act = a.act;
   p.err = a.err;
   p.timeout_ns = kTimeoutNs;
+  p.sorted_slots = a.sorted_slots;
+  p.w = a.w;
+  p.T = a.T;
+  p.k = a.k;
 
   const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + sizeof(Ctl) +
                       sizeof(int32_t) * (size_t)(a.G + 1);
@@ -415,7 +456,12 @@ __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
-  return a.mode == 0 ? launch_mode<0>(a, st) : launch_mode<1>(a, st);
+  switch (a.mode) {
+    case 0: return launch_mode<0>(a, st);
+    case 1: return launch_mode<1>(a, st);
+    case 2: return launch_mode<2>(a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,

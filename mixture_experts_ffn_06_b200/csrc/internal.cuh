@@ -32,7 +32,7 @@ struct WsMap {
   size_t lt_rank;      // [T*k] int32 stable rank inside the layout block
   size_t x_perm;       // [cap,H] bf16 gathered activations
   size_t h;            // [cap,I] bf16 gated intermediate
-  size_t y_perm;       // [cap,H] bf16 expert outputs (moe_forward)
+  size_t acc;          // [T,H] fp32 layer accumulator (moe_forward)
   size_t total;
   int64_t cap;
   int64_t n_lt;
@@ -50,17 +50,26 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
                           cudaStream_t st);
 
+// Gathers x rows into x_perm; when acc is given also zeroes acc[0, n_acc).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
-                          int H, int64_t cap, __nv_bfloat16* x_perm,
-                          cudaStream_t st);
+                          int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
+                          int64_t n_acc, cudaStream_t st);
 
-cudaError_t launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row,
+cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,
                            __nv_bfloat16* out, cudaStream_t st);
 
-// Grouped GEMMs on tcgen05.  mode 0: h = Act(A W1^T) (*) (A W3^T) with B the
-// packed [G][2N][K] gate/up rows; mode 1: y = A W^T with B = [G][N][K].
+// out[i] = bf16 round-to-nearest-even of acc[i], i < n (n % 8 == 0).
+cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
+                            cudaStream_t st);
+
+// Grouped GEMMs on tcgen05.
+//   mode 0: h = Act(A W1^T) (*) (A W3^T), B = packed [G][2N][K] gate/up rows,
+//           bf16 out [cap, N];
+//   mode 1: y = A W^T, B = [G][N][K], fp32 out [cap, N] (unweighted rows);
+//   mode 2: as mode 1, but row r adds w_r * y_r into the fp32 accumulator
+//           row of its token (the fused combine).
 struct GroupedGemmArgs {
   int mode;
   const __nv_bfloat16* A;       // [cap, K]
@@ -70,9 +79,14 @@ struct GroupedGemmArgs {
   int G, E;                     // groups, routed groups
   int N, K;                     // output columns, reduction length
   int64_t cap;                  // rows of A / out
-  __nv_bfloat16* out;           // [cap, N]
+  void* out;                    // mode 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T,N]
   int act;
   uint32_t* err;
+  // mode 2 only
+  const int32_t* sorted_slots;  // [cap]
+  const float* w;               // [T,k]
+  int64_t T;
+  int k;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
 

@@ -35,7 +35,7 @@ WsMap workspace_map(const moe_shape& s) {
   m.lt_rank = take(sizeof(int32_t) * T * k);
   m.x_perm = take(2ull * m.cap * s.H);
   m.h = take(2ull * m.cap * Imax);
-  m.y_perm = take(2ull * m.cap * s.H);
+  m.acc = take(4ull * T * s.H);
   m.total = o;
   return m;
 }
@@ -79,14 +79,17 @@ static bool mark(void* const* ev, int i, cudaStream_t st) {
   return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
 }
 
+// gather -> w13 GEMM (+activation) -> w2 GEMM.  With acc == nullptr the w2
+// GEMM writes unweighted fp32 rows to y_perm (moe_expert_ffn); otherwise it
+// adds w * y into the fp32 [T,H] accumulator acc (moe_forward).
 static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
                                  const int32_t* offsets,
                                  const int32_t* sorted_slots,
                                  const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                  const __nv_bfloat16* w13_sh,
-                                 const __nv_bfloat16* w2_sh, __nv_bfloat16* y_perm,
-                                 void* ws, cudaStream_t st,
-                                 void* const* ev = nullptr) {
+                                 const __nv_bfloat16* w2_sh, float* y_perm,
+                                 float* acc, const float* w, void* ws,
+                                 cudaStream_t st, void* const* ev = nullptr) {
   const WsMap m = workspace_map(s);
   const int G = s.E + s.n_shared;
   auto* x_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.x_perm));
@@ -94,7 +97,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
   if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
   cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
-                                x_perm, st);
+                                x_perm, acc, acc ? s.T * (int64_t)s.H : 0, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 3, st)) return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
@@ -114,13 +117,17 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   e = launch_grouped_gemm(a, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
-  a.mode = 1;
+  a.mode = acc ? 2 : 1;
   a.A = h;
   a.B = w2;
   a.B_sh = w2_sh;
   a.N = s.H;
   a.K = s.I;
-  a.out = y_perm;
+  a.out = acc ? static_cast<void*>(acc) : static_cast<void*>(y_perm);
+  a.sorted_slots = sorted_slots;
+  a.w = w;
+  a.T = s.T;
+  a.k = s.k;
   return from_cuda(launch_grouped_gemm(a, st));
 }
 
@@ -172,7 +179,7 @@ moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
                           const int32_t* offsets, const int32_t* sorted_slots,
                           const moe_bf16* w13, const moe_bf16* w2,
                           const moe_bf16* w13_sh, const moe_bf16* w2_sh,
-                          moe_bf16* y_perm, void* ws, size_t ws_bytes,
+                          float* y_perm, void* ws, size_t ws_bytes,
                           cudaStream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -186,36 +193,36 @@ moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
                         sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
                         reinterpret_cast<const __nv_bfloat16*>(w2),
                         reinterpret_cast<const __nv_bfloat16*>(w13_sh),
-                        reinterpret_cast<const __nv_bfloat16*>(w2_sh),
-                        reinterpret_cast<__nv_bfloat16*>(y_perm), ws, stream);
+                        reinterpret_cast<const __nv_bfloat16*>(w2_sh), y_perm,
+                        nullptr, nullptr, ws, stream);
 }
 
-moe_status moe_combine(const moe_shape* shape, const moe_bf16* y_perm,
+moe_status moe_combine(const moe_shape* shape, const float* y_perm,
                        const int32_t* slot_row, const float* w, moe_bf16* out,
                        cudaStream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   if (!y_perm || !slot_row || !w || !out) return MOE_ERR_INVALID_ARG;
-  return from_cuda(launch_combine(reinterpret_cast<const __nv_bfloat16*>(y_perm),
-                                  slot_row, w, shape->T, shape->k,
+  return from_cuda(launch_combine(y_perm, slot_row, w, shape->T, shape->k,
                                   shape->n_shared, shape->H,
                                   reinterpret_cast<__nv_bfloat16*>(out), stream));
 }
 
-moe_status moe_forward_staged(const moe_shape* shape, const moe_bf16* x,
-                              const float* logits, const moe_bf16* w13,
-                              const moe_bf16* w2, const float* scale,
-                              const moe_bf16* w13_sh, const moe_bf16* w2_sh,
-                              moe_bf16* out, int32_t* ids_out, float* w_out,
-                              void* ws, size_t ws_bytes, void* const* ev,
-                              cudaStream_t stream) {
+moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
+                          const float* logits, const moe_bf16* w13,
+                          const moe_bf16* w2, const float* scale,
+                          const moe_bf16* w13_sh, const moe_bf16* w2_sh,
+                          moe_bf16* out, int32_t* ids_out, float* w_out, void* ws,
+                          size_t ws_bytes, const moe_forward_opts* opts,
+                          cudaStream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (!w13 || !w2 || (shape->T > 0 && (!x || !logits || !out)))
     return MOE_ERR_INVALID_ARG;
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  void* const* ev = opts ? opts->stage_events : nullptr;
   if (ev)
     for (int i = 0; i <= MOE_NUM_STAGES; ++i)
       if (!ev[i]) return MOE_ERR_INVALID_ARG;
@@ -231,7 +238,8 @@ moe_status moe_forward_staged(const moe_shape* shape, const moe_bf16* x,
   auto* offsets = reinterpret_cast<int32_t*>(at(ws, m.offsets));
   auto* sorted_slots = reinterpret_cast<int32_t*>(at(ws, m.sorted_slots));
   auto* slot_row = reinterpret_cast<int32_t*>(at(ws, m.slot_row));
-  auto* y_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.y_perm));
+  float* acc = (opts && opts->out_f32) ? opts->out_f32
+                                       : reinterpret_cast<float*>(at(ws, m.acc));
   if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
   if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -246,12 +254,12 @@ moe_status moe_forward_staged(const moe_shape* shape, const moe_bf16* x,
                       sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
                       reinterpret_cast<const __nv_bfloat16*>(w2),
                       reinterpret_cast<const __nv_bfloat16*>(w13_sh),
-                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), y_perm, ws,
-                      stream, ev);
+                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), nullptr, acc,
+                      w, ws, stream, ev);
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
-  if (launch_combine(y_perm, slot_row, w, s.T, s.k, s.n_shared, s.H,
-                     reinterpret_cast<__nv_bfloat16*>(out), stream) != cudaSuccess)
+  if (launch_finalize(acc, s.T * (int64_t)s.H,
+                      reinterpret_cast<__nv_bfloat16*>(out), stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -262,8 +270,8 @@ moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        const moe_bf16* w13_sh, const moe_bf16* w2_sh,
                        moe_bf16* out, int32_t* ids_out, float* w_out, void* ws,
                        size_t ws_bytes, cudaStream_t stream) {
-  return moe_forward_staged(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
-                            ids_out, w_out, ws, ws_bytes, nullptr, stream);
+  return moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
+                        ids_out, w_out, ws, ws_bytes, nullptr, stream);
 }
 
 moe_status moe_read_error(void* ws, size_t ws_bytes, cudaStream_t stream) {

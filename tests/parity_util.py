@@ -20,18 +20,24 @@ def to_device(inp: inputs.MoEInputs, device="cuda") -> inputs.MoEInputs:
 
 
 def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True):
+    """moe_forward_ex through the C ABI -> (out bf16, out_f32, ids, w).
+    Checks that the bf16 output is exactly the round-to-nearest-even of the
+    fp32 layer output."""
     s = api.shape_from(inp.shape)
     T, H, k = inp.shape.T, inp.shape.H, inp.shape.k
     dev = inp.x.device
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    out_f32 = torch.empty(T, H, dtype=torch.float32, device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev) if with_routing else None
     w = torch.empty(T, k, dtype=torch.float32, device=dev) if with_routing else None
     ws = api.alloc_workspace(s, dev)
-    api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
-                    inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w)
+    api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                       inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w,
+                       out_f32=out_f32)
     torch.cuda.synchronize()
     assert api.moe_read_error(ws) == 0
-    return out, ids, w
+    assert torch.equal(out, out_f32.to(torch.bfloat16)), "bf16 rounding step"
+    return out, out_f32, ids, w
 
 
 def oracle_forward(inp: inputs.MoEInputs, tokens=None):
@@ -40,8 +46,10 @@ def oracle_forward(inp: inputs.MoEInputs, tokens=None):
                           w2_sh=inp.w2_sh, tokens=tokens)
 
 
-def assert_out_close(got_bf16: torch.Tensor, want: np.ndarray, what=""):
-    got = got_bf16.float().cpu().numpy().astype(np.float64)
+def assert_out_close(got_t: torch.Tensor, want: np.ndarray, what=""):
+    """Literal bound on the layer output before its final bf16 rounding:
+    max|got - want| <= OUT_TOL * RMS(want)."""
+    got = got_t.float().cpu().numpy().astype(np.float64)
     assert got.shape == want.shape, (got.shape, want.shape)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     rms = float(np.sqrt(np.mean(want ** 2)))

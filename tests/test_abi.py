@@ -62,7 +62,7 @@ def test_capacity_and_workspace_size(api):
     assert api.moe_layout_capacity(s) == 64 * 2 + 8 * 127
     ws = api.moe_workspace_size(s)
     cap = 64 * 2 + 8 * 127
-    assert ws >= cap * 256 * 2 * 2 + cap * 512 * 2  # x_perm, y_perm, h
+    assert ws >= cap * 256 * 2 + cap * 512 * 2 + 64 * 256 * 4  # x_perm, h, acc
     sh = _shape(api, n_shared=2, I_shared=512)
     assert api.moe_layout_capacity(sh) == 64 * 2 + 64 * 2 + 10 * 127
     assert api.moe_workspace_size(sh) > ws

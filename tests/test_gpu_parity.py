@@ -1,9 +1,13 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
 Bars: top-k ids, the permutation and the slot maps bit-exact; gate weights
-within 1e-6 relative; layer outputs within max|err| <= 2e-2 x RMS(oracle).
-Small shapes are compared on every output element; the full-size workloads
-on every routing decision and on a token sample that covers every expert.
+within 1e-6 relative; the layer output within max|err| <= 2e-2 x RMS(oracle),
+checked on the fp32 result before its final rounding, while the bf16 output
+must be exactly the round-to-nearest-even of that fp32 result (rounding a
+heavy-tailed output to bf16 alone can exceed 2e-2 x RMS, so the bound cannot
+be put on the bf16 tensor itself).  Small shapes are compared on every output
+element; the full-size workloads on every routing decision and on a token
+sample that covers every expert.
 """
 import numpy as np
 import pytest
@@ -49,9 +53,9 @@ def _small(name, seed=0):
 def test_forward_small_every_element(api, name):
     inp = _small(name)
     want, ids_ref, w_ref = oracle_forward(inp)
-    out, ids, w = gpu_forward(api, to_device(inp))
+    out, out32, ids, w = gpu_forward(api, to_device(inp))
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out, want, name)
+    assert_out_close(out32, want, name)
 
 
 def test_all_tokens_on_one_expert(api):
@@ -61,9 +65,9 @@ def test_all_tokens_on_one_expert(api):
     inp.logits[:, 5] += 50.0
     want, ids_ref, w_ref = oracle_forward(inp)
     assert (ids_ref == 5).all()
-    out, ids, w = gpu_forward(api, to_device(inp))
+    out, out32, ids, w = gpu_forward(api, to_device(inp))
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out, want, "one hot expert")
+    assert_out_close(out32, want, "one hot expert")
 
 
 def _layout_gpu(api, s, ids_dev, E, S):
@@ -106,7 +110,8 @@ def test_permute_large_random_ids(api):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "tail704"])
-def test_four_call_chain_matches_fused_and_oracle_rows(api, name):
+def test_four_call_chain_against_oracle_rows(api, name):
+    """moe_route -> moe_permute -> moe_expert_ffn -> moe_combine."""
     inp = _small(name)
     shp = inp.shape
     d = to_device(inp)
@@ -121,15 +126,13 @@ def test_four_call_chain_matches_fused_and_oracle_rows(api, name):
     slot_row = torch.empty(T, k + S, dtype=torch.int32, device="cuda")
     ws = api.alloc_workspace(s)
     api.moe_permute(s, ids, offsets, sorted_slots, slot_row, ws)
-    y_perm = torch.empty(cap, H, dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.empty(cap, H, dtype=torch.float32, device="cuda")
     api.moe_expert_ffn(s, d.x, offsets, sorted_slots, d.w13, d.w2, d.w13_sh,
                        d.w2_sh, y_perm, ws)
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
     api.moe_combine(s, y_perm, slot_row, w, out)
     torch.cuda.synchronize()
     assert api.moe_read_error(ws) == 0
-    fused, _, _ = gpu_forward(api, d)
-    assert torch.equal(out, fused)  # same kernels, same order: bit-exact
 
     # unweighted expert rows against the oracle, every row in use
     used = int(offsets[-1])
@@ -139,30 +142,50 @@ def test_four_call_chain_matches_fused_and_oracle_rows(api, name):
     R = T * k
     routed = sl < R
     ids_np = ids.cpu().numpy().ravel()
-    y = y_perm[:used].float().cpu().numpy()
+    y = y_perm[:used].cpu().numpy().astype(np.float64)
     if routed.any():
-        tok = sl[routed] // k
-        ex = ids_np[sl[routed]]
-        want = oracle.expert_rows(inp.x, inp.w13, inp.w2, tok, ex, shp.act)
-        got = y[rows[routed]].astype(np.float64)
+        want = oracle.expert_rows(inp.x, inp.w13, inp.w2, sl[routed] // k,
+                                  ids_np[sl[routed]], shp.act)
         rms = np.sqrt(np.mean(want ** 2))
-        assert np.abs(got - want).max() <= 2e-2 * rms
+        assert np.abs(y[rows[routed]] - want).max() <= 2e-2 * rms
     if S:
         q = sl[~routed] - R
         want = oracle.expert_rows(inp.x, inp.w13_sh, inp.w2_sh, q % T, q // T,
                                   shp.act)
-        got = y[rows[~routed]].astype(np.float64)
         rms = np.sqrt(np.mean(want ** 2))
-        assert np.abs(got - want).max() <= 2e-2 * rms
+        assert np.abs(y[rows[~routed]] - want).max() <= 2e-2 * rms
     pad = np.nonzero(slots < 0)[0]
     assert (y[pad] == 0).all()  # padding rows hold zeros
 
+    # combine: fixed-order fp32 sum of the rows it was given, rounded once
+    sr = slot_row.long().cpu()
+    yt = y_perm.cpu()
+    acc = torch.zeros(T, H, dtype=torch.float32)
+    wt = w.cpu()
+    for j in range(k):
+        acc = torch.addcmul(acc, wt[:, j:j + 1], yt[sr[:, j]])
+    for sh in range(S):
+        acc = acc + yt[sr[:, k + sh]]
+    ref = acc.to(torch.bfloat16).float()
+    diff = (out.cpu().float() - ref).abs()
+    ulp = ref.abs().clamp_min(1e-30) * 2.0 ** -7
+    assert (diff <= ulp).all()  # within one bf16 ulp (fma vs mul+add)
 
-def test_deterministic_across_calls(api):
+    # the chain's fp32 sum and the fused call both meet the output bound
+    want, _, _ = oracle_forward(inp)
+    assert_out_close(acc, want, name + " chain")
+    _, out32, _, _ = gpu_forward(api, d)
+    assert_out_close(out32, want, name + " fused")
+
+
+def test_repeat_calls_agree(api):
+    # the fused combine adds in fp32 in no fixed order: repeat calls agree to
+    # fp32 rounding, not bit for bit
     inp = to_device(_small("gemma_shapes_T130"))
-    a, _, _ = gpu_forward(api, inp)
-    b, _, _ = gpu_forward(api, inp)
-    assert torch.equal(a, b)
+    _, a, _, _ = gpu_forward(api, inp)
+    _, b, _, _ = gpu_forward(api, inp)
+    scale = a.abs().max().item()
+    assert (a - b).abs().max().item() <= 1e-5 * scale
 
 
 def test_device_wait_limit_reports_timeout(api):
@@ -172,7 +195,7 @@ def test_device_wait_limit_reports_timeout(api):
     assert api.moe_read_error(ws) == 5  # MOE_ERR_TIMEOUT, context still usable
     assert api.moe_read_error(ws) == 0  # cleared
     inp = to_device(inputs.make_inputs(inputs.Shape(T=8, H=64, E=4, k=2, I=64)))
-    out, _, _ = gpu_forward(api, inp)
+    out, _, _, _ = gpu_forward(api, inp)
     assert torch.isfinite(out.float()).all()
 
 
@@ -213,10 +236,10 @@ def _cover_tokens(ids: np.ndarray, E: int, extra: int, seed: int) -> np.ndarray:
                                   "decode_t64", "decode_t256"])
 def test_decode_sweep_every_element(api, name):
     inp = inputs.make_inputs(name, seed=0, device="cuda")
-    out, ids, w = gpu_forward(api, inp)
+    out, out32, ids, w = gpu_forward(api, inp)
     want, ids_ref, w_ref = oracle_forward(inp)
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out, want, name)
+    assert_out_close(out32, want, name)
 
 
 @pytest.mark.parametrize("name", ["mixtral_prefill", "many_small_prefill",
@@ -224,7 +247,7 @@ def test_decode_sweep_every_element(api, name):
 def test_prefill_full_size(api, name):
     inp = inputs.make_inputs(name, seed=0, device="cuda")
     shp = inp.shape
-    out, ids, w = gpu_forward(api, inp)
+    out, out32, ids, w = gpu_forward(api, inp)
     # routing of every token, bit-exact ids
     ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
     assert_routing_exact(ids, w, ids_ref, w_ref)
@@ -237,4 +260,4 @@ def test_prefill_full_size(api, name):
     # outputs on a token sample covering every expert
     tok = _cover_tokens(ids_ref, shp.E, extra=6, seed=1)
     want_out, _, _ = oracle_forward(inp, tokens=tok)
-    assert_out_close(out[torch.from_numpy(tok).cuda()], want_out, name)
+    assert_out_close(out32[torch.from_numpy(tok).cuda()], want_out, name)
