@@ -47,7 +47,21 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", default="mixtral_prefill")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--shape", default=None,
+                    help="override the workload shape, e.g. T=4096,I=2048")
+    ap.add_argument("--profile", action="store_true",
+                    help="device timing only: skip the e2e and CPU legs")
     return ap.parse_args()
+
+
+def make_workload(args, device, seed):
+    from mixture_experts_ffn_06_b200 import inputs
+    over = {}
+    if args.shape:
+        for kv in args.shape.split(","):
+            key, val = kv.split("=")
+            over[key.strip()] = int(val)
+    return inputs.make_inputs(args.config, seed=seed, device=device, **over)
 
 
 def dist_env():
@@ -191,6 +205,43 @@ def cpu_oracle_rate(inp, budget_s: float = 12.0, max_rounds: int = 64):
 
 # ---------------------------------------------------------------- our arm
 
+def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks):
+    """Same metric through the C ABI with the token inputs copied from pinned
+    host memory and the output copied back, inside the timed region."""
+    import torch
+    shp = inp.shape
+    x_h = inp.x.cpu().pin_memory()
+    z_h = inp.logits.cpu().pin_memory()
+    out_h = torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(inp.x)
+    z_d = torch.empty_like(inp.logits)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        z_d.copy_(z_h, non_blocking=True)
+        api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                        inp.w2_sh, out, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+    return e2e_ms, h2d, d2h
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -204,7 +255,7 @@ def run_ours(args):
         dist.init_process_group("nccl", device_id=dev,
                                 timeout=__import__("datetime").timedelta(seconds=120))
 
-    inp = inputs.make_inputs(args.config, seed=args.seed + rank, device=dev)
+    inp = make_workload(args, dev, args.seed + rank)
     shp = inp.shape
     s = api.shape_from(shp)
     ws = api.alloc_workspace(s, dev)
@@ -242,6 +293,9 @@ def run_ours(args):
     nst = api.NUM_STAGES
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
                 for _ in range(args.steps)]
+    for evs in stage_ev:  # create the events before the timed region
+        for e in evs:
+            e.record(stream)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -265,35 +319,8 @@ def run_ours(args):
         raise RuntimeError(f"device error in the timed region: {status}")
 
     # ---- end to end: pinned host inputs in, host output back, every step
-    x_h = inp.x.cpu().pin_memory()
-    z_h = inp.logits.cpu().pin_memory()
-    out_h = torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(inp.x)
-    z_d = torch.empty_like(inp.logits)
-
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        z_d.copy_(z_h, non_blocking=True)
-        api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
-                        inp.w2_sh, out, ws)
-        out_h.copy_(out, non_blocking=True)
-
-    for _ in range(max(args.warmup, 3)):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
-    d2h = out_h.numel() * out_h.element_size()
+    e2e_ms, h2d, d2h = run_e2e(args, api, inp, s, ws, out, stream, barrier,
+                               max_over_ranks) if not args.profile else (None, 0, 0)
 
     result = None
     if rank == 0:
@@ -310,7 +337,7 @@ def run_ours(args):
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
         launches_per_step = 9  # route, layout x4, gather, 2 GEMMs, round
         cpu = None
-        if world == 1:
+        if world == 1 and not args.profile:
             rate, cores, ntok, secs = cpu_oracle_rate(inp)
             cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                    "sample": f"{ntok} tokens drawn from the same {shp.T}-token "
@@ -338,7 +365,8 @@ def run_ours(args):
             "layer_tflops": layer_tflops,
             "stage_ms": dict(zip(api.STAGE_NAMES, stage_ms)),
             "cpu_baseline": cpu,
-            "e2e": {"value": world * shp.T / (e2e_ms / 1e3), "unit": UNIT,
+            "e2e": None if e2e_ms is None else
+                   {"value": world * shp.T / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
@@ -361,7 +389,7 @@ def run_reference(args):
     import oracle
     from mixture_experts_ffn_06_b200 import inputs
 
-    inp = inputs.make_inputs(args.config, seed=args.seed, device="cpu")
+    inp = make_workload(args, "cpu", args.seed)
     shp = inp.shape
     cores = oracle.num_threads()
     per_step = min(cores, shp.T)
