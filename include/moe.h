@@ -192,6 +192,35 @@ MOE_API moe_status moe_forward_ex(
     const moe_forward_opts* opts, cudaStream_t stream);
 
 /*
+ * moe_permute_noalloc -- moe_permute for callers that cannot hand the library
+ * a workspace: code that runs while a CUDA graph is being captured (where
+ * cudaMalloc is not allowed), runtimes whose memory pool is fully reserved up
+ * front, and plug-in hosts that pass only the input and output buffers at
+ * launch time.  The pages have no counterpart of this entry point; it is a
+ * deployment convenience.
+ *
+ * Same inputs, outputs and results as moe_permute.  Its scratch (per-block
+ * histograms, bases and ranks of the counting sort, 1 MiB) is a fixed array
+ * in device memory that the library holds on every GPU it is loaded on
+ * until the process exits.  Nothing is allocated or freed by the call.
+ *   - Limit: T*k <= MOE_NOALLOC_MAX_SLOTS; larger batches (and every shape
+ *     moe_permute rejects) return MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG
+ *     before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one array: calls that may run at the same time on
+ *     the GPU (other streams, other host threads) race and must not overlap.
+ *     Every call writes the scratch it later reads, so nothing in the array
+ *     has to start at zero and the previous call's leftovers do no harm.
+ */
+#define MOE_NOALLOC_MAX_SLOTS 131072
+MOE_API moe_status moe_permute_noalloc(const moe_shape* shape,
+                                       const int32_t* ids, int32_t* offsets,
+                                       int32_t* sorted_slots,
+                                       int32_t* slot_row, cudaStream_t stream);
+
+/*
  * moe_read_error -- SYNCHRONISES ``stream``, then returns the status recorded
  * in the workspace error word by earlier calls on it (MOE_OK if none) and
  * clears the word.  ws is the device workspace used by those calls.

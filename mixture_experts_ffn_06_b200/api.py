@@ -26,7 +26,8 @@ STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act",
 EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_route",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_ex",
-           "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string")
+           "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string",
+           "moe_permute_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
                                    ctypes.c_size_t,
                                    ctypes.POINTER(moe_forward_opts), P]
     lib.moe_read_error.argtypes = [P, ctypes.c_size_t, P]
+    lib.moe_permute_noalloc.argtypes = [S, P, P, P, P, P]
+    lib.moe_permute_noalloc.restype = st
     lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t,
                                               ctypes.c_uint32, P]
     lib.moe_status_string.argtypes = [st]
@@ -147,6 +150,16 @@ def moe_permute(shape, ids, offsets, sorted_slots, slot_row, ws, stream=None):
     _check(lib.moe_permute(ctypes.byref(shape), _p(ids), _p(offsets),
                            _p(sorted_slots), _p(slot_row), _p(ws), ws.numel(),
                            _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(shape, ids, offsets, sorted_slots, slot_row,
+                        stream=None):
+    """moe_permute without a workspace (scratch in a fixed 1 MiB device array
+    inside the library; T*k <= MOE_NOALLOC_MAX_SLOTS; calls must not overlap
+    on the GPU)."""
+    _check(lib.moe_permute_noalloc(ctypes.byref(shape), _p(ids), _p(offsets),
+                                   _p(sorted_slots), _p(slot_row),
+                                   _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_expert_ffn(shape, x, offsets, sorted_slots, w13, w2, w13_sh, w2_sh,

@@ -40,6 +40,9 @@ struct WsMap {
 
 WsMap workspace_map(const moe_shape& s);
 
+// Shape validation shared by every entry point (MOE_OK or the error status).
+moe_status validate_shape(const moe_shape* s);
+
 // ---- launch wrappers (return cudaGetLastError of the launch) ----
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
                          int E, int k, int32_t* ids, float* w, cudaStream_t st);

@@ -57,6 +57,8 @@ static moe_status check_shape(const moe_shape* s) {
   return MOE_OK;
 }
 
+moe_status validate_shape(const moe_shape* s) { return check_shape(s); }
+
 static moe_status from_cuda(cudaError_t e) {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
