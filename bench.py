@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--shape", default=None,
                     help="override the workload shape, e.g. T=4096,I=2048")
+    ap.add_argument("--path", choices=("auto", "prefill", "decode"),
+                    default="auto", help="force the kernel path")
     ap.add_argument("--profile", action="store_true",
                     help="device timing only: skip the e2e and CPU legs")
     return ap.parse_args()
@@ -205,6 +207,17 @@ def cpu_oracle_rate(inp, budget_s: float = 12.0, max_rounds: int = 64):
 
 # ---------------------------------------------------------------- our arm
 
+def touched_experts(api, s, inp, ws) -> int:
+    """Distinct experts the batch routes to (+ shared experts), from one call
+    of the library's own routing."""
+    import torch
+    shp = inp.shape
+    ids = torch.empty(shp.T, shp.k, dtype=torch.int32, device=inp.x.device)
+    w = torch.empty(shp.T, shp.k, dtype=torch.float32, device=inp.x.device)
+    api.moe_route(s, inp.logits, inp.scale, ids, w)
+    return int(torch.unique(ids).numel()) + shp.n_shared
+
+
 def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks):
     """Same metric through the C ABI with the token inputs copied from pinned
     host memory and the output copied back, inside the timed region."""
@@ -262,14 +275,15 @@ def run_ours(args):
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    path = {"auto": api.PATH_AUTO, "prefill": api.PATH_PREFILL,
+            "decode": api.PATH_DECODE}[args.path]
+    decode = path == api.PATH_DECODE or (path == api.PATH_AUTO
+                                         and shp.T <= api.DECODE_MAX_T)
+
     def step(events=None):
-        if events is None:
-            api.moe_forward(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
-                            inp.w13_sh, inp.w2_sh, out, ws)
-        else:
-            api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2,
-                               inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
-                               events=events)
+        api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                           inp.w13_sh, inp.w2_sh, out, ws, events=events,
+                           path=path)
 
     def barrier():
         if world > 1:
@@ -326,16 +340,38 @@ def run_ours(args):
     if rank == 0:
         peaks, peak_src = load_peaks()
         value = world * shp.T / (ms_per_step / 1e3)
-        # dominant kernel: the w13 grouped GEMM with the fused activation
-        # (2/3 of the layer's FLOPs); algorithmic FLOPs count real rows only
+        # dominant kernel: the w13 product with the fused activation (2/3 of
+        # the layer's FLOPs and of its weight bytes); FLOPs count real rows
+        # only, bytes count each touched expert once
         w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) \
             * shp.H * 2
         w13_ms = stage_ms[3]
-        achieved = w13_flops / (w13_ms / 1e3) / 1e12
-        peak = float(peaks["bf16_tflops"])
-        traffic = traffic_for("gemm_tc.cu")
+        touched = touched_experts(api, s, inp, ws)
+        expert_bytes = 3.0 * shp.H * shp.I * 2
+        layer_bytes = touched * expert_bytes
+        if decode:
+            achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roof = {"bound": "hbm", "kernel": "decode_w13_kernel (w13 + act)",
+                    "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak,
+                    "peak_source": f"{peak_src} hbm_gbs",
+                    "traffic": traffic_for("decode.cu"),
+                    "layer_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peak,
+                    "touched_experts": touched}
+        else:
+            achieved = w13_flops / (w13_ms / 1e3) / 1e12
+            peak = float(peaks["bf16_tflops"])
+            roof = {"bound": "tensor", "kernel": "grouped_gemm_kernel<0> "
+                    "(w13 + activation)", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": f"{peak_src} bf16_tflops (burst)",
+                    "traffic": traffic_for("gemm_tc.cu"),
+                    "layer_frac": shp.flops() / (ms_per_step / 1e3) / 1e12 / peak}
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
-        launches_per_step = 9  # route, layout x4, gather, 2 GEMMs, round
+        # our kernels per step: prefill route, layout x4, gather, 2 GEMMs,
+        # row sum; decode route, w13, w2, row sum
+        launches_per_step = 4 if decode else 9
         cpu = None
         if world == 1 and not args.profile:
             rate, cores, ntok, secs = cpu_oracle_rate(inp)
@@ -351,17 +387,13 @@ def run_ours(args):
             "data": "synthetic: seeded N(0,1) tokens, N(0,0.02) bf16 random-init "
                     "expert weights, fp32 router logits with a 1e-3 top-k margin",
             "config": {"workload": workload_name(args.config, shp),
+                       "path": "decode" if decode else "prefill",
                        "global_batch": world * shp.T, "seq_len": shp.T,
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2: expert weights "
                              f"{(inp.w13.numel() + inp.w2.numel()) * 2 / 1e9:.2f} GB "
                              "streamed every step"},
-            "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<0> "
-                         "(w13 + activation)",
-                         "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "traffic": traffic},
+            "roofline": roof,
             "layer_tflops": layer_tflops,
             "stage_ms": dict(zip(api.STAGE_NAMES, stage_ms)),
             "cpu_baseline": cpu,

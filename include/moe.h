@@ -142,8 +142,8 @@ MOE_API moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
  * moe_combine -- weighted combine (walkthrough section 7 step 4; the weighted
  * sum after ggml_mul_mat_id in lesson 35), with shared experts at weight 1.
  *   y_perm [cap,H] fp32, slot_row [T,k+S] int32, w [T,k] fp32
- *   out    [T,H] bf16 out: sum over j in order 0..k-1, then the shared
- *          experts, in fp32, rounded once to bf16 (deterministic)
+ *   out    [T,H] bf16 out: w[t,j] * y rounded, then added in fp32 in order
+ *          j = 0..k-1, then the shared experts; rounded once to bf16
  */
 MOE_API moe_status moe_combine(const moe_shape* shape, const float* y_perm,
                        const int32_t* slot_row, const float* w, moe_bf16* out,
@@ -155,11 +155,10 @@ MOE_API moe_status moe_combine(const moe_shape* shape, const float* y_perm,
  * walkthrough's section 6 describes it).  ids_out [T,k] and w_out [T,k] may
  * be NULL; when given they receive the routing.
  * Here the combine is fused into the w2 GEMM's epilogue: each expert row is
- * multiplied by its gate weight and added into an fp32 [T,H] accumulator
- * with atomic vector adds, which a last pass rounds to bf16.  The order of
- * those fp32 additions is not fixed, so two calls may differ in the last bit
- * of the fp32 sum (and rarely in one bf16 ulp); moe_combine is the
- * deterministic alternative.
+ * multiplied by its gate weight and stored at its (token, choice) position;
+ * a last pass adds each token's k + S rows in a fixed order in fp32 and
+ * rounds once to bf16.  The result is deterministic and bit-identical to
+ * moe_expert_ffn followed by moe_combine.
  */
 MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        const float* logits, const moe_bf16* w13,
@@ -174,14 +173,28 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
  *                 caller; event i is recorded before stage i and event
  *                 MOE_NUM_STAGES after the last one, on ``stream``.  Stages:
  *                 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
- *                 4 w2 GEMM + weighted combine, 5 bf16 rounding.
- *   out_f32       NULL or [T,H] fp32: receives the layer output before its
- *                 rounding to bf16 (it is then used as the accumulator).
+ *                 4 w2 GEMM + gate weight + un-permute, 5 sum over the
+ *                 k + S rows of each token and bf16 rounding.
+ *   out_f32       NULL or [T,H] fp32: also receives the layer output before
+ *                 its rounding to bf16.
+ *   path          which kernels run (moe_path).  The decode path (T small)
+ *                 routes in one block and streams each touched expert's
+ *                 weights once through skinny tensor-core kernels; its
+ *                 stages 1 and 2 are empty (folded into stage 0).  Both
+ *                 paths compute the same function; they differ in the order
+ *                 of fp32 additions inside the products.
  */
 #define MOE_NUM_STAGES 6
+typedef enum {
+  MOE_PATH_AUTO = 0,     /* decode path when T <= MOE_DECODE_MAX_T */
+  MOE_PATH_PREFILL = 1,  /* tcgen05 grouped GEMMs over padded expert segments */
+  MOE_PATH_DECODE = 2    /* touched experts streamed by skinny kernels; T <= 1024 */
+} moe_path;
+#define MOE_DECODE_MAX_T 64
 typedef struct {
   void* const* stage_events;
   float* out_f32;
+  int32_t path;  /* moe_path */
 } moe_forward_opts;
 
 MOE_API moe_status moe_forward_ex(

@@ -10,8 +10,11 @@
 // (grid-stride over tokens); each thread owns 4 hidden columns at a time and
 // sums the k+S fp32 rows of y_perm that slot_row names in a fixed order.
 // HBM-bound: reads (k+S)*H*4 bytes, writes H*2.
-// finalize_kernel (the fused path): the w2 epilogue has already added every
-// weighted expert row into an fp32 [T,H] accumulator; this pass rounds it.
+// sum_rows_kernel (the fused path): the w2 epilogue has already stored every
+// weighted expert row at its (token, choice) position; this pass adds the
+// k+S contiguous rows of each token in order and rounds once.  Both paths
+// use the same arithmetic (product rounded, then added, in order j), so
+// they give bit-identical outputs.
 #include "internal.cuh"
 
 namespace moe {
@@ -36,13 +39,15 @@ combine_kernel(const float4* __restrict__ y_perm,
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       // fixed order: routed choices j = 0..k-1, then the shared experts
+      // product rounded, then added (no fma), the same arithmetic as the
+      // fused path's weighted epilogue followed by sum_rows_kernel
       for (int j = 0; j < ks; ++j) {
         const float4 v = __ldg(y_perm + rows[j] + c);
         const float wt = wts[j];
-        a0 = fmaf(wt, v.x, a0);
-        a1 = fmaf(wt, v.y, a1);
-        a2 = fmaf(wt, v.z, a2);
-        a3 = fmaf(wt, v.w, a3);
+        a0 = __fadd_rn(a0, __fmul_rn(wt, v.x));
+        a1 = __fadd_rn(a1, __fmul_rn(wt, v.y));
+        a2 = __fadd_rn(a2, __fmul_rn(wt, v.z));
+        a3 = __fadd_rn(a3, __fmul_rn(wt, v.w));
       }
       const __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
       const __nv_bfloat162 hi = __floats2bfloat162_rn(a2, a3);
@@ -54,25 +59,50 @@ combine_kernel(const float4* __restrict__ y_perm,
   }
 }
 
-// bf16 rounding of the fp32 accumulator, 8 values per thread-iteration.
+// Sum of the k+S weighted rows of a token, which the fused w2 epilogue has
+// stored contiguously, in order j = 0..k+S-1; one bf16 rounding.  Each thread
+// owns 8 columns (two float4) of one token at a time.
 __global__ void __launch_bounds__(256)
-finalize_kernel(const float4* __restrict__ acc, int64_t n8,
-                uint4* __restrict__ out) {
+sum_rows_kernel(const float4* __restrict__ stage, int64_t T, int ks, int H,
+                uint4* __restrict__ out, float4* __restrict__ out_f32) {
+  // when launched as a programmatic dependent, wait for the rows' producer
+  // (returns at once otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int c8 = H >> 3;
+  const int64_t n = T * c8;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += stride) {
-    const float4 a = __ldg(acc + 2 * i);
-    const float4 b = __ldg(acc + 2 * i + 1);
-    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
-    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
-    const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
-    const __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+    const int64_t t = i / c8;
+    const int c = (int)(i - t * c8);
+    const float4* src = stage + (t * ks) * (int64_t)(H >> 2) + 2 * c;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < ks; ++j) {
+      const float4 u = __ldg(src + (int64_t)j * (H >> 2));
+      const float4 v = __ldg(src + (int64_t)j * (H >> 2) + 1);
+      a[0] = __fadd_rn(a[0], u.x);
+      a[1] = __fadd_rn(a[1], u.y);
+      a[2] = __fadd_rn(a[2], u.z);
+      a[3] = __fadd_rn(a[3], u.w);
+      a[4] = __fadd_rn(a[4], v.x);
+      a[5] = __fadd_rn(a[5], v.y);
+      a[6] = __fadd_rn(a[6], v.z);
+      a[7] = __fadd_rn(a[7], v.w);
+    }
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a[0], a[1]);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a[2], a[3]);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[4], a[5]);
+    const __nv_bfloat162 p3 = __floats2bfloat162_rn(a[6], a[7]);
     uint4 o;
     o.x = *reinterpret_cast<const uint32_t*>(&p0);
     o.y = *reinterpret_cast<const uint32_t*>(&p1);
     o.z = *reinterpret_cast<const uint32_t*>(&p2);
     o.w = *reinterpret_cast<const uint32_t*>(&p3);
     out[i] = o;
+    if (out_f32) {
+      out_f32[2 * i] = make_float4(a[0], a[1], a[2], a[3]);
+      out_f32[2 * i + 1] = make_float4(a[4], a[5], a[6], a[7]);
+    }
   }
 }
 
@@ -91,15 +121,26 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
   return cudaGetLastError();
 }
 
-cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
-                            cudaStream_t st) {
-  const int64_t n8 = n / 8;
-  if (n8 == 0) return cudaSuccess;
-  const int64_t want = (n8 + 255) / 256;
+cudaError_t launch_sum_rows(const float* stage, int64_t T, int ks, int H,
+                            __nv_bfloat16* out, float* out_f32, cudaStream_t st,
+                            bool pdl) {
+  const int64_t n = T * (H / 8);
+  if (n == 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256;
   const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
-  finalize_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc), n8,
-                                          reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, sum_rows_kernel,
+                            reinterpret_cast<const float4*>(stage), T, ks, H,
+                            reinterpret_cast<uint4*>(out),
+                            reinterpret_cast<float4*>(out_f32));
 }
 
 }  // namespace moe

@@ -1,0 +1,430 @@
+// decode.cu -- the layer for small token counts, where it is bound by HBM:
+// every touched expert's weights must be streamed once, and each weight is
+// used by only a few tokens.  llama-cpp-visual-guide lesson 35 (cost
+// section) notes that decode moves the bottleneck from compute to moving
+// data; the design below streams only the touched experts' weights.
+//
+// Four kernels on one stream, the last three launched as programmatic
+// dependents (PDL) so each one's launch overlaps the previous one's tail:
+//   decode_route  one block: routes all T tokens (route_impl.cuh), counts
+//                 tokens per expert, lists the touched experts in ascending
+//                 id (shared experts last) and, per expert, its slots;
+//   decode_w13    one CTA per (touched expert, 16 rows of I): h = Act(x W1^T)
+//                 (*) (x W3^T) for the expert's tokens, rounded to bf16;
+//   decode_w2     one CTA per (touched expert, 16 rows of H): y = h W2^T,
+//                 times the gate weight, stored at the (token, choice) row;
+//   sum_rows      (combine.cu) adds each token's k+S rows in order, bf16 out.
+//
+// The skinny products use mma.sync m16n8k16 (bf16 in, fp32 accumulate) with
+// weight rows as the 16-row A operand and up to 8 tokens per B tile.  The K
+// order inside each 32-column chunk is permuted so that every thread loads
+// its A and B elements as one 16-byte vector: thread (g, c) of the warp reads
+// columns [8c, 8c+8) of rows g and g+8, and the same columns of its tokens;
+// MMA step s takes the words 2s and 2s+1 of those vectors.  A dot product is
+// indifferent to the order of its terms as long as A and B share it.  The 4
+// warps of a CTA split K and add their partial sums through shared memory.
+#include "route_impl.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kDecThreads = 128;
+constexpr int kDecRows = 16;
+constexpr int kDecNT = 8;                    // token tiles of 8 per pass
+constexpr int kDecPass = kDecNT * 8;         // tokens per pass
+
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                         uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// d += A(rows g, g+8; 32 permuted columns) x B(token; same columns)
+__device__ __forceinline__ void mma_chunk(float (&d)[4], const uint4& ar0,
+                                          const uint4& ar8, const uint4& b) {
+  mma16816(d, ar0.x, ar8.x, ar0.y, ar8.y, b.x, b.y);
+  mma16816(d, ar0.z, ar8.z, ar0.w, ar8.w, b.z, b.w);
+}
+
+__device__ __forceinline__ float dec_act(int act, float g) {
+  if (act == MOE_ACT_SILU) return g / (1.0f + expf(-g));
+  const float c = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * g * (1.0f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
+}
+
+// Exclusive scan of one value per thread over a 1024-thread block.
+__device__ int block_scan_excl(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int ws = warp_sums[lane];
+    int wi = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += n;
+    }
+    warp_sums[lane] = wi - ws;
+    if (lane == 31) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  const int r = incl - v + warp_sums[warp];
+  *total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
+
+// meta layout (int32): [0] n touched groups; [1 + i] group id of the i-th
+// touched group; [1 + G + i] first slot-list entry of group i (i <= n).
+__global__ void __launch_bounds__(1024)
+decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
+                    int T, int E, int k, int S, int32_t* __restrict__ ids,
+                    float* __restrict__ w, int32_t* __restrict__ meta,
+                    int32_t* __restrict__ slots) {
+  extern __shared__ int32_t dsm[];
+  const int G = E + S, R = T * k;
+  int32_t* cnt = dsm;            // [G]
+  int32_t* pos = cnt + G;        // [G]
+  int32_t* ids_s = pos + G;      // [R]
+  __shared__ int warp_sums[33];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  for (int i = tid; i < G; i += blockDim.x) cnt[i] = (i < E) ? 0 : T;
+  __syncthreads();
+  for (int t = warp; t < T; t += blockDim.x >> 5) {
+    int id;
+    float wt;
+    route_token_warp(logits + (int64_t)t * E, scale, E, k, &id, &wt);
+    if (lane < k) {
+      ids[t * k + lane] = id;
+      w[t * k + lane] = wt;
+      ids_s[t * k + lane] = id;
+    }
+  }
+  __syncthreads();
+  for (int s = tid; s < R; s += blockDim.x) atomicAdd(&cnt[ids_s[s]], 1);
+  __syncthreads();
+  const int c = (tid < G) ? cnt[tid] : 0;
+  const int f = c > 0 ? 1 : 0;
+  int total_c, total_f;
+  const int base = block_scan_excl(c, warp_sums, &total_c);
+  const int idx = block_scan_excl(f, warp_sums, &total_f);
+  if (tid < G) {
+    pos[tid] = base;
+    if (f) {
+      meta[1 + idx] = tid;
+      meta[1 + G + idx] = base;
+    }
+  }
+  if (tid == 0) {
+    meta[0] = total_f;
+    meta[1 + G + total_f] = total_c;
+  }
+  __syncthreads();
+  // slot lists: routed slots by atomic position (the order inside an expert's
+  // list only decides which MMA column a token uses, not its result)
+  for (int s = tid; s < R; s += blockDim.x) {
+    const int p = atomicAdd(&pos[ids_s[s]], 1);
+    slots[p] = s;
+  }
+  for (int q = tid; q < T * S; q += blockDim.x) {
+    const int sh = q / T, t = q - sh * T;
+    slots[pos[E + sh] + t] = R + q;
+  }
+}
+
+struct DecGroup {
+  int g, base, n;
+};
+
+__device__ __forceinline__ bool load_group(const int32_t* meta, int G, int idx,
+                                           DecGroup* out) {
+  const int n_groups = meta[0];
+  if (idx >= n_groups) return false;
+  out->g = meta[1 + idx];
+  out->base = meta[1 + G + idx];
+  out->n = meta[1 + G + idx + 1] - out->base;
+  return true;
+}
+
+__global__ void __launch_bounds__(kDecThreads, 4)
+decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
+                  const __nv_bfloat16* __restrict__ w13,
+                  const __nv_bfloat16* __restrict__ w13_sh,
+                  const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
+                  int T, int H, int I, int E, int k, int S, int act,
+                  __nv_bfloat16* __restrict__ h_dec) {
+  __shared__ int32_t tok_s[kDecPass];
+  __shared__ int32_t slot_s[kDecPass];
+  __shared__ float red[4][kDecNT][32][8];
+  pdl_trigger();
+  pdl_wait();  // routing (meta, slots) comes from decode_route
+  DecGroup grp;
+  if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
+  const int R = T * k;
+  const __nv_bfloat16* W = grp.g < E ? w13 + (int64_t)grp.g * 2 * I * H
+                                     : w13_sh + (int64_t)(grp.g - E) * 2 * I * H;
+  const int i0 = blockIdx.y * kDecRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, c = lane & 3;
+  const int nch = (H + 31) / 32;
+  const int ch0 = warp * nch / 4, ch1 = (warp + 1) * nch / 4;
+  const int ra = i0 + gq, rb = i0 + gq + 8;  // gate rows; up rows are +I
+  const bool va = ra < I, vb = rb < I;
+  const __nv_bfloat16* pga = W + (int64_t)ra * H;
+  const __nv_bfloat16* pgb = W + (int64_t)rb * H;
+  const __nv_bfloat16* pua = W + (int64_t)(I + ra) * H;
+  const __nv_bfloat16* pub = W + (int64_t)(I + rb) * H;
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+
+  for (int p0 = 0; p0 < grp.n; p0 += kDecPass) {
+    const int np = min(kDecPass, grp.n - p0);
+    const int NT = (np + 7) >> 3;
+    __syncthreads();
+    for (int i = threadIdx.x; i < np; i += kDecThreads) {
+      const int s = slots[grp.base + p0 + i];
+      slot_s[i] = s;
+      tok_s[i] = s < R ? s / k : (s - R) % T;
+    }
+    __syncthreads();
+    float ag[kDecNT][4], au[kDecNT][4];
+#pragma unroll
+    for (int nt = 0; nt < kDecNT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ag[nt][e] = au[nt][e] = 0.f;
+    // weights of chunk ch+1 are requested before chunk ch is multiplied
+    auto load_w = [&](int ch, uint4& ga, uint4& gb, uint4& ua, uint4& ub) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = ch < ch1 && col < H;
+      ga = (va && vc) ? ld_stream(pga + col) : z4;
+      gb = (vb && vc) ? ld_stream(pgb + col) : z4;
+      ua = (va && vc) ? ld_stream(pua + col) : z4;
+      ub = (vb && vc) ? ld_stream(pub + col) : z4;
+    };
+    uint4 nga, ngb, nua, nub;
+    load_w(ch0, nga, ngb, nua, nub);
+    for (int ch = ch0; ch < ch1; ++ch) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = col < H;
+      const uint4 wga = nga, wgb = ngb, wua = nua, wub = nub;
+      load_w(ch + 1, nga, ngb, nua, nub);
+#pragma unroll
+      for (int nt = 0; nt < kDecNT; ++nt) {
+        if (nt < NT) {
+          const int tk = nt * 8 + gq;
+          const uint4 xv = (tk < np && vc)
+              ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)tok_s[tk] * H + col))
+              : z4;
+          mma_chunk(ag[nt], wga, wgb, xv);
+          mma_chunk(au[nt], wua, wub, xv);
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < kDecNT; ++nt) {
+      if (nt < NT) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          red[warp][nt][lane][e] = ag[nt][e];
+          red[warp][nt][lane][4 + e] = au[nt][e];
+        }
+      }
+    }
+    __syncthreads();
+    for (int nt = warp; nt < NT; nt += 4) {
+      float g4[4], u4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        g4[e] = red[0][nt][lane][e] + red[1][nt][lane][e] + red[2][nt][lane][e] +
+                red[3][nt][lane][e];
+        u4[e] = red[0][nt][lane][4 + e] + red[1][nt][lane][4 + e] +
+                red[2][nt][lane][4 + e] + red[3][nt][lane][4 + e];
+      }
+      // fragment element e: row gq (+8 for e >= 2), token 2c + (e & 1)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = i0 + gq + (e >= 2 ? 8 : 0);
+        const int tk = nt * 8 + 2 * c + (e & 1);
+        if (row < I && tk < np)
+          h_dec[(int64_t)slot_s[tk] * I + row] =
+              __float2bfloat16_rn(dec_act(act, g4[e]) * u4[e]);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kDecThreads, 4)
+decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
+                 const __nv_bfloat16* __restrict__ w2,
+                 const __nv_bfloat16* __restrict__ w2_sh,
+                 const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
+                 const float* __restrict__ wgt, int T, int H, int I, int E, int k,
+                 int S, float* __restrict__ stage) {
+  __shared__ int32_t slot_s[kDecPass];
+  __shared__ float red[4][kDecNT][32][4];
+  pdl_trigger();
+  pdl_wait();  // h_dec comes from decode_w13 (which itself waited for routing)
+  DecGroup grp;
+  if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
+  const int R = T * k, ks = k + S;
+  const __nv_bfloat16* W = grp.g < E ? w2 + (int64_t)grp.g * H * I
+                                     : w2_sh + (int64_t)(grp.g - E) * H * I;
+  const int r0 = blockIdx.y * kDecRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, c = lane & 3;
+  const int nch = (I + 31) / 32;
+  const int ch0 = warp * nch / 4, ch1 = (warp + 1) * nch / 4;
+  const int ra = r0 + gq, rb = r0 + gq + 8;
+  const bool va = ra < H, vb = rb < H;
+  const __nv_bfloat16* pa = W + (int64_t)ra * I;
+  const __nv_bfloat16* pb = W + (int64_t)rb * I;
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+
+  for (int p0 = 0; p0 < grp.n; p0 += kDecPass) {
+    const int np = min(kDecPass, grp.n - p0);
+    const int NT = (np + 7) >> 3;
+    __syncthreads();
+    for (int i = threadIdx.x; i < np; i += kDecThreads)
+      slot_s[i] = slots[grp.base + p0 + i];
+    __syncthreads();
+    float acc[kDecNT][4];
+#pragma unroll
+    for (int nt = 0; nt < kDecNT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    auto load_w = [&](int ch, uint4& a, uint4& b) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = ch < ch1 && col < I;
+      a = (va && vc) ? ld_stream(pa + col) : z4;
+      b = (vb && vc) ? ld_stream(pb + col) : z4;
+    };
+    uint4 na, nb;
+    load_w(ch0, na, nb);
+    for (int ch = ch0; ch < ch1; ++ch) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = col < I;
+      const uint4 wa = na, wb = nb;
+      load_w(ch + 1, na, nb);
+#pragma unroll
+      for (int nt = 0; nt < kDecNT; ++nt) {
+        if (nt < NT) {
+          const int tk = nt * 8 + gq;
+          const uint4 hv = (tk < np && vc)
+              ? __ldg(reinterpret_cast<const uint4*>(h_dec + (int64_t)slot_s[tk] * I + col))
+              : z4;
+          mma_chunk(acc[nt], wa, wb, hv);
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < kDecNT; ++nt)
+      if (nt < NT)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) red[warp][nt][lane][e] = acc[nt][e];
+    __syncthreads();
+    for (int nt = warp; nt < NT; nt += 4) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = red[0][nt][lane][e] + red[1][nt][lane][e] +
+                        red[2][nt][lane][e] + red[3][nt][lane][e];
+        const int row = r0 + gq + (e >= 2 ? 8 : 0);
+        const int tk = nt * 8 + 2 * c + (e & 1);
+        if (row < H && tk < np) {
+          const int s = slot_s[tk];
+          int64_t dst;
+          float wt;
+          if (s < R) {
+            const int t = s / k;
+            dst = (int64_t)t * ks + (s - t * k);
+            wt = __ldg(wgt + s);
+          } else {
+            const int q = s - R, sh = q / T;
+            dst = (int64_t)(q - sh * T) * ks + k + sh;
+            wt = 1.0f;
+          }
+          stage[dst * H + row] = __fmul_rn(wt, y);
+        }
+      }
+    }
+  }
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace
+
+size_t decode_meta_ints(int G) { return 2 + 2 * (size_t)G; }
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev) {
+  auto mark = [&](int i) -> bool {
+    return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+  };
+  const int G = a.E + a.S, R = a.T * a.k;
+  if (!mark(0)) return cudaErrorUnknown;
+  const size_t smem = sizeof(int32_t) * (2 * (size_t)G + R);
+  decode_route_kernel<<<1, 1024, smem, st>>>(a.logits, a.scale, a.T, a.E, a.k, a.S,
+                                             a.ids, a.w, a.meta, a.slots);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
+  const int max_groups = (R < a.E ? R : a.E) + a.S;
+  e = launch_pdl(decode_w13_kernel, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
+                 dim3(kDecThreads), st, a.x, a.w13, a.w13_sh,
+                 (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
+                 a.k, a.S, a.act, a.h_dec);
+  if (e != cudaSuccess) return e;
+  if (!mark(4)) return cudaErrorUnknown;
+  e = launch_pdl(decode_w2_kernel, dim3(max_groups, (a.H + kDecRows - 1) / kDecRows),
+                 dim3(kDecThreads), st, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
+                 (const int32_t*)a.meta, (const int32_t*)a.slots, (const float*)a.w,
+                 a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
+  if (e != cudaSuccess) return e;
+  if (!mark(5)) return cudaErrorUnknown;
+  e = launch_sum_rows(a.stage, a.T, a.k + a.S, a.H, a.out, a.out_f32, st,
+                      /*pdl=*/true);
+  if (e != cudaSuccess) return e;
+  if (!mark(6)) return cudaErrorUnknown;
+  return cudaSuccess;
+}
+
+}  // namespace moe

@@ -20,9 +20,11 @@
 //     into one of two 256-column TMEM accumulators and releases ring slots
 //     and accumulators with tcgen05.commit;
 //   * warps 2-5 are the epilogue: tcgen05.ld of their 32 TMEM lanes, the
-//     gate activation fused in mode 0 (so g and u never reach HBM), bf16
-//     stores.  Two accumulators let the epilogue of tile i overlap the MMAs
-//     of tile i+1.
+//     gate activation fused in mode 0 (so g and u never reach HBM) with bf16
+//     h stores; in mode 2 each row is multiplied by its gate weight and
+//     stored at its (token, choice) position, so the combine that follows
+//     only sums k+S contiguous rows.  Two accumulators let the epilogue of
+//     tile i overlap the MMAs of tile i+1.
 // Every wait is bounded (tc_ptx.cuh: mbar_wait); on a timeout the block
 // records MOE_ERR_TIMEOUT, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -64,7 +66,7 @@ struct KParams {
   const int32_t* sorted_slots;  // mode 2
   const float* w;               // mode 2
   int64_t T;                    // mode 2
-  int k;                        // mode 2
+  int k, S;                     // mode 2
 };
 
 struct Tile {
@@ -99,14 +101,6 @@ __device__ __forceinline__ float act_apply(int act, float g) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Vector fp32 reduction into global memory (16-byte aligned destination).
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c,
-                                           float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 
 template <int MODE>
@@ -275,7 +269,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       } else {
-        // mode 1: plain fp32 rows; mode 2: weight and add into the token row
+        // mode 1: plain fp32 rows in permuted order; mode 2: the row times its
+        // gate weight, stored at its (token, choice) position (un-permute)
         float* orow;
         float wt = 1.0f;
         bool live = true;
@@ -285,16 +280,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const int32_t slot = p.sorted_slots[row];
           live = slot >= 0;
           const int64_t R = p.T * p.k;
-          int64_t tok = 0;
+          const int64_t ks = p.k + p.S;
+          int64_t dst = 0;
           if (live) {
             if (slot < R) {
-              tok = slot / p.k;
+              const int64_t t = slot / p.k;
+              dst = t * ks + (slot - t * p.k);
               wt = __ldg(p.w + slot);
             } else {
-              tok = (slot - R) % p.T;
+              const int64_t q = slot - R, sh = q / p.T;
+              dst = (q - sh * p.T) * ks + p.k + sh;
             }
           }
-          orow = static_cast<float*>(p.out) + tok * (int64_t)p.N;
+          orow = static_cast<float*>(p.out) + dst * (int64_t)p.N;
         }
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -314,7 +312,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               if (MODE == 1) {
                 *reinterpret_cast<float4*>(dst) = make_float4(a0, a1, a2, a3);
               } else {
-                red_add_v4(dst, wt * a0, wt * a1, wt * a2, wt * a3);
+                *reinterpret_cast<float4*>(dst) =
+                    make_float4(__fmul_rn(wt, a0), __fmul_rn(wt, a1),
+                                __fmul_rn(wt, a2), __fmul_rn(wt, a3));
               }
             }
           }
@@ -422,6 +422,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
   p.w = a.w;
   p.T = a.T;
   p.k = a.k;
+  p.S = a.G - a.E;
 
   const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + sizeof(Ctl) +
                       sizeof(int32_t) * (size_t)(a.G + 1);

@@ -32,7 +32,8 @@ struct WsMap {
   size_t lt_rank;      // [T*k] int32 stable rank inside the layout block
   size_t x_perm;       // [cap,H] bf16 gathered activations
   size_t h;            // [cap,I] bf16 gated intermediate
-  size_t acc;          // [T,H] fp32 layer accumulator (moe_forward)
+  size_t stage;        // [T,k+S,H] fp32 weighted expert rows (moe_forward)
+  size_t dec_meta;     // decode path: touched-expert lists
   size_t total;
   int64_t cap;
   int64_t n_lt;
@@ -53,26 +54,51 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
                           cudaStream_t st);
 
-// Gathers x rows into x_perm; when acc is given also zeroes acc[0, n_acc).
+// Gathers x rows into x_perm (zeros on padding rows).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
-                          int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
-                          int64_t n_acc, cudaStream_t st);
+                          int H, int64_t cap, __nv_bfloat16* x_perm,
+                          cudaStream_t st);
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,
                            __nv_bfloat16* out, cudaStream_t st);
 
-// out[i] = bf16 round-to-nearest-even of acc[i], i < n (n % 8 == 0).
-cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
-                            cudaStream_t st);
+// out[t] = bf16(sum_{j < ks} stage[t*ks + j]) summed in order j = 0..ks-1;
+// out_f32 (optional) receives the fp32 sum.
+// pdl: launch as a programmatic dependent of the previous kernel.
+cudaError_t launch_sum_rows(const float* stage, int64_t T, int ks, int H,
+                            __nv_bfloat16* out, float* out_f32, cudaStream_t st,
+                            bool pdl = false);
+
+// The small-T path (decode.cu).
+constexpr int kDecodeMaxT = MOE_DECODE_MAX_T;
+constexpr int kDecodeForcedMaxT = 1024;
+struct DecodeArgs {
+  const __nv_bfloat16* x;
+  const float* logits;
+  const float* scale;
+  const __nv_bfloat16 *w13, *w2, *w13_sh, *w2_sh;
+  int T, H, E, k, I, S, act;
+  int32_t* ids;          // [T,k] out
+  float* w;              // [T,k] out
+  int32_t* meta;         // [decode_meta_ints(E+S)] scratch
+  int32_t* slots;        // [T*(k+S)] scratch
+  __nv_bfloat16* h_dec;  // [T*(k+S), I] scratch
+  float* stage;          // [T*(k+S), H] scratch
+  __nv_bfloat16* out;    // [T,H]
+  float* out_f32;        // [T,H] or nullptr
+};
+size_t decode_meta_ints(int G);
+// ev: nullptr or MOE_NUM_STAGES + 1 events (see moe_forward_ex)
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev);
 
 // Grouped GEMMs on tcgen05.
 //   mode 0: h = Act(A W1^T) (*) (A W3^T), B = packed [G][2N][K] gate/up rows,
 //           bf16 out [cap, N];
 //   mode 1: y = A W^T, B = [G][N][K], fp32 out [cap, N] (unweighted rows);
-//   mode 2: as mode 1, but row r adds w_r * y_r into the fp32 accumulator
-//           row of its token (the fused combine).
+//   mode 2: as mode 1, but row r stores w_r * y_r (fp32) at row
+//           t*(k+S) + j of out, the (token, choice) order (un-permute).
 struct GroupedGemmArgs {
   int mode;
   const __nv_bfloat16* A;       // [cap, K]
@@ -82,7 +108,7 @@ struct GroupedGemmArgs {
   int G, E;                     // groups, routed groups
   int N, K;                     // output columns, reduction length
   int64_t cap;                  // rows of A / out
-  void* out;                    // mode 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T,N]
+  void* out;                    // mode 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T*(k+S),N]
   int act;
   uint32_t* err;
   // mode 2 only

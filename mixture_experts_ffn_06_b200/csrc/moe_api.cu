@@ -35,7 +35,8 @@ WsMap workspace_map(const moe_shape& s) {
   m.lt_rank = take(sizeof(int32_t) * T * k);
   m.x_perm = take(2ull * m.cap * s.H);
   m.h = take(2ull * m.cap * Imax);
-  m.acc = take(4ull * T * s.H);
+  m.stage = take(4ull * T * (k + S) * s.H);
+  m.dec_meta = take(sizeof(int32_t) * decode_meta_ints((int)G));
   m.total = o;
   return m;
 }
@@ -81,16 +82,17 @@ static bool mark(void* const* ev, int i, cudaStream_t st) {
   return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
 }
 
-// gather -> w13 GEMM (+activation) -> w2 GEMM.  With acc == nullptr the w2
-// GEMM writes unweighted fp32 rows to y_perm (moe_expert_ffn); otherwise it
-// adds w * y into the fp32 [T,H] accumulator acc (moe_forward).
+// gather -> w13 GEMM (+activation) -> w2 GEMM.  With stage == nullptr the w2
+// GEMM writes unweighted fp32 rows to y_perm in permuted order
+// (moe_expert_ffn); otherwise it stores w * y at the row's (token, choice)
+// position of stage [T, k+S, H] (moe_forward).
 static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
                                  const int32_t* offsets,
                                  const int32_t* sorted_slots,
                                  const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                  const __nv_bfloat16* w13_sh,
                                  const __nv_bfloat16* w2_sh, float* y_perm,
-                                 float* acc, const float* w, void* ws,
+                                 float* stage, const float* w, void* ws,
                                  cudaStream_t st, void* const* ev = nullptr) {
   const WsMap m = workspace_map(s);
   const int G = s.E + s.n_shared;
@@ -99,7 +101,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
   if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
   cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
-                                x_perm, acc, acc ? s.T * (int64_t)s.H : 0, st);
+                                x_perm, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 3, st)) return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
@@ -119,13 +121,13 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   e = launch_grouped_gemm(a, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
-  a.mode = acc ? 2 : 1;
+  a.mode = stage ? 2 : 1;
   a.A = h;
   a.B = w2;
   a.B_sh = w2_sh;
   a.N = s.H;
   a.K = s.I;
-  a.out = acc ? static_cast<void*>(acc) : static_cast<void*>(y_perm);
+  a.out = stage ? static_cast<void*>(stage) : static_cast<void*>(y_perm);
   a.sorted_slots = sorted_slots;
   a.w = w;
   a.T = s.T;
@@ -240,8 +242,38 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
   auto* offsets = reinterpret_cast<int32_t*>(at(ws, m.offsets));
   auto* sorted_slots = reinterpret_cast<int32_t*>(at(ws, m.sorted_slots));
   auto* slot_row = reinterpret_cast<int32_t*>(at(ws, m.slot_row));
-  float* acc = (opts && opts->out_f32) ? opts->out_f32
-                                       : reinterpret_cast<float*>(at(ws, m.acc));
+  auto* stage = reinterpret_cast<float*>(at(ws, m.stage));
+  const int path = opts ? opts->path : MOE_PATH_AUTO;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE)
+    return MOE_ERR_INVALID_ARG;
+  if (path == MOE_PATH_DECODE && s.T > kDecodeForcedMaxT) return MOE_ERR_UNSUPPORTED;
+  if (path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && s.T <= kDecodeMaxT)) {
+    // few tokens: stream only the touched experts (decode.cu)
+    DecodeArgs d{};
+    d.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    d.logits = logits;
+    d.scale = scale;
+    d.w13 = reinterpret_cast<const __nv_bfloat16*>(w13);
+    d.w2 = reinterpret_cast<const __nv_bfloat16*>(w2);
+    d.w13_sh = reinterpret_cast<const __nv_bfloat16*>(w13_sh);
+    d.w2_sh = reinterpret_cast<const __nv_bfloat16*>(w2_sh);
+    d.T = (int)s.T;
+    d.H = s.H;
+    d.E = s.E;
+    d.k = s.k;
+    d.I = s.I;
+    d.S = s.n_shared;
+    d.act = s.act;
+    d.ids = ids;
+    d.w = w;
+    d.meta = reinterpret_cast<int32_t*>(at(ws, m.dec_meta));
+    d.slots = sorted_slots;
+    d.h_dec = reinterpret_cast<__nv_bfloat16*>(at(ws, m.h));
+    d.stage = stage;
+    d.out = reinterpret_cast<__nv_bfloat16*>(out);
+    d.out_f32 = opts ? opts->out_f32 : nullptr;
+    return from_cuda(launch_decode(d, stream, ev));
+  }
   if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
   if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -256,12 +288,13 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                       sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
                       reinterpret_cast<const __nv_bfloat16*>(w2),
                       reinterpret_cast<const __nv_bfloat16*>(w13_sh),
-                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), nullptr, acc,
-                      w, ws, stream, ev);
+                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), nullptr,
+                      stage, w, ws, stream, ev);
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
-  if (launch_finalize(acc, s.T * (int64_t)s.H,
-                      reinterpret_cast<__nv_bfloat16*>(out), stream) != cudaSuccess)
+  if (launch_sum_rows(stage, s.T, s.k + s.n_shared, s.H,
+                      reinterpret_cast<__nv_bfloat16*>(out),
+                      opts ? opts->out_f32 : nullptr, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
 }

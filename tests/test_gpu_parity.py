@@ -49,25 +49,31 @@ def _small(name, seed=0):
     return inputs.make_inputs(shp, seed=seed, bias=bias, scale=scale)
 
 
+PATHS = {"prefill": 1, "decode": 2}
+
+
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(SMALL))
-def test_forward_small_every_element(api, name):
+def test_forward_small_every_element(api, name, path):
     inp = _small(name)
     want, ids_ref, w_ref = oracle_forward(inp)
-    out, out32, ids, w = gpu_forward(api, to_device(inp))
+    out, out32, ids, w = gpu_forward(api, to_device(inp), path=PATHS[path])
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out32, want, name)
+    assert_out_close(out32, want, f"{name} ({path})")
 
 
-def test_all_tokens_on_one_expert(api):
-    # one expert takes every token: a segment of several M tiles, others empty
+@pytest.mark.parametrize("path", list(PATHS))
+def test_all_tokens_on_one_expert(api, path):
+    # one expert takes every token: a segment of several M tiles (prefill)
+    # or several 64-token passes (decode); the other experts are empty
     shp = inputs.Shape(T=300, H=128, E=8, k=1, I=256)
     inp = inputs.make_inputs(shp, seed=1)
     inp.logits[:, 5] += 50.0
     want, ids_ref, w_ref = oracle_forward(inp)
     assert (ids_ref == 5).all()
-    out, out32, ids, w = gpu_forward(api, to_device(inp))
+    out, out32, ids, w = gpu_forward(api, to_device(inp), path=PATHS[path])
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out32, want, "one hot expert")
+    assert_out_close(out32, want, f"one hot expert ({path})")
 
 
 def _layout_gpu(api, s, ids_dev, E, S):
@@ -171,21 +177,21 @@ def test_four_call_chain_against_oracle_rows(api, name):
     ulp = ref.abs().clamp_min(1e-30) * 2.0 ** -7
     assert (diff <= ulp).all()  # within one bf16 ulp (fma vs mul+add)
 
-    # the chain's fp32 sum and the fused call both meet the output bound
+    # the chain's fp32 sum and the fused call both meet the output bound, and
+    # the two paths use the same arithmetic: bit-identical outputs
     want, _, _ = oracle_forward(inp)
     assert_out_close(acc, want, name + " chain")
-    _, out32, _, _ = gpu_forward(api, d)
+    fused, out32, _, _ = gpu_forward(api, d, path=PATHS["prefill"])
     assert_out_close(out32, want, name + " fused")
+    assert torch.equal(out, fused)  # same GEMM kernels, same additions
 
 
-def test_repeat_calls_agree(api):
-    # the fused combine adds in fp32 in no fixed order: repeat calls agree to
-    # fp32 rounding, not bit for bit
+@pytest.mark.parametrize("path", list(PATHS))
+def test_repeat_calls_are_bit_identical(api, path):
     inp = to_device(_small("gemma_shapes_T130"))
-    _, a, _, _ = gpu_forward(api, inp)
-    _, b, _, _ = gpu_forward(api, inp)
-    scale = a.abs().max().item()
-    assert (a - b).abs().max().item() <= 1e-5 * scale
+    a, a32, _, _ = gpu_forward(api, inp, path=PATHS[path])
+    b, b32, _, _ = gpu_forward(api, inp, path=PATHS[path])
+    assert torch.equal(a, b) and torch.equal(a32, b32)
 
 
 def test_device_wait_limit_reports_timeout(api):
@@ -232,11 +238,12 @@ def _cover_tokens(ids: np.ndarray, E: int, extra: int, seed: int) -> np.ndarray:
     return np.array(sorted(set(chosen)), np.int64)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", ["decode_t1", "decode_t4", "decode_t16",
                                   "decode_t64", "decode_t256"])
-def test_decode_sweep_every_element(api, name):
+def test_decode_sweep_every_element(api, name, path):
     inp = inputs.make_inputs(name, seed=0, device="cuda")
-    out, out32, ids, w = gpu_forward(api, inp)
+    out, out32, ids, w = gpu_forward(api, inp, path=PATHS[path])
     want, ids_ref, w_ref = oracle_forward(inp)
     assert_routing_exact(ids, w, ids_ref, w_ref)
     assert_out_close(out32, want, name)
