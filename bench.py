@@ -51,6 +51,10 @@ def parse():
                     help="override the workload shape, e.g. T=4096,I=2048")
     ap.add_argument("--path", choices=("auto", "prefill", "decode"),
                     default="auto", help="force the kernel path")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="fixed-order combine on the prefill path")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain stream launches instead of one CUDA graph")
     ap.add_argument("--profile", action="store_true",
                     help="device timing only: skip the e2e and CPU legs")
     return ap.parse_args()
@@ -273,7 +277,10 @@ def run_ours(args):
     s = api.shape_from(shp)
     ws = api.alloc_workspace(s, dev)
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+    # all work on a side stream (CUDA graphs are captured off the default one)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
 
     path = {"auto": api.PATH_AUTO, "prefill": api.PATH_PREFILL,
             "decode": api.PATH_DECODE}[args.path]
@@ -283,7 +290,7 @@ def run_ours(args):
     def step(events=None):
         api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                            inp.w13_sh, inp.w2_sh, out, ws, events=events,
-                           path=path)
+                           path=path, deterministic=args.deterministic)
 
     def barrier():
         if world > 1:
@@ -303,13 +310,33 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {status}")
 
-    # ---- device-resident timed region (per-stage events on the stream)
+    # ---- device-resident timed region (per-stage events on the stream).
+    # By default the K steps are captured once into a CUDA graph and the
+    # timed region is one replay of it, so that host launch overhead does
+    # not pace small batches; the library makes no allocation or
+    # synchronisation, so its calls capture as they are.
     nst = api.NUM_STAGES
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
                 for _ in range(args.steps)]
     for evs in stage_ev:  # create the events before the timed region
         for e in evs:
             e.record(stream)
+    graph = staged = None
+    if not args.no_graph:
+        # one graph of K plain steps (the timed region) and one of K steps
+        # with stage events (per-kernel times: an event node adds a few
+        # microseconds, so it stays out of the step time)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(args.steps):
+                step()
+        staged = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(staged, stream=stream):
+            for i in range(args.steps):
+                step(stage_ev[i])
+        graph.replay()  # untimed first replays
+        staged.replay()
+        torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -318,16 +345,35 @@ def run_ours(args):
     clocks.start()
     time.sleep(0.3)  # let the sampler start before the timed work
     t_start.record(stream)
-    for i in range(args.steps):
-        step(stage_ev[i])
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            step()
     t_end.record(stream)
+    if staged is not None:
+        staged.replay()
+    else:
+        for i in range(args.steps):
+            step(stage_ev[i])
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    if graph is not None:
+        del graph, staged
     ms_total = max_over_ranks(t_start.elapsed_time(t_end))
     ms_per_step = ms_total / args.steps
-    stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev)
-                for j in range(nst)]
+    try:
+        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
+                                    for ev in stage_ev) for j in range(nst)]
+    except RuntimeError:
+        # events inside the graph could not be timed: take the stage times
+        # from the same K steps launched on the stream instead
+        for i in range(args.steps):
+            step(stage_ev[i])
+        torch.cuda.synchronize()
+        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
+                                    for ev in stage_ev) for j in range(nst)]
     status = api.moe_read_error(ws)
     if status != 0:
         raise RuntimeError(f"device error in the timed region: {status}")
@@ -388,6 +434,10 @@ def run_ours(args):
                     "expert weights, fp32 router logits with a 1e-3 top-k margin",
             "config": {"workload": workload_name(args.config, shp),
                        "path": "decode" if decode else "prefill",
+                       "combine": "fixed-order" if (decode or args.deterministic)
+                                  else "fp32 reductions",
+                       "timing": "one CUDA-graph replay of the K steps"
+                                 if not args.no_graph else "stream launches",
                        "global_batch": world * shp.T, "seq_len": shp.T,
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2: expert weights "

@@ -155,10 +155,15 @@ MOE_API moe_status moe_combine(const moe_shape* shape, const float* y_perm,
  * walkthrough's section 6 describes it).  ids_out [T,k] and w_out [T,k] may
  * be NULL; when given they receive the routing.
  * Here the combine is fused into the w2 GEMM's epilogue: each expert row is
- * multiplied by its gate weight and stored at its (token, choice) position;
- * a last pass adds each token's k + S rows in a fixed order in fp32 and
- * rounds once to bf16.  The result is deterministic and bit-identical to
- * moe_expert_ffn followed by moe_combine.
+ * multiplied by its gate weight and added into an fp32 [T,H] accumulator
+ * with vector reductions, which a last pass rounds once to bf16.  The order
+ * of those fp32 additions is not fixed, so two calls may differ in the last
+ * bits of the fp32 sum (and rarely by one bf16 ulp).  moe_forward_ex with
+ * deterministic = 1 instead stores each weighted row at its (token, choice)
+ * position and adds the k + S rows of a token in a fixed order: then the
+ * result is reproducible and bit-identical to moe_expert_ffn followed by
+ * moe_combine, at the cost of writing and reading T*(k+S)*H*4 more bytes.
+ * The decode path is always deterministic.
  */
 MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        const float* logits, const moe_bf16* w13,
@@ -173,8 +178,9 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
  *                 caller; event i is recorded before stage i and event
  *                 MOE_NUM_STAGES after the last one, on ``stream``.  Stages:
  *                 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
- *                 4 w2 GEMM + gate weight + un-permute, 5 sum over the
- *                 k + S rows of each token and bf16 rounding.
+ *                 4 w2 GEMM + gate weight + combine, 5 bf16 rounding
+ *                 (with deterministic = 1: the fixed-order sum over the
+ *                 k + S rows of each token, then the rounding).
  *   out_f32       NULL or [T,H] fp32: also receives the layer output before
  *                 its rounding to bf16.
  *   path          which kernels run (moe_path).  The decode path (T small)
@@ -194,7 +200,8 @@ typedef enum {
 typedef struct {
   void* const* stage_events;
   float* out_f32;
-  int32_t path;  /* moe_path */
+  int32_t path;           /* moe_path */
+  int32_t deterministic;  /* prefill path: fixed-order combine (see above) */
 } moe_forward_opts;
 
 MOE_API moe_status moe_forward_ex(

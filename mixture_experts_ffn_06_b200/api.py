@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 NUM_STAGES = 6
 STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act",
-               "w2_gemm_weight_unpermute", "sum_rows_bf16")
+               "w2_gemm_weight_combine", "round_bf16")
 EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_route",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_ex",
@@ -43,7 +43,8 @@ DECODE_MAX_T = 64
 class moe_forward_opts(ctypes.Structure):
     _fields_ = [("stage_events", ctypes.c_void_p),
                 ("out_f32", ctypes.c_void_p),
-                ("path", ctypes.c_int32)]
+                ("path", ctypes.c_int32),
+                ("deterministic", ctypes.c_int32)]
 
 
 class moe_shape(ctypes.Structure):
@@ -190,11 +191,12 @@ def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
 
 def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                    ids_out=None, w_out=None, events=None, out_f32=None,
-                   path=PATH_AUTO, stream=None):
+                   path=PATH_AUTO, deterministic=False, stream=None):
     """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
     created with enable_timing=True) recorded around the stages, ``out_f32``
     ([T,H] fp32) receiving the output before its bf16 rounding, and ``path``
-    (PATH_AUTO, PATH_PREFILL or PATH_DECODE)."""
+    (PATH_AUTO, PATH_PREFILL or PATH_DECODE); ``deterministic`` selects the
+    fixed-order combine on the prefill path."""
     arr = None
     if events is not None:
         if len(events) != NUM_STAGES + 1:
@@ -207,7 +209,7 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
             *[ctypes.c_void_p(e.cuda_event) for e in events])
     opts = moe_forward_opts(
         ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
-        _p(out_f32), path)
+        _p(out_f32), path, int(bool(deterministic)))
     _check(lib.moe_forward_ex(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
                               _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
                               _p(ids_out), _p(w_out), _p(ws), ws.numel(),

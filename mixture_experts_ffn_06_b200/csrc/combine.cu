@@ -10,7 +10,9 @@
 // (grid-stride over tokens); each thread owns 4 hidden columns at a time and
 // sums the k+S fp32 rows of y_perm that slot_row names in a fixed order.
 // HBM-bound: reads (k+S)*H*4 bytes, writes H*2.
-// sum_rows_kernel (the fused path): the w2 epilogue has already stored every
+// finalize_kernel (the fused fast path): the w2 epilogue has already added
+// every weighted expert row into an fp32 [T,H] accumulator; this rounds it.
+// sum_rows_kernel (the fused deterministic path): the w2 epilogue has stored every
 // weighted expert row at its (token, choice) position; this pass adds the
 // k+S contiguous rows of each token in order and rounds once.  Both paths
 // use the same arithmetic (product rounded, then added, in order j), so
@@ -106,7 +108,46 @@ sum_rows_kernel(const float4* __restrict__ stage, int64_t T, int ks, int H,
   }
 }
 
+// out = bf16 RNE of the fp32 accumulator the w2 epilogue added into (and an
+// fp32 copy when asked), 8 values per thread-iteration.
+__global__ void __launch_bounds__(256)
+finalize_kernel(const float4* __restrict__ acc, int64_t n8, uint4* __restrict__ out,
+                float4* __restrict__ out_f32) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += stride) {
+    const float4 a = __ldg(acc + 2 * i);
+    const float4 b = __ldg(acc + 2 * i + 1);
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
+    const __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&p0);
+    o.y = *reinterpret_cast<const uint32_t*>(&p1);
+    o.z = *reinterpret_cast<const uint32_t*>(&p2);
+    o.w = *reinterpret_cast<const uint32_t*>(&p3);
+    out[i] = o;
+    if (out_f32) {
+      out_f32[2 * i] = a;
+      out_f32[2 * i + 1] = b;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
+                            float* out_f32, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  const int64_t want = (n8 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  finalize_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc), n8,
+                                          reinterpret_cast<uint4*>(out),
+                                          reinterpret_cast<float4*>(out_f32));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,

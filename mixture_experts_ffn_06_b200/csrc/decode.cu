@@ -11,7 +11,7 @@
 //                 id (shared experts last) and, per expert, its slots;
 //   decode_w13    one CTA per (touched expert, 16 rows of I): h = Act(x W1^T)
 //                 (*) (x W3^T) for the expert's tokens, rounded to bf16;
-//   decode_w2     one CTA per (touched expert, 16 rows of H): y = h W2^T,
+//   decode_w2     one CTA per (touched expert, 64 rows of H): y = h W2^T,
 //                 times the gate weight, stored at the (token, choice) row;
 //   sum_rows      (combine.cu) adds each token's k+S rows in order, bf16 out.
 //
@@ -21,8 +21,10 @@
 // its A and B elements as one 16-byte vector: thread (g, c) of the warp reads
 // columns [8c, 8c+8) of rows g and g+8, and the same columns of its tokens;
 // MMA step s takes the words 2s and 2s+1 of those vectors.  A dot product is
-// indifferent to the order of its terms as long as A and B share it.  The 4
-// warps of a CTA split K and add their partial sums through shared memory.
+// indifferent to the order of its terms as long as A and B share it.  In
+// decode_w13 the 4 warps of a CTA split K (H is long) and add their partial
+// sums through shared memory; in decode_w2 each warp owns 16 rows and all of
+// K (I is short).
 #include "route_impl.cuh"
 
 namespace moe {
@@ -183,8 +185,8 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
   __shared__ int32_t tok_s[kDecPass];
   __shared__ int32_t slot_s[kDecPass];
   __shared__ float red[4][kDecNT][32][8];
-  pdl_trigger();
   pdl_wait();  // routing (meta, slots) comes from decode_route
+  pdl_trigger();
   DecGroup grp;
   if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
   const int R = T * k;
@@ -279,6 +281,11 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
   }
 }
 
+// One CTA per (touched expert, 64 rows of H); each warp owns 16 rows and the
+// whole of K = I, so no cross-warp reduction is needed.  The weight loads run
+// two 32-column chunks ahead of the MMAs.
+constexpr int kW2Rows = 64;
+
 __global__ void __launch_bounds__(kDecThreads, 4)
 decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const __nv_bfloat16* __restrict__ w2,
@@ -287,24 +294,28 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const float* __restrict__ wgt, int T, int H, int I, int E, int k,
                  int S, float* __restrict__ stage) {
   __shared__ int32_t slot_s[kDecPass];
-  __shared__ float red[4][kDecNT][32][4];
-  pdl_trigger();
   pdl_wait();  // h_dec comes from decode_w13 (which itself waited for routing)
+  pdl_trigger();
   DecGroup grp;
   if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
   const int R = T * k, ks = k + S;
   const __nv_bfloat16* W = grp.g < E ? w2 + (int64_t)grp.g * H * I
                                      : w2_sh + (int64_t)(grp.g - E) * H * I;
-  const int r0 = blockIdx.y * kDecRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, c = lane & 3;
+  const int r0 = blockIdx.y * kW2Rows + warp * kDecRows;
   const int nch = (I + 31) / 32;
-  const int ch0 = warp * nch / 4, ch1 = (warp + 1) * nch / 4;
   const int ra = r0 + gq, rb = r0 + gq + 8;
   const bool va = ra < H, vb = rb < H;
   const __nv_bfloat16* pa = W + (int64_t)ra * I;
   const __nv_bfloat16* pb = W + (int64_t)rb * I;
   const uint4 z4 = make_uint4(0, 0, 0, 0);
+  auto load_w = [&](int ch, uint4& a, uint4& b) {
+    const int col = ch * 32 + 8 * c;
+    const bool vc = ch < nch && col < I;
+    a = (va && vc) ? ld_stream(pa + col) : z4;
+    b = (vb && vc) ? ld_stream(pb + col) : z4;
+  };
 
   for (int p0 = 0; p0 < grp.n; p0 += kDecPass) {
     const int np = min(kDecPass, grp.n - p0);
@@ -318,19 +329,16 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
     for (int nt = 0; nt < kDecNT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-    auto load_w = [&](int ch, uint4& a, uint4& b) {
-      const int col = ch * 32 + 8 * c;
-      const bool vc = ch < ch1 && col < I;
-      a = (va && vc) ? ld_stream(pa + col) : z4;
-      b = (vb && vc) ? ld_stream(pb + col) : z4;
-    };
-    uint4 na, nb;
-    load_w(ch0, na, nb);
-    for (int ch = ch0; ch < ch1; ++ch) {
+    uint4 qa0, qb0, qa1, qb1;  // chunks ch and ch+1 in flight
+    load_w(0, qa0, qb0);
+    load_w(1, qa1, qb1);
+    for (int ch = 0; ch < nch; ++ch) {
       const int col = ch * 32 + 8 * c;
       const bool vc = col < I;
-      const uint4 wa = na, wb = nb;
-      load_w(ch + 1, na, nb);
+      const uint4 wa = qa0, wb = qb0;
+      qa0 = qa1;
+      qb0 = qb1;
+      load_w(ch + 2, qa1, qb1);
 #pragma unroll
       for (int nt = 0; nt < kDecNT; ++nt) {
         if (nt < NT) {
@@ -343,32 +351,27 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < kDecNT; ++nt)
-      if (nt < NT)
+    for (int nt = 0; nt < kDecNT; ++nt) {
+      if (nt < NT) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) red[warp][nt][lane][e] = acc[nt][e];
-    __syncthreads();
-    for (int nt = warp; nt < NT; nt += 4) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float y = red[0][nt][lane][e] + red[1][nt][lane][e] +
-                        red[2][nt][lane][e] + red[3][nt][lane][e];
-        const int row = r0 + gq + (e >= 2 ? 8 : 0);
-        const int tk = nt * 8 + 2 * c + (e & 1);
-        if (row < H && tk < np) {
-          const int s = slot_s[tk];
-          int64_t dst;
-          float wt;
-          if (s < R) {
-            const int t = s / k;
-            dst = (int64_t)t * ks + (s - t * k);
-            wt = __ldg(wgt + s);
-          } else {
-            const int q = s - R, sh = q / T;
-            dst = (int64_t)(q - sh * T) * ks + k + sh;
-            wt = 1.0f;
+        for (int e = 0; e < 4; ++e) {
+          const int row = r0 + gq + (e >= 2 ? 8 : 0);
+          const int tk = nt * 8 + 2 * c + (e & 1);
+          if (row < H && tk < np) {
+            const int s = slot_s[tk];
+            int64_t dst;
+            float wt;
+            if (s < R) {
+              const int t = s / k;
+              dst = (int64_t)t * ks + (s - t * k);
+              wt = __ldg(wgt + s);
+            } else {
+              const int q = s - R, sh = q / T;
+              dst = (int64_t)(q - sh * T) * ks + k + sh;
+              wt = 1.0f;
+            }
+            stage[dst * H + row] = __fmul_rn(wt, acc[nt][e]);
           }
-          stage[dst * H + row] = __fmul_rn(wt, y);
         }
       }
     }
@@ -396,9 +399,7 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, cudaStream_t st,
 size_t decode_meta_ints(int G) { return 2 + 2 * (size_t)G; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev) {
-  auto mark = [&](int i) -> bool {
-    return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
-  };
+  auto mark = [&](int i) -> bool { return !ev || record_stage_event(ev[i], st); };
   const int G = a.E + a.S, R = a.T * a.k;
   if (!mark(0)) return cudaErrorUnknown;
   const size_t smem = sizeof(int32_t) * (2 * (size_t)G + R);
@@ -414,7 +415,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
                  a.k, a.S, a.act, a.h_dec);
   if (e != cudaSuccess) return e;
   if (!mark(4)) return cudaErrorUnknown;
-  e = launch_pdl(decode_w2_kernel, dim3(max_groups, (a.H + kDecRows - 1) / kDecRows),
+  e = launch_pdl(decode_w2_kernel, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
                  dim3(kDecThreads), st, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
                  (const int32_t*)a.meta, (const int32_t*)a.slots, (const float*)a.w,
                  a.T, a.H, a.I, a.E, a.k, a.S, a.stage);

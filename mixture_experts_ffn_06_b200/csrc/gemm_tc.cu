@@ -21,10 +21,12 @@
 //     and accumulators with tcgen05.commit;
 //   * warps 2-5 are the epilogue: tcgen05.ld of their 32 TMEM lanes, the
 //     gate activation fused in mode 0 (so g and u never reach HBM) with bf16
-//     h stores; in mode 2 each row is multiplied by its gate weight and
-//     stored at its (token, choice) position, so the combine that follows
-//     only sums k+S contiguous rows.  Two accumulators let the epilogue of
-//     tile i overlap the MMAs of tile i+1.
+//     h stores; in modes 2 and 3 each row is multiplied by its gate weight
+//     and either added into its token's fp32 output row (mode 2, vector
+//     reductions) or stored at its (token, choice) position for a fixed-order
+//     sum (mode 3).  Stores go through a shared-memory transpose so each
+//     warp instruction writes whole row segments.  Two accumulators let the
+//     epilogue of tile i overlap the MMAs of tile i+1.
 // Every wait is bounded (tc_ptx.cuh: mbar_wait); on a timeout the block
 // records MOE_ERR_TIMEOUT, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -52,6 +54,22 @@ struct Ctl {
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort_flag;
+};
+
+// Vector fp32 reduction into global memory (16-byte aligned destination).
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c,
+                                           float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// Epilogue scratch: one padded 32x33 fp32 tile per epilogue warp, and the
+// destination row / gate weight of each tile row (modes 2 and 3).
+struct EpiSmem {
+  float buf[4][32][33];
+  int64_t rdst[4][32];
+  float rw[4][32];
 };
 
 struct KParams {
@@ -114,7 +132,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * A_STAGE;
-  Ctl* ctl = reinterpret_cast<Ctl*>(gbase + STAGES * (A_STAGE + B_STAGE));
+  EpiSmem* epi = reinterpret_cast<EpiSmem*>(gbase + STAGES * (A_STAGE + B_STAGE));
+  Ctl* ctl = reinterpret_cast<Ctl*>(epi + 1);
   int32_t* offs = reinterpret_cast<int32_t*>(ctl + 1);
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
@@ -231,94 +250,111 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q+32)
+    // Each warp owns TMEM lanes [32q, 32q+32), i.e. 32 rows of the tile.
+    // Per 32-column chunk it loads its rows' accumulators (one row per
+    // lane), parks them in a padded 32x33 shared tile and writes them out
+    // transposed, so that every store (or reduction) instruction of the warp
+    // covers whole 64/128-byte row segments instead of 32 scattered rows.
+    const int q = warp & 3;
+    float(*tbuf)[33] = epi->buf[q];
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile tl = map_tile<MODE>(t, offs, p.G, p.NT);
+      if (MODE >= 2) {
+        // destination row and gate weight of this lane's tile row
+        const int64_t row = tl.row0 + q * 32 + lane;
+        const int32_t slot = p.sorted_slots[row];
+        const int64_t R = p.T * p.k;
+        int64_t dst = -1;
+        float wt = 1.0f;
+        if (slot >= 0) {
+          int64_t tok, j;
+          if (slot < R) {
+            tok = slot / p.k;
+            j = slot - tok * p.k;
+            wt = __ldg(p.w + slot);
+          } else {
+            const int64_t qq = slot - R, sh = qq / p.T;
+            tok = qq - sh * p.T;
+            j = p.k + sh;
+          }
+          dst = MODE == 2 ? tok : tok * (p.k + p.S) + j;
+        }
+        epi->rdst[q][lane] = dst;
+        epi->rw[q][lane] = wt;
+      }
       const bool got = mbar_wait(smem_u32(&ctl->tmem_full[acc]), acc_phase,
                                  abort_flag, p.timeout_ns, p.err);
       // warp-uniform decision; also reconverges the warp for tcgen05.ld
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
-      const int64_t row = tl.row0 + q * 32 + lane;
-      if (MODE == 0) {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + row * (int64_t)p.N;
+      const int64_t wrow0 = tl.row0 + q * 32;  // first tile row of this warp
+      constexpr int CHUNKS = MODE == 0 ? 4 : 8;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          const int col0 = tl.n0 + c * 32;
-          if (col0 >= p.N) break;
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int col0 = tl.n0 + c * 32;
+        if (col0 >= p.N) break;
+        if (MODE == 0) {
           uint32_t g[32], u[32];
           tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (col0 + v * 8 < p.N) {
-              uint4 o;
-              uint32_t* op = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int i0 = v * 8 + 2 * e;
-                const float h0 = act_apply(p.act, __uint_as_float(g[i0])) *
-                                 __uint_as_float(u[i0]);
-                const float h1 = act_apply(p.act, __uint_as_float(g[i0 + 1])) *
-                                 __uint_as_float(u[i0 + 1]);
-                op[e] = pack_bf16x2(h0, h1);
-              }
-              *reinterpret_cast<uint4*>(orow + col0 + v * 8) = o;
-            }
-          }
-        }
-      } else {
-        // mode 1: plain fp32 rows in permuted order; mode 2: the row times its
-        // gate weight, stored at its (token, choice) position (un-permute)
-        float* orow;
-        float wt = 1.0f;
-        bool live = true;
-        if (MODE == 1) {
-          orow = static_cast<float*>(p.out) + row * (int64_t)p.N;
+          for (int j = 0; j < 32; ++j)
+            tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) *
+                            __uint_as_float(u[j]);
         } else {
-          const int32_t slot = p.sorted_slots[row];
-          live = slot >= 0;
-          const int64_t R = p.T * p.k;
-          const int64_t ks = p.k + p.S;
-          int64_t dst = 0;
-          if (live) {
-            if (slot < R) {
-              const int64_t t = slot / p.k;
-              dst = t * ks + (slot - t * p.k);
-              wt = __ldg(p.w + slot);
-            } else {
-              const int64_t q = slot - R, sh = q / p.T;
-              dst = (q - sh * p.T) * ks + p.k + sh;
+          uint32_t y[32];
+          tmem_ld32(tb + c * 32, y);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tbuf[lane][j] = __uint_as_float(y[j]);
+        }
+        __syncwarp();
+        if (MODE == 0) {
+          // 8 rows x 64 bytes per instruction
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+          const int cc = (lane & 3) * 8;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = i * 8 + (lane >> 2);
+            if (col0 + cc < p.N) {
+              uint4 o;
+              o.x = pack_bf16x2(tbuf[r][cc + 0], tbuf[r][cc + 1]);
+              o.y = pack_bf16x2(tbuf[r][cc + 2], tbuf[r][cc + 3]);
+              o.z = pack_bf16x2(tbuf[r][cc + 4], tbuf[r][cc + 5]);
+              o.w = pack_bf16x2(tbuf[r][cc + 6], tbuf[r][cc + 7]);
+              *reinterpret_cast<uint4*>(out + (wrow0 + r) * (int64_t)p.N + col0 + cc) = o;
             }
           }
-          orow = static_cast<float*>(p.out) + dst * (int64_t)p.N;
-        }
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          const int col0 = tl.n0 + c * 32;
-          if (col0 >= p.N) break;
-          uint32_t y[32];
-          tmem_ld32(tb + c * 32, y);  // warp-collective: every lane loads
-          if (!live) continue;
+        } else {
+          // 4 rows x 128 bytes per instruction
+          float* out = static_cast<float*>(p.out);
+          const int cc = (lane & 7) * 4;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            if (col0 + v * 4 < p.N) {
-              float* dst = orow + col0 + v * 4;
-              const float a0 = __uint_as_float(y[v * 4 + 0]);
-              const float a1 = __uint_as_float(y[v * 4 + 1]);
-              const float a2 = __uint_as_float(y[v * 4 + 2]);
-              const float a3 = __uint_as_float(y[v * 4 + 3]);
+          for (int i = 0; i < 8; ++i) {
+            const int r = i * 4 + (lane >> 3);
+            if (col0 + cc < p.N) {
+              const float a0 = tbuf[r][cc + 0], a1 = tbuf[r][cc + 1];
+              const float a2 = tbuf[r][cc + 2], a3 = tbuf[r][cc + 3];
               if (MODE == 1) {
-                *reinterpret_cast<float4*>(dst) = make_float4(a0, a1, a2, a3);
+                *reinterpret_cast<float4*>(out + (wrow0 + r) * (int64_t)p.N + col0 + cc) =
+                    make_float4(a0, a1, a2, a3);
               } else {
-                *reinterpret_cast<float4*>(dst) =
-                    make_float4(__fmul_rn(wt, a0), __fmul_rn(wt, a1),
-                                __fmul_rn(wt, a2), __fmul_rn(wt, a3));
+                const int64_t dst = epi->rdst[q][r];
+                const float wt = epi->rw[q][r];
+                if (dst >= 0) {
+                  float* d = out + dst * (int64_t)p.N + col0 + cc;
+                  const float b0 = __fmul_rn(wt, a0), b1 = __fmul_rn(wt, a1);
+                  const float b2 = __fmul_rn(wt, a2), b3 = __fmul_rn(wt, a3);
+                  if (MODE == 2)
+                    red_add_v4(d, b0, b1, b2, b3);
+                  else
+                    *reinterpret_cast<float4*>(d) = make_float4(b0, b1, b2, b3);
+                }
               }
             }
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
@@ -424,7 +460,8 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
   p.k = a.k;
   p.S = a.G - a.E;
 
-  const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + sizeof(Ctl) +
+  const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) +
+                      sizeof(EpiSmem) + sizeof(Ctl) +
                       sizeof(int32_t) * (size_t)(a.G + 1);
   static bool attr_set = false;
   if (!attr_set) {
@@ -461,6 +498,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
     case 0: return launch_mode<0>(a, st);
     case 1: return launch_mode<1>(a, st);
     case 2: return launch_mode<2>(a, st);
+    case 3: return launch_mode<3>(a, st);
   }
   return cudaErrorInvalidValue;
 }

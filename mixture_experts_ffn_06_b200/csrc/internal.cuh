@@ -33,6 +33,7 @@ struct WsMap {
   size_t x_perm;       // [cap,H] bf16 gathered activations
   size_t h;            // [cap,I] bf16 gated intermediate
   size_t stage;        // [T,k+S,H] fp32 weighted expert rows (moe_forward)
+  size_t acc;          // [T,H] fp32 accumulator (moe_forward, fast combine)
   size_t dec_meta;     // decode path: touched-expert lists
   size_t total;
   int64_t cap;
@@ -44,6 +45,9 @@ WsMap workspace_map(const moe_shape& s);
 // Shape validation shared by every entry point (MOE_OK or the error status).
 moe_status validate_shape(const moe_shape* s);
 
+// cudaEventRecord of a caller's stage event; an event node under capture.
+bool record_stage_event(void* ev, cudaStream_t st);
+
 // ---- launch wrappers (return cudaGetLastError of the launch) ----
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
                          int E, int k, int32_t* ids, float* w, cudaStream_t st);
@@ -54,11 +58,16 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
                           cudaStream_t st);
 
-// Gathers x rows into x_perm (zeros on padding rows).
+// Gathers x rows into x_perm (zeros on padding rows); when acc is given it
+// also zeroes acc[0, n_acc) (n_acc % 4 == 0).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
-                          int H, int64_t cap, __nv_bfloat16* x_perm,
-                          cudaStream_t st);
+                          int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
+                          int64_t n_acc, cudaStream_t st);
+
+// out = bf16(acc) (round to nearest even), out_f32 = acc if given; n % 8 == 0.
+cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
+                            float* out_f32, cudaStream_t st);
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,
@@ -97,8 +106,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
 //   mode 0: h = Act(A W1^T) (*) (A W3^T), B = packed [G][2N][K] gate/up rows,
 //           bf16 out [cap, N];
 //   mode 1: y = A W^T, B = [G][N][K], fp32 out [cap, N] (unweighted rows);
-//   mode 2: as mode 1, but row r stores w_r * y_r (fp32) at row
-//           t*(k+S) + j of out, the (token, choice) order (un-permute).
+//   mode 2: as mode 1, but row r adds w_r * y_r into row t of the fp32
+//           accumulator out [T, N] (vector reductions: fast, the order of
+//           the additions is not fixed);
+//   mode 3: as mode 1, but row r stores w_r * y_r at row t*(k+S) + j of
+//           out [T*(k+S), N], the (token, choice) order (un-permute), for a
+//           fixed-order sum afterwards.
 struct GroupedGemmArgs {
   int mode;
   const __nv_bfloat16* A;       // [cap, K]
@@ -108,7 +121,7 @@ struct GroupedGemmArgs {
   int G, E;                     // groups, routed groups
   int N, K;                     // output columns, reduction length
   int64_t cap;                  // rows of A / out
-  void* out;                    // mode 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T*(k+S),N]
+  void* out;                    // 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T,N]; 3: fp32 [T*(k+S),N]
   int act;
   uint32_t* err;
   // mode 2 only

@@ -18,7 +18,8 @@
 //   layout_scatter every slot writes sorted_slots[row] and slot_row;
 //   layout_pad     padding rows and rows past the last segment get -1.
 // gather_rows then copies x[token] into x_perm[row] (zeros on padding) with
-// 16-byte vector loads, one warp per row.
+// 16-byte vector loads, one warp per row, and zeroes the fp32 accumulator of
+// the fast combine.
 #include "internal.cuh"
 
 namespace moe {
@@ -165,7 +166,8 @@ layout_pad(const int32_t* __restrict__ offsets, const int32_t* __restrict__ lt_b
 __global__ void __launch_bounds__(256)
 gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slots,
             const int32_t* __restrict__ offsets, int G, int64_t T, int k,
-            int H, uint4* __restrict__ x_perm) {
+            int H, uint4* __restrict__ x_perm, uint4* __restrict__ acc,
+            int64_t n_acc4) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t rows = offsets[G];
@@ -184,6 +186,12 @@ gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slot
     const uint4* src = x + t * chunks;
     for (int c = lane; c < chunks; c += 32) dst[c] = __ldg(src + c);
   }
+  // zero the fp32 accumulator the w2 epilogue adds into (fast combine)
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_acc4;
+       i += stride)
+    acc[i] = z;
 }
 
 }  // namespace
@@ -223,13 +231,14 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
-                          int H, int64_t cap, __nv_bfloat16* x_perm,
-                          cudaStream_t st) {
+                          int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
+                          int64_t n_acc, cudaStream_t st) {
   const int64_t want = (cap + 7) / 8;
   const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
   gather_rows<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(
       reinterpret_cast<const uint4*>(x), sorted_slots, offsets, G, T, k, H,
-      reinterpret_cast<uint4*>(x_perm));
+      reinterpret_cast<uint4*>(x_perm), reinterpret_cast<uint4*>(acc),
+      acc ? n_acc / 4 : 0);
   return cudaGetLastError();
 }
 

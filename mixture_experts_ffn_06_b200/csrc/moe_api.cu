@@ -36,6 +36,7 @@ WsMap workspace_map(const moe_shape& s) {
   m.x_perm = take(2ull * m.cap * s.H);
   m.h = take(2ull * m.cap * Imax);
   m.stage = take(4ull * T * (k + S) * s.H);
+  m.acc = take(4ull * T * s.H);
   m.dec_meta = take(sizeof(int32_t) * decode_meta_ints((int)G));
   m.total = o;
   return m;
@@ -60,6 +61,15 @@ static moe_status check_shape(const moe_shape* s) {
 
 moe_status validate_shape(const moe_shape* s) { return check_shape(s); }
 
+bool record_stage_event(void* ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return false;
+  const unsigned flags =
+      cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u;
+  return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), st, flags) ==
+         cudaSuccess;
+}
+
 static moe_status from_cuda(cudaError_t e) {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -76,23 +86,26 @@ static uint8_t* at(P* base, size_t off) {
   return reinterpret_cast<uint8_t*>(const_cast<void*>(static_cast<const void*>(base))) + off;
 }
 
-// Record stage event i (if the caller asked for stage events).
+// Record stage event i (if the caller asked for stage events).  Under stream
+// capture the record becomes an event node of the graph, so the caller can
+// time the stages of each replay.
 static bool mark(void* const* ev, int i, cudaStream_t st) {
   if (!ev) return true;
-  return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+  return record_stage_event(ev[i], st);
 }
 
-// gather -> w13 GEMM (+activation) -> w2 GEMM.  With stage == nullptr the w2
-// GEMM writes unweighted fp32 rows to y_perm in permuted order
-// (moe_expert_ffn); otherwise it stores w * y at the row's (token, choice)
-// position of stage [T, k+S, H] (moe_forward).
+// gather -> w13 GEMM (+activation) -> w2 GEMM.  The w2 GEMM writes
+//   combine 0: unweighted fp32 rows to y_perm in permuted order (moe_expert_ffn);
+//   combine 2: adds w * y into the fp32 accumulator y_perm = acc [T, H];
+//   combine 3: stores w * y at the row's (token, choice) position of
+//              y_perm = stage [T, k+S, H].
 static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
                                  const int32_t* offsets,
                                  const int32_t* sorted_slots,
                                  const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                  const __nv_bfloat16* w13_sh,
                                  const __nv_bfloat16* w2_sh, float* y_perm,
-                                 float* stage, const float* w, void* ws,
+                                 int combine, const float* w, void* ws,
                                  cudaStream_t st, void* const* ev = nullptr) {
   const WsMap m = workspace_map(s);
   const int G = s.E + s.n_shared;
@@ -101,7 +114,8 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
   if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
   cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
-                                x_perm, st);
+                                x_perm, combine == 2 ? y_perm : nullptr,
+                                s.T * (int64_t)s.H, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 3, st)) return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
@@ -121,13 +135,13 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   e = launch_grouped_gemm(a, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
-  a.mode = stage ? 2 : 1;
+  a.mode = combine == 0 ? 1 : combine;
   a.A = h;
   a.B = w2;
   a.B_sh = w2_sh;
   a.N = s.H;
   a.K = s.I;
-  a.out = stage ? static_cast<void*>(stage) : static_cast<void*>(y_perm);
+  a.out = y_perm;
   a.sorted_slots = sorted_slots;
   a.w = w;
   a.T = s.T;
@@ -198,7 +212,7 @@ moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
                         reinterpret_cast<const __nv_bfloat16*>(w2),
                         reinterpret_cast<const __nv_bfloat16*>(w13_sh),
                         reinterpret_cast<const __nv_bfloat16*>(w2_sh), y_perm,
-                        nullptr, nullptr, ws, stream);
+                        0, nullptr, ws, stream);
 }
 
 moe_status moe_combine(const moe_shape* shape, const float* y_perm,
@@ -284,18 +298,23 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                     reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt,
                     stream) != cudaSuccess)
     return MOE_ERR_CUDA;
+  const bool det = opts && opts->deterministic;
+  float* acc = reinterpret_cast<float*>(at(ws, m.acc));
   st = run_expert_ffn(s, reinterpret_cast<const __nv_bfloat16*>(x), offsets,
                       sorted_slots, reinterpret_cast<const __nv_bfloat16*>(w13),
                       reinterpret_cast<const __nv_bfloat16*>(w2),
                       reinterpret_cast<const __nv_bfloat16*>(w13_sh),
-                      reinterpret_cast<const __nv_bfloat16*>(w2_sh), nullptr,
-                      stage, w, ws, stream, ev);
+                      reinterpret_cast<const __nv_bfloat16*>(w2_sh),
+                      det ? stage : acc, det ? 3 : 2, w, ws, stream, ev);
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
-  if (launch_sum_rows(stage, s.T, s.k + s.n_shared, s.H,
-                      reinterpret_cast<__nv_bfloat16*>(out),
-                      opts ? opts->out_f32 : nullptr, stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  float* out_f32 = opts ? opts->out_f32 : nullptr;
+  const cudaError_t e =
+      det ? launch_sum_rows(stage, s.T, s.k + s.n_shared, s.H,
+                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream)
+          : launch_finalize(acc, s.T * (int64_t)s.H,
+                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
   return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -50,16 +50,20 @@ def _small(name, seed=0):
 
 
 PATHS = {"prefill": 1, "decode": 2}
+# (path, deterministic combine) variants of moe_forward_ex
+VARIANTS = {"prefill": (1, False), "prefill_det": (1, True), "decode": (2, False)}
 
 
-@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("variant", list(VARIANTS))
 @pytest.mark.parametrize("name", list(SMALL))
-def test_forward_small_every_element(api, name, path):
+def test_forward_small_every_element(api, name, variant):
     inp = _small(name)
     want, ids_ref, w_ref = oracle_forward(inp)
-    out, out32, ids, w = gpu_forward(api, to_device(inp), path=PATHS[path])
+    path, det = VARIANTS[variant]
+    out, out32, ids, w = gpu_forward(api, to_device(inp), path=path,
+                                     deterministic=det)
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out32, want, f"{name} ({path})")
+    assert_out_close(out32, want, f"{name} ({variant})")
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -181,17 +185,29 @@ def test_four_call_chain_against_oracle_rows(api, name):
     # the two paths use the same arithmetic: bit-identical outputs
     want, _, _ = oracle_forward(inp)
     assert_out_close(acc, want, name + " chain")
-    fused, out32, _, _ = gpu_forward(api, d, path=PATHS["prefill"])
+    fused, out32, _, _ = gpu_forward(api, d, path=PATHS["prefill"],
+                                     deterministic=True)
     assert_out_close(out32, want, name + " fused")
     assert torch.equal(out, fused)  # same GEMM kernels, same additions
+    fast, fast32, _, _ = gpu_forward(api, d, path=PATHS["prefill"])
+    assert_out_close(fast32, want, name + " fused, fp32 reductions")
 
 
-@pytest.mark.parametrize("path", list(PATHS))
-def test_repeat_calls_are_bit_identical(api, path):
+@pytest.mark.parametrize("variant", ["prefill_det", "decode"])
+def test_repeat_calls_are_bit_identical(api, variant):
     inp = to_device(_small("gemma_shapes_T130"))
-    a, a32, _, _ = gpu_forward(api, inp, path=PATHS[path])
-    b, b32, _, _ = gpu_forward(api, inp, path=PATHS[path])
+    path, det = VARIANTS[variant]
+    a, a32, _, _ = gpu_forward(api, inp, path=path, deterministic=det)
+    b, b32, _, _ = gpu_forward(api, inp, path=path, deterministic=det)
     assert torch.equal(a, b) and torch.equal(a32, b32)
+
+
+def test_fast_combine_repeats_within_fp32_rounding(api):
+    inp = to_device(_small("gemma_shapes_T130"))
+    _, a32, _, _ = gpu_forward(api, inp, path=PATHS["prefill"])
+    _, b32, _, _ = gpu_forward(api, inp, path=PATHS["prefill"])
+    # k + S <= 9 fp32 terms per element, added in any order
+    assert (a32 - b32).abs().max().item() <= 1e-5 * a32.abs().max().item()
 
 
 def test_device_wait_limit_reports_timeout(api):
@@ -249,12 +265,13 @@ def test_decode_sweep_every_element(api, name, path):
     assert_out_close(out32, want, name)
 
 
+@pytest.mark.parametrize("det", [False, True])
 @pytest.mark.parametrize("name", ["mixtral_prefill", "many_small_prefill",
                                   "skewed_shared_prefill"])
-def test_prefill_full_size(api, name):
+def test_prefill_full_size(api, name, det):
     inp = inputs.make_inputs(name, seed=0, device="cuda")
     shp = inp.shape
-    out, out32, ids, w = gpu_forward(api, inp)
+    out, out32, ids, w = gpu_forward(api, inp, deterministic=det)
     # routing of every token, bit-exact ids
     ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
     assert_routing_exact(ids, w, ids_ref, w_ref)
