@@ -395,14 +395,23 @@ def run_ours(args):
         touched = touched_experts(api, s, inp, ws)
         expert_bytes = 3.0 * shp.H * shp.I * 2
         layer_bytes = touched * expert_bytes
-        if decode:
+        # the w13 product does 2 FLOP per weight byte per token routed to the
+        # expert; below the ridge point (peak FLOP/s / peak B/s) it is bound
+        # by streaming the touched experts' weights from HBM
+        rows = shp.T * shp.k + shp.T * shp.n_shared
+        tokens_per_expert = rows / max(touched, 1)
+        ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+        hbm_bound = tokens_per_expert < ridge
+        if hbm_bound:
             achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
             peak = float(peaks["hbm_gbs"])
-            roof = {"bound": "hbm", "kernel": "decode_w13_kernel (w13 + act)",
+            roof = {"bound": "hbm",
+                    "kernel": "decode_w13_kernel (w13 + act)" if decode
+                    else "grouped_gemm_kernel<0> (w13 + activation)",
                     "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak,
                     "peak_source": f"{peak_src} hbm_gbs",
-                    "traffic": traffic_for("decode.cu"),
+                    "traffic": traffic_for("decode.cu" if decode else "gemm_tc.cu"),
                     "layer_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peak,
                     "touched_experts": touched}
         else:

@@ -67,9 +67,8 @@ combine_kernel(const float4* __restrict__ y_perm,
 __global__ void __launch_bounds__(256)
 sum_rows_kernel(const float4* __restrict__ stage, int64_t T, int ks, int H,
                 uint4* __restrict__ out, float4* __restrict__ out_f32) {
-  // when launched as a programmatic dependent, wait for the rows' producer
-  // (returns at once otherwise)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
+  pdl_trigger();
   const int c8 = H >> 3;
   const int64_t n = T * c8;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -113,6 +112,8 @@ sum_rows_kernel(const float4* __restrict__ stage, int64_t T, int ks, int H,
 __global__ void __launch_bounds__(256)
 finalize_kernel(const float4* __restrict__ acc, int64_t n8, uint4* __restrict__ out,
                 float4* __restrict__ out_f32) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
        i += stride) {
@@ -138,15 +139,14 @@ finalize_kernel(const float4* __restrict__ acc, int64_t n8, uint4* __restrict__ 
 }  // namespace
 
 cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
-                            float* out_f32, cudaStream_t st) {
+                            float* out_f32, cudaStream_t st, bool pdl) {
   const int64_t n8 = n / 8;
   if (n8 == 0) return cudaSuccess;
   const int64_t want = (n8 + 255) / 256;
   const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
-  finalize_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc), n8,
-                                          reinterpret_cast<uint4*>(out),
-                                          reinterpret_cast<float4*>(out_f32));
-  return cudaGetLastError();
+  return launch_ex(finalize_kernel, dim3(blocks), dim3(256), 0, st, pdl,
+                   reinterpret_cast<const float4*>(acc), n8,
+                   reinterpret_cast<uint4*>(out), reinterpret_cast<float4*>(out_f32));
 }
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
@@ -169,19 +169,9 @@ cudaError_t launch_sum_rows(const float* stage, int64_t T, int ks, int H,
   if (n == 0) return cudaSuccess;
   const int64_t want = (n + 255) / 256;
   const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(blocks);
-  cfg.blockDim = dim3(256);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, sum_rows_kernel,
-                            reinterpret_cast<const float4*>(stage), T, ks, H,
-                            reinterpret_cast<uint4*>(out),
-                            reinterpret_cast<float4*>(out_f32));
+  return launch_ex(sum_rows_kernel, dim3(blocks), dim3(256), 0, st, pdl,
+                   reinterpret_cast<const float4*>(stage), T, ks, H,
+                   reinterpret_cast<uint4*>(out), reinterpret_cast<float4*>(out_f32));
 }
 
 }  // namespace moe

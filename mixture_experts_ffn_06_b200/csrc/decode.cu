@@ -35,13 +35,6 @@ constexpr int kDecRows = 16;
 constexpr int kDecNT = 8;                    // token tiles of 8 per pass
 constexpr int kDecPass = kDecNT * 8;         // tokens per pass
 
-__device__ __forceinline__ void pdl_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_trigger() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -378,22 +371,6 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
   }
 }
 
-template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, cudaStream_t st,
-                       Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 }  // namespace
 
 size_t decode_meta_ints(int G) { return 2 + 2 * (size_t)G; }
@@ -409,14 +386,14 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   const int max_groups = (R < a.E ? R : a.E) + a.S;
-  e = launch_pdl(decode_w13_kernel, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
-                 dim3(kDecThreads), st, a.x, a.w13, a.w13_sh,
+  e = launch_ex(decode_w13_kernel, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
+                 dim3(kDecThreads), 0, st, true, a.x, a.w13, a.w13_sh,
                  (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
                  a.k, a.S, a.act, a.h_dec);
   if (e != cudaSuccess) return e;
   if (!mark(4)) return cudaErrorUnknown;
-  e = launch_pdl(decode_w2_kernel, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
-                 dim3(kDecThreads), st, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
+  e = launch_ex(decode_w2_kernel, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
+                 dim3(kDecThreads), 0, st, true, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
                  (const int32_t*)a.meta, (const int32_t*)a.slots, (const float*)a.w,
                  a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
   if (e != cudaSuccess) return e;

@@ -138,7 +138,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i <= p.G; i += THREADS) offs[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
@@ -156,6 +155,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     tma_prefetch_desc(&tmBs);
   }
   if (warp == 1) tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+  // everything above overlaps the previous kernel when launched with PDL;
+  // the expert offsets and the operands are its outputs
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i <= p.G; i += THREADS) offs[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -424,7 +428,7 @@ int num_sms() {
 }
 
 template <int MODE>
-cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
+cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
   CUtensorMap mA, mB, mBs;
   cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM);
@@ -474,8 +478,8 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st) {
   const int64_t max_tiles = (a.cap / BM) * p.NT;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  grouped_gemm_kernel<MODE><<<grid, THREADS, smem, st>>>(mA, mB, mBs, p);
-  return cudaGetLastError();
+  return launch_ex(grouped_gemm_kernel<MODE>, dim3(grid), dim3(THREADS), smem, st, pdl,
+                   mA, mB, mBs, p);
 }
 
 __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
@@ -493,12 +497,12 @@ __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
 
 }  // namespace
 
-cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   switch (a.mode) {
-    case 0: return launch_mode<0>(a, st);
-    case 1: return launch_mode<1>(a, st);
-    case 2: return launch_mode<2>(a, st);
-    case 3: return launch_mode<3>(a, st);
+    case 0: return launch_mode<0>(a, st, pdl);
+    case 1: return launch_mode<1>(a, st, pdl);
+    case 2: return launch_mode<2>(a, st, pdl);
+    case 3: return launch_mode<3>(a, st, pdl);
   }
   return cudaErrorInvalidValue;
 }

@@ -52,22 +52,25 @@ bool record_stage_event(void* ev, cudaStream_t st);
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
                          int E, int k, int32_t* ids, float* w, cudaStream_t st);
 
+// pdl on any launch function: launch its first kernel as a programmatic
+// dependent of the previous kernel on the stream (later kernels of the same
+// function always are).
 cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* offsets, int32_t* sorted_slots,
                           int32_t* slot_row, int64_t cap, int32_t* lt_count,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
-                          cudaStream_t st);
+                          cudaStream_t st, bool pdl = false);
 
 // Gathers x rows into x_perm (zeros on padding rows); when acc is given it
 // also zeroes acc[0, n_acc) (n_acc % 4 == 0).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
                           int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
-                          int64_t n_acc, cudaStream_t st);
+                          int64_t n_acc, cudaStream_t st, bool pdl = false);
 
 // out = bf16(acc) (round to nearest even), out_f32 = acc if given; n % 8 == 0.
 cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
-                            float* out_f32, cudaStream_t st);
+                            float* out_f32, cudaStream_t st, bool pdl = false);
 
 cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
                            const float* w, int64_t T, int k, int S, int H,
@@ -130,7 +133,8 @@ struct GroupedGemmArgs {
   int64_t T;
   int k;
 };
-cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st,
+                                bool pdl = false);
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
                                  cudaStream_t st);
@@ -150,6 +154,35 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
   if (err) atomicCAS(err, 0u, code);
+}
+
+// Programmatic dependent launch.  A kernel launched with the PDL attribute
+// may start while its predecessor on the stream is still running; it must
+// call pdl_wait() before touching anything the predecessor writes (the wait
+// returns at once when there is no such predecessor).  pdl_trigger() lets the
+// next kernel start launching.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// cudaLaunchKernelEx with the programmatic-serialisation attribute when pdl.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 #endif  // __CUDACC__

@@ -30,6 +30,8 @@ layout_count(const int32_t* __restrict__ ids, int64_t R, int E,
              int32_t* __restrict__ lt_count, int32_t* __restrict__ lt_rank) {
   extern __shared__ int32_t wc[];  // [32 warps][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int i = tid; i < 32 * E; i += blockDim.x) wc[i] = 0;
   __syncthreads();
 
@@ -62,6 +64,8 @@ layout_scan(const int32_t* __restrict__ lt_count, int64_t n_lt, int E, int S,
   __shared__ int32_t seg[kMaxExperts + kMaxShared + 1];
   __shared__ int32_t warp_sum[32];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int G = E + S;
   // per-expert running sum over layout blocks
   for (int e = tid; e < G; e += blockDim.x) {
@@ -114,6 +118,8 @@ layout_scatter(const int32_t* __restrict__ ids, int64_t T, int k, int E, int S,
                int32_t* __restrict__ slot_row) {
   const int64_t R = T * k, RS = T * S;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < R + RS;
        i += stride) {
     if (i < R) {
@@ -141,6 +147,8 @@ layout_pad(const int32_t* __restrict__ offsets, const int32_t* __restrict__ lt_b
            int64_t T, int P, int64_t cap, int32_t* __restrict__ sorted_slots) {
   const int G = E + S;
   const int g = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (g < G) {
     int64_t count;
     if (g < E) {
@@ -170,6 +178,8 @@ gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slot
             int64_t n_acc4) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   const int64_t rows = offsets[G];
   const int chunks = H >> 3;  // 8 bf16 per 16-byte chunk
   const int64_t R = T * k;
@@ -179,12 +189,24 @@ gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slot
     uint4* dst = x_perm + r * chunks;
     if (s < 0) {
       const uint4 z = make_uint4(0, 0, 0, 0);
-      for (int c = lane; c < chunks; c += 32) dst[c] = z;
+      for (int c = lane; c < chunks; c += 32) __stcs(dst + c, z);
       continue;
     }
     const int64_t t = (s < R) ? (int64_t)s / k : ((int64_t)s - R) % T;
     const uint4* src = x + t * chunks;
-    for (int c = lane; c < chunks; c += 32) dst[c] = __ldg(src + c);
+    // four 16-byte loads in flight per lane before the stores; the copies
+    // are written with the streaming hint so they do not push x (read k
+    // times) out of L2
+    int c = lane;
+    for (; c + 96 < chunks; c += 128) {
+      const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32);
+      const uint4 v2 = __ldg(src + c + 64), v3 = __ldg(src + c + 96);
+      __stcs(dst + c, v0);
+      __stcs(dst + c + 32, v1);
+      __stcs(dst + c + 64, v2);
+      __stcs(dst + c + 96, v3);
+    }
+    for (; c < chunks; c += 32) __stcs(dst + c, __ldg(src + c));
   }
   // zero the fp32 accumulator the w2 epilogue adds into (fast combine)
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -200,46 +222,56 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* offsets, int32_t* sorted_slots,
                           int32_t* slot_row, int64_t cap, int32_t* lt_count,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool pdl) {
   const int64_t R = s.T * s.k;
   const int E = s.E, S = s.n_shared, G = E + S;
   const int P = s.pad ? s.pad : kSegPad;
+  cudaError_t e;
+  bool chained = pdl;  // every launch after the first is a dependent
   if (R > 0) {
     const size_t smem = sizeof(int32_t) * 32 * (size_t)E;
     if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(
-          layout_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(layout_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
       if (e != cudaSuccess) return e;
     }
-    layout_count<<<(unsigned)n_lt, kLayoutTile, smem, st>>>(ids, R, E, lt_count,
-                                                           lt_rank);
+    e = launch_ex(layout_count, dim3((unsigned)n_lt), dim3(kLayoutTile), smem, st,
+                  chained, ids, R, E, lt_count, lt_rank);
+    if (e != cudaSuccess) return e;
+    chained = true;
   }
-  layout_scan<<<1, 1024, 0, st>>>(lt_count, R > 0 ? n_lt : 0, E, S, s.T, P,
-                                  lt_base, offsets);
+  e = launch_ex(layout_scan, dim3(1), dim3(1024), 0, st, chained,
+                (const int32_t*)lt_count, R > 0 ? n_lt : (int64_t)0, E, S, s.T, P,
+                lt_base, offsets);
+  if (e != cudaSuccess) return e;
   const int64_t work = R + s.T * S;
   if (work > 0) {
     const int64_t blocks = (work + 255) / 256;
-    layout_scatter<<<(unsigned)(blocks < 65535 * 16 ? blocks : 65535 * 16), 256,
-                     0, st>>>(ids, s.T, s.k, E, S, offsets, lt_base, lt_rank,
-                              sorted_slots, slot_row);
+    e = launch_ex(layout_scatter,
+                  dim3((unsigned)(blocks < 65535 * 16 ? blocks : 65535 * 16)),
+                  dim3(256), 0, st, true, ids, s.T, s.k, E, S,
+                  (const int32_t*)offsets, (const int32_t*)lt_base,
+                  (const int32_t*)lt_rank, sorted_slots, slot_row);
+    if (e != cudaSuccess) return e;
   }
-  layout_pad<<<(unsigned)(G + 148), 256, 0, st>>>(
-      offsets, lt_base, lt_count, R > 0 ? n_lt : 0, E, S, s.T, P, cap,
-      sorted_slots);
+  e = launch_ex(layout_pad, dim3((unsigned)(G + 148)), dim3(256), 0, st, true,
+                (const int32_t*)offsets, (const int32_t*)lt_base,
+                (const int32_t*)lt_count, R > 0 ? n_lt : (int64_t)0, E, S, s.T, P,
+                cap, sorted_slots);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
                           int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
-                          int64_t n_acc, cudaStream_t st) {
+                          int64_t n_acc, cudaStream_t st, bool pdl) {
   const int64_t want = (cap + 7) / 8;
   const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
-  gather_rows<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(
-      reinterpret_cast<const uint4*>(x), sorted_slots, offsets, G, T, k, H,
-      reinterpret_cast<uint4*>(x_perm), reinterpret_cast<uint4*>(acc),
-      acc ? n_acc / 4 : 0);
-  return cudaGetLastError();
+  return launch_ex(gather_rows, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st, pdl,
+                   reinterpret_cast<const uint4*>(x), sorted_slots, offsets, G, T, k,
+                   H, reinterpret_cast<uint4*>(x_perm), reinterpret_cast<uint4*>(acc),
+                   acc ? n_acc / 4 : (int64_t)0);
 }
 
 }  // namespace moe

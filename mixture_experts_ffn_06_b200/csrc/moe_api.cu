@@ -106,7 +106,8 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
                                  const __nv_bfloat16* w13_sh,
                                  const __nv_bfloat16* w2_sh, float* y_perm,
                                  int combine, const float* w, void* ws,
-                                 cudaStream_t st, void* const* ev = nullptr) {
+                                 cudaStream_t st, void* const* ev = nullptr,
+                                 bool pdl = false) {
   const WsMap m = workspace_map(s);
   const int G = s.E + s.n_shared;
   auto* x_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.x_perm));
@@ -115,7 +116,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
   cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
                                 x_perm, combine == 2 ? y_perm : nullptr,
-                                s.T * (int64_t)s.H, st);
+                                s.T * (int64_t)s.H, st, pdl);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 3, st)) return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
@@ -132,7 +133,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   a.out = h;
   a.act = s.act;
   a.err = err;
-  e = launch_grouped_gemm(a, st);
+  e = launch_grouped_gemm(a, st, true);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
   a.mode = combine == 0 ? 1 : combine;
@@ -296,7 +297,7 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                     reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
                     reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
                     reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt,
-                    stream) != cudaSuccess)
+                    stream, /*pdl=*/true) != cudaSuccess)
     return MOE_ERR_CUDA;
   const bool det = opts && opts->deterministic;
   float* acc = reinterpret_cast<float*>(at(ws, m.acc));
@@ -305,15 +306,17 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                       reinterpret_cast<const __nv_bfloat16*>(w2),
                       reinterpret_cast<const __nv_bfloat16*>(w13_sh),
                       reinterpret_cast<const __nv_bfloat16*>(w2_sh),
-                      det ? stage : acc, det ? 3 : 2, w, ws, stream, ev);
+                      det ? stage : acc, det ? 3 : 2, w, ws, stream, ev, true);
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
   float* out_f32 = opts ? opts->out_f32 : nullptr;
   const cudaError_t e =
       det ? launch_sum_rows(stage, s.T, s.k + s.n_shared, s.H,
-                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream)
+                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream,
+                            true)
           : launch_finalize(acc, s.T * (int64_t)s.H,
-                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream);
+                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream,
+                            true);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -13,6 +13,8 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
              float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();  // let the layout kernels start launching
   if (t >= T) return;
   int id;
   float wt;
