@@ -53,6 +53,8 @@ def parse():
                     default="auto", help="force the kernel path")
     ap.add_argument("--deterministic", action="store_true",
                     help="fixed-order combine on the prefill path")
+    ap.add_argument("--pairs", choices=("auto", "off", "on"), default="auto",
+                    help="prefill GEMMs on single CTAs or on CTA pairs")
     ap.add_argument("--no-graph", action="store_true",
                     help="time plain stream launches instead of one CUDA graph")
     ap.add_argument("--profile", action="store_true",
@@ -290,7 +292,8 @@ def run_ours(args):
     def step(events=None):
         api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                            inp.w13_sh, inp.w2_sh, out, ws, events=events,
-                           path=path, deterministic=args.deterministic)
+                           path=path, deterministic=args.deterministic,
+                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs])
 
     def barrier():
         if world > 1:

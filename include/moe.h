@@ -202,6 +202,8 @@ typedef struct {
   float* out_f32;
   int32_t path;           /* moe_path */
   int32_t deterministic;  /* prefill path: fixed-order combine (see above) */
+  int32_t cta_pairs;      /* prefill GEMMs: 0 auto, 1 one CTA per tile, 2 CTA
+                             pairs (2-SM MMA, M = 256); results are identical */
 } moe_forward_opts;
 
 MOE_API moe_status moe_forward_ex(

@@ -44,7 +44,8 @@ class moe_forward_opts(ctypes.Structure):
     _fields_ = [("stage_events", ctypes.c_void_p),
                 ("out_f32", ctypes.c_void_p),
                 ("path", ctypes.c_int32),
-                ("deterministic", ctypes.c_int32)]
+                ("deterministic", ctypes.c_int32),
+                ("cta_pairs", ctypes.c_int32)]
 
 
 class moe_shape(ctypes.Structure):
@@ -191,12 +192,14 @@ def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
 
 def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                    ids_out=None, w_out=None, events=None, out_f32=None,
-                   path=PATH_AUTO, deterministic=False, stream=None):
+                   path=PATH_AUTO, deterministic=False, cta_pairs=0,
+                   stream=None):
     """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
     created with enable_timing=True) recorded around the stages, ``out_f32``
     ([T,H] fp32) receiving the output before its bf16 rounding, and ``path``
     (PATH_AUTO, PATH_PREFILL or PATH_DECODE); ``deterministic`` selects the
-    fixed-order combine on the prefill path."""
+    fixed-order combine on the prefill path; ``cta_pairs`` picks the GEMM
+    form (0 auto, 1 single CTAs, 2 CTA pairs)."""
     arr = None
     if events is not None:
         if len(events) != NUM_STAGES + 1:
@@ -209,7 +212,7 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
             *[ctypes.c_void_p(e.cuda_event) for e in events])
     opts = moe_forward_opts(
         ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
-        _p(out_f32), path, int(bool(deterministic)))
+        _p(out_f32), path, int(bool(deterministic)), cta_pairs)
     _check(lib.moe_forward_ex(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
                               _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
                               _p(ids_out), _p(w_out), _p(ws), ws.numel(),

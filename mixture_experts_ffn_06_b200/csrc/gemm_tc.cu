@@ -39,16 +39,25 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int BN_ACC = 256;
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK * 2;       // 16 KiB
-constexpr int B_STAGE = BN_ACC * BK * 2;   // 32 KiB
+constexpr int A_STAGE = BM * BK * 2;  // 16 KiB
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN_ACC;
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+constexpr int kMaxStages = 6;
+
+// CG = CTAs per MMA: 1 (M=128 per CTA, B tile 256 rows per CTA, 4 stages) or
+// 2 (a CTA pair computes M=256: each CTA loads its own 128 A rows and half of
+// the 256 B rows, so a stage is 32 KiB instead of 48 KiB and 6 fit).
+template <int CG>
+struct Cfg {
+  static constexpr int B_ROWS = BN_ACC / CG;        // B rows loaded per CTA
+  static constexpr int B_STAGE = B_ROWS * BK * 2;
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+};
 
 struct Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -81,33 +90,38 @@ struct KParams {
   int act;
   uint32_t* err;
   uint64_t timeout_ns;
-  const int32_t* sorted_slots;  // mode 2
-  const float* w;               // mode 2
-  int64_t T;                    // mode 2
-  int k, S;                     // mode 2
+  const int32_t* sorted_slots;  // modes 2, 3
+  const float* w;               // modes 2, 3
+  int64_t T;                    // modes 2, 3
+  int k, S;                     // modes 2, 3
 };
 
+// A work unit is (group g, block of CG m-tiles, n-tile); units are ordered
+// group-major, then n-tile, then m-block, so the CTAs running at once share
+// B tiles through L2.  ub[g] = units of the groups before g.
 struct Tile {
   int g;
-  int64_t row0;
+  int64_t row0;  // first row of this CTA's m-tile
   int n0;
+  bool valid;    // this CTA's m-tile lies inside the group's segment
 };
 
-template <int MODE>
-__device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs, int G,
-                                         int NT) {
+template <int MODE, int CG>
+__device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs,
+                                         const int64_t* ub, int G, int NT,
+                                         uint32_t rank) {
   constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
-  int lo = 0, hi = G - 1;  // last g with (offs[g]/BM)*NT <= i
+  int lo = 0, hi = G - 1;  // last g with ub[g] <= i
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if ((int64_t)(offs[mid] / BM) * NT <= i) lo = mid; else hi = mid - 1;
+    if (ub[mid] <= i) lo = mid; else hi = mid - 1;
   }
-  const int64_t mt0 = offs[lo] / BM;
   const int64_t mtg = (offs[lo + 1] - offs[lo]) / BM;
-  const int64_t local = i - mt0 * NT;
-  const int64_t nt = local / mtg;
-  const int64_t mt = local - nt * mtg;
-  return Tile{lo, (mt0 + mt) * BM, (int)nt * BN_OUT};
+  const int64_t mbg = (mtg + CG - 1) / CG;
+  const int64_t local = i - ub[lo];
+  const int64_t nt = local / mbg;
+  const int64_t mt = (local - nt * mbg) * CG + rank;
+  return Tile{lo, offs[lo] + mt * BM, (int)nt * BN_OUT, mt < mtg};
 }
 
 __device__ __forceinline__ float act_apply(int act, float g) {
@@ -121,11 +135,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmBs, const KParams p) {
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int B_STAGE = C::B_STAGE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -134,10 +151,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t sB = base + STAGES * A_STAGE;
   EpiSmem* epi = reinterpret_cast<EpiSmem*>(gbase + STAGES * (A_STAGE + B_STAGE));
   Ctl* ctl = reinterpret_cast<Ctl*>(epi + 1);
-  int32_t* offs = reinterpret_cast<int32_t*>(ctl + 1);
+  int64_t* ub = reinterpret_cast<int64_t*>(ctl + 1);        // [G+1]
+  int32_t* offs = reinterpret_cast<int32_t*>(ub + p.G + 1);  // [G+1]
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int64_t unit0 = CG == 2 ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
+  const int64_t unit_step = CG == 2 ? (int64_t)nclusters_x() : (int64_t)gridDim.x;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
@@ -145,7 +167,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&ctl->tmem_full[a]), 1);
-      mbar_init(smem_u32(&ctl->tmem_empty[a]), 128);
+      mbar_init(smem_u32(&ctl->tmem_empty[a]), 4 * CG);  // one per epilogue warp
     }
     mbar_init(smem_u32(&ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -154,17 +176,47 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmBs);
   }
-  if (warp == 1) tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+  if (warp == 1) {
+    if (CG == 2)
+      tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    else
+      tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+  }
   // everything above overlaps the previous kernel when launched with PDL;
   // the expert offsets and the operands are its outputs
   pdl_wait();
   pdl_trigger();
   for (int i = threadIdx.x; i <= p.G; i += THREADS) offs[i] = p.offsets[i];
+  __syncthreads();
+  if (warp == 0) {
+    // units before each group: lane l sums a contiguous run of groups
+    const int per = (p.G + 31) / 32;
+    const int g0 = lane * per, g1 = min(g0 + per, p.G);
+    int64_t run = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int64_t mtg = (offs[g + 1] - offs[g]) / BM;
+      run += (mtg + CG - 1) / CG * p.NT;
+    }
+    int64_t incl = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += n;
+    }
+    int64_t acc = incl - run;
+    for (int g = g0; g < g1; ++g) {
+      ub[g] = acc;
+      const int64_t mtg = (offs[g + 1] - offs[g]) / BM;
+      acc += (mtg + CG - 1) / CG * p.NT;
+    }
+    if (lane == 31) ub[p.G] = incl;
+  }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const int64_t total = (int64_t)(offs[p.G] / BM) * p.NT;
+  const int64_t total = ub[p.G];
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -173,12 +225,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       int32_t last_fill[STAGES];
       for (int s = 0; s < STAGES; ++s) last_fill[s] = -1;
       bool ok = true;
-      for (int64_t t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tl = map_tile<MODE>(t, offs, p.G, p.NT);
+      for (int64_t t = unit0; ok && t < total; t += unit_step) {
+        const Tile tl = map_tile<MODE, CG>(t, offs, ub, p.G, p.NT, rank);
         const bool routed = tl.g < p.E;
         const CUtensorMap* mb = routed ? &tmB : &tmBs;
         const int32_t gl = routed ? tl.g : tl.g - p.E;
-        const int32_t brow = gl * p.b_rows_per_group + tl.n0;
+        // B rows this CTA loads: mode 0 -- gate rows then up rows (CG = 1),
+        // or CTA 0 the gate rows and CTA 1 the up rows (CG = 2); otherwise
+        // 256 rows, or CTA r rows [128r, 128r + 128)
+        const int32_t brow = gl * p.b_rows_per_group + tl.n0 +
+                             (int32_t)rank * (MODE == 0 ? p.up_off : C::B_ROWS);
         for (int kb = 0; kb < p.KB; ++kb) {
           const uint32_t fb = smem_u32(&ctl->full[stage]);
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
@@ -186,20 +242,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             ok = false;
             break;
           }
-          mbar_expect_tx(fb, A_STAGE + B_STAGE);
-          tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0, fb);
-          if (MODE == 0) {
-            tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
-            tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * BK,
-                        brow + p.up_off, fb);
+          if (CG == 1) {
+            mbar_expect_tx(fb, A_STAGE + B_STAGE);
+            tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0, fb);
+            if (MODE == 0) {
+              tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+              tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * BK,
+                          brow + p.up_off, fb);
+            } else {
+              tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+            }
           } else {
-            tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+            // both CTAs' bytes complete on CTA 0's full barrier
+            if (rank == 0) mbar_expect_tx(fb, 2 * (A_STAGE + B_STAGE));
+            const uint32_t fb0 = fb & kPeerBitMask;
+            tma_load_2d_pair(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0,
+                             fb0);
+            tma_load_2d_pair(sB + stage * B_STAGE, mb, kb * BK, brow, fb0);
           }
           last_fill[stage] = (int32_t)phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok && (CG == 1 || rank == 0)) {
         // let the copies already issued land before the block exits
         int32_t none = 0;
         volatile int32_t* never = &none;
@@ -211,13 +276,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN_ACC);
+    // (CTA 0 of the pair issues for both when CG = 2)
+    if (lane == 0 && (CG == 1 || rank == 0)) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN_ACC);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        if (!mbar_wait(smem_u32(&ctl->tmem_empty[acc]), acc_phase ^ 1u, abort_flag,
-                       p.timeout_ns, p.err)) {
+      for (int64_t t = unit0; ok && t < total; t += unit_step) {
+        const uint32_t eb = smem_u32(&ctl->tmem_empty[acc]);
+        const bool got = CG == 2
+            ? mbar_wait_cluster(eb, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.err)
+            : mbar_wait(eb, acc_phase ^ 1u, abort_flag, p.timeout_ns, p.err);
+        if (!got) {
           ok = false;
           break;
         }
@@ -233,14 +302,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint64_t ad = sw128_kmajor_desc(sA + stage * A_STAGE);
           const uint64_t bd = sw128_kmajor_desc(sB + stage * B_STAGE);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d, ad + 2u * kk, bd + 2u * kk, idesc,
-                      (kb | kk) != 0 ? 1u : 0u);
-          umma_commit(smem_u32(&ctl->empty[stage]));
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if (CG == 2)
+              umma_bf16_pair(d, ad + 2u * kk, bd + 2u * kk, idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d, ad + 2u * kk, bd + 2u * kk, idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+          if (CG == 2)
+            umma_commit_pair_mc(smem_u32(&ctl->empty[stage]), 0x3);
+          else
+            umma_commit(smem_u32(&ctl->empty[stage]));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(smem_u32(&ctl->tmem_full[acc]));
+        if (CG == 2)
+          umma_commit_pair_mc(smem_u32(&ctl->tmem_full[acc]), 0x3);
+        else
+          umma_commit(smem_u32(&ctl->tmem_full[acc]));
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -248,41 +328,48 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         // wait for the MMAs already issued before TMEM is released
         int32_t none = 0;
         volatile int32_t* never = &none;
-        umma_commit(smem_u32(&ctl->drain));
+        if (CG == 2)
+          umma_commit_pair(smem_u32(&ctl->drain));
+        else
+          umma_commit(smem_u32(&ctl->drain));
         mbar_wait(smem_u32(&ctl->drain), 0, never, p.timeout_ns, p.err);
       }
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    // Each warp owns TMEM lanes [32q, 32q+32), i.e. 32 rows of the tile.
-    // Per 32-column chunk it loads its rows' accumulators (one row per
-    // lane), parks them in a padded 32x33 shared tile and writes them out
+    // Each warp owns TMEM lanes [32q, 32q+32), i.e. 32 rows of this CTA's
+    // m-tile.  Per 32-column chunk it loads its rows' accumulators (one row
+    // per lane), parks them in a padded 32x33 shared tile and writes them out
     // transposed, so that every store (or reduction) instruction of the warp
     // covers whole 64/128-byte row segments instead of 32 scattered rows.
     const int q = warp & 3;
     float(*tbuf)[33] = epi->buf[q];
+    const uint32_t empty0 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[0]), 0) : 0u;
+    const uint32_t empty1 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[1]), 0) : 0u;
     uint32_t acc = 0, acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = map_tile<MODE>(t, offs, p.G, p.NT);
+    for (int64_t t = unit0; t < total; t += unit_step) {
+      const Tile tl = map_tile<MODE, CG>(t, offs, ub, p.G, p.NT, rank);
       if (MODE >= 2) {
         // destination row and gate weight of this lane's tile row
-        const int64_t row = tl.row0 + q * 32 + lane;
-        const int32_t slot = p.sorted_slots[row];
-        const int64_t R = p.T * p.k;
         int64_t dst = -1;
         float wt = 1.0f;
-        if (slot >= 0) {
-          int64_t tok, j;
-          if (slot < R) {
-            tok = slot / p.k;
-            j = slot - tok * p.k;
-            wt = __ldg(p.w + slot);
-          } else {
-            const int64_t qq = slot - R, sh = qq / p.T;
-            tok = qq - sh * p.T;
-            j = p.k + sh;
+        if (tl.valid) {
+          const int64_t row = tl.row0 + q * 32 + lane;
+          const int32_t slot = p.sorted_slots[row];
+          const int64_t R = p.T * p.k;
+          if (slot >= 0) {
+            int64_t tok, j;
+            if (slot < R) {
+              tok = slot / p.k;
+              j = slot - tok * p.k;
+              wt = __ldg(p.w + slot);
+            } else {
+              const int64_t qq = slot - R, sh = qq / p.T;
+              tok = qq - sh * p.T;
+              j = p.k + sh;
+            }
+            dst = MODE == 2 ? tok : tok * (p.k + p.S) + j;
           }
-          dst = MODE == 2 ? tok : tok * (p.k + p.S) + j;
         }
         epi->rdst[q][lane] = dst;
         epi->rw[q][lane] = wt;
@@ -302,6 +389,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (MODE == 0) {
           uint32_t g[32], u[32];
           tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
+          if (!tl.valid) continue;  // the pair's empty half: nothing to store
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) *
@@ -309,6 +397,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         } else {
           uint32_t y[32];
           tmem_ld32(tb + c * 32, y);
+          if (!tl.valid) continue;
 #pragma unroll
           for (int j = 0; j < 32; ++j) tbuf[lane][j] = __uint_as_float(y[j]);
         }
@@ -360,8 +449,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         __syncwarp();
       }
+      // this warp is done with the accumulator: one arrival per warp (on
+      // CTA 0's barrier when the pair shares the MMA)
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(acc ? empty1 : empty0);
+        else
+          mbar_arrive(smem_u32(&ctl->tmem_empty[acc]));
+      }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -369,10 +466,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // no peer still uses this CTA's barriers or TMEM
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -427,14 +528,17 @@ int num_sms() {
   return n;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
+  using C = Cfg<CG>;
   constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
   CUtensorMap mA, mB, mBs;
   cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM);
   if (e != cudaSuccess) return e;
   const uint64_t rows_per_group = MODE == 0 ? 2ull * a.N : (uint64_t)a.N;
-  const uint32_t box_rows = MODE == 0 ? BN_ACC / 2 : BN_ACC;
+  // per-CTA B box: mode 0 loads 128 gate (and 128 up) rows; the others 256
+  // rows, or 128 per CTA of a pair
+  const uint32_t box_rows = MODE == 0 ? BN_ACC / 2 : (uint32_t)C::B_ROWS;
   e = make_map(&mB, a.B, (uint64_t)a.K, rows_per_group * (uint64_t)a.E, box_rows);
   if (e != cudaSuccess) return e;
   if (a.B_sh && a.G > a.E) {
@@ -464,22 +568,43 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   p.k = a.k;
   p.S = a.G - a.E;
 
-  const size_t smem = 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) +
+  const size_t smem = 1024 + (size_t)C::STAGES * (A_STAGE + C::B_STAGE) +
                       sizeof(EpiSmem) + sizeof(Ctl) +
-                      sizeof(int32_t) * (size_t)(a.G + 1);
+                      (sizeof(int64_t) + sizeof(int32_t)) * (size_t)(a.G + 1);
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int64_t max_tiles = (a.cap / BM) * p.NT;
-  int grid = num_sms();
-  if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  return launch_ex(grouped_gemm_kernel<MODE>, dim3(grid), dim3(THREADS), smem, st, pdl,
-                   mA, mB, mBs, p);
+  // units: at most (cap / BM) m-tiles, grouped CG at a time, per n-tile
+  const int64_t max_units = ((a.cap / BM) / CG + a.G) * p.NT;
+  int64_t groups = num_sms() / CG;  // CTAs (or CTA pairs) resident at once
+  if (max_units < groups) groups = max_units > 0 ? max_units : 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(groups * CG));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (CG == 2) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG>, mA, mB, mBs, p);
 }
 
 __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
@@ -498,11 +623,14 @@ __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
+  // CTA pairs when the experts' segments are large enough that most m-blocks
+  // hold two full m-tiles; single CTAs for few rows per expert (decode-sized)
+  const bool pair = a.pair;
   switch (a.mode) {
-    case 0: return launch_mode<0>(a, st, pdl);
-    case 1: return launch_mode<1>(a, st, pdl);
-    case 2: return launch_mode<2>(a, st, pdl);
-    case 3: return launch_mode<3>(a, st, pdl);
+    case 0: return pair ? launch_mode<0, 2>(a, st, pdl) : launch_mode<0, 1>(a, st, pdl);
+    case 1: return pair ? launch_mode<1, 2>(a, st, pdl) : launch_mode<1, 1>(a, st, pdl);
+    case 2: return pair ? launch_mode<2, 2>(a, st, pdl) : launch_mode<2, 1>(a, st, pdl);
+    case 3: return pair ? launch_mode<3, 2>(a, st, pdl) : launch_mode<3, 1>(a, st, pdl);
   }
   return cudaErrorInvalidValue;
 }

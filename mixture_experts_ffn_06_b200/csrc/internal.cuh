@@ -132,6 +132,7 @@ struct GroupedGemmArgs {
   const float* w;               // [T,k]
   int64_t T;
   int k;
+  bool pair;                    // run on CTA pairs (2-SM MMA, M = 256)
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st,
                                 bool pdl = false);

@@ -107,7 +107,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
                                  const __nv_bfloat16* w2_sh, float* y_perm,
                                  int combine, const float* w, void* ws,
                                  cudaStream_t st, void* const* ev = nullptr,
-                                 bool pdl = false) {
+                                 bool pdl = false, int cta_pairs = 0) {
   const WsMap m = workspace_map(s);
   const int G = s.E + s.n_shared;
   auto* x_perm = reinterpret_cast<__nv_bfloat16*>(at(ws, m.x_perm));
@@ -133,10 +133,17 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   a.out = h;
   a.act = s.act;
   a.err = err;
+  // CTA pairs (2-SM MMA) when asked; by default only for the w2 GEMM with
+  // a long reduction (I >= 1024) once an expert averages two or more full
+  // 128-row m-tiles -- measured on B200, pairs help w2 there and cost the
+  // w13 GEMM and short reductions a few percent
+  const bool big = s.T * (int64_t)s.k >= 2 * 128 * (int64_t)s.E;
+  a.pair = cta_pairs == 2;
   e = launch_grouped_gemm(a, st, true);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(ev, 4, st)) return MOE_ERR_CUDA;
   a.mode = combine == 0 ? 1 : combine;
+  a.pair = cta_pairs == 2 || (cta_pairs == 0 && big && s.I >= 1024);
   a.A = h;
   a.B = w2;
   a.B_sh = w2_sh;
@@ -259,6 +266,7 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
   auto* slot_row = reinterpret_cast<int32_t*>(at(ws, m.slot_row));
   auto* stage = reinterpret_cast<float*>(at(ws, m.stage));
   const int path = opts ? opts->path : MOE_PATH_AUTO;
+  if (opts && (opts->cta_pairs < 0 || opts->cta_pairs > 2)) return MOE_ERR_INVALID_ARG;
   if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE)
     return MOE_ERR_INVALID_ARG;
   if (path == MOE_PATH_DECODE && s.T > kDecodeForcedMaxT) return MOE_ERR_UNSUPPORTED;
@@ -306,7 +314,8 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                       reinterpret_cast<const __nv_bfloat16*>(w2),
                       reinterpret_cast<const __nv_bfloat16*>(w13_sh),
                       reinterpret_cast<const __nv_bfloat16*>(w2_sh),
-                      det ? stage : acc, det ? 3 : 2, w, ws, stream, ev, true);
+                      det ? stage : acc, det ? 3 : 2, w, ws, stream, ev, true,
+                      opts ? opts->cta_pairs : 0);
   if (st != MOE_OK) return st;
   if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
   float* out_f32 = opts ? opts->out_f32 : nullptr;

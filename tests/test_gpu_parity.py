@@ -41,6 +41,12 @@ SMALL = {
     "gemma_shapes_T130": (inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),
                           "zero", "uniform"),
     "wide_tiles": (inputs.Shape(T=300, H=520, E=3, k=2, I=392), "normal0.5", "uniform"),
+    # T*k >= 256*E: the grouped GEMMs run on CTA pairs (M = 256), with odd
+    # m-tile counts per expert, K and N tails, and shared experts
+    "pairs_ragged": (inputs.Shape(T=700, H=200, E=3, k=2, I=104, act=1),
+                     "normal0.5", "uniform"),
+    "pairs_shared": (inputs.Shape(T=600, H=128, E=4, k=2, I=96, n_shared=1,
+                                  I_shared=96), "zero", "ones"),
 }
 
 
@@ -119,7 +125,8 @@ def test_permute_large_random_ids(api):
         assert (g == w_).all(), what
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "tail704"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "tail704",
+                                  "pairs_ragged", "pairs_shared"])
 def test_four_call_chain_against_oracle_rows(api, name):
     """moe_route -> moe_permute -> moe_expert_ffn -> moe_combine."""
     inp = _small(name)
@@ -167,19 +174,19 @@ def test_four_call_chain_against_oracle_rows(api, name):
     pad = np.nonzero(slots < 0)[0]
     assert (y[pad] == 0).all()  # padding rows hold zeros
 
-    # combine: fixed-order fp32 sum of the rows it was given, rounded once
+    # combine: the fixed-order fp32 sum of the rows it was given (each
+    # product rounded to fp32, then added, j = 0..k-1, then the shared
+    # experts), rounded once -- redone here op by op, so bit for bit
     sr = slot_row.long().cpu()
     yt = y_perm.cpu()
     acc = torch.zeros(T, H, dtype=torch.float32)
     wt = w.cpu()
     for j in range(k):
-        acc = torch.addcmul(acc, wt[:, j:j + 1], yt[sr[:, j]])
+        prod = wt[:, j:j + 1] * yt[sr[:, j]]
+        acc = acc + prod
     for sh in range(S):
         acc = acc + yt[sr[:, k + sh]]
-    ref = acc.to(torch.bfloat16).float()
-    diff = (out.cpu().float() - ref).abs()
-    ulp = ref.abs().clamp_min(1e-30) * 2.0 ** -7
-    assert (diff <= ulp).all()  # within one bf16 ulp (fma vs mul+add)
+    assert torch.equal(out.cpu(), acc.to(torch.bfloat16))
 
     # the chain's fp32 sum and the fused call both meet the output bound, and
     # the two paths use the same arithmetic: bit-identical outputs
