@@ -160,9 +160,10 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def traffic_for(kernel_src: str):
-    """DRAM bytes per launch from the committed ncu summary, only while the
-    kernel source still matches the one the counters were taken on."""
+def traffic_for(kernel_src: str, config: str, shape_override):
+    """DRAM bytes per launch from the committed ncu summary, only for the
+    workload it was captured on and while the kernel source still matches
+    the one the counters were taken on."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -176,6 +177,8 @@ def traffic_for(kernel_src: str):
         return None
     ent = d.get(kernel_src)
     if not ent or ent.get("source_sha256_16") != sha:
+        return None
+    if shape_override or ent.get("config") != config:
         return None
     return ent.get("bytes_per_launch")
 
@@ -414,7 +417,8 @@ def run_ours(args):
                     "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak,
                     "peak_source": f"{peak_src} hbm_gbs",
-                    "traffic": traffic_for("decode.cu" if decode else "gemm_tc.cu"),
+                    "traffic": traffic_for("decode.cu" if decode else "gemm_tc.cu",
+                                           args.config, args.shape),
                     "layer_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peak,
                     "touched_experts": touched}
         else:
@@ -424,7 +428,7 @@ def run_ours(args):
                     "(w13 + activation)", "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
                     "peak_source": f"{peak_src} bf16_tflops (burst)",
-                    "traffic": traffic_for("gemm_tc.cu"),
+                    "traffic": traffic_for("gemm_tc.cu", args.config, args.shape),
                     "layer_frac": shp.flops() / (ms_per_step / 1e3) / 1e12 / peak}
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
         # our kernels per step: prefill route, layout x4, gather, 2 GEMMs,

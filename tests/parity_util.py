@@ -20,7 +20,7 @@ def to_device(inp: inputs.MoEInputs, device="cuda") -> inputs.MoEInputs:
 
 
 def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
-                deterministic=False):
+                deterministic=False, cta_pairs=0):
     """moe_forward_ex through the C ABI -> (out bf16, out_f32, ids, w).
     Checks that the bf16 output is exactly the round-to-nearest-even of the
     fp32 layer output."""
@@ -34,7 +34,8 @@ def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
     ws = api.alloc_workspace(s, dev)
     api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                        inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w,
-                       out_f32=out_f32, path=path, deterministic=deterministic)
+                       out_f32=out_f32, path=path, deterministic=deterministic,
+                       cta_pairs=cta_pairs)
     torch.cuda.synchronize()
     assert api.moe_read_error(ws) == 0
     assert torch.equal(out, out_f32.to(torch.bfloat16)), "bf16 rounding step"

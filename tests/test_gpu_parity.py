@@ -47,6 +47,10 @@ SMALL = {
                      "normal0.5", "uniform"),
     "pairs_shared": (inputs.Shape(T=600, H=128, E=4, k=2, I=96, n_shared=1,
                                   I_shared=96), "zero", "ones"),
+    # I >= 1024 and two m-tiles per expert: the w2 GEMM picks CTA pairs by
+    # itself (also in moe_expert_ffn)
+    "pairs_wide_I": (inputs.Shape(T=600, H=128, E=2, k=2, I=1024), "zero",
+                     "uniform"),
 }
 
 
@@ -56,8 +60,10 @@ def _small(name, seed=0):
 
 
 PATHS = {"prefill": 1, "decode": 2}
-# (path, deterministic combine) variants of moe_forward_ex
-VARIANTS = {"prefill": (1, False), "prefill_det": (1, True), "decode": (2, False)}
+# (path, deterministic combine, cta_pairs) variants of moe_forward_ex
+VARIANTS = {"prefill": (1, False, 0), "prefill_det": (1, True, 0),
+            "prefill_pairs": (1, False, 2), "prefill_pairs_det": (1, True, 2),
+            "decode": (2, False, 0)}
 
 
 @pytest.mark.parametrize("variant", list(VARIANTS))
@@ -65,9 +71,9 @@ VARIANTS = {"prefill": (1, False), "prefill_det": (1, True), "decode": (2, False
 def test_forward_small_every_element(api, name, variant):
     inp = _small(name)
     want, ids_ref, w_ref = oracle_forward(inp)
-    path, det = VARIANTS[variant]
+    path, det, pairs = VARIANTS[variant]
     out, out32, ids, w = gpu_forward(api, to_device(inp), path=path,
-                                     deterministic=det)
+                                     deterministic=det, cta_pairs=pairs)
     assert_routing_exact(ids, w, ids_ref, w_ref)
     assert_out_close(out32, want, f"{name} ({variant})")
 
@@ -126,7 +132,7 @@ def test_permute_large_random_ids(api):
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "shared", "tail704",
-                                  "pairs_ragged", "pairs_shared"])
+                                  "pairs_ragged", "pairs_shared", "pairs_wide_I"])
 def test_four_call_chain_against_oracle_rows(api, name):
     """moe_route -> moe_permute -> moe_expert_ffn -> moe_combine."""
     inp = _small(name)
@@ -200,12 +206,14 @@ def test_four_call_chain_against_oracle_rows(api, name):
     assert_out_close(fast32, want, name + " fused, fp32 reductions")
 
 
-@pytest.mark.parametrize("variant", ["prefill_det", "decode"])
+@pytest.mark.parametrize("variant", ["prefill_det", "prefill_pairs_det", "decode"])
 def test_repeat_calls_are_bit_identical(api, variant):
     inp = to_device(_small("gemma_shapes_T130"))
-    path, det = VARIANTS[variant]
-    a, a32, _, _ = gpu_forward(api, inp, path=path, deterministic=det)
-    b, b32, _, _ = gpu_forward(api, inp, path=path, deterministic=det)
+    path, det, pairs = VARIANTS[variant]
+    a, a32, _, _ = gpu_forward(api, inp, path=path, deterministic=det,
+                               cta_pairs=pairs)
+    b, b32, _, _ = gpu_forward(api, inp, path=path, deterministic=det,
+                               cta_pairs=pairs)
     assert torch.equal(a, b) and torch.equal(a32, b32)
 
 
@@ -272,13 +280,14 @@ def test_decode_sweep_every_element(api, name, path):
     assert_out_close(out32, want, name)
 
 
-@pytest.mark.parametrize("det", [False, True])
+@pytest.mark.parametrize("det,pairs", [(False, 0), (True, 0), (False, 2)])
 @pytest.mark.parametrize("name", ["mixtral_prefill", "many_small_prefill",
                                   "skewed_shared_prefill"])
-def test_prefill_full_size(api, name, det):
+def test_prefill_full_size(api, name, det, pairs):
     inp = inputs.make_inputs(name, seed=0, device="cuda")
     shp = inp.shape
-    out, out32, ids, w = gpu_forward(api, inp, deterministic=det)
+    out, out32, ids, w = gpu_forward(api, inp, deterministic=det,
+                                     cta_pairs=pairs)
     # routing of every token, bit-exact ids
     ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
     assert_routing_exact(ids, w, ids_ref, w_ref)
