@@ -196,7 +196,7 @@ typedef enum {
   MOE_PATH_PREFILL = 1,  /* tcgen05 grouped GEMMs over padded expert segments */
   MOE_PATH_DECODE = 2    /* touched experts streamed by skinny kernels; T <= 1024 */
 } moe_path;
-#define MOE_DECODE_MAX_T 64
+#define MOE_DECODE_MAX_T 8
 typedef struct {
   void* const* stage_events;
   float* out_f32;

@@ -37,7 +37,7 @@ class MoEError(RuntimeError):
 
 
 PATH_AUTO, PATH_PREFILL, PATH_DECODE = 0, 1, 2
-DECODE_MAX_T = 64
+DECODE_MAX_T = 8
 
 
 class moe_forward_opts(ctypes.Structure):

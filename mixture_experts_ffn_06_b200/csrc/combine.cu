@@ -156,10 +156,10 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
   const int64_t blocks = T < 148 * 64 ? T : 148 * 64;
   const int chunks = H / 4;
   const int threads = chunks >= 256 ? 256 : ((chunks + 31) / 32) * 32;
-  combine_kernel<<<(unsigned)blocks, threads < 64 ? 64 : threads, 0, st>>>(
-      reinterpret_cast<const float4*>(y_perm), slot_row, w, T, k, S, H,
-      reinterpret_cast<uint2*>(out));
-  return cudaGetLastError();
+  return launch_ex(combine_kernel, dim3((unsigned)blocks),
+                   dim3(threads < 64 ? 64 : threads), 0, st, false,
+                   reinterpret_cast<const float4*>(y_perm), slot_row, w, T, k, S, H,
+                   reinterpret_cast<uint2*>(out));
 }
 
 cudaError_t launch_sum_rows(const float* stage, int64_t T, int ks, int H,

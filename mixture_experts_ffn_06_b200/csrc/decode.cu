@@ -32,8 +32,7 @@ namespace {
 
 constexpr int kDecThreads = 128;
 constexpr int kDecRows = 16;
-constexpr int kDecNT = 8;                    // token tiles of 8 per pass
-constexpr int kDecPass = kDecNT * 8;         // tokens per pass
+constexpr int kDecNT = 8;  // token tiles of 8 per pass (64 tokens) for T > 8
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -41,6 +40,12 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// Asks L2 to fetch [p, p + bytes) (16-byte aligned, multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -168,16 +173,24 @@ __device__ __forceinline__ bool load_group(const int32_t* meta, int G, int idx,
   return true;
 }
 
-__global__ void __launch_bounds__(kDecThreads, 4)
+// NTMAX: token tiles kept in registers per pass (8 -> up to 64 tokens of an
+// expert at once; 1 -> up to 8, which frees registers for a deeper weight
+// prefetch: two 32-column chunks ahead instead of one, and lets the token
+// rows sit in shared memory).
+template <int NTMAX>
+__global__ void __launch_bounds__(kDecThreads, NTMAX == 1 ? 3 : 4)
 decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
                   const __nv_bfloat16* __restrict__ w13,
                   const __nv_bfloat16* __restrict__ w13_sh,
                   const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
                   int T, int H, int I, int E, int k, int S, int act,
                   __nv_bfloat16* __restrict__ h_dec) {
-  __shared__ int32_t tok_s[kDecPass];
-  __shared__ int32_t slot_s[kDecPass];
-  __shared__ float red[4][kDecNT][32][8];
+  constexpr int PASS = NTMAX * 8;
+  constexpr int AHEAD = NTMAX == 1 ? 2 : 1;
+  __shared__ int32_t tok_s[PASS];
+  __shared__ int32_t slot_s[PASS];
+  __shared__ float red[4][NTMAX][32][8];
+  extern __shared__ __align__(16) uint4 xs[];  // NTMAX == 1: [8][H/8] token rows
   pdl_wait();  // routing (meta, slots) comes from decode_route
   pdl_trigger();
   DecGroup grp;
@@ -197,52 +210,84 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
   const __nv_bfloat16* pua = W + (int64_t)(I + ra) * H;
   const __nv_bfloat16* pub = W + (int64_t)(I + rb) * H;
   const uint4 z4 = make_uint4(0, 0, 0, 0);
+  struct W4 {
+    uint4 ga, gb, ua, ub;
+  };
+  auto load_w = [&](int ch) -> W4 {
+    const int col = ch * 32 + 8 * c;
+    const bool vc = ch < ch1 && col < H;
+    W4 r;
+    r.ga = (va && vc) ? ld_stream(pga + col) : z4;
+    r.gb = (vb && vc) ? ld_stream(pgb + col) : z4;
+    r.ua = (va && vc) ? ld_stream(pua + col) : z4;
+    r.ub = (vb && vc) ? ld_stream(pub + col) : z4;
+    return r;
+  };
 
-  for (int p0 = 0; p0 < grp.n; p0 += kDecPass) {
-    const int np = min(kDecPass, grp.n - p0);
+  for (int p0 = 0; p0 < grp.n; p0 += PASS) {
+    const int np = min(PASS, grp.n - p0);
     const int NT = (np + 7) >> 3;
     __syncthreads();
+    // weights of the next AHEAD chunks are requested before a chunk is
+    // multiplied (the first ones before the token rows are even looked up)
+    W4 q0 = load_w(ch0), q1, q2;
+    if (AHEAD >= 2) q1 = load_w(ch0 + 1);
+    if (AHEAD >= 3) q2 = load_w(ch0 + 2);
     for (int i = threadIdx.x; i < np; i += kDecThreads) {
       const int s = slots[grp.base + p0 + i];
       slot_s[i] = s;
       tok_s[i] = s < R ? s / k : (s - R) % T;
     }
     __syncthreads();
-    float ag[kDecNT][4], au[kDecNT][4];
+    if (NTMAX == 1) {
+      // the (at most 8) token rows of x, staged once: no L2 round trip per
+      // chunk in the loop below
+      const int hv = H >> 3;
+      for (int i = threadIdx.x; i < 8 * hv; i += kDecThreads) {
+        const int tk = i / hv, cc = i - tk * hv;
+        xs[i] = tk < np ? __ldg(reinterpret_cast<const uint4*>(x) +
+                                (int64_t)tok_s[tk] * hv + cc)
+                        : z4;
+      }
+      __syncthreads();
+    }
+    float ag[NTMAX][4], au[NTMAX][4];
 #pragma unroll
-    for (int nt = 0; nt < kDecNT; ++nt)
+    for (int nt = 0; nt < NTMAX; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) ag[nt][e] = au[nt][e] = 0.f;
-    // weights of chunk ch+1 are requested before chunk ch is multiplied
-    auto load_w = [&](int ch, uint4& ga, uint4& gb, uint4& ua, uint4& ub) {
-      const int col = ch * 32 + 8 * c;
-      const bool vc = ch < ch1 && col < H;
-      ga = (va && vc) ? ld_stream(pga + col) : z4;
-      gb = (vb && vc) ? ld_stream(pgb + col) : z4;
-      ua = (va && vc) ? ld_stream(pua + col) : z4;
-      ub = (vb && vc) ? ld_stream(pub + col) : z4;
-    };
-    uint4 nga, ngb, nua, nub;
-    load_w(ch0, nga, ngb, nua, nub);
     for (int ch = ch0; ch < ch1; ++ch) {
       const int col = ch * 32 + 8 * c;
       const bool vc = col < H;
-      const uint4 wga = nga, wgb = ngb, wua = nua, wub = nub;
-      load_w(ch + 1, nga, ngb, nua, nub);
+      const W4 cur = q0;
+      if (AHEAD == 1) {
+        q0 = load_w(ch + 1);
+      } else if (AHEAD == 2) {
+        q0 = q1;
+        q1 = load_w(ch + 2);
+      } else {
+        q0 = q1;
+        q1 = q2;
+        q2 = load_w(ch + 3);
+      }
 #pragma unroll
-      for (int nt = 0; nt < kDecNT; ++nt) {
+      for (int nt = 0; nt < NTMAX; ++nt) {
         if (nt < NT) {
           const int tk = nt * 8 + gq;
-          const uint4 xv = (tk < np && vc)
-              ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)tok_s[tk] * H + col))
-              : z4;
-          mma_chunk(ag[nt], wga, wgb, xv);
-          mma_chunk(au[nt], wua, wub, xv);
+          uint4 xv;
+          if (NTMAX == 1)
+            xv = vc ? xs[gq * (H >> 3) + (col >> 3)] : z4;  // zero rows past np
+          else
+            xv = (tk < np && vc)
+                ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)tok_s[tk] * H + col))
+                : z4;
+          mma_chunk(ag[nt], cur.ga, cur.gb, xv);
+          mma_chunk(au[nt], cur.ua, cur.ub, xv);
         }
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < kDecNT; ++nt) {
+    for (int nt = 0; nt < NTMAX; ++nt) {
       if (nt < NT) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -279,6 +324,7 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
 // two 32-column chunks ahead of the MMAs.
 constexpr int kW2Rows = 64;
 
+template <int NTMAX>
 __global__ void __launch_bounds__(kDecThreads, 4)
 decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const __nv_bfloat16* __restrict__ w2,
@@ -286,15 +332,28 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
                  const float* __restrict__ wgt, int T, int H, int I, int E, int k,
                  int S, float* __restrict__ stage) {
-  __shared__ int32_t slot_s[kDecPass];
-  pdl_wait();  // h_dec comes from decode_w13 (which itself waited for routing)
-  pdl_trigger();
+  constexpr int PASS = NTMAX * 8;
+  __shared__ int32_t slot_s[PASS];
+  extern __shared__ __align__(16) uint4 hs[];  // NTMAX == 1: [8][I/8] h rows
+  // This kernel is launched once every decode_w13 block has passed its own
+  // wait for the routing, so the expert lists are final here: the weight rows
+  // of this block are pulled into L2 while decode_w13 still streams its own.
   DecGroup grp;
-  if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
-  const int R = T * k, ks = k + S;
-  const __nv_bfloat16* W = grp.g < E ? w2 + (int64_t)grp.g * H * I
-                                     : w2_sh + (int64_t)(grp.g - E) * H * I;
+  const bool live = load_group(meta, E + S, blockIdx.x, &grp);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* W = nullptr;
+  if (live) {
+    W = grp.g < E ? w2 + (int64_t)grp.g * H * I : w2_sh + (int64_t)(grp.g - E) * H * I;
+    const int rows = min(kDecRows, H - (int)(blockIdx.y * kW2Rows + warp * kDecRows));
+    if (lane == 0 && rows > 0)
+      prefetch_l2_bulk(W + (int64_t)(blockIdx.y * kW2Rows + warp * kDecRows) * I,
+                       (uint32_t)rows * I * 2);
+  }
+  pdl_wait();  // h_dec comes from decode_w13
+  pdl_trigger();
+  if (!live) return;
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  const int R = T * k, ks = k + S;
   const int gq = lane >> 2, c = lane & 3;
   const int r0 = blockIdx.y * kW2Rows + warp * kDecRows;
   const int nch = (I + 31) / 32;
@@ -302,7 +361,6 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
   const bool va = ra < H, vb = rb < H;
   const __nv_bfloat16* pa = W + (int64_t)ra * I;
   const __nv_bfloat16* pb = W + (int64_t)rb * I;
-  const uint4 z4 = make_uint4(0, 0, 0, 0);
   auto load_w = [&](int ch, uint4& a, uint4& b) {
     const int col = ch * 32 + 8 * c;
     const bool vc = ch < nch && col < I;
@@ -310,16 +368,26 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
     b = (vb && vc) ? ld_stream(pb + col) : z4;
   };
 
-  for (int p0 = 0; p0 < grp.n; p0 += kDecPass) {
-    const int np = min(kDecPass, grp.n - p0);
+  for (int p0 = 0; p0 < grp.n; p0 += PASS) {
+    const int np = min(PASS, grp.n - p0);
     const int NT = (np + 7) >> 3;
     __syncthreads();
     for (int i = threadIdx.x; i < np; i += kDecThreads)
       slot_s[i] = slots[grp.base + p0 + i];
     __syncthreads();
-    float acc[kDecNT][4];
+    if (NTMAX == 1) {
+      const int iv = I >> 3;
+      for (int i = threadIdx.x; i < 8 * iv; i += kDecThreads) {
+        const int tk = i / iv, cc = i - tk * iv;
+        hs[i] = tk < np ? __ldg(reinterpret_cast<const uint4*>(h_dec) +
+                                (int64_t)slot_s[tk] * iv + cc)
+                        : z4;
+      }
+      __syncthreads();
+    }
+    float acc[NTMAX][4];
 #pragma unroll
-    for (int nt = 0; nt < kDecNT; ++nt)
+    for (int nt = 0; nt < NTMAX; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
     uint4 qa0, qb0, qa1, qb1;  // chunks ch and ch+1 in flight
@@ -333,18 +401,22 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
       qb0 = qb1;
       load_w(ch + 2, qa1, qb1);
 #pragma unroll
-      for (int nt = 0; nt < kDecNT; ++nt) {
+      for (int nt = 0; nt < NTMAX; ++nt) {
         if (nt < NT) {
           const int tk = nt * 8 + gq;
-          const uint4 hv = (tk < np && vc)
-              ? __ldg(reinterpret_cast<const uint4*>(h_dec + (int64_t)slot_s[tk] * I + col))
-              : z4;
+          uint4 hv;
+          if (NTMAX == 1)
+            hv = vc ? hs[gq * (I >> 3) + (col >> 3)] : z4;
+          else
+            hv = (tk < np && vc)
+                ? __ldg(reinterpret_cast<const uint4*>(h_dec + (int64_t)slot_s[tk] * I + col))
+                : z4;
           mma_chunk(acc[nt], wa, wb, hv);
         }
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < kDecNT; ++nt) {
+    for (int nt = 0; nt < NTMAX; ++nt) {
       if (nt < NT) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -380,20 +452,36 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   const int G = a.E + a.S, R = a.T * a.k;
   if (!mark(0)) return cudaErrorUnknown;
   const size_t smem = sizeof(int32_t) * (2 * (size_t)G + R);
-  decode_route_kernel<<<1, 1024, smem, st>>>(a.logits, a.scale, a.T, a.E, a.k, a.S,
-                                             a.ids, a.w, a.meta, a.slots);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_ex(decode_route_kernel, dim3(1), dim3(1024), smem, st, false,
+                            a.logits, a.scale, a.T, a.E, a.k, a.S, a.ids, a.w,
+                            a.meta, a.slots);
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   const int max_groups = (R < a.E ? R : a.E) + a.S;
-  e = launch_ex(decode_w13_kernel, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
-                 dim3(kDecThreads), 0, st, true, a.x, a.w13, a.w13_sh,
+  // every expert (and shared expert) has at most T tokens: with T <= 8 the
+  // token rows of x and of h fit in shared memory
+  const bool few = a.T <= 8;
+  auto w13k = few ? decode_w13_kernel<1> : decode_w13_kernel<kDecNT>;
+  auto w2k = few ? decode_w2_kernel<1> : decode_w2_kernel<kDecNT>;
+  const size_t xs_bytes = few ? (size_t)8 * a.H * 2 : 0;
+  const size_t hs_bytes = few ? (size_t)8 * a.I * 2 : 0;
+  // dynamic + static shared memory above 48 KiB needs the opt-in
+  if (few) {
+    if ((e = cudaFuncSetAttribute(w13k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)xs_bytes)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(w2k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)hs_bytes)) != cudaSuccess)
+      return e;
+  }
+  e = launch_ex(w13k, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
+                 dim3(kDecThreads), xs_bytes, st, true, a.x, a.w13, a.w13_sh,
                  (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
                  a.k, a.S, a.act, a.h_dec);
   if (e != cudaSuccess) return e;
   if (!mark(4)) return cudaErrorUnknown;
-  e = launch_ex(decode_w2_kernel, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
-                 dim3(kDecThreads), 0, st, true, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
+  e = launch_ex(w2k, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
+                 dim3(kDecThreads), hs_bytes, st, true, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
                  (const int32_t*)a.meta, (const int32_t*)a.slots, (const float*)a.w,
                  a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
   if (e != cudaSuccess) return e;

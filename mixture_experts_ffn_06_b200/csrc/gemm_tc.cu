@@ -637,8 +637,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool 
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
                                  cudaStream_t st) {
-  wait_selftest_kernel<<<1, 32, 0, st>>>(err, (uint64_t)timeout_us * 1000ull);
-  return cudaGetLastError();
+  return launch_ex(wait_selftest_kernel, dim3(1), dim3(32), 0, st, false, err,
+                   (uint64_t)timeout_us * 1000ull);
 }
 
 }  // namespace moe

@@ -258,8 +258,7 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                 (const int32_t*)offsets, (const int32_t*)lt_base,
                 (const int32_t*)lt_count, R > 0 ? n_lt : (int64_t)0, E, S, s.T, P,
                 cap, sorted_slots);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,

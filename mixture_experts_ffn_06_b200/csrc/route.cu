@@ -33,9 +33,8 @@ cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
-  route_kernel<<<(unsigned)blocks, warps * 32, 0, st>>>(logits, scale, T, E, k,
-                                                       ids, w);
-  return cudaGetLastError();
+  return launch_ex(route_kernel, dim3((unsigned)blocks), dim3(warps * 32), 0, st,
+                   false, logits, scale, T, E, k, ids, w);
 }
 
 }  // namespace moe
