@@ -90,7 +90,7 @@ struct KParams {
   int act;
   uint32_t* err;
   uint64_t timeout_ns;
-  const int32_t* sorted_slots;  // modes 2, 3
+  const int32_t* sorted_slots;  // row -> slot (-1: padding row)
   const float* w;               // modes 2, 3
   int64_t T;                    // modes 2, 3
   int k, S;                     // modes 2, 3
@@ -349,7 +349,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = unit0; t < total; t += unit_step) {
       const Tile tl = map_tile<MODE, CG>(t, offs, ub, p.G, p.NT, rank);
-      if (MODE >= 2) {
+      if (MODE <= 1) {
+        // 1: a real row.  Padding rows (only in a segment's last tile) feed
+        // nothing: mode 0 leaves them as they are (-1), mode 1 writes zeros
+        // there (0) so that the caller's y_perm holds no stale values
+        const bool real = tl.row0 + BM < (int64_t)offs[tl.g + 1] ||
+                          (tl.valid && p.sorted_slots[tl.row0 + q * 32 + lane] >= 0);
+        epi->rdst[q][lane] = real ? 1 : (MODE == 1 ? 0 : -1);
+      } else {
         // destination row and gate weight of this lane's tile row
         int64_t dst = -1;
         float wt = 1.0f;
@@ -409,7 +416,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int r = i * 8 + (lane >> 2);
-            if (col0 + cc < p.N) {
+            const int64_t rd = epi->rdst[q][r];
+            if (col0 + cc < p.N && rd > 0) {
               uint4 o;
               o.x = pack_bf16x2(tbuf[r][cc + 0], tbuf[r][cc + 1]);
               o.y = pack_bf16x2(tbuf[r][cc + 2], tbuf[r][cc + 3]);
@@ -430,7 +438,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               const float a2 = tbuf[r][cc + 2], a3 = tbuf[r][cc + 3];
               if (MODE == 1) {
                 *reinterpret_cast<float4*>(out + (wrow0 + r) * (int64_t)p.N + col0 + cc) =
-                    make_float4(a0, a1, a2, a3);
+                    epi->rdst[q][r] > 0 ? make_float4(a0, a1, a2, a3)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
               } else {
                 const int64_t dst = epi->rdst[q][r];
                 const float wt = epi->rw[q][r];

@@ -61,8 +61,8 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
                           cudaStream_t st, bool pdl = false);
 
-// Gathers x rows into x_perm (zeros on padding rows); when acc is given it
-// also zeroes acc[0, n_acc) (n_acc % 4 == 0).
+// Gathers x rows into x_perm (padding rows are left as they are); when acc
+// is given it also zeroes acc[0, n_acc) (n_acc % 4 == 0).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
                           int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
@@ -127,8 +127,8 @@ struct GroupedGemmArgs {
   void* out;                    // 0: bf16 [cap,N]; 1: fp32 [cap,N]; 2: fp32 [T,N]; 3: fp32 [T*(k+S),N]
   int act;
   uint32_t* err;
-  // mode 2 only
-  const int32_t* sorted_slots;  // [cap]
+  const int32_t* sorted_slots;  // [cap] row -> slot, -1 on padding rows
+  // modes 2, 3
   const float* w;               // [T,k]
   int64_t T;
   int k;

@@ -133,6 +133,10 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   a.out = h;
   a.act = s.act;
   a.err = err;
+  a.sorted_slots = sorted_slots;  // both GEMMs look up which rows are real
+  a.w = w;
+  a.T = s.T;
+  a.k = s.k;
   // CTA pairs (2-SM MMA) when asked; by default only for the w2 GEMM with
   // a long reduction (I >= 1024) once an expert averages two or more full
   // 128-row m-tiles -- measured on B200, pairs help w2 there and cost the
@@ -150,10 +154,6 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   a.N = s.H;
   a.K = s.I;
   a.out = y_perm;
-  a.sorted_slots = sorted_slots;
-  a.w = w;
-  a.T = s.T;
-  a.k = s.k;
   return from_cuda(launch_grouped_gemm(a, st));
 }
 

@@ -20,10 +20,11 @@ def to_device(inp: inputs.MoEInputs, device="cuda") -> inputs.MoEInputs:
 
 
 def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
-                deterministic=False, cta_pairs=0):
+                deterministic=False, cta_pairs=0, ws_fill=None):
     """moe_forward_ex through the C ABI -> (out bf16, out_f32, ids, w).
     Checks that the bf16 output is exactly the round-to-nearest-even of the
-    fp32 layer output."""
+    fp32 layer output.  ws_fill: byte written over the workspace past its
+    zeroed header before the call (stale contents)."""
     s = api.shape_from(inp.shape)
     T, H, k = inp.shape.T, inp.shape.H, inp.shape.k
     dev = inp.x.device
@@ -32,6 +33,8 @@ def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
     ids = torch.empty(T, k, dtype=torch.int32, device=dev) if with_routing else None
     w = torch.empty(T, k, dtype=torch.float32, device=dev) if with_routing else None
     ws = api.alloc_workspace(s, dev)
+    if ws_fill is not None:
+        ws[256:].fill_(ws_fill)
     api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                        inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w,
                        out_f32=out_f32, path=path, deterministic=deterministic,

@@ -217,6 +217,23 @@ def test_repeat_calls_are_bit_identical(api, variant):
     assert torch.equal(a, b) and torch.equal(a32, b32)
 
 
+@pytest.mark.parametrize("variant", ["prefill_det", "prefill_pairs_det", "decode"])
+@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_shapes_T130"])
+def test_stale_workspace_changes_nothing(api, name, variant):
+    # Padding rows of the gathered activations and of h are never written;
+    # each MMA row depends on its own A row only, so whatever they hold may
+    # reach only padding rows of the products.  0xFF bytes are NaN in both
+    # bf16 and fp32: one leaking into a real output would show.
+    inp = to_device(_small(name))
+    path, det, pairs = VARIANTS[variant]
+    a, a32, _, _ = gpu_forward(api, inp, path=path, deterministic=det,
+                               cta_pairs=pairs)
+    b, b32, _, _ = gpu_forward(api, inp, path=path, deterministic=det,
+                               cta_pairs=pairs, ws_fill=0xFF)
+    assert torch.isfinite(b32).all()
+    assert torch.equal(a, b) and torch.equal(a32, b32)
+
+
 def test_fast_combine_repeats_within_fp32_rounding(api):
     inp = to_device(_small("gemma_shapes_T130"))
     _, a32, _, _ = gpu_forward(api, inp, path=PATHS["prefill"])
