@@ -8,7 +8,9 @@ batch of synthetic tokens, through the C ABI call ``moe_forward``.  The
 default workload is the Mixtral-shaped prefill (T=4096, H=4096, E=8, k=2,
 I=14336, SiLU).  Inputs are resident in HBM when the timed region starts; the
 expert weights (2.8 GB) are far larger than L2, so every step streams them
-from HBM.  ``e2e`` repeats the measurement with the token inputs copied from
+from HBM.  A small batch that touches few experts (weights under four times
+the L2 size) gets an L2 flush before every step, outside that step's CUDA
+events.  ``e2e`` repeats the measurement with the token inputs copied from
 pinned host memory and the output copied back inside the timed region.
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own replica of
@@ -227,9 +229,12 @@ def touched_experts(api, s, inp, ws) -> int:
     return int(torch.unique(ids).numel()) + shp.n_shared
 
 
-def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks):
+def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
+            flush=None):
     """Same metric through the C ABI with the token inputs copied from pinned
-    host memory and the output copied back, inside the timed region."""
+    host memory and the output copied back, inside the timed region.  With
+    ``flush`` (an L2 flush), it runs before every step, outside that step's
+    events, and the step time is the mean of the per-step event pairs."""
     import torch
     shp = inp.shape
     x_h = inp.x.cpu().pin_memory()
@@ -248,17 +253,26 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks):
     for _ in range(max(args.warmup, 3)):
         e2e_step()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    n = args.steps if flush is not None else 1
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    if flush is None:
+        e0[0].record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1[0].record(stream)
+    else:
+        for i in range(args.steps):
+            flush(i)
+            e0[i].record(stream)
+            e2e_step()
+            e1[i].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    total = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
+    e2e_ms = max_over_ranks(total) / args.steps
     h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
     return e2e_ms, h2d, d2h
@@ -316,6 +330,23 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {status}")
 
+    # ---- L2.  A step whose expert weights (the distinct experts it routes
+    # to) fit a few times over in L2 would find them there on the next step:
+    # then every step is preceded by a write of twice the L2 size, outside
+    # that step's events, and the step time is the mean of the per-step
+    # event pairs.  Larger working sets stream from HBM by themselves.
+    touched = touched_experts(api, s, inp, ws)
+    expert_bytes = 3.0 * shp.H * shp.I * 2
+    weight_set = touched * expert_bytes
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = None
+    if weight_set < 4 * l2_bytes:
+        flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+
+    def flush(i):
+        if flush_buf is not None:
+            flush_buf.fill_(i & 0xFF)
+
     # ---- device-resident timed region (per-stage events on the stream).
     # By default the K steps are captured once into a CUDA graph and the
     # timed region is one replay of it, so that host launch overhead does
@@ -324,9 +355,24 @@ def run_ours(args):
     nst = api.NUM_STAGES
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
                 for _ in range(args.steps)]
-    for evs in stage_ev:  # create the events before the timed region
+    # with the flush: only the first and last event of each step, so that no
+    # event node sits between the step's kernels
+    step_ev = [[e[0]] + [None] * (nst - 1) + [e[nst]] for e in
+               [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+                for _ in range(args.steps)]]
+    for evs in stage_ev + step_ev:  # create the events before the timed region
         for e in evs:
-            e.record(stream)
+            if e is not None:
+                e.record(stream)
+
+    def plain_step(i):
+        flush(i)
+        step(step_ev[i] if flush_buf is not None else None)
+
+    def staged_step(i):
+        flush(i)
+        step(stage_ev[i])
+
     graph = staged = None
     if not args.no_graph:
         # one graph of K plain steps (the timed region) and one of K steps
@@ -335,11 +381,11 @@ def run_ours(args):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             for i in range(args.steps):
-                step()
+                plain_step(i)
         staged = torch.cuda.CUDAGraph()
         with torch.cuda.graph(staged, stream=stream):
             for i in range(args.steps):
-                step(stage_ev[i])
+                staged_step(i)
         graph.replay()  # untimed first replays
         staged.replay()
         torch.cuda.synchronize()
@@ -355,20 +401,23 @@ def run_ours(args):
         graph.replay()
     else:
         for i in range(args.steps):
-            step()
+            plain_step(i)
     t_end.record(stream)
     if staged is not None:
         staged.replay()
     else:
         for i in range(args.steps):
-            step(stage_ev[i])
+            staged_step(i)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     if graph is not None:
         del graph, staged
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
-    ms_per_step = ms_total / args.steps
+    if flush_buf is None:
+        ms_total = t_start.elapsed_time(t_end)
+    else:
+        ms_total = sum(e[0].elapsed_time(e[nst]) for e in step_ev)
+    ms_per_step = max_over_ranks(ms_total) / args.steps
     try:
         stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
                                     for ev in stage_ev) for j in range(nst)]
@@ -376,7 +425,7 @@ def run_ours(args):
         # events inside the graph could not be timed: take the stage times
         # from the same K steps launched on the stream instead
         for i in range(args.steps):
-            step(stage_ev[i])
+            staged_step(i)
         torch.cuda.synchronize()
         stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
                                     for ev in stage_ev) for j in range(nst)]
@@ -385,8 +434,9 @@ def run_ours(args):
         raise RuntimeError(f"device error in the timed region: {status}")
 
     # ---- end to end: pinned host inputs in, host output back, every step
-    e2e_ms, h2d, d2h = run_e2e(args, api, inp, s, ws, out, stream, barrier,
-                               max_over_ranks) if not args.profile else (None, 0, 0)
+    e2e_ms, h2d, d2h = run_e2e(
+        args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
+        flush if flush_buf is not None else None) if not args.profile else (None, 0, 0)
 
     result = None
     if rank == 0:
@@ -398,9 +448,7 @@ def run_ours(args):
         w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) \
             * shp.H * 2
         w13_ms = stage_ms[3]
-        touched = touched_experts(api, s, inp, ws)
-        expert_bytes = 3.0 * shp.H * shp.I * 2
-        layer_bytes = touched * expert_bytes
+        layer_bytes = weight_set
         # the w13 product does 2 FLOP per weight byte per token routed to the
         # expert; below the ridge point (peak FLOP/s / peak B/s) it is bound
         # by streaming the touched experts' weights from HBM
@@ -452,13 +500,19 @@ def run_ours(args):
                        "path": "decode" if decode else "prefill",
                        "combine": "fixed-order" if (decode or args.deterministic)
                                   else "fp32 reductions",
-                       "timing": "one CUDA-graph replay of the K steps"
-                                 if not args.no_graph else "stream launches",
+                       "timing": ("one CUDA-graph replay of the K steps"
+                                  if not args.no_graph else "stream launches")
+                                 + ("; step time = mean of per-step event pairs"
+                                    if flush_buf is not None else ""),
                        "global_batch": world * shp.T, "seq_len": shp.T,
                        "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "inputs larger than L2: expert weights "
-                             f"{(inp.w13.numel() + inp.w2.numel()) * 2 / 1e9:.2f} GB "
-                             "streamed every step"},
+                       "l2": (f"L2 flushed before every step ({2 * l2_bytes / 1e6:.0f}"
+                              " MB write outside the step's events): the step "
+                              f"touches {weight_set / 1e6:.0f} MB of expert weights"
+                              if flush_buf is not None else
+                              "inputs larger than L2: the step streams the "
+                              f"{weight_set / 1e9:.2f} GB of the {touched} experts "
+                              "it routes to")},
             "roofline": roof,
             "layer_tflops": layer_tflops,
             "stage_ms": dict(zip(api.STAGE_NAMES, stage_ms)),

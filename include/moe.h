@@ -175,8 +175,9 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
 /*
  * moe_forward_ex -- moe_forward with options (opts may be NULL):
  *   stage_events  NULL or MOE_NUM_STAGES + 1 cudaEvent_t created by the
- *                 caller; event i is recorded before stage i and event
- *                 MOE_NUM_STAGES after the last one, on ``stream``.  Stages:
+ *                 caller (a NULL entry records nothing); event i is recorded
+ *                 before stage i and event MOE_NUM_STAGES after the last one,
+ *                 on ``stream``.  Stages:
  *                 0 route, 1 permute, 2 gather, 3 w13 GEMM + activation,
  *                 4 w2 GEMM + gate weight + combine, 5 bf16 rounding
  *                 (with deterministic = 1: the fixed-order sum over the

@@ -195,7 +195,8 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                    path=PATH_AUTO, deterministic=False, cta_pairs=0,
                    stream=None):
     """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
-    created with enable_timing=True) recorded around the stages, ``out_f32``
+    created with enable_timing=True, or None to skip one) recorded around
+    the stages, ``out_f32``
     ([T,H] fp32) receiving the output before its bf16 rounding, and ``path``
     (PATH_AUTO, PATH_PREFILL or PATH_DECODE); ``deterministic`` selects the
     fixed-order combine on the prefill path; ``cta_pairs`` picks the GEMM
@@ -206,10 +207,11 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
             raise ValueError("need NUM_STAGES + 1 events")
         st = stream if stream is not None else torch.cuda.current_stream()
         for e in events:
-            if not e.cuda_event:  # torch creates its events lazily
+            if e is not None and not e.cuda_event:  # torch creates them lazily
                 e.record(st)
         arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
-            *[ctypes.c_void_p(e.cuda_event) for e in events])
+            *[ctypes.c_void_p(e.cuda_event if e is not None else 0)
+              for e in events])
     opts = moe_forward_opts(
         ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
         _p(out_f32), path, int(bool(deterministic)), cta_pairs)

@@ -448,7 +448,7 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
 size_t decode_meta_ints(int G) { return 2 + 2 * (size_t)G; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev) {
-  auto mark = [&](int i) -> bool { return !ev || record_stage_event(ev[i], st); };
+  auto mark = [&](int i) -> bool { return !ev || !ev[i] || record_stage_event(ev[i], st); };
   const int G = a.E + a.S, R = a.T * a.k;
   if (!mark(0)) return cudaErrorUnknown;
   const size_t smem = sizeof(int32_t) * (2 * (size_t)G + R);

@@ -234,6 +234,30 @@ def test_stale_workspace_changes_nothing(api, name, variant):
     assert torch.equal(a, b) and torch.equal(a32, b32)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
+def test_stage_events_may_be_left_out(api, path):
+    # only the first and the last event: the step's time with no event
+    # between its kernels
+    inp = to_device(_small("gemma_shapes_T130" if path != "decode" else "one_token"))
+    want, _, _, _ = gpu_forward(api, inp, path=PATHS[path])
+    s = api.shape_from(inp.shape)
+    out = torch.empty_like(want)
+    ws = api.alloc_workspace(s)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    events = [ev[0]] + [None] * (api.NUM_STAGES - 1) + [ev[1]]
+    api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
+                       inp.w13_sh, inp.w2_sh, out, ws, events=events,
+                       path=PATHS[path])
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    assert ev[0].elapsed_time(ev[1]) > 0
+    if path == "decode":
+        assert torch.equal(out, want)  # the decode path is deterministic
+    else:  # fp32 reductions in any order, then one bf16 rounding
+        assert (out.float() - want.float()).abs().max() <= \
+            1e-2 * want.float().abs().max()
+
+
 def test_fast_combine_repeats_within_fp32_rounding(api):
     inp = to_device(_small("gemma_shapes_T130"))
     _, a32, _, _ = gpu_forward(api, inp, path=PATHS["prefill"])
