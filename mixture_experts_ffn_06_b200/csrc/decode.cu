@@ -25,6 +25,8 @@
 // decode_w13 the 4 warps of a CTA split K (H is long) and add their partial
 // sums through shared memory; in decode_w2 each warp owns 16 rows and all of
 // K (I is short).
+#include <algorithm>
+
 #include "route_impl.cuh"
 
 namespace moe {
@@ -71,37 +73,16 @@ __device__ __forceinline__ float dec_act(int act, float g) {
   return 0.5f * g * (1.0f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
 }
 
-// Exclusive scan of one value per thread over a 1024-thread block.
-__device__ int block_scan_excl(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += n;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int ws = warp_sums[lane];
-    int wi = ws;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += n;
-    }
-    warp_sums[lane] = wi - ws;
-    if (lane == 31) warp_sums[32] = wi;
-  }
-  __syncthreads();
-  const int r = incl - v + warp_sums[warp];
-  *total = warp_sums[32];
-  __syncthreads();
-  return r;
-}
-
 // meta layout (int32): [0] n touched groups; [1 + i] group id of the i-th
 // touched group; [1 + G + i] first slot-list entry of group i (i <= n).
+//
+// One block of 32 * ceil(G / 32) threads (at least one warp per token up to
+// 32 warps): thread g owns group g.  One block-wide scan of the packed pair
+// (touched ? 1 : 0) << 16 | tokens of g gives both the touched index and
+// the first slot-list entry of every group (both sums stay below 2^16:
+// G <= 520 groups, T (k + S) <= 1024 * 40 slots).  PER logits per lane
+// (route_impl.cuh).
+template <int PER>
 __global__ void __launch_bounds__(1024)
 decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
                     int T, int E, int k, int S, int32_t* __restrict__ ids,
@@ -109,18 +90,18 @@ decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ 
                     int32_t* __restrict__ slots) {
   extern __shared__ int32_t dsm[];
   const int G = E + S, R = T * k;
-  int32_t* cnt = dsm;            // [G]
-  int32_t* pos = cnt + G;        // [G]
-  int32_t* ids_s = pos + G;      // [R]
-  __shared__ int warp_sums[33];
+  int32_t* cnt = dsm;            // [G] tokens, then first slot-list entry
+  int32_t* ids_s = cnt + G;      // [R]
+  __shared__ uint32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
   pdl_trigger();
   for (int i = tid; i < G; i += blockDim.x) cnt[i] = (i < E) ? 0 : T;
   __syncthreads();
-  for (int t = warp; t < T; t += blockDim.x >> 5) {
+  for (int t = warp; t < T; t += nwarps) {
     int id;
     float wt;
-    route_token_warp(logits + (int64_t)t * E, scale, E, k, &id, &wt);
+    route_token_warp<PER>(logits + (int64_t)t * E, scale, E, k, &id, &wt);
     if (lane < k) {
       ids[t * k + lane] = id;
       w[t * k + lane] = wt;
@@ -131,31 +112,49 @@ decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ 
   for (int s = tid; s < R; s += blockDim.x) atomicAdd(&cnt[ids_s[s]], 1);
   __syncthreads();
   const int c = (tid < G) ? cnt[tid] : 0;
-  const int f = c > 0 ? 1 : 0;
-  int total_c, total_f;
-  const int base = block_scan_excl(c, warp_sums, &total_c);
-  const int idx = block_scan_excl(f, warp_sums, &total_f);
+  const uint32_t v = (c > 0 ? 1u << 16 : 0u) | (uint32_t)c;
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t ws = lane < nwarps ? warp_sums[lane] : 0u;
+    uint32_t wi = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += o;
+    }
+    warp_sums[lane] = wi - ws;  // exclusive prefix of the warps before
+    if (lane == 31) {
+      meta[0] = (int32_t)(wi >> 16);                 // touched groups
+      meta[1 + G + (wi >> 16)] = (int32_t)(wi & 0xffffu);  // total slots
+    }
+  }
+  __syncthreads();
+  const uint32_t excl = incl - v + warp_sums[warp];
   if (tid < G) {
-    pos[tid] = base;
-    if (f) {
+    const int base = (int)(excl & 0xffffu), idx = (int)(excl >> 16);
+    cnt[tid] = base;
+    if (c > 0) {
       meta[1 + idx] = tid;
       meta[1 + G + idx] = base;
     }
-  }
-  if (tid == 0) {
-    meta[0] = total_f;
-    meta[1 + G + total_f] = total_c;
   }
   __syncthreads();
   // slot lists: routed slots by atomic position (the order inside an expert's
   // list only decides which MMA column a token uses, not its result)
   for (int s = tid; s < R; s += blockDim.x) {
-    const int p = atomicAdd(&pos[ids_s[s]], 1);
+    const int p = atomicAdd(&cnt[ids_s[s]], 1);
     slots[p] = s;
   }
   for (int q = tid; q < T * S; q += blockDim.x) {
     const int sh = q / T, t = q - sh * T;
-    slots[pos[E + sh] + t] = R + q;
+    slots[cnt[E + sh] + t] = R + q;
   }
 }
 
@@ -451,10 +450,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   auto mark = [&](int i) -> bool { return !ev || !ev[i] || record_stage_event(ev[i], st); };
   const int G = a.E + a.S, R = a.T * a.k;
   if (!mark(0)) return cudaErrorUnknown;
-  const size_t smem = sizeof(int32_t) * (2 * (size_t)G + R);
-  cudaError_t e = launch_ex(decode_route_kernel, dim3(1), dim3(1024), smem, st, false,
-                            a.logits, a.scale, a.T, a.E, a.k, a.S, a.ids, a.w,
-                            a.meta, a.slots);
+  const size_t smem = sizeof(int32_t) * ((size_t)G + R);
+  const int rthreads = 32 * std::min(32, std::max((G + 31) / 32, std::min(a.T, 32)));
+  auto rk = a.E <= 32 ? decode_route_kernel<1> : a.E <= 64 ? decode_route_kernel<2>
+            : a.E <= 128 ? decode_route_kernel<4> : a.E <= 256 ? decode_route_kernel<8>
+            : decode_route_kernel<16>;
+  cudaError_t e = launch_ex(rk, dim3(1), dim3(rthreads), smem, st, false, a.logits, a.scale,
+                            a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots);
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   const int max_groups = (R < a.E ? R : a.E) + a.S;

@@ -7,6 +7,7 @@
 namespace moe {
 namespace {
 
+template <int PER>
 __global__ void __launch_bounds__(256)
 route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
              int64_t T, int E, int k, int32_t* __restrict__ ids,
@@ -18,7 +19,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
   if (t >= T) return;
   int id;
   float wt;
-  route_token_warp(logits + t * E, scale, E, k, &id, &wt);
+  route_token_warp<PER>(logits + t * E, scale, E, k, &id, &wt);
   if (lane < k) {
     ids[t * k + lane] = id;
     w[t * k + lane] = wt;
@@ -33,8 +34,11 @@ cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
-  return launch_ex(route_kernel, dim3((unsigned)blocks), dim3(warps * 32), 0, st,
-                   false, logits, scale, T, E, k, ids, w);
+  // logits per lane: the fewest that cover E (E <= 512)
+  auto kern = E <= 32 ? route_kernel<1> : E <= 64 ? route_kernel<2> : E <= 128 ? route_kernel<4>
+              : E <= 256 ? route_kernel<8> : route_kernel<16>;
+  return launch_ex(kern, dim3((unsigned)blocks), dim3(warps * 32), 0, st, false, logits, scale,
+                   T, E, k, ids, w);
 }
 
 }  // namespace moe

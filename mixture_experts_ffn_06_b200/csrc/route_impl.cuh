@@ -8,10 +8,13 @@
 // alone (the all-E denominator cancels), so that closed form is evaluated:
 // it needs no pass over the unselected experts and cannot underflow.
 //
-// Lane l holds logits e = l, l+32, ... (E <= 512: at most 16 per lane).  Each
-// of the k rounds is a warp-wide argmax under (larger logit, then lower id),
-// so ids come out in the order of a stable descending sort.  The weights are
-// formed in fp64 and rounded once to fp32.
+// Lane l holds logits e = l, l+32, ... (PER per lane, E <= 32 PER; at most
+// 16 for E <= 512).  Each of the k rounds is a warp-wide argmax under
+// (larger logit, then lower id), so ids come out in the order of a stable
+// descending sort.  The weights are formed in fp64 and rounded once to fp32.
+// PER is a template parameter so that a round scans only the entries that
+// exist (measured on B200: scanning 16 per lane with E = 128 and k = 8 took
+// the prefill route kernel 28 us instead of 22 on 8192 tokens).
 #pragma once
 
 #include "internal.cuh"
@@ -25,12 +28,14 @@ __device__ __forceinline__ bool route_precedes(float va, int ia, float vb, int i
   return va > vb || (va == vb && ia < ib);
 }
 
-// Routes token row z[0..E) with the calling warp.  Lane j < k returns the
-// j-th choice in (*id, *wt); the other lanes return id 0, weight 0.
+// Routes token row z[0..E) with the calling warp (E <= 32 PER).  Lane j < k
+// returns the j-th choice in (*id, *wt); the other lanes return id 0,
+// weight 0.
+template <int PER = kMaxExperts / 32>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
                                                  const float* __restrict__ scale,
                                                  int E, int k, int* id, float* wt) {
-  constexpr int kPerLane = kMaxExperts / 32;
+  constexpr int kPerLane = PER;
   const int lane = threadIdx.x & 31;
   float v[kPerLane];
 #pragma unroll
