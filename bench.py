@@ -231,51 +231,102 @@ def touched_experts(api, s, inp, ws) -> int:
 
 def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
             flush=None):
-    """Same metric through the C ABI with the token inputs copied from pinned
-    host memory and the output copied back, inside the timed region.  With
-    ``flush`` (an L2 flush), it runs before every step, outside that step's
-    events, and the step time is the mean of the per-step event pairs."""
+    """Same metric through the C ABI with every step's token inputs copied
+    from pinned host memory and its output copied back, inside the timed
+    region.
+
+    Without ``flush`` the steps are pipelined the way a serving loop runs
+    them: the input copies on one stream, moe_forward on the compute stream,
+    the output copies on a third, over two device buffers per tensor, so
+    that step i+1's inputs and step i-1's output cross PCIe while step i
+    computes.  Each step still copies its own inputs in and its own output
+    out.  With ``flush`` (an L2 flush; small batches, whose copies are a few
+    KB) the flush runs before every step, outside that step's events, the
+    steps run one after another, and the step time is the mean of the
+    per-step event pairs."""
     import torch
     shp = inp.shape
+    dev = inp.x.device
     x_h = inp.x.cpu().pin_memory()
     z_h = inp.logits.cpu().pin_memory()
-    out_h = torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(inp.x)
-    z_d = torch.empty_like(inp.logits)
+    h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
+    d2h = shp.T * shp.H * 2
+    if flush is not None:
+        out_h = torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
+        x_d = torch.empty_like(inp.x)
+        z_d = torch.empty_like(inp.logits)
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        z_d.copy_(z_h, non_blocking=True)
-        api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
-                        inp.w2_sh, out, ws)
-        out_h.copy_(out, non_blocking=True)
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            z_d.copy_(z_h, non_blocking=True)
+            api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                            inp.w2_sh, out, ws)
+            out_h.copy_(out, non_blocking=True)
 
-    for _ in range(max(args.warmup, 3)):
-        e2e_step()
-    torch.cuda.synchronize()
-    n = args.steps if flush is not None else 1
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    barrier()
-    torch.cuda.synchronize()
-    if flush is None:
-        e0[0].record(stream)
-        for _ in range(args.steps):
+        for _ in range(max(args.warmup, 3)):
             e2e_step()
-        e1[0].record(stream)
-    else:
+        torch.cuda.synchronize()
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
         for i in range(args.steps):
             flush(i)
             e0[i].record(stream)
             e2e_step()
             e1[i].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        total = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
+        return max_over_ranks(total) / args.steps, h2d, d2h
+
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    x_d = [torch.empty_like(inp.x) for _ in range(2)]
+    z_d = [torch.empty_like(inp.logits) for _ in range(2)]
+    o_d = [torch.empty_like(out) for _ in range(2)]
+    out_h = [torch.empty(shp.T, shp.H, dtype=torch.bfloat16).pin_memory()
+             for _ in range(2)]
+
+    def run(n):
+        """n pipelined steps; returns (start event, end event)."""
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        ev_in = [ev() for _ in range(n)]
+        ev_c = [ev() for _ in range(n)]
+        ev_out = [ev() for _ in range(n)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[i - 2])  # step i-2 has read buffer b
+                x_d[b].copy_(x_h, non_blocking=True)
+                z_d[b].copy_(z_h, non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev_in[i])
+                if i >= 2:
+                    stream.wait_event(ev_out[i - 2])  # output buffer b copied out
+                api.moe_forward(s, x_d[b], z_d[b], inp.w13, inp.w2, inp.scale,
+                                inp.w13_sh, inp.w2_sh, o_d[b], ws, stream=stream)
+                ev_c[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[i])
+                out_h[b].copy_(o_d[b], non_blocking=True)
+                ev_out[i].record(s_out)
+        t1.record(s_out)  # after the last output copy, hence after every step
+        return t0, t1
+
+    run(max(args.warmup, 3))
     torch.cuda.synchronize()
     barrier()
-    total = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
-    e2e_ms = max_over_ranks(total) / args.steps
-    h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
-    d2h = out_h.numel() * out_h.element_size()
-    return e2e_ms, h2d, d2h
+    torch.cuda.synchronize()
+    t0, t1 = run(args.steps)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(t0.elapsed_time(t1)) / args.steps, h2d, d2h
 
 
 def run_ours(args):
@@ -519,7 +570,11 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": None if e2e_ms is None else
                    {"value": world * shp.T / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "timing": "steps one after another, L2 flushed before each"
+                              if flush_buf is not None else
+                              "pipelined: input copies, moe_forward and output "
+                              "copies on three streams, two buffers each"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
