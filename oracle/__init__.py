@@ -12,7 +12,11 @@ walkthrough's worked example (yeyulingfeng.com/587419.html section 4), the
 closed form of the same section, brute-force top-k and counting sort, a dense
 "run every expert then mask" evaluation (llama-cpp-visual-guide lesson 35,
 ggml_mul_mat_id section), the E=1/k=1 plain gated MLP, and torch's own SiLU
-and tanh-GELU in float64.
+and tanh-GELU in float64.  The router ahead of the routing (walkthrough
+section 3, Gemma4Router) is pinned by the closed form of a constant row, the
+unit RMS of the normalised row, exact invariance under power-of-two row
+scaling, exact linearity in the scale and the weight, bf16-valued
+activations, and a finite zero row.
 """
 from __future__ import annotations
 
@@ -59,8 +63,11 @@ def _load():
         lib.oracle_forward.argtypes = [i64, i32, i32, i32, i32, i32, i32, i32,
                                        P, P, P, P, P, P, P, P, i64, i32, i32,
                                        P, P, P]
+        lib.oracle_router_logits.argtypes = [i64, i32, i32, ctypes.c_double, P, P,
+                                             P, P]
         for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
-                  lib.oracle_expert_rows, lib.oracle_forward):
+                  lib.oracle_expert_rows, lib.oracle_forward,
+                  lib.oracle_router_logits):
             f.restype = i32
         _lib = lib
     return _lib
@@ -153,6 +160,19 @@ def expert_rows(x, w13, w2, tok, exp_id, act_kind: int, round_h: bool = False,
                                       int(round_h), nthreads, _ptr(y)),
            "expert_rows")
     return y
+
+
+def router_logits(x, w_router, scale, eps: float) -> np.ndarray:
+    """Router logits [T,E] float32 from the bf16 residual [T,H], the bf16
+    GateLinear weight [E,H] and the bf16 per-dimension scale [H]."""
+    xu, wu, su = _u16(x), _u16(w_router), _u16(scale)
+    T, H = xu.shape
+    E = wu.shape[0]
+    assert wu.shape == (E, H) and su.shape == (H,)
+    z = np.empty((T, E), np.float32)
+    _check(_load().oracle_router_logits(T, H, E, float(eps), _ptr(xu), _ptr(wu),
+                                        _ptr(su), _ptr(z)), "router_logits")
+    return z
 
 
 def forward(x, logits, w13, w2, k: int, act_kind: int, scale=None,

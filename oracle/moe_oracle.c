@@ -406,3 +406,57 @@ int oracle_forward(int64_t T, int H, int E, int k, int I, int act, int S,
   if (!w_out) free(w);
   return rc;
 }
+
+/* ----------------------------------------------------------------- router */
+
+/*
+ * router -- the step ahead of the routing: "Gemma4Router-MoE 的入口"
+ * (section 3 of the Gemma 4 walkthrough, yeyulingfeng.com/587419.html) and
+ * the Gemma4Router class on the vLLM API page.  For every residual row r
+ * (bf16, H values):
+ *   1. RMSNorm with no gamma, computed in fp32 and returned in the input
+ *      dtype: n_h = bf16( fl(r_h * fl(1 / fl(sqrt(fl(v + eps))))) ), where
+ *      v = fl(mean_h r_h^2) is taken in double and rounded once to fp32 and
+ *      fl() is an fp32 operation (IEEE, round to nearest even);
+ *   2. times the constant hidden_size^-0.5, itself cast to bf16 first (the
+ *      fp32 buffer .to(x.dtype)): a_h = bf16( n_h * bf16(fl(H^-0.5)) );
+ *   3. times the learned per-dimension scale in bf16: b_h = bf16(a_h * s_h);
+ *   4. GateLinear: bf16 activations and weights, fp32 output:
+ *      z[e] = fl( sum_h b_h * W[e,h] ), the sum in double.
+ * Products of two bf16 values are exact in double (and in fp32), so steps 2
+ * and 3 round exactly once each, as a bf16 multiply does.
+ */
+int oracle_router_logits(int64_t T, int H, int E, double eps, const uint16_t* x,
+                         const uint16_t* w_router, const uint16_t* scale,
+                         float* logits) {
+  if (T < 0 || H < 1 || E < 1 || !(eps >= 0.0) || !x || !w_router || !scale || !logits)
+    return EINVAL_ARG;
+  double* b = (double*)malloc(sizeof(double) * (size_t)H);
+  if (!b) return ENOMEM_ARG;
+  const double root = round_to_bf16((double)(float)pow((double)H, -0.5));
+  for (int64_t t = 0; t < T; ++t) {
+    const uint16_t* r = x + t * (int64_t)H;
+    double ss = 0.0;
+    for (int h = 0; h < H; ++h) {
+      const double v = bf16_to_double(r[h]);
+      ss += v * v;
+    }
+    const float var = (float)(ss / (double)H);
+    const float den = sqrtf(var + (float)eps);
+    const float inv = 1.0f / den;
+    for (int h = 0; h < H; ++h) {
+      const float n = (float)bf16_to_double(r[h]) * inv;
+      const double nb = round_to_bf16((double)n);
+      const double a = round_to_bf16(nb * root);
+      b[h] = round_to_bf16(a * bf16_to_double(scale[h]));
+    }
+    for (int e = 0; e < E; ++e) {
+      const uint16_t* wr = w_router + (int64_t)e * H;
+      double z = 0.0;
+      for (int h = 0; h < H; ++h) z += b[h] * bf16_to_double(wr[h]);
+      logits[t * (int64_t)E + e] = (float)z;
+    }
+  }
+  free(b);
+  return OK;
+}

@@ -275,3 +275,83 @@ def test_parameter_counts_from_the_page():
     # lesson 35: top-2 of 8 computes a quarter of the equal-capacity dense
     mix = inputs.shape_of("mixtral_prefill")
     assert mix.flops() / (6.0 * mix.H * mix.I * mix.T * mix.E) == 0.25
+
+
+# ------------------------------------------------------------------ router
+# The router ahead of the routing: section 3 of the Gemma 4 walkthrough
+# ("Gemma4Router-MoE 的入口") and the Gemma4Router class of the vLLM page --
+# RMSNorm without gamma, times bf16(H^-0.5), times the per-dimension scale,
+# then GateLinear with fp32 output.
+
+def _bf(a) -> torch.Tensor:
+    return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _router_case(T, H, E, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    w = torch.randn(E, H, generator=g).to(torch.bfloat16)
+    s = (0.5 + torch.rand(H, generator=g)).to(torch.bfloat16)
+    return x, w, s
+
+
+def test_router_constant_row_closed_form():
+    # A constant row normalises to exactly +-1 (eps = 0), so with a unit
+    # scale and an all-ones weight row the logit is H * bf16(H^-0.5): the
+    # constant is rounded to bf16 before it multiplies (H = 100 turns 0.1
+    # into 0.10009765625, so the logit is 10.009765625, not 10).
+    for H, want in ((64, 8.0), (100, 10.009765625), (256, 16.0)):
+        x = _bf([[3.0] * H, [-0.25] * H])
+        w = _bf([[1.0] * H, [-1.0] * H])
+        z = oracle.router_logits(x, w, _bf([1.0] * H), 0.0)
+        assert z[0, 0] == np.float32(want) and z[0, 1] == np.float32(-want)
+        assert z[1, 0] == np.float32(-want) and z[1, 1] == np.float32(want)
+
+
+def test_router_norm_gives_unit_rms():
+    # H = 64 makes H^-0.5 = 1/8 exact; with the identity as GateLinear weight
+    # and a unit scale, 8 z is the normalised row rounded to bf16, whose RMS
+    # is 1 up to that rounding -- a mean-absolute or L2 norm would not give 1
+    H = 64
+    x, _, _ = _router_case(8, H, 1, 3)
+    z = oracle.router_logits(x, torch.eye(H).to(torch.bfloat16), _bf([1.0] * H), 0.0)
+    rms = np.sqrt(np.mean((8.0 * z.astype(np.float64)) ** 2, axis=1))
+    assert np.all(np.abs(rms - 1.0) <= 2.0 ** -8)
+
+
+def test_router_power_of_two_row_scaling_changes_nothing():
+    # RMSNorm removes the row's scale; a power of two passes through every
+    # rounding exactly (eps = 0)
+    x, w, s = _router_case(5, 96, 7, 0)
+    z = oracle.router_logits(x, w, s, 0.0)
+    for j in (-3, 1, 4):
+        assert np.array_equal(oracle.router_logits(x * 2.0 ** j, w, s, 0.0), z)
+
+
+def test_router_is_linear_in_the_scale_and_the_weight():
+    x, w, s = _router_case(4, 80, 5, 1)
+    z = oracle.router_logits(x, w, s, 1e-6)
+    assert np.array_equal(oracle.router_logits(x, w * 2, s, 1e-6), 2 * z)
+    assert np.array_equal(oracle.router_logits(x, w, s * 2, 1e-6), 2 * z)
+    # each expert's logit uses its own weight row only
+    perm = torch.tensor([3, 0, 4, 1, 2])
+    assert np.array_equal(oracle.router_logits(x, w[perm], s, 1e-6), z[:, perm.numpy()])
+
+
+def test_router_activations_are_bf16_before_the_projection():
+    # with a one-hot weight row the logit is one activation b_h itself, which
+    # must be a bf16 value: the norm, the constant and the scale each round
+    x, _, s = _router_case(6, 48, 1, 2)
+    for h in (0, 17, 47):
+        w = torch.zeros(1, 48, dtype=torch.bfloat16)
+        w[0, h] = 1.0
+        z = oracle.router_logits(x, w, s, 1e-6)[:, 0]
+        assert np.array_equal(torch.tensor(z).to(torch.bfloat16).float().numpy(), z)
+
+
+def test_router_zero_row_stays_finite():
+    # eps keeps the norm of an all-zero row finite: its logits are zero
+    x, w, s = _router_case(3, 64, 4, 4)
+    x[1] = 0.0
+    z = oracle.router_logits(x, w, s, 1e-6)
+    assert np.all(z[1] == 0.0) and np.all(np.isfinite(z))
