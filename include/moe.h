@@ -86,6 +86,25 @@ MOE_API int64_t moe_layout_capacity(const moe_shape* shape);
 MOE_API size_t moe_workspace_size(const moe_shape* shape);
 
 /*
+ * moe_router_logits -- the router ahead of the routing (walkthrough section
+ * 3, "Gemma4Router-MoE 的入口"; the Gemma4Router class on the vLLM page):
+ *   x        [T,H] bf16 residual-stream rows (the router's own input, not
+ *            the experts' normalised input)
+ *   w_router [E,H] bf16 GateLinear weight
+ *   scale    [H] bf16 learned per-dimension scale
+ *   eps      RMSNorm epsilon (>= 0)
+ *   logits   [T,E] fp32 out: z = GateLinear(bf16(bf16(bf16(RMSNorm(x))
+ *            * bf16(H^-0.5)) * scale)); the norm in fp32 with no gamma, the
+ *            projection accumulated in fp32.  The activations before the
+ *            projection match the oracle exactly; the logits within the
+ *            fp32 accumulation error.
+ * Uses no workspace.  shape->k, I, n_shared, act are not read.
+ */
+MOE_API moe_status moe_router_logits(const moe_shape* shape, const moe_bf16* x,
+                                     const moe_bf16* w_router, const moe_bf16* scale,
+                                     float eps, float* logits, cudaStream_t stream);
+
+/*
  * moe_route -- routing of every token (walkthrough section 4 steps 1-5 and
  * section 5; Gemma4MoE.routing_function on the vLLM page).
  *   logits [T,E] fp32, scale [E] fp32 or NULL (all ones)

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 NUM_STAGES = 6
 STAGE_NAMES = ("route", "permute", "gather", "w13_gemm_act",
                "w2_gemm_weight_combine", "round_bf16")
-EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_route",
+EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_router_logits",
+           "moe_route",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_ex",
            "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string",
@@ -68,6 +69,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_layout_capacity.restype = ctypes.c_int64
     lib.moe_workspace_size.argtypes = [S]
     lib.moe_workspace_size.restype = ctypes.c_size_t
+    lib.moe_router_logits.argtypes = [S, P, P, P, ctypes.c_float, P, P]
     lib.moe_route.argtypes = [S, P, P, P, P, P]
     lib.moe_permute.argtypes = [S, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_expert_ffn.argtypes = [S, P, P, P, P, P, P, P, P, P,
@@ -85,7 +87,8 @@ def _load() -> ctypes.CDLL:
                                               ctypes.c_uint32, P]
     lib.moe_status_string.argtypes = [st]
     lib.moe_status_string.restype = ctypes.c_char_p
-    for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+    for name in ("moe_router_logits", "moe_route", "moe_permute", "moe_expert_ffn",
+                 "moe_combine",
                  "moe_forward", "moe_forward_ex", "moe_read_error",
                  "moe_selftest_wait_timeout"):
         getattr(lib, name).restype = st
@@ -146,6 +149,14 @@ def alloc_workspace(shape: moe_shape, device="cuda") -> torch.Tensor:
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     ws[:256].zero_()
     return ws
+
+
+def moe_router_logits(shape, x, w_router, scale, eps, logits, stream=None):
+    """Router logits [T,E] fp32 from the bf16 residual x [T,H], the bf16
+    GateLinear weight [E,H] and the bf16 per-dimension scale [H]."""
+    _check(lib.moe_router_logits(ctypes.byref(shape), _p(x), _p(w_router), _p(scale),
+                                 ctypes.c_float(eps), _p(logits), _stream(stream)),
+           "moe_router_logits")
 
 
 def moe_route(shape, logits, scale, ids, w, stream=None):

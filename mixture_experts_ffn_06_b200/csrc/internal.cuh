@@ -52,6 +52,13 @@ bool record_stage_event(void* ev, cudaStream_t st);
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
                          int E, int k, int32_t* ids, float* w, cudaStream_t st);
 
+// Router logits [T,E] fp32 from the bf16 residual [T,H], the GateLinear
+// weight [E,H] and the per-dimension scale [H] (router.cu).
+cudaError_t launch_router_logits(const __nv_bfloat16* x, const __nv_bfloat16* w_router,
+                                 const __nv_bfloat16* scale, int64_t T, int H, int E,
+                                 float eps, float* logits, cudaStream_t st,
+                                 bool pdl = false);
+
 // pdl on any launch function: launch its first kernel as a programmatic
 // dependent of the previous kernel on the stream (later kernels of the same
 // function always are).

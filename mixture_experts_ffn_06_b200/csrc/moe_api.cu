@@ -2,6 +2,8 @@
 // checks, the workspace map, and the launch sequence of each call.  Every
 // argument error is returned before anything is enqueued; nothing here
 // allocates, frees or synchronises (moe_read_error excepted, as documented).
+#include <cmath>
+
 #include "internal.cuh"
 
 namespace moe {
@@ -171,6 +173,24 @@ int64_t moe_layout_capacity(const moe_shape* shape) {
 size_t moe_workspace_size(const moe_shape* shape) {
   if (check_shape(shape) != MOE_OK) return 0;
   return workspace_map(*shape).total;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status moe_router_logits(const moe_shape* shape, const moe_bf16* x,
+                             const moe_bf16* w_router, const moe_bf16* scale, float eps,
+                             float* logits, cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) return MOE_OK;
+  if (!x || !w_router || !scale || !logits) return MOE_ERR_INVALID_ARG;
+  // the kernel reads 16-byte vectors
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(scale)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_router_logits(reinterpret_cast<const __nv_bfloat16*>(x),
+                                        reinterpret_cast<const __nv_bfloat16*>(w_router),
+                                        reinterpret_cast<const __nv_bfloat16*>(scale),
+                                        shape->T, shape->H, shape->E, eps, logits, stream));
 }
 
 moe_status moe_route(const moe_shape* shape, const float* logits,

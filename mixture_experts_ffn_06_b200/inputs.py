@@ -140,6 +140,17 @@ def router_logits(T: int, E: int, k: int, gen: torch.Generator, device,
     raise RuntimeError("could not meet the top-k margin")
 
 
+def router_inputs(T: int, H: int, E: int, gen: torch.Generator, device):
+    """Inputs of the router ahead of the routing: the residual rows [T,H]
+    (N(0, 4) in bf16 -- the router normalises them away), the GateLinear
+    weight [E,H] (N(0,1) in bf16, so that the logits come out near unit
+    scale) and the per-dimension scale [H] (U[0.5, 1.5] in bf16)."""
+    x = (2.0 * torch.randn(T, H, generator=gen, device=device)).to(torch.bfloat16)
+    w = torch.randn(E, H, generator=gen, device=device).to(torch.bfloat16)
+    s = (0.5 + torch.rand(H, generator=gen, device=device)).to(torch.bfloat16)
+    return x.contiguous(), w.contiguous(), s.contiguous()
+
+
 def _normal_bf16(shape, std: float, gen: torch.Generator, device) -> torch.Tensor:
     out = torch.empty(shape, dtype=torch.bfloat16, device=device)
     if out.dim() == 3:

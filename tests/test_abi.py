@@ -128,3 +128,18 @@ def test_status_strings(api):
     assert api.moe_status_string(0) == "MOE_OK"
     assert api.moe_status_string(5) == "MOE_ERR_TIMEOUT"
     assert api.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_router_logits_refuses_bad_arguments(api):
+    # rejected on the host before any launch: no GPU needed
+    s = api.make_shape(T=4, H=64, E=8, k=1, I=8)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    null = ctypes.c_void_p(0)
+    f = api.lib.moe_router_logits
+    assert f(ctypes.byref(s), fake, fake, fake, ctypes.c_float(-1.0), fake, null) == 1
+    assert f(ctypes.byref(s), fake, fake, fake, ctypes.c_float(float("inf")), fake, null) == 1
+    assert f(ctypes.byref(s), odd, fake, fake, ctypes.c_float(1e-6), fake, null) == 1
+    assert f(ctypes.byref(s), null, fake, fake, ctypes.c_float(1e-6), fake, null) == 1
+    empty = api.make_shape(T=0, H=64, E=8, k=1, I=8)
+    assert f(ctypes.byref(empty), null, null, null, ctypes.c_float(1e-6), null, null) == 0

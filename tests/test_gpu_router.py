@@ -1,0 +1,104 @@
+"""Parity of the router kernel (moe_router_logits) with the fp64 oracle.
+
+The router ahead of the routing: section 3 of the Gemma 4 walkthrough
+("Gemma4Router-MoE 的入口") and the Gemma4Router class of the vLLM page.  Both
+sides form the same bf16 activations (RMSNorm in fp32 with the normaliser of
+an exact-in-double mean, then the bf16 roundings the page's casts fix); the
+logits differ only by the accumulation of the projection, fp32 on the GPU and
+double in the oracle.  The bar for that: max|err| <= 3e-4 x RMS(oracle
+logits) (fp32 accumulation of H products: relative error ~ sqrt(H/16)
+2^-24 times the sum of |products|, a few 1e-5 of the RMS at H = 4096).
+Routing on the GPU's logits must then match the oracle's routing of the same
+logits bit for bit, and the oracle's routing of its own logits wherever the
+k-th and (k+1)-th logits are further apart than the logit error.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_ffn_06_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = 3e-4
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixture_experts_ffn_06_b200 import api as a
+    return a
+
+
+def _case(T, H, E, seed):
+    g = torch.Generator().manual_seed(seed)
+    return inputs.router_inputs(T, H, E, g, "cpu")
+
+
+def _gpu_logits(api, x, w, s, eps):
+    T, H = x.shape
+    E = w.shape[0]
+    shape = api.make_shape(T=T, H=H, E=E, k=1, I=8)
+    z = torch.full((T, E), float("nan"), dtype=torch.float32, device="cuda")
+    api.moe_router_logits(shape, x.cuda(), w.cuda(), s.cuda(), eps, z)
+    torch.cuda.synchronize()
+    return z.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,H,E", [
+    (64, 256, 8),       # one CTA, Mixtral's E
+    (130, 2816, 128),   # ragged token tail, the many-small shape
+    (37, 200, 5),       # H not a multiple of 32: a partial 32-column chunk
+    (16, 64, 130),      # E > 128: two expert blocks, the second ragged
+    (1, 4096, 8),       # one token
+])
+def test_router_logits_match_oracle(api, T, H, E):
+    x, w, s = _case(T, H, E, seed=T + H + E)
+    want = oracle.router_logits(x, w, s, 1e-6)
+    got = _gpu_logits(api, x, w, s, 1e-6)
+    assert np.isfinite(got).all()
+    rms = float(np.sqrt(np.mean(want.astype(np.float64) ** 2)))
+    err = float(np.abs(got.astype(np.float64) - want).max())
+    assert err <= TOL * rms, f"max|err| {err:.3e} > {TOL} x RMS {rms:.3e}"
+
+
+def test_zero_and_constant_rows(api):
+    # all-zero rows stay finite (eps); constant rows normalise to +-1
+    x, w, s = _case(20, 128, 8, seed=7)
+    x[3] = 0.0
+    x[5] = 1.5
+    want = oracle.router_logits(x, w, s, 1e-6)
+    got = _gpu_logits(api, x, w, s, 1e-6)
+    assert np.all(got[3] == 0.0)
+    rms = float(np.sqrt(np.mean(want.astype(np.float64) ** 2)))
+    assert float(np.abs(got - want).max()) <= TOL * rms
+
+
+@pytest.mark.parametrize("k", [2, 8])
+def test_routing_on_router_logits(api, k):
+    T, H, E = 200, 2816, 128
+    x, w, s = _case(T, H, E, seed=11 + k)
+    zo = oracle.router_logits(x, w, s, 1e-6)
+    zg = _gpu_logits(api, x, w, s, 1e-6)
+    shape = api.make_shape(T=T, H=H, E=E, k=k, I=8)
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    api.moe_route(shape, torch.from_numpy(zg).cuda(), None, ids, wt)
+    torch.cuda.synchronize()
+    ids = ids.cpu().numpy()
+    # the same logits: the same decisions, bit for bit
+    ref_ids, _ = oracle.route(zg, k)
+    assert np.array_equal(ids, ref_ids)
+    # the oracle's own logits: the same decisions wherever the k-th and
+    # (k+1)-th logits are further apart than the logit error
+    own_ids, _ = oracle.route(zo, k)
+    srt = -np.sort(-zo.astype(np.float64), axis=1)
+    gap = srt[:, k - 1] - srt[:, k]
+    rms = float(np.sqrt(np.mean(zo.astype(np.float64) ** 2)))
+    clear = gap > 2 * TOL * rms
+    assert clear.mean() > 0.9
+    assert np.array_equal(np.sort(ids[clear], axis=1), np.sort(own_ids[clear], axis=1))
