@@ -209,6 +209,13 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
  *                 stages 1 and 2 are empty (folded into stage 0).  Both
  *                 paths compute the same function; they differ in the order
  *                 of fp32 additions inside the products.
+ *   router_w      NULL, or the router ahead of the routing (see
+ *                 moe_router_logits): with router_w [E,H], router_x [T,H]
+ *                 (the residual rows the router reads) and router_scale [H]
+ *                 given, the logits are first computed from them into the
+ *                 workspace with RMSNorm epsilon router_eps, and ``logits``
+ *                 may be NULL.  On the prefill path this is part of stage 0;
+ *                 on the decode path it runs before stage 0.
  */
 #define MOE_NUM_STAGES 6
 typedef enum {
@@ -224,6 +231,10 @@ typedef struct {
   int32_t deterministic;  /* prefill path: fixed-order combine (see above) */
   int32_t cta_pairs;      /* prefill GEMMs: 0 auto, 1 one CTA per tile, 2 CTA
                              pairs (2-SM MMA, M = 256); results are identical */
+  const moe_bf16* router_x;      /* see router_w above */
+  const moe_bf16* router_w;
+  const moe_bf16* router_scale;
+  float router_eps;
 } moe_forward_opts;
 
 MOE_API moe_status moe_forward_ex(

@@ -46,7 +46,11 @@ class moe_forward_opts(ctypes.Structure):
                 ("out_f32", ctypes.c_void_p),
                 ("path", ctypes.c_int32),
                 ("deterministic", ctypes.c_int32),
-                ("cta_pairs", ctypes.c_int32)]
+                ("cta_pairs", ctypes.c_int32),
+                ("router_x", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p),
+                ("router_scale", ctypes.c_void_p),
+                ("router_eps", ctypes.c_float)]
 
 
 class moe_shape(ctypes.Structure):
@@ -204,14 +208,16 @@ def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
 def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                    ids_out=None, w_out=None, events=None, out_f32=None,
                    path=PATH_AUTO, deterministic=False, cta_pairs=0,
-                   stream=None):
+                   router=None, stream=None):
     """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
     created with enable_timing=True, or None to skip one) recorded around
     the stages, ``out_f32``
     ([T,H] fp32) receiving the output before its bf16 rounding, and ``path``
     (PATH_AUTO, PATH_PREFILL or PATH_DECODE); ``deterministic`` selects the
     fixed-order combine on the prefill path; ``cta_pairs`` picks the GEMM
-    form (0 auto, 1 single CTAs, 2 CTA pairs)."""
+    form (0 auto, 1 single CTAs, 2 CTA pairs); ``router`` = (router_x [T,H],
+    router_w [E,H], router_scale [H], eps) computes the logits first
+    (``logits`` may then be None)."""
     arr = None
     if events is not None:
         if len(events) != NUM_STAGES + 1:
@@ -223,9 +229,11 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
         arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
             *[ctypes.c_void_p(e.cuda_event if e is not None else 0)
               for e in events])
+    rx, rw, rs, reps = router if router is not None else (None, None, None, 0.0)
     opts = moe_forward_opts(
         ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
-        _p(out_f32), path, int(bool(deterministic)), cta_pairs)
+        _p(out_f32), path, int(bool(deterministic)), cta_pairs,
+        _p(rx), _p(rw), _p(rs), float(reps))
     _check(lib.moe_forward_ex(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
                               _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
                               _p(ids_out), _p(w_out), _p(ws), ws.numel(),

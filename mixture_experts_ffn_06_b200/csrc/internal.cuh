@@ -35,6 +35,7 @@ struct WsMap {
   size_t stage;        // [T,k+S,H] fp32 weighted expert rows (moe_forward)
   size_t acc;          // [T,H] fp32 accumulator (moe_forward, fast combine)
   size_t dec_meta;     // decode path: touched-expert lists
+  size_t logits;       // [T,E] fp32 router logits (moe_forward_ex with a router)
   size_t total;
   int64_t cap;
   int64_t n_lt;

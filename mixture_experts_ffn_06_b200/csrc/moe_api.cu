@@ -40,6 +40,7 @@ WsMap workspace_map(const moe_shape& s) {
   m.stage = take(4ull * T * (k + S) * s.H);
   m.acc = take(4ull * T * s.H);
   m.dec_meta = take(sizeof(int32_t) * decode_meta_ints((int)G));
+  m.logits = take(sizeof(float) * T * s.E);
   m.total = o;
   return m;
 }
@@ -264,8 +265,17 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                           cudaStream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
-  if (!w13 || !w2 || (shape->T > 0 && (!x || !logits || !out)))
+  const bool use_router = opts && opts->router_w;
+  if (!w13 || !w2 || (shape->T > 0 && (!x || (!logits && !use_router) || !out)))
     return MOE_ERR_INVALID_ARG;
+  if (use_router) {
+    if (!(opts->router_eps >= 0.0f) || !std::isfinite(opts->router_eps))
+      return MOE_ERR_INVALID_ARG;
+    if (shape->T > 0 && (!opts->router_x || !opts->router_scale ||
+                         !aligned16(opts->router_x) || !aligned16(opts->router_w) ||
+                         !aligned16(opts->router_scale)))
+      return MOE_ERR_INVALID_ARG;
+  }
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   void* const* ev = opts ? opts->stage_events : nullptr;
@@ -287,6 +297,17 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
   if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE)
     return MOE_ERR_INVALID_ARG;
   if (path == MOE_PATH_DECODE && s.T > kDecodeForcedMaxT) return MOE_ERR_UNSUPPORTED;
+  // the router ahead of the routing (moe_router_logits), when given: its
+  // logits go to the workspace and the routing reads them there
+  if (use_router) logits = reinterpret_cast<float*>(at(ws, m.logits));
+  auto run_router = [&]() {
+    return !use_router ||
+           launch_router_logits(reinterpret_cast<const __nv_bfloat16*>(opts->router_x),
+                                reinterpret_cast<const __nv_bfloat16*>(opts->router_w),
+                                reinterpret_cast<const __nv_bfloat16*>(opts->router_scale),
+                                s.T, s.H, s.E, opts->router_eps,
+                                const_cast<float*>(logits), stream) == cudaSuccess;
+  };
   if (path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && s.T <= kDecodeMaxT)) {
     // few tokens: stream only the touched experts (decode.cu)
     DecodeArgs d{};
@@ -312,9 +333,11 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
     d.stage = stage;
     d.out = reinterpret_cast<__nv_bfloat16*>(out);
     d.out_f32 = opts ? opts->out_f32 : nullptr;
+    if (!run_router()) return MOE_ERR_CUDA;
     return from_cuda(launch_decode(d, stream, ev));
   }
   if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
+  if (!run_router()) return MOE_ERR_CUDA;
   if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (!mark(ev, 1, stream)) return MOE_ERR_CUDA;

@@ -102,3 +102,34 @@ def test_routing_on_router_logits(api, k):
     clear = gap > 2 * TOL * rms
     assert clear.mean() > 0.9
     assert np.array_equal(np.sort(ids[clear], axis=1), np.sort(own_ids[clear], axis=1))
+
+
+@pytest.mark.parametrize("path,T", [(1, 37), (2, 4)])  # prefill, decode
+def test_forward_from_hidden_states(api, path, T):
+    # moe_forward_ex with the router options: logits computed from the
+    # residual first.  The oracle runs the layer on the GPU router's own
+    # logits (checked against the oracle router above), so both take the
+    # same routing decisions; ids bit-exact, output within 2e-2 x RMS.
+    from parity_util import assert_out_close, to_device
+    shp = inputs.Shape(T=T, H=256, E=8, k=2, I=128, act=1)
+    inp = to_device(inputs.make_inputs(shp, seed=3, scale="uniform"))
+    g = torch.Generator().manual_seed(5)
+    rx, rw, rs = (t.cuda() for t in inputs.router_inputs(T, 256, 8, g, "cpu"))
+    s = api.shape_from(shp)
+    ws = api.alloc_workspace(s)
+    out = torch.empty(T, 256, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty(T, 256, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, 2, dtype=torch.int32, device="cuda")
+    wt = torch.empty(T, 2, dtype=torch.float32, device="cuda")
+    api.moe_forward_ex(s, inp.x, None, inp.w13, inp.w2, inp.scale, None, None, out, ws,
+                       ids_out=ids, w_out=wt, out_f32=out32, path=path,
+                       router=(rx, rw, rs, 1e-6))
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    zg = _gpu_logits(api, rx.cpu(), rw.cpu(), rs.cpu(), 1e-6)
+    want, ref_ids, ref_w = oracle.forward(inp.x, zg, inp.w13, inp.w2, 2, 1,
+                                          scale=inp.scale)
+    assert np.array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.allclose(wt.cpu().numpy(), ref_w, rtol=1e-6, atol=0)
+    assert_out_close(out32, want, f"path {path}")
+    assert torch.equal(out, out32.to(torch.bfloat16))
