@@ -61,6 +61,9 @@ def parse():
                     help="time plain stream launches instead of one CUDA graph")
     ap.add_argument("--profile", action="store_true",
                     help="device timing only: skip the e2e and CPU legs")
+    ap.add_argument("--router", action="store_true",
+                    help="start from hidden states: the router (RMSNorm, scale, "
+                         "GateLinear) computes the logits inside every step")
     return ap.parse_args()
 
 
@@ -357,11 +360,17 @@ def run_ours(args):
     decode = path == api.PATH_DECODE or (path == api.PATH_AUTO
                                          and shp.T <= api.DECODE_MAX_T)
 
+    router = None
+    if args.router:
+        rg = torch.Generator(device=dev).manual_seed(args.seed + 1000 + rank)
+        router = (*inputs.router_inputs(shp.T, shp.H, shp.E, rg, dev), 1e-6)
+
     def step(events=None):
-        api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
-                           inp.w13_sh, inp.w2_sh, out, ws, events=events,
-                           path=path, deterministic=args.deterministic,
-                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs])
+        api.moe_forward_ex(s, inp.x, inp.logits if router is None else None, inp.w13,
+                           inp.w2, inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
+                           events=events, path=path, deterministic=args.deterministic,
+                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs],
+                           router=router)
 
     def barrier():
         if world > 1:
@@ -396,7 +405,8 @@ def run_ours(args):
 
     def flush(i):
         if flush_buf is not None:
-            flush_buf.fill_(i & 0xFF)
+            with torch.cuda.stream(stream):  # ordered before the step's kernels
+                flush_buf.fill_(i & 0xFF)
 
     # ---- device-resident timed region (per-stage events on the stream).
     # By default the K steps are captured once into a CUDA graph and the
@@ -484,10 +494,38 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device error in the timed region: {status}")
 
+    # ---- the router kernel alone (--router): L2 flushed before each launch
+    router_stats = None
+    if router is not None:
+        rz = torch.empty(shp.T, shp.E, dtype=torch.float32, device=dev)
+        fl = flush_buf if flush_buf is not None else \
+            torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            api.moe_router_logits(s, *router, rz, stream=stream)
+        rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i, (ra, rb) in enumerate(rev):
+            with torch.cuda.stream(stream):
+                fl.fill_(i & 0xFF)
+            ra.record(stream)
+            api.moe_router_logits(s, *router, rz, stream=stream)
+            rb.record(stream)
+        torch.cuda.synchronize()
+        r_ms = max_over_ranks(statistics.mean(ra.elapsed_time(rb) for ra, rb in rev))
+        # residual rows, GateLinear weight and scale read; logits written
+        r_bytes = (shp.T * shp.H + shp.E * shp.H + shp.H) * 2 + shp.T * shp.E * 4
+        router_stats = {"kernel": "router_logits_kernel (RMSNorm, scale, GateLinear)",
+                        "us": r_ms * 1e3, "bytes": r_bytes,
+                        "achieved_gbs": r_bytes / (r_ms / 1e3) / 1e9,
+                        "tflops": 2.0 * shp.T * shp.H * shp.E / (r_ms / 1e3) / 1e12,
+                        "timing": "L2 flushed before each launch"}
+        del fl
+
     # ---- end to end: pinned host inputs in, host output back, every step
     e2e_ms, h2d, d2h = run_e2e(
         args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
-        flush if flush_buf is not None else None) if not args.profile else (None, 0, 0)
+        flush if flush_buf is not None else None) \
+        if not (args.profile or args.router) else (None, 0, 0)
 
     result = None
     if rank == 0:
@@ -575,9 +613,14 @@ def run_ours(args):
                               if flush_buf is not None else
                               "pipelined: input copies, moe_forward and output "
                               "copies on three streams, two buffers each"},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": (launches_per_step + (1 if router is not None else 0))
+                            * args.steps,
             "clocks": clk,
         }
+        if router_stats is not None:
+            router_stats["frac_hbm"] = router_stats["achieved_gbs"] / float(peaks["hbm_gbs"])
+            result["router"] = router_stats
+            result["config"]["workload"] += " + router (from hidden states)"
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.barrier()

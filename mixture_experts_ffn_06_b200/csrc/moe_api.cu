@@ -333,8 +333,13 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
     d.stage = stage;
     d.out = reinterpret_cast<__nv_bfloat16*>(out);
     d.out_f32 = opts ? opts->out_f32 : nullptr;
+    if (!use_router) return from_cuda(launch_decode(d, stream, ev));
+    // the router counts in the first stage: event 0 goes ahead of it
+    void* dev[MOE_NUM_STAGES + 1] = {};
+    for (int i = 1; ev && i <= MOE_NUM_STAGES; ++i) dev[i] = ev[i];
+    if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
     if (!run_router()) return MOE_ERR_CUDA;
-    return from_cuda(launch_decode(d, stream, ev));
+    return from_cuda(launch_decode(d, stream, ev ? dev : nullptr));
   }
   if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
   if (!run_router()) return MOE_ERR_CUDA;

@@ -12,19 +12,26 @@
 // sequential double sum unless the two land on different sides of an fp32
 // rounding point, which takes a difference in the 53rd bit; 1/sqrt is the
 // IEEE fp32 division and square root, not the approximate reciprocal square
-// root.  Steps 2 and 3 multiply two bf16 values, exact in fp32, and round
-// once to bf16.  The activations are therefore the oracle's; the logits
-// differ from it only by the fp32 accumulation of the projection.
+// root.  Step 1 is an fp32 product rounded to bf16; steps 2 and 3 multiply
+// two bf16 values, whose product is exact in fp32, so the bf16x2 multiply
+// (one rounding of the exact product) gives the same bf16 as the fp32
+// product cast to bf16.  The activations are therefore the oracle's; the
+// logits differ from it only by the fp32 accumulation of the projection.
 //
-// One CTA of 4 warps takes 64 tokens and 128 experts (grid.y covers larger
-// E); warp w multiplies its 16 tokens (one 16-row MMA tile of activations)
-// by the 128 experts' weight rows (16 n8 tiles) with mma.sync m16n8k16 over
-// K = H.  Inside each 32-column chunk of K the column order is permuted so
-// that every fragment is one 16-byte load: thread (g, c) takes columns
-// [8c, 8c + 8) of token rows g and g + 8 and of expert row g; both operands
-// share the order, so the dot products are unchanged.  The activations of a
-// chunk are formed in registers from the residual and the scale; the weight
-// rows come through L1, which the 4 warps share.
+// One CTA of 8 warps takes 64 tokens and up to 128 experts (grid.y covers
+// larger E).  It streams the tokens' rows twice through a ring of shared-
+// memory slots: once to sum their squares, then with the experts' weight rows
+// and the scale for the projection; the second read of the residual comes
+// from L2.  Warp w multiplies token group w % 4 (16 tokens, one 16-row MMA
+// tile of activations) by the experts' weight rows (n8 tiles) with mma.sync
+// m16n8k16 over half of each staged K-block (w / 4 picks the half); the two
+// halves are added through shared memory in a fixed order at the end.
+// Inside each 32-column chunk of K the column order is permuted so that
+// every fragment is one 16-byte shared-memory load: thread (g, c) takes
+// columns [8c, 8c + 8) of token rows g and g + 8 and of expert row g; both
+// operands share the order, so the dot products are unchanged.  The
+// activations of a chunk are formed in registers from the staged residual
+// and scale.
 #include <cmath>
 
 #include "internal.cuh"
@@ -32,9 +39,10 @@
 namespace moe {
 namespace {
 
-constexpr int kRtWarps = 4;
-constexpr int kRtTokens = 16 * kRtWarps;  // tokens per CTA
-constexpr int kRtExperts = 128;           // experts per CTA (16 n8 tiles)
+constexpr int kRtWarps = 8;
+constexpr int kRtGroups = 4;                 // 16-token groups per CTA
+constexpr int kRtTokens = 16 * kRtGroups;    // tokens per CTA
+constexpr int kRtThreads = kRtWarps * 32;
 
 __device__ __forceinline__ void rt_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                        uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -48,103 +56,231 @@ __device__ __forceinline__ void rt_mma(float (&d)[4], uint32_t a0, uint32_t a1, 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
-__device__ __forceinline__ uint32_t bf_round(float f) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+// Steps 1-3 for one bf16 pair of a token row: bf16(bf16(bf16(x inv) root) s),
+// root2 = bf16(H^-0.5) in both halves
+__device__ __forceinline__ uint32_t rt_act2(uint32_t x2, uint32_t s2, float inv,
+                                            uint32_t root2) {
+  const float lo = __fmul_rn(bf_lo(x2), inv), hi = __fmul_rn(bf_hi(x2), inv);
+  uint32_t n2, a2, b2;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(n2) : "f"(hi), "f"(lo));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(a2) : "r"(n2), "r"(root2));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(b2) : "r"(a2), "r"(s2));
+  return b2;
 }
 
-// Steps 1-3 for one bf16 pair of a token row: bf16(bf16(bf16(x inv) root) s)
-__device__ __forceinline__ uint32_t rt_act2(uint32_t x2, uint32_t s2, float inv, float root) {
-  uint32_t out = 0;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const float x = half ? bf_hi(x2) : bf_lo(x2);
-    const float s = half ? bf_hi(s2) : bf_lo(s2);
-    const float n = __uint_as_float(bf_round(__fmul_rn(x, inv)) << 16);
-    const float a = __uint_as_float(bf_round(__fmul_rn(n, root)) << 16);
-    const uint32_t b = bf_round(__fmul_rn(a, s));
-    out |= half ? (b << 16) : b;
-  }
-  return out;
+__device__ __forceinline__ uint4 rt_act8(const uint4& x, const uint4& s, float inv,
+                                         uint32_t root2) {
+  return make_uint4(rt_act2(x.x, s.x, inv, root2), rt_act2(x.y, s.y, inv, root2),
+                    rt_act2(x.z, s.z, inv, root2), rt_act2(x.w, s.w, inv, root2));
 }
 
-__device__ __forceinline__ uint4 rt_act8(const uint4& x, const uint4& s, float inv, float root) {
-  return make_uint4(rt_act2(x.x, s.x, inv, root), rt_act2(x.y, s.y, inv, root),
-                    rt_act2(x.z, s.z, inv, root), rt_act2(x.w, s.w, inv, root));
+// 16-byte asynchronous copy global -> shared; src_bytes 0 fills zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__global__ void __launch_bounds__(kRtWarps * 32)
-router_logits_kernel(const uint4* __restrict__ x, const uint4* __restrict__ w,
-                     const uint4* __restrict__ scale, int64_t T, int H, int E, float eps,
-                     float root, float* __restrict__ logits) {
+__device__ __forceinline__ uint4 rt_lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+constexpr int kRtKB = 256;  // K columns per staged block
+// Bytes per staged row: 512 + 64, so rows g and g + 1 fall 16 banks apart
+// and the 8 lanes of one shared-memory phase -- two rows, four 16-byte
+// vectors each -- cover the 32 banks once.
+constexpr int kRtPitch = kRtKB * 2 + 64;
+constexpr uint32_t kRtRingMax = 224 * 1024;
+static_assert(kRtKB / 8 == 32, "one staged row is 32 16-byte vectors");
+
+// Rows of one staged block: 8 NT expert rows of W, the 64 token rows of the
+// residual, and the scale.
+__host__ __device__ constexpr int rt_rows(int NT) { return 8 * NT + kRtTokens + 1; }
+// Ring depth: as many blocks as fit in kRtRingMax bytes, at most 4.
+__host__ __device__ constexpr int rt_stages(int NT) {
+  return kRtRingMax / ((uint32_t)rt_rows(NT) * kRtPitch) > 4
+             ? 4
+             : (int)(kRtRingMax / ((uint32_t)rt_rows(NT) * kRtPitch));
+}
+
+// NT n8 tiles: the CTA's 8 NT experts (<= 128).  The CTA runs 2 nkb jobs
+// through a ring of rt_stages(NT) shared-memory slots filled with 16-byte
+// asynchronous copies, up to S - 1 jobs ahead: job j < nkb stages K-block j
+// of the token rows, whose squares the norm pass sums; job nkb + kb stages
+// K-block kb of the expert rows, the token rows (again, now from L2) and
+// the scale, which the projection multiplies.  Only rows that exist are
+// copied; columns past H are filled with zeros, so the ragged K tail adds
+// nothing.  Rows past T or E of a slot hold stale data: a token row past T
+// enters the MMA as zeros, and an expert row past E only feeds its own
+// output column, which is not stored.
+template <int NT>
+__global__ void __launch_bounds__(kRtThreads)
+router_logits_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                     const __nv_bfloat16* __restrict__ scale, int64_t T, int H, int E, float eps,
+                     uint32_t root2, float* __restrict__ logits) {
+  constexpr int EB = 8 * NT;           // experts per CTA
+  constexpr int S = rt_stages(NT);
+  static_assert(S >= 2, "the ring needs two slots");
+  constexpr uint32_t BLK = (uint32_t)rt_rows(NT) * kRtPitch;
+  constexpr int XR = EB;               // first token row of a slot
+  constexpr int SR = EB + kRtTokens;   // the scale row
+  static_assert(kRtGroups * NT * 4 * 32 * 4 <= BLK, "the K-half partial sums fit in a slot");
+  extern __shared__ __align__(16) uint8_t ring[];  // [S][rt_rows(NT)][kRtPitch]
   __shared__ float inv_s[kRtTokens];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = lane & 3;
-  const int hv = H >> 3;  // 16-byte vectors per row
   const int64_t t0 = (int64_t)blockIdx.x * kRtTokens;
-  const int e0 = blockIdx.y * kRtExperts;
-  pdl_wait();
-  pdl_trigger();
-  // ---- step 1: 1 / sqrt(mean(r^2) + eps) of this warp's 16 tokens
-  for (int i = 0; i < 16; ++i) {
-    const int64_t t = t0 + warp * 16 + i;
-    double ss = 0.0;
-    if (t < T) {
-      const uint4* row = x + t * hv;
-      for (int v = lane; v < hv; v += 32) {
-        const uint4 q = __ldg(row + v);
-        const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+  const int e0 = blockIdx.y * EB;
+  const int nt = T - t0 < kRtTokens ? (int)(T - t0) : kRtTokens;  // token rows of the CTA
+  const int ne = min(EB, E - e0);                                   // expert rows of the CTA
+  const int nkb = (H + kRtKB - 1) / kRtKB;
+  const uint32_t ring0 = smem_u32(ring);
+  // thread t stages 16-byte vector t % 32 of rows t / 32, t / 32 + 8, ...
+  const int sv = tid & 31, sr0 = tid >> 5;
+  auto stage = [&](int j) {
+    if (j < 2 * nkb) {
+      const bool proj = j >= nkb;
+      const int kb = proj ? j - nkb : j;
+      const int col = kb * kRtKB + sv * 8;
+      const bool ok = col < H;
+      const uint32_t nbytes = ok ? 16u : 0u;
+      const int cc = ok ? col : 0;
+      const uint32_t base = ring0 + (uint32_t)(j % S) * BLK + (uint32_t)sv * 16;
+      for (int r = sr0; r < nt; r += kRtWarps)
+        cp_async16(base + (uint32_t)(XR + r) * kRtPitch, x + (t0 + r) * H + cc, nbytes);
+      if (proj) {
+        for (int r = sr0; r < ne; r += kRtWarps)
+          cp_async16(base + (uint32_t)r * kRtPitch, w + (int64_t)(e0 + r) * H + cc, nbytes);
+        if (sr0 == 0) cp_async16(base + (uint32_t)SR * kRtPitch, scale + cc, nbytes);
+      }
+    }
+    cp_async_commit();  // one group per job, empty past the last
+  };
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const double lo = bf_lo(wd[j]), hi = bf_hi(wd[j]);
-          ss = fma(lo, lo, ss);
-          ss = fma(hi, hi, ss);
+  for (int p = 0; p < S - 1; ++p) stage(p);
+
+  // norm pass: lane l of warp w sums row 8w + l / 4, vectors l % 4 + 4i
+  const int nr = warp * 8 + (lane >> 2);
+  const bool nr_ok = nr < nt;
+  double ss = 0.0;
+  // projection: warp w multiplies token rows 16 (w % 4) + g and + g + 8 over
+  // chunks [4 (w / 4), 4 (w / 4) + 4) of each K-block
+  const int tg = warp & (kRtGroups - 1), kh = warp / kRtGroups;
+  const int ra = tg * 16 + gq, rb = ra + 8;
+  const bool va = ra < nt, vb = rb < nt, live = tg * 16 < nt;
+  float inv_a = 0.f, inv_b = 0.f;
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+
+  for (int j = 0; j < 2 * nkb; ++j) {
+    stage(j + S - 1);
+    cp_async_wait<S - 1>();  // job j has landed (this thread's copies)
+    __syncthreads();         // ... and everyone's
+    const uint32_t slot = ring0 + (uint32_t)(j % S) * BLK;
+    if (j < nkb) {
+      // ---- step 1: sum of squares, in double
+      if (nr_ok) {
+        const uint32_t row = slot + (uint32_t)(XR + nr) * kRtPitch + (uint32_t)(lane & 3) * 16;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = rt_lds128(row + i * 64);
+          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const double lo = bf_lo(wd[u]), hi = bf_hi(wd[u]);
+            ss = fma(lo, lo, ss);
+            ss = fma(hi, hi, ss);
+          }
+        }
+      }
+      if (j == nkb - 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        if ((lane & 3) == 0 && nr_ok) {
+          const float var = (float)(ss / (double)H);
+          inv_s[nr] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
+        }
+        __syncthreads();  // rows of other warps
+        if (va) inv_a = inv_s[ra];
+        if (vb) inv_b = inv_s[rb];
+      }
+    } else if (live) {
+      // ---- steps 2-4 on this warp's half of K-block kb
+      const int kb = j - nkb;
+      const int ch_end = min(4 * kh + 4, (H - kb * kRtKB + 31) / 32);
+      const uint32_t xa = slot + (uint32_t)(XR + ra) * kRtPitch;
+      const uint32_t xb = xa + 8 * kRtPitch;
+      const uint32_t srow = slot + (uint32_t)SR * kRtPitch;
+      for (int ch = 4 * kh; ch < ch_end; ++ch) {
+        const uint32_t col_b = (uint32_t)(ch * 32 + 8 * cq) * 2;
+        const uint4 cs = rt_lds128(srow + col_b);
+        const uint4 a0 = va ? rt_act8(rt_lds128(xa + col_b), cs, inv_a, root2) : z4;
+        const uint4 a8 = vb ? rt_act8(rt_lds128(xb + col_b), cs, inv_b, root2) : z4;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const uint4 bv = rt_lds128(slot + (uint32_t)(n * 8 + gq) * kRtPitch + col_b);
+          rt_mma(acc[n], a0.x, a8.x, a0.y, a8.y, bv.x, bv.y);
+          rt_mma(acc[n], a0.z, a8.z, a0.w, a8.w, bv.z, bv.w);
         }
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (lane == 0) {
-      const float var = (float)(ss / (double)H);
-      inv_s[warp * 16 + i] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
-    }
+    __syncthreads();  // slot j % S is refilled by job j + S
   }
-  __syncwarp();
-  // ---- steps 2-4: this warp's 16 tokens x 128 experts over K = H
-  const int64_t ta = t0 + warp * 16 + gq, tb = ta + 8;  // A rows g and g + 8
-  const bool va = ta < T, vb = tb < T;
-  const float inv_a = inv_s[warp * 16 + gq], inv_b = inv_s[warp * 16 + gq + 8];
-  const uint4* xa = x + (va ? ta : 0) * hv;
-  const uint4* xb = x + (vb ? tb : 0) * hv;
-  float acc[16][4];
+  cp_async_wait<0>();
+  // ---- the two K-halves: the second half's tiles go through slot 0 (free
+  // now), the first half adds them and stores
+  float* red = reinterpret_cast<float*>(ring);  // [group][n][e][lane]
+  if (kh == 1 && live) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  const int nch = (H + 31) >> 5;
-  for (int ch = 0; ch < nch; ++ch) {
-    const int v = ch * 4 + cq;  // 16-byte column group of this thread
-    const bool vc = v < hv;
-    const uint4 s = vc ? __ldg(scale + v) : z4;
-    const uint4 a0 = va && vc ? rt_act8(__ldg(xa + v), s, inv_a, root) : z4;
-    const uint4 a8 = vb && vc ? rt_act8(__ldg(xb + v), s, inv_b, root) : z4;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int e = e0 + j * 8 + gq;  // B column (expert) of this thread
-      const uint4 b = (e < E && vc) ? __ldg(w + (int64_t)e * hv + v) : z4;
-      rt_mma(acc[j], a0.x, a8.x, a0.y, a8.y, b.x, b.y);
-      rt_mma(acc[j], a0.z, a8.z, a0.w, a8.w, b.z, b.w);
-    }
+      for (int e = 0; e < 4; ++e) red[((tg * NT + n) * 4 + e) * 32 + lane] = acc[n][e];
   }
-  // ---- fragment element e: token row g (+8 for e >= 2), expert 2c + e % 2
+  __syncthreads();
+  if (kh == 1 || !live) return;
+  // fragment element e: token row g (+8 for e >= 2), expert 2c + e % 2
+  const int64_t ta = t0 + ra, tb = t0 + rb;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int e = e0 + j * 8 + 2 * cq;
-    if (va && e < E) logits[ta * E + e] = acc[j][0];
-    if (va && e + 1 < E) logits[ta * E + e + 1] = acc[j][1];
-    if (vb && e < E) logits[tb * E + e] = acc[j][2];
-    if (vb && e + 1 < E) logits[tb * E + e + 1] = acc[j][3];
+  for (int n = 0; n < NT; ++n) {
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = acc[n][e] + red[((tg * NT + n) * 4 + e) * 32 + lane];
+    const int c = n * 8 + 2 * cq;
+    const int e = e0 + c;
+    if (va && c < ne) logits[ta * E + e] = o[0];
+    if (va && c + 1 < ne) logits[ta * E + e + 1] = o[1];
+    if (vb && c < ne) logits[tb * E + e] = o[2];
+    if (vb && c + 1 < ne) logits[tb * E + e + 1] = o[3];
   }
+}
+
+template <int NT>
+cudaError_t launch_router_nt(const __nv_bfloat16* x, const __nv_bfloat16* w,
+                             const __nv_bfloat16* scale, int64_t T, int H, int E, float eps,
+                             uint32_t root2, float* logits, cudaStream_t st, bool pdl) {
+  const size_t smem = (size_t)rt_stages(NT) * rt_rows(NT) * kRtPitch;
+  const cudaError_t e = cudaFuncSetAttribute(
+      router_logits_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((T + kRtTokens - 1) / kRtTokens),
+                  (unsigned)((E + 8 * NT - 1) / (8 * NT)));
+  return launch_ex(router_logits_kernel<NT>, grid, dim3(kRtThreads), smem, st, pdl, x, w,
+                   scale, T, H, E, eps, root2, logits);
 }
 
 }  // namespace
@@ -159,12 +295,25 @@ cudaError_t launch_router_logits(const __nv_bfloat16* x, const __nv_bfloat16* w_
                                  const __nv_bfloat16* scale, int64_t T, int H, int E,
                                  float eps, float* logits, cudaStream_t st, bool pdl) {
   if (T == 0) return cudaSuccess;
-  const dim3 grid((unsigned)((T + kRtTokens - 1) / kRtTokens),
-                  (unsigned)((E + kRtExperts - 1) / kRtExperts));
-  return launch_ex(router_logits_kernel, grid, dim3(kRtWarps * 32), 0, st, pdl,
-                   reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(w_router),
-                   reinterpret_cast<const uint4*>(scale), T, H, E, eps, router_root(H),
-                   logits);
+  const uint32_t rb = __bfloat16_as_ushort(__float2bfloat16_rn(router_root(H)));
+  const uint32_t root2 = rb | (rb << 16);
+  // experts per CTA: the fewest n8 tiles that cover E, at most 16 (grid.y
+  // takes the rest); with few token tiles, fewer, so that the weight rows
+  // stream through more SMs
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int nt = E <= 8 ? 1 : E <= 16 ? 2 : E <= 32 ? 4 : E <= 64 ? 8 : 16;
+  const int64_t tiles_t = (T + kRtTokens - 1) / kRtTokens;
+  while (nt > 1 && tiles_t * ((E + 8 * nt - 1) / (8 * nt)) <= sms / 2) nt >>= 1;
+  switch (nt) {
+    case 1: return launch_router_nt<1>(x, w_router, scale, T, H, E, eps, root2, logits, st, pdl);
+    case 2: return launch_router_nt<2>(x, w_router, scale, T, H, E, eps, root2, logits, st, pdl);
+    case 4: return launch_router_nt<4>(x, w_router, scale, T, H, E, eps, root2, logits, st, pdl);
+    case 8: return launch_router_nt<8>(x, w_router, scale, T, H, E, eps, root2, logits, st, pdl);
+    default:
+      return launch_router_nt<16>(x, w_router, scale, T, H, E, eps, root2, logits, st, pdl);
+  }
 }
 
 }  // namespace moe
