@@ -114,12 +114,20 @@ __host__ __device__ constexpr int rt_stages(int NT) {
              : (int)(kRtRingMax / ((uint32_t)rt_rows(NT) * kRtPitch));
 }
 
+// Norm-pass ring depth: the same shared memory cut into slots of the 64
+// token rows alone, at most 6.
+__host__ __device__ constexpr int rt_norm_stages(int NT) {
+  return rt_stages(NT) * rt_rows(NT) / kRtTokens > 6 ? 6
+                                                       : rt_stages(NT) * rt_rows(NT) / kRtTokens;
+}
+
 // NT n8 tiles: the CTA's 8 NT experts (<= 128).  The CTA runs 2 nkb jobs
-// through a ring of rt_stages(NT) shared-memory slots filled with 16-byte
-// asynchronous copies, up to S - 1 jobs ahead: job j < nkb stages K-block j
-// of the token rows, whose squares the norm pass sums; job nkb + kb stages
-// K-block kb of the expert rows, the token rows (again, now from L2) and
-// the scale, which the projection multiplies.  Only rows that exist are
+// through shared memory filled with 16-byte asynchronous copies: the norm
+// pass stages K-block j of the token rows into a ring of rt_norm_stages(NT)
+// slots, up to Q - 1 blocks ahead, and sums their squares; the projection
+// stages K-block kb of the expert rows, the token rows (again, now from L2)
+// and the scale into a ring of rt_stages(NT) larger slots over the same
+// memory, up to S - 1 blocks ahead.  Only rows that exist are
 // copied; columns past H are filled with zeros, so the ragged K tail adds
 // nothing.  Rows past T or E of a slot hold stale data: a token row past T
 // enters the MMA as zeros, and an expert row past E only feeds its own
@@ -135,9 +143,13 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
   constexpr uint32_t BLK = (uint32_t)rt_rows(NT) * kRtPitch;
   constexpr int XR = EB;               // first token row of a slot
   constexpr int SR = EB + kRtTokens;   // the scale row
+  constexpr int Q = rt_norm_stages(NT);
+  static_assert(Q >= 2, "the norm ring needs two slots");
+  constexpr uint32_t NB = (uint32_t)kRtTokens * kRtPitch;  // one norm slot
   static_assert(kRtGroups * NT * 4 * 32 * 4 <= BLK, "the K-half partial sums fit in a slot");
   extern __shared__ __align__(16) uint8_t ring[];  // [S][rt_rows(NT)][kRtPitch]
   __shared__ float inv_s[kRtTokens];
+  __shared__ double part_s[kRtTokens];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = lane & 3;
   const int64_t t0 = (int64_t)blockIdx.x * kRtTokens;
@@ -146,34 +158,61 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
   const int ne = min(EB, E - e0);                                   // expert rows of the CTA
   const int nkb = (H + kRtKB - 1) / kRtKB;
   const uint32_t ring0 = smem_u32(ring);
-  // thread t stages 16-byte vector t % 32 of rows t / 32, t / 32 + 8, ...
+  // thread t stages 16-byte vector t % 32 of rows t / 32, t / 32 + 8, ...;
+  // a vector past H is a zero fill whose source is the row's start
   const int sv = tid & 31, sr0 = tid >> 5;
-  auto stage = [&](int j) {
-    if (j < 2 * nkb) {
-      const bool proj = j >= nkb;
-      const int kb = proj ? j - nkb : j;
-      const int col = kb * kRtKB + sv * 8;
-      const bool ok = col < H;
+  const __nv_bfloat16* const xs = x + (t0 + sr0) * H;
+  const __nv_bfloat16* const ws = w + (int64_t)(e0 + sr0) * H;
+  const int64_t rstep = (int64_t)kRtWarps * H;
+  // token rows of K-block kb into the slot at dst (rows from row0 on)
+  auto stage_x = [&](int kb, uint32_t dst, int row0) {
+    const bool ok = kb * kRtKB + sv * 8 < H;
+    const uint32_t nbytes = ok ? 16u : 0u;
+    uint32_t d = dst + (uint32_t)(row0 + sr0) * kRtPitch + (uint32_t)sv * 16;
+    const __nv_bfloat16* src = xs + (ok ? kb * kRtKB + sv * 8 : 0);
+    for (int r = sr0; r < nt; r += kRtWarps, d += kRtWarps * kRtPitch, src += rstep)
+      cp_async16(d, src, nbytes);
+  };
+  // Norm job j -> norm slot j % Q.  With R = the least power of two >= nt,
+  // one job holds m = 64 / R K-blocks: block j m + p in rows [p R, p R + nt).
+  // One group per job, empty past the last.
+  int R = kRtTokens;
+  while (R > 1 && nt <= R / 2) R >>= 1;
+  const int m = kRtTokens / R;
+  const int nnj = (nkb + m - 1) / m;
+  auto stage_n = [&](int j) {
+    if (j < nnj)
+      for (int p = 0; p < m && j * m + p < nkb; ++p)
+        stage_x(j * m + p, ring0 + (uint32_t)(j % Q) * NB, p * R);
+    cp_async_commit();
+  };
+  // projection job kb -> slot kb % S
+  auto stage_p = [&](int kb) {
+    if (kb < nkb) {
+      const uint32_t dst = ring0 + (uint32_t)(kb % S) * BLK;
+      stage_x(kb, dst, XR);
+      const bool ok = kb * kRtKB + sv * 8 < H;
       const uint32_t nbytes = ok ? 16u : 0u;
-      const int cc = ok ? col : 0;
-      const uint32_t base = ring0 + (uint32_t)(j % S) * BLK + (uint32_t)sv * 16;
-      for (int r = sr0; r < nt; r += kRtWarps)
-        cp_async16(base + (uint32_t)(XR + r) * kRtPitch, x + (t0 + r) * H + cc, nbytes);
-      if (proj) {
-        for (int r = sr0; r < ne; r += kRtWarps)
-          cp_async16(base + (uint32_t)r * kRtPitch, w + (int64_t)(e0 + r) * H + cc, nbytes);
-        if (sr0 == 0) cp_async16(base + (uint32_t)SR * kRtPitch, scale + cc, nbytes);
-      }
+      const int cc = ok ? kb * kRtKB + sv * 8 : 0;
+      uint32_t d = dst + (uint32_t)sr0 * kRtPitch + (uint32_t)sv * 16;
+      const __nv_bfloat16* src = ws + cc;
+      for (int r = sr0; r < ne; r += kRtWarps, d += kRtWarps * kRtPitch, src += rstep)
+        cp_async16(d, src, nbytes);
+      if (sr0 == 0)
+        cp_async16(dst + (uint32_t)SR * kRtPitch + (uint32_t)sv * 16, scale + cc, nbytes);
     }
-    cp_async_commit();  // one group per job, empty past the last
+    cp_async_commit();
   };
 #pragma unroll
-  for (int p = 0; p < S - 1; ++p) stage(p);
+  for (int p = 0; p < Q - 1; ++p) stage_n(p);
 
-  // norm pass: lane l of warp w sums row 8w + l / 4, vectors l % 4 + 4i
+  // norm pass: lane l of warp w sums slot row nr = 8w + l / 4 -- token nr % R
+  // of the job's block nr / R -- vectors l % 4 + 4i
   const int nr = warp * 8 + (lane >> 2);
-  const bool nr_ok = nr < nt;
-  double ss = 0.0;
+  const bool nr_ok = nr % R < nt;
+  double ss[8];  // one partial sum per vector slot: eight independent chains
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss[i] = 0.0;
   // projection: warp w multiplies token rows 16 (w % 4) + g and + g + 8 over
   // chunks [4 (w / 4), 4 (w / 4) + 4) of each K-block
   const int tg = warp & (kRtGroups - 1), kh = warp / kRtGroups;
@@ -187,41 +226,55 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
     for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
   const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
 
-  for (int j = 0; j < 2 * nkb; ++j) {
-    stage(j + S - 1);
-    cp_async_wait<S - 1>();  // job j has landed (this thread's copies)
+  // ---- step 1: sum of squares, in double
+  for (int j = 0; j < nnj; ++j) {
+    stage_n(j + Q - 1);
+    cp_async_wait<Q - 1>();  // job j has landed (this thread's copies)
     __syncthreads();         // ... and everyone's
-    const uint32_t slot = ring0 + (uint32_t)(j % S) * BLK;
-    if (j < nkb) {
-      // ---- step 1: sum of squares, in double
-      if (nr_ok) {
-        const uint32_t row = slot + (uint32_t)(XR + nr) * kRtPitch + (uint32_t)(lane & 3) * 16;
+    if (nr_ok && j * m + nr / R < nkb) {
+      const uint32_t row = ring0 + (uint32_t)(j % Q) * NB + (uint32_t)nr * kRtPitch +
+                           (uint32_t)(lane & 3) * 16;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = rt_lds128(row + i * 64);
-          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = rt_lds128(row + i * 64);
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const double lo = bf_lo(wd[u]), hi = bf_hi(wd[u]);
-            ss = fma(lo, lo, ss);
-            ss = fma(hi, hi, ss);
-          }
+        for (int u = 0; u < 4; ++u) {
+          const double lo = bf_lo(wd[u]), hi = bf_hi(wd[u]);
+          ss[i] = fma(lo, lo, ss[i]);
+          ss[i] = fma(hi, hi, ss[i]);
         }
       }
-      if (j == nkb - 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        if ((lane & 3) == 0 && nr_ok) {
-          const float var = (float)(ss / (double)H);
-          inv_s[nr] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
-        }
-        __syncthreads();  // rows of other warps
-        if (va) inv_a = inv_s[ra];
-        if (vb) inv_b = inv_s[rb];
-      }
-    } else if (live) {
-      // ---- steps 2-4 on this warp's half of K-block kb
-      const int kb = j - nkb;
+    }
+    __syncthreads();  // norm slot j % Q is refilled by job j + Q
+  }
+  // the projection's first blocks stream while the normalisers are formed
+#pragma unroll
+  for (int p = 0; p < S - 1; ++p) stage_p(p);
+  {
+    double sum = ((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7]));
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    if ((lane & 3) == 0) part_s[nr] = sum;
+    __syncthreads();
+    // token r: its m partial sums in order of the block
+    if (tid < nt) {
+      double tot = 0.0;
+      for (int p = 0; p < m; ++p) tot += part_s[p * R + tid];
+      const float var = (float)(tot / (double)H);
+      inv_s[tid] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
+    }
+    __syncthreads();
+    if (va) inv_a = inv_s[ra];
+    if (vb) inv_b = inv_s[rb];
+  }
+  // ---- steps 2-4: this warp's half of each K-block
+  for (int kb = 0; kb < nkb; ++kb) {
+    stage_p(kb + S - 1);
+    cp_async_wait<S - 1>();
+    __syncthreads();
+    const uint32_t slot = ring0 + (uint32_t)(kb % S) * BLK;
+    if (live) {
       const int ch_end = min(4 * kh + 4, (H - kb * kRtKB + 31) / 32);
       const uint32_t xa = slot + (uint32_t)(XR + ra) * kRtPitch;
       const uint32_t xb = xa + 8 * kRtPitch;
@@ -239,7 +292,7 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
         }
       }
     }
-    __syncthreads();  // slot j % S is refilled by job j + S
+    __syncthreads();  // slot kb % S is refilled by block kb + S
   }
   cp_async_wait<0>();
   // ---- the two K-halves: the second half's tiles go through slot 0 (free
