@@ -25,6 +25,15 @@
 // decode_w13 the 4 warps of a CTA split K (H is long) and add their partial
 // sums through shared memory; in decode_w2 each warp owns 16 rows and all of
 // K (I is short).
+//
+// With at most 8 tokens (one B tile) the kernels take their "few" form: the
+// weights stream through a per-warp ring of shared-memory slots filled with
+// 16-byte cp.async copies several chunks ahead, so a lane keeps 5-7 chunks
+// in flight without holding them in registers (the register-prefetch form
+// holds one or two and is bound by DRAM latency at this size).  Each lane
+// reads back only the bytes it copied itself, so the ring needs no barrier.
+// decode_w13 also asks L2 for the w2 rows of its expert when the touched
+// w2 set is small, and decode_w2 starts its ring before it waits for h.
 #include <algorithm>
 
 #include "route_impl.cuh"
@@ -48,6 +57,31 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
                : "memory");
+}
+
+// L2 policy for weights that are read once: evict them first, so that what
+// is read again (the w2 rows asked for early, the token rows) stays.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte global -> shared copy that skips L1; when !valid nothing is read
+// and the 16 bytes are zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid,
+                                           uint64_t pol) {
+  asm volatile(
+      "cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+      "l"(src), "r"(valid ? 16 : 0), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -172,24 +206,21 @@ __device__ __forceinline__ bool load_group(const int32_t* meta, int G, int idx,
   return true;
 }
 
-// NTMAX: token tiles kept in registers per pass (8 -> up to 64 tokens of an
-// expert at once; 1 -> up to 8, which frees registers for a deeper weight
-// prefetch: two 32-column chunks ahead instead of one, and lets the token
-// rows sit in shared memory).
-template <int NTMAX>
-__global__ void __launch_bounds__(kDecThreads, NTMAX == 1 ? 3 : 4)
+// The many-token form (T > 8): NTMAX token tiles kept in registers per pass
+// (up to 64 tokens of a group at once), weights loaded one 32-column chunk
+// ahead into registers.
+__global__ void __launch_bounds__(kDecThreads, 4)
 decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
                   const __nv_bfloat16* __restrict__ w13,
                   const __nv_bfloat16* __restrict__ w13_sh,
                   const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
                   int T, int H, int I, int E, int k, int S, int act,
                   __nv_bfloat16* __restrict__ h_dec) {
+  constexpr int NTMAX = kDecNT;
   constexpr int PASS = NTMAX * 8;
-  constexpr int AHEAD = NTMAX == 1 ? 2 : 1;
   __shared__ int32_t tok_s[PASS];
   __shared__ int32_t slot_s[PASS];
   __shared__ float red[4][NTMAX][32][8];
-  extern __shared__ __align__(16) uint4 xs[];  // NTMAX == 1: [8][H/8] token rows
   pdl_wait();  // routing (meta, slots) comes from decode_route
   pdl_trigger();
   DecGroup grp;
@@ -227,29 +258,15 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
     const int np = min(PASS, grp.n - p0);
     const int NT = (np + 7) >> 3;
     __syncthreads();
-    // weights of the next AHEAD chunks are requested before a chunk is
-    // multiplied (the first ones before the token rows are even looked up)
-    W4 q0 = load_w(ch0), q1, q2;
-    if (AHEAD >= 2) q1 = load_w(ch0 + 1);
-    if (AHEAD >= 3) q2 = load_w(ch0 + 2);
+    // the next chunk's weights are requested before a chunk is multiplied
+    // (the first ones before the token rows are even looked up)
+    W4 q0 = load_w(ch0);
     for (int i = threadIdx.x; i < np; i += kDecThreads) {
       const int s = slots[grp.base + p0 + i];
       slot_s[i] = s;
       tok_s[i] = s < R ? s / k : (s - R) % T;
     }
     __syncthreads();
-    if (NTMAX == 1) {
-      // the (at most 8) token rows of x, staged once: no L2 round trip per
-      // chunk in the loop below
-      const int hv = H >> 3;
-      for (int i = threadIdx.x; i < 8 * hv; i += kDecThreads) {
-        const int tk = i / hv, cc = i - tk * hv;
-        xs[i] = tk < np ? __ldg(reinterpret_cast<const uint4*>(x) +
-                                (int64_t)tok_s[tk] * hv + cc)
-                        : z4;
-      }
-      __syncthreads();
-    }
     float ag[NTMAX][4], au[NTMAX][4];
 #pragma unroll
     for (int nt = 0; nt < NTMAX; ++nt)
@@ -259,27 +276,15 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
       const int col = ch * 32 + 8 * c;
       const bool vc = col < H;
       const W4 cur = q0;
-      if (AHEAD == 1) {
-        q0 = load_w(ch + 1);
-      } else if (AHEAD == 2) {
-        q0 = q1;
-        q1 = load_w(ch + 2);
-      } else {
-        q0 = q1;
-        q1 = q2;
-        q2 = load_w(ch + 3);
-      }
+      q0 = load_w(ch + 1);
 #pragma unroll
       for (int nt = 0; nt < NTMAX; ++nt) {
         if (nt < NT) {
           const int tk = nt * 8 + gq;
-          uint4 xv;
-          if (NTMAX == 1)
-            xv = vc ? xs[gq * (H >> 3) + (col >> 3)] : z4;  // zero rows past np
-          else
-            xv = (tk < np && vc)
-                ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)tok_s[tk] * H + col))
-                : z4;
+          const uint4 xv =
+              (tk < np && vc)
+                  ? __ldg(reinterpret_cast<const uint4*>(x + (int64_t)tok_s[tk] * H + col))
+                  : z4;
           mma_chunk(ag[nt], cur.ga, cur.gb, xv);
           mma_chunk(au[nt], cur.ua, cur.ub, xv);
         }
@@ -323,7 +328,6 @@ decode_w13_kernel(const __nv_bfloat16* __restrict__ x,
 // two 32-column chunks ahead of the MMAs.
 constexpr int kW2Rows = 64;
 
-template <int NTMAX>
 __global__ void __launch_bounds__(kDecThreads, 4)
 decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const __nv_bfloat16* __restrict__ w2,
@@ -331,9 +335,9 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
                  const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
                  const float* __restrict__ wgt, int T, int H, int I, int E, int k,
                  int S, float* __restrict__ stage) {
+  constexpr int NTMAX = kDecNT;
   constexpr int PASS = NTMAX * 8;
   __shared__ int32_t slot_s[PASS];
-  extern __shared__ __align__(16) uint4 hs[];  // NTMAX == 1: [8][I/8] h rows
   // This kernel is launched once every decode_w13 block has passed its own
   // wait for the routing, so the expert lists are final here: the weight rows
   // of this block are pulled into L2 while decode_w13 still streams its own.
@@ -374,16 +378,6 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
     for (int i = threadIdx.x; i < np; i += kDecThreads)
       slot_s[i] = slots[grp.base + p0 + i];
     __syncthreads();
-    if (NTMAX == 1) {
-      const int iv = I >> 3;
-      for (int i = threadIdx.x; i < 8 * iv; i += kDecThreads) {
-        const int tk = i / iv, cc = i - tk * iv;
-        hs[i] = tk < np ? __ldg(reinterpret_cast<const uint4*>(h_dec) +
-                                (int64_t)slot_s[tk] * iv + cc)
-                        : z4;
-      }
-      __syncthreads();
-    }
     float acc[NTMAX][4];
 #pragma unroll
     for (int nt = 0; nt < NTMAX; ++nt)
@@ -403,13 +397,10 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
       for (int nt = 0; nt < NTMAX; ++nt) {
         if (nt < NT) {
           const int tk = nt * 8 + gq;
-          uint4 hv;
-          if (NTMAX == 1)
-            hv = vc ? hs[gq * (I >> 3) + (col >> 3)] : z4;
-          else
-            hv = (tk < np && vc)
-                ? __ldg(reinterpret_cast<const uint4*>(h_dec + (int64_t)slot_s[tk] * I + col))
-                : z4;
+          const uint4 hv =
+              (tk < np && vc)
+                  ? __ldg(reinterpret_cast<const uint4*>(h_dec + (int64_t)slot_s[tk] * I + col))
+                  : z4;
           mma_chunk(acc[nt], wa, wb, hv);
         }
       }
@@ -442,6 +433,235 @@ decode_w2_kernel(const __nv_bfloat16* __restrict__ h_dec,
   }
 }
 
+
+// ---- the few-token form (T <= 8: one B tile, one pass per group) ----
+
+// ring slots per warp (D - 1 chunks in flight) and the shared memory of each
+// kernel: the rings, then the token rows (min(T, 8) rows of x or of h)
+constexpr int kW13Ring = 6;
+constexpr int kW2Ring = 8;
+__host__ __device__ constexpr size_t w13_ring_bytes() { return 4u * kW13Ring * 4 * 512; }
+__host__ __device__ constexpr size_t w2_ring_bytes() { return 4u * kW2Ring * 2 * 512; }
+
+// One CTA per (touched group, 16 rows of I), as decode_w13_kernel, with the
+// gate and up rows streamed through the warp's ring: slot j holds the four
+// 16-byte pieces (gate rows g, g+8; up rows g, g+8) of a lane at
+// [(j * 4 + part) * 32 + lane], so a warp's reads of one part are
+// contiguous.  w2_l2 != 0: ask L2 for each touched group's w2 block, split
+// over the CTAs of the group (set only when those blocks fit in L2 together).
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
+                      const __nv_bfloat16* __restrict__ w13,
+                      const __nv_bfloat16* __restrict__ w13_sh,
+                      const __nv_bfloat16* __restrict__ w2,
+                      const __nv_bfloat16* __restrict__ w2_sh,
+                      const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
+                      int T, int H, int I, int E, int k, int S, int act, int w2_l2,
+                      __nv_bfloat16* __restrict__ h_dec) {
+  __shared__ int32_t tok_s[8];
+  __shared__ int32_t slot_s[8];
+  __shared__ float red[4][32][8];
+  extern __shared__ __align__(16) uint4 dyn[];
+  pdl_wait();  // routing (meta, slots) comes from decode_route
+  pdl_trigger();
+  DecGroup grp;
+  if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
+  const int R = T * k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (w2_l2 > 0 && warp == 0) {
+    // this CTA's share of the group's w2 block, in pieces of <= 32 KB
+    const __nv_bfloat16* W2 = grp.g < E ? w2 + (int64_t)grp.g * H * I
+                                        : w2_sh + (int64_t)(grp.g - E) * H * I;
+    const uint32_t total = (uint32_t)H * I * 2;
+    const uint32_t per = ((total + gridDim.y - 1) / gridDim.y + 15) & ~15u;
+    const uint32_t b0 = blockIdx.y * per;
+    const uint32_t b1 = min(total, b0 + per);
+    for (uint32_t o = b0 + lane * 32768u; o < b1; o += 32u * 32768u)
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(W2) + o, min(32768u, b1 - o));
+  }
+  const __nv_bfloat16* W = grp.g < E ? w13 + (int64_t)grp.g * 2 * I * H
+                                     : w13_sh + (int64_t)(grp.g - E) * 2 * I * H;
+  const int i0 = blockIdx.y * kDecRows;
+  const int gq = lane >> 2, c = lane & 3;
+  const int nch = (H + 31) / 32;
+  const int ch0 = warp * nch / 4, ch1 = (warp + 1) * nch / 4;
+  const int ra = i0 + gq, rb = i0 + gq + 8;  // gate rows; up rows are +I
+  const bool va = ra < I, vb = rb < I;
+  // rows past I are zero-filled from a valid address (nothing is read)
+  const __nv_bfloat16* pga = W + (int64_t)(va ? ra : 0) * H;
+  const __nv_bfloat16* pgb = W + (int64_t)(vb ? rb : 0) * H;
+  const __nv_bfloat16* pua = W + (int64_t)(I + (va ? ra : 0)) * H;
+  const __nv_bfloat16* pub = W + (int64_t)(I + (vb ? rb : 0)) * H;
+  const uint64_t pol = evict_first_policy();
+  uint4* ring = dyn + warp * (D * 4 * 32);
+  const uint32_t ring_s = smem_u32(ring + lane);
+  auto issue = [&](int ch, int slot) {
+    if (ch < ch1) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = col < H;
+      const int cc = vc ? col : 0;
+      const uint32_t d = ring_s + (uint32_t)slot * 4 * 512;
+      cp_async16(d, pga + cc, va && vc, pol);
+      cp_async16(d + 512, pgb + cc, vb && vc, pol);
+      cp_async16(d + 1024, pua + cc, va && vc, pol);
+      cp_async16(d + 1536, pub + cc, vb && vc, pol);
+    }
+    cp_async_commit();  // empty groups past the end keep the count uniform
+  };
+#pragma unroll
+  for (int j = 0; j < D - 1; ++j) issue(ch0 + j, j);
+
+  const int np = grp.n;  // <= T <= 8
+  if (threadIdx.x < np) {
+    const int s = slots[grp.base + threadIdx.x];
+    slot_s[threadIdx.x] = s;
+    tok_s[threadIdx.x] = s < R ? s / k : (s - R) % T;
+  }
+  __syncthreads();
+  const int hv = H >> 3;
+  uint4* xs = dyn + 4 * (D * 4 * 32);  // [np][H/8]
+  for (int i = threadIdx.x; i < np * hv; i += kDecThreads) {
+    const int tk = i / hv, cc = i - tk * hv;
+    xs[i] = __ldg(reinterpret_cast<const uint4*>(x) + (int64_t)tok_s[tk] * hv + cc);
+  }
+  __syncthreads();
+
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+  int slot = 0;
+  for (int ch = ch0; ch < ch1; ++ch) {
+    cp_async_wait<D - 2>();  // chunk ch has landed (this lane's pieces)
+    // refill the slot read in the previous iteration, whose values the MMAs
+    // there have already consumed
+    issue(ch + D - 1, slot == 0 ? D - 1 : slot - 1);
+    const uint4* q = ring + slot * 4 * 32;
+    const uint4 ga = q[lane], gb = q[32 + lane], ua = q[64 + lane], ub = q[96 + lane];
+    const int col = ch * 32 + 8 * c;
+    const uint4 xv = (gq < np && col < H) ? xs[gq * hv + (col >> 3)] : z4;
+    mma_chunk(ag, ga, gb, xv);
+    mma_chunk(au, ua, ub, xv);
+    slot = slot == D - 1 ? 0 : slot + 1;
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    red[warp][lane][e] = ag[e];
+    red[warp][lane][4 + e] = au[e];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // fragment element e: row gq (+8 for e >= 2), token 2c + (e & 1)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float g = red[0][lane][e] + red[1][lane][e] + red[2][lane][e] + red[3][lane][e];
+      const float u = red[0][lane][4 + e] + red[1][lane][4 + e] + red[2][lane][4 + e] +
+                      red[3][lane][4 + e];
+      const int row = i0 + gq + (e >= 2 ? 8 : 0);
+      const int tk = 2 * c + (e & 1);
+      if (row < I && tk < np)
+        h_dec[(int64_t)slot_s[tk] * I + row] = __float2bfloat16_rn(dec_act(act, g) * u);
+    }
+  }
+}
+
+// One CTA per (touched group, 64 rows of H), as decode_w2_kernel, with the
+// w2 rows streamed through the warp's ring (slot j: [(j * 2 + part) * 32 +
+// lane], parts = rows g and g+8).  The weights do not depend on the previous
+// kernel, so the ring is started before the wait for h.
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+decode_w2_few_kernel(const __nv_bfloat16* __restrict__ h_dec,
+                     const __nv_bfloat16* __restrict__ w2,
+                     const __nv_bfloat16* __restrict__ w2_sh,
+                     const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
+                     const float* __restrict__ wgt, int T, int H, int I, int E, int k,
+                     int S, float* __restrict__ stage) {
+  __shared__ int32_t slot_s[8];
+  extern __shared__ __align__(16) uint4 dyn[];
+  // Launched once every decode_w13 block has passed its own wait for the
+  // routing, so the group lists are final here.
+  DecGroup grp;
+  const bool live = load_group(meta, E + S, blockIdx.x, &grp);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, c = lane & 3;
+  const int r0 = blockIdx.y * kW2Rows + warp * kDecRows;
+  const int nch = (I + 31) / 32;
+  const int ra = r0 + gq, rb = r0 + gq + 8;
+  const bool va = ra < H, vb = rb < H;
+  const __nv_bfloat16* W = nullptr;
+  const __nv_bfloat16 *pa = nullptr, *pb = nullptr;
+  uint4* ring = dyn + warp * (D * 2 * 32);
+  const uint32_t ring_s = smem_u32(ring + lane);
+  const uint64_t pol = evict_first_policy();
+  auto issue = [&](int ch, int slot) {
+    if (ch < nch) {
+      const int col = ch * 32 + 8 * c;
+      const bool vc = col < I;
+      const int cc = vc ? col : 0;
+      const uint32_t d = ring_s + (uint32_t)slot * 2 * 512;
+      cp_async16(d, pa + cc, va && vc, pol);
+      cp_async16(d + 512, pb + cc, vb && vc, pol);
+    }
+    cp_async_commit();
+  };
+  if (live) {
+    W = grp.g < E ? w2 + (int64_t)grp.g * H * I : w2_sh + (int64_t)(grp.g - E) * H * I;
+    pa = W + (int64_t)(va ? ra : 0) * I;
+    pb = W + (int64_t)(vb ? rb : 0) * I;
+#pragma unroll
+    for (int j = 0; j < D - 1; ++j) issue(j, j);
+  }
+  pdl_wait();  // h_dec comes from decode_w13
+  pdl_trigger();
+  if (!live) return;
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  const int R = T * k, ks = k + S;
+  const int np = grp.n;  // <= T <= 8
+  if (threadIdx.x < np) slot_s[threadIdx.x] = slots[grp.base + threadIdx.x];
+  __syncthreads();
+  const int iv = I >> 3;
+  uint4* hs = dyn + 4 * (D * 2 * 32);  // [np][I/8]
+  for (int i = threadIdx.x; i < np * iv; i += kDecThreads) {
+    const int tk = i / iv, cc = i - tk * iv;
+    hs[i] = __ldg(reinterpret_cast<const uint4*>(h_dec) + (int64_t)slot_s[tk] * iv + cc);
+  }
+  __syncthreads();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int slot = 0;
+  for (int ch = 0; ch < nch; ++ch) {
+    cp_async_wait<D - 2>();
+    issue(ch + D - 1, slot == 0 ? D - 1 : slot - 1);
+    const uint4* q = ring + slot * 2 * 32;
+    const uint4 wa = q[lane], wb = q[32 + lane];
+    const int col = ch * 32 + 8 * c;
+    const uint4 hv = (gq < np && col < I) ? hs[gq * iv + (col >> 3)] : z4;
+    mma_chunk(acc, wa, wb, hv);
+    slot = slot == D - 1 ? 0 : slot + 1;
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int row = r0 + gq + (e >= 2 ? 8 : 0);
+    const int tk = 2 * c + (e & 1);
+    if (row < H && tk < np) {
+      const int s = slot_s[tk];
+      int64_t dst;
+      float wt;
+      if (s < R) {
+        const int t = s / k;
+        dst = (int64_t)t * ks + (s - t * k);
+        wt = __ldg(wgt + s);
+      } else {
+        const int q = s - R, sh = q / T;
+        dst = (int64_t)(q - sh * T) * ks + k + sh;
+        wt = 1.0f;
+      }
+      stage[dst * H + row] = __fmul_rn(wt, acc[e]);
+    }
+  }
+}
+
 }  // namespace
 
 size_t decode_meta_ints(int G) { return 2 + 2 * (size_t)G; }
@@ -460,33 +680,51 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   const int max_groups = (R < a.E ? R : a.E) + a.S;
-  // every expert (and shared expert) has at most T tokens: with T <= 8 the
-  // token rows of x and of h fit in shared memory
-  const bool few = a.T <= 8;
-  auto w13k = few ? decode_w13_kernel<1> : decode_w13_kernel<kDecNT>;
-  auto w2k = few ? decode_w2_kernel<1> : decode_w2_kernel<kDecNT>;
-  const size_t xs_bytes = few ? (size_t)8 * a.H * 2 : 0;
-  const size_t hs_bytes = few ? (size_t)8 * a.I * 2 : 0;
-  // dynamic + static shared memory above 48 KiB needs the opt-in
+  // every expert (and shared expert) has at most T tokens: with T <= 8 one
+  // B tile holds them all, and the ring kernels keep those token rows in
+  // shared memory next to the rings
+  const int nx = a.T < 8 ? a.T : 8;
+  const size_t w13_smem = w13_ring_bytes() + (size_t)nx * a.H * 2;
+  const size_t w2_smem = w2_ring_bytes() + (size_t)nx * a.I * 2;
+  const bool few = a.T <= 8 && w13_smem <= 200 * 1024 && w2_smem <= 200 * 1024;
   if (few) {
+    auto w13k = decode_w13_few_kernel<kW13Ring>;
+    auto w2k = decode_w2_few_kernel<kW2Ring>;
+    // dynamic shared memory above 48 KiB needs the opt-in
     if ((e = cudaFuncSetAttribute(w13k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)xs_bytes)) != cudaSuccess)
+                                  (int)w13_smem)) != cudaSuccess)
       return e;
     if ((e = cudaFuncSetAttribute(w2k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)hs_bytes)) != cudaSuccess)
+                                  (int)w2_smem)) != cudaSuccess)
       return e;
+    // the w2 blocks of the touched groups are asked for early when they fit
+    // in a third of L2 together (32 MB: 8 experts at H=2816, I=704)
+    const double w2_set = (double)max_groups * a.H * a.I * 2;
+    const int w2_l2 = w2_set <= 32.0 * (1 << 20) ? 1 : 0;
+    e = launch_ex(w13k, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
+                  dim3(kDecThreads), w13_smem, st, true, a.x, a.w13, a.w13_sh, a.w2,
+                  a.w2_sh, (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H,
+                  a.I, a.E, a.k, a.S, a.act, w2_l2, a.h_dec);
+    if (e != cudaSuccess) return e;
+    if (!mark(4)) return cudaErrorUnknown;
+    e = launch_ex(w2k, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
+                  dim3(kDecThreads), w2_smem, st, true, (const __nv_bfloat16*)a.h_dec,
+                  a.w2, a.w2_sh, (const int32_t*)a.meta, (const int32_t*)a.slots,
+                  (const float*)a.w, a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
+    if (e != cudaSuccess) return e;
+  } else {
+    e = launch_ex(decode_w13_kernel, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
+                  dim3(kDecThreads), 0, st, true, a.x, a.w13, a.w13_sh,
+                  (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
+                  a.k, a.S, a.act, a.h_dec);
+    if (e != cudaSuccess) return e;
+    if (!mark(4)) return cudaErrorUnknown;
+    e = launch_ex(decode_w2_kernel, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
+                  dim3(kDecThreads), 0, st, true, (const __nv_bfloat16*)a.h_dec, a.w2,
+                  a.w2_sh, (const int32_t*)a.meta, (const int32_t*)a.slots,
+                  (const float*)a.w, a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
+    if (e != cudaSuccess) return e;
   }
-  e = launch_ex(w13k, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
-                 dim3(kDecThreads), xs_bytes, st, true, a.x, a.w13, a.w13_sh,
-                 (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
-                 a.k, a.S, a.act, a.h_dec);
-  if (e != cudaSuccess) return e;
-  if (!mark(4)) return cudaErrorUnknown;
-  e = launch_ex(w2k, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
-                 dim3(kDecThreads), hs_bytes, st, true, (const __nv_bfloat16*)a.h_dec, a.w2, a.w2_sh,
-                 (const int32_t*)a.meta, (const int32_t*)a.slots, (const float*)a.w,
-                 a.T, a.H, a.I, a.E, a.k, a.S, a.stage);
-  if (e != cudaSuccess) return e;
   if (!mark(5)) return cudaErrorUnknown;
   e = launch_sum_rows(a.stage, a.T, a.k + a.S, a.H, a.out, a.out_f32, st,
                       /*pdl=*/true);

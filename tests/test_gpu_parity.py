@@ -38,6 +38,13 @@ SMALL = {
     "single_expert": (inputs.Shape(T=19, H=64, E=1, k=1, I=64), "zero", "uniform"),
     "k_equals_E": (inputs.Shape(T=33, H=64, E=4, k=4, I=32, act=1), "zero", "uniform"),
     "one_token": (inputs.Shape(T=1, H=128, E=8, k=2, I=128), "zero", "uniform"),
+    # T <= 8 on the decode path: the ring form of the skinny kernels, with a
+    # K tail in both products (H % 32, I % 32), a partial 16-row block of I
+    # and a partial 64-row block of H, and shared experts
+    "few_ragged": (inputs.Shape(T=3, H=200, E=5, k=3, I=104, act=1), "zero",
+                   "uniform"),
+    "few_shared": (inputs.Shape(T=8, H=136, E=6, k=2, I=88, n_shared=2,
+                                I_shared=88), "zero", "ones"),
     "gemma_shapes_T130": (inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),
                           "zero", "uniform"),
     "wide_tiles": (inputs.Shape(T=300, H=520, E=3, k=2, I=392), "normal0.5", "uniform"),
@@ -218,7 +225,8 @@ def test_repeat_calls_are_bit_identical(api, variant):
 
 
 @pytest.mark.parametrize("variant", ["prefill_det", "prefill_pairs_det", "decode"])
-@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_shapes_T130"])
+@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_shapes_T130",
+                                  "few_ragged"])
 def test_stale_workspace_changes_nothing(api, name, variant):
     # Padding rows of the gathered activations and of h are never written;
     # each MMA row depends on its own A row only, so whatever they hold may
