@@ -11,8 +11,9 @@
 // B200:
 //
 //   * persistent: one 192-thread CTA per SM walks the tile list
-//     (expert-major, then n-tile, then m-tile, so the CTAs running at once
-//     share weight tiles through L2);
+//     (expert-major, then panels of 16 m-tiles, then n-tile, then m-tile,
+//     so the CTAs running at once share weight and activation tiles
+//     through L2);
 //   * warp 0 lane 0 is the TMA producer: 128x64 A tiles and 256x64 B tiles
 //     (mode 0: 128 gate rows + the matching 128 up rows) into a 4-stage ring
 //     of 128-byte-swizzled shared memory;
@@ -44,6 +45,7 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN_ACC;
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kMaxStages = 6;
+constexpr int kPanel = 16;  // m-blocks per panel of the tile order
 
 // CG = CTAs per MMA: 1 (M=128 per CTA, B tile 256 rows per CTA, 4 stages) or
 // 2 (a CTA pair computes M=256: each CTA loads its own 128 A rows and half of
@@ -97,8 +99,12 @@ struct KParams {
 };
 
 // A work unit is (group g, block of CG m-tiles, n-tile); units are ordered
-// group-major, then n-tile, then m-block, so the CTAs running at once share
-// B tiles through L2.  ub[g] = units of the groups before g.
+// group-major, then by panels of kPanel m-blocks, then n-tile, then m-block
+// inside the panel.  The CTAs running at once share B tiles through L2, and
+// a group with many m-tiles (a popular expert, a shared expert) is swept a
+// panel at a time, so the A rows they re-read for every n-tile stay in L2
+// too (kPanel m-tiles, instead of all of the group's).  ub[g] = units of the
+// groups before g.
 struct Tile {
   int g;
   int64_t row0;  // first row of this CTA's m-tile
@@ -119,8 +125,12 @@ __device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs,
   const int64_t mtg = (offs[lo + 1] - offs[lo]) / BM;
   const int64_t mbg = (mtg + CG - 1) / CG;
   const int64_t local = i - ub[lo];
-  const int64_t nt = local / mbg;
-  const int64_t mt = (local - nt * mbg) * CG + rank;
+  const int64_t panel = local / ((int64_t)kPanel * NT);
+  const int64_t p0 = panel * kPanel;                          // first m-block
+  const int64_t pw = mbg - p0 < kPanel ? mbg - p0 : kPanel;   // m-blocks in it
+  const int64_t in = local - panel * kPanel * NT;
+  const int64_t nt = in / pw;
+  const int64_t mt = (p0 + in - nt * pw) * CG + rank;
   return Tile{lo, offs[lo] + mt * BM, (int)nt * BN_OUT, mt < mtg};
 }
 

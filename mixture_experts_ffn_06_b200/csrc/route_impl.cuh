@@ -11,7 +11,8 @@
 // Lane l holds logits e = l, l+32, ... (PER per lane, E <= 32 PER; at most
 // 16 for E <= 512).  Each of the k rounds is a warp-wide argmax under
 // (larger logit, then lower id), so ids come out in the order of a stable
-// descending sort.  The weights are formed in fp64 and rounded once to fp32.
+// descending sort.  The argmax compares order-preserving integer keys of the
+// fp32 logits, which rank them exactly as the float comparison does.  The weights are formed in fp64 and rounded once to fp32.
 // PER is a template parameter so that a round scans only the entries that
 // exist (measured on B200: scanning 16 per lane with E = 128 and k = 8 took
 // the prefill route kernel 28 us instead of 22 on 8192 tokens).
@@ -21,16 +22,24 @@
 
 namespace moe {
 
-// true if (va, ia) precedes (vb, ib): larger value, ties to the lower id.
-// NaN never precedes anything, so a NaN logit is chosen only when nothing
-// else is left (it still yields a valid id).
-__device__ __forceinline__ bool route_precedes(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
+// Order-preserving key of a logit: a larger key is a larger value.  -0 is
+// keyed as +0 (the two compare equal, so the lower id wins the tie) and NaN
+// as 0, below every number: a NaN logit is chosen only when nothing else is
+// left (it still yields a valid id).
+__device__ __forceinline__ uint32_t route_key(float v) {
+  if (v != v) return 0u;
+  if (v == 0.0f) v = 0.0f;
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Routes token row z[0..E) with the calling warp (E <= 32 PER).  Lane j < k
 // returns the j-th choice in (*id, *wt); the other lanes return id 0,
 // weight 0.
+//
+// Each round, every lane takes its best untaken entry, and two warp
+// reductions (redux.sync) pick the winner: the largest key, then the lowest
+// id among the lanes holding it.
 template <int PER = kMaxExperts / 32>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
                                                  const float* __restrict__ scale,
@@ -38,40 +47,39 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
   constexpr int kPerLane = PER;
   const int lane = threadIdx.x & 31;
   float v[kPerLane];
+  uint32_t key[kPerLane];
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? __ldg(z + e) : -INFINITY;
+    v[i] = (e < E) ? __ldg(z + e) : 0.f;
+    key[i] = route_key(v[i]);
   }
-  uint32_t taken = 0;  // bit i: expert lane+32i already chosen
+  // bit i: entry lane + 32 i is not (or no longer) a candidate
+  uint32_t gone = 0;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i)
+    if (lane + 32 * i >= E) gone |= 1u << i;
   float my_v = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    // best untaken entry of this lane: larger key, then lower id (lower i)
+    uint32_t bk = 0;
+    int bi = -1;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u)) {
-        if (bi == 0x7fffffff || route_precedes(v[i], e, bv, bi)) {
-          bv = v[i];
-          bi = e;
-        }
+      if (!((gone >> i) & 1u) && (bi < 0 || key[i] > bk)) {
+        bk = key[i];
+        bi = i;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || route_precedes(ov, oi, bv, bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const uint32_t cand = (bi >= 0 && bk == kmax) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+    const int win = (int)__reduce_min_sync(0xffffffffu, cand);
+    if ((win & 31) == lane) gone |= 1u << (win >> 5);
     if (lane == j) {
-      my_v = bv;
-      my_id = bi;
+      my_id = win;
+      // the winner's value from its key (NaN for key 0)
+      my_v = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax);
     }
   }
   const float zmax = __shfl_sync(0xffffffffu, my_v, 0);

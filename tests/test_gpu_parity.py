@@ -350,3 +350,27 @@ def test_prefill_full_size(api, name, det, pairs):
     tok = _cover_tokens(ids_ref, shp.E, extra=6, seed=1)
     want_out, _, _ = oracle_forward(inp, tokens=tok)
     assert_out_close(out32[torch.from_numpy(tok).cuda()], want_out, name)
+
+
+@pytest.mark.parametrize("E,k", [(5, 3), (128, 8), (64, 6), (512, 32), (40, 32)])
+def test_route_ties_and_signed_zeros(api, E, k):
+    # Logits drawn from a handful of values, so that most rows hold exact ties
+    # (-0.0 and +0.0 among them, which compare equal): the ids must follow
+    # (larger logit, then lower id) and the weights the oracle's.
+    gen = torch.Generator().manual_seed(E * 100 + k)
+    T = 300
+    vals = torch.tensor([-1.5, -0.0, 0.0, 0.25, 0.25, 2.0, -3.0],
+                        dtype=torch.float32)
+    z = vals[torch.randint(0, len(vals), (T, E), generator=gen)]
+    z[0] = 0.0
+    z[1] = -0.0
+    z[2, ::2] = -0.0
+    z[2, 1::2] = 0.0
+    s = api.make_shape(T=T, H=64, E=E, k=k, I=64)
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    api.moe_route(s, z.cuda(), None, ids, w)
+    torch.cuda.synchronize()
+    ids_ref, w_ref = oracle.route(z.numpy(), k)
+    assert (ids.cpu().numpy() == ids_ref).all()
+    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-6, atol=0)
