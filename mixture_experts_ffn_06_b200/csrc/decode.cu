@@ -484,8 +484,9 @@ decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
                                      : w13_sh + (int64_t)(grp.g - E) * 2 * I * H;
   const int i0 = blockIdx.y * kDecRows;
   const int gq = lane >> 2, c = lane & 3;
+  // warp w takes the 32-column chunks w, w + 4, ...: the four warps read
+  // 256 contiguous bytes of each weight row at a time
   const int nch = (H + 31) / 32;
-  const int ch0 = warp * nch / 4, ch1 = (warp + 1) * nch / 4;
   const int ra = i0 + gq, rb = i0 + gq + 8;  // gate rows; up rows are +I
   const bool va = ra < I, vb = rb < I;
   // rows past I are zero-filled from a valid address (nothing is read)
@@ -496,8 +497,9 @@ decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
   const uint64_t pol = evict_first_policy();
   uint4* ring = dyn + warp * (D * 4 * 32);
   const uint32_t ring_s = smem_u32(ring + lane);
-  auto issue = [&](int ch, int slot) {
-    if (ch < ch1) {
+  auto issue = [&](int i, int slot) {  // the warp's i-th chunk
+    const int ch = warp + 4 * i;
+    if (ch < nch) {
       const int col = ch * 32 + 8 * c;
       const bool vc = col < H;
       const int cc = vc ? col : 0;
@@ -510,7 +512,7 @@ decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
     cp_async_commit();  // empty groups past the end keep the count uniform
   };
 #pragma unroll
-  for (int j = 0; j < D - 1; ++j) issue(ch0 + j, j);
+  for (int j = 0; j < D - 1; ++j) issue(j, j);
 
   const int np = grp.n;  // <= T <= 8
   if (threadIdx.x < np) {
@@ -530,11 +532,11 @@ decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
   const uint4 z4 = make_uint4(0, 0, 0, 0);
   float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
   int slot = 0;
-  for (int ch = ch0; ch < ch1; ++ch) {
+  for (int i = 0, ch = warp; ch < nch; ++i, ch += 4) {
     cp_async_wait<D - 2>();  // chunk ch has landed (this lane's pieces)
     // refill the slot read in the previous iteration, whose values the MMAs
     // there have already consumed
-    issue(ch + D - 1, slot == 0 ? D - 1 : slot - 1);
+    issue(i + D - 1, slot == 0 ? D - 1 : slot - 1);
     const uint4* q = ring + slot * 4 * 32;
     const uint4 ga = q[lane], gb = q[32 + lane], ua = q[64 + lane], ub = q[96 + lane];
     const int col = ch * 32 + 8 * c;

@@ -50,11 +50,16 @@ constexpr int kPanel = 16;  // m-blocks per panel of the tile order
 // CG = CTAs per MMA: 1 (M=128 per CTA, B tile 256 rows per CTA, 4 stages) or
 // 2 (a CTA pair computes M=256: each CTA loads its own 128 A rows and half of
 // the 256 B rows, so a stage is 32 KiB instead of 48 KiB and 6 fit).
-template <int CG>
+// NH (mode 0, CG = 1): gate rows per tile.  128 gives N = 256; 88 gives
+// N = 176 (88 gate + 88 up rows), which tiles I = 704 (the Gemma-4 expert
+// width) without the half-empty last n-tile of the 128-row form, and with a
+// 38 KiB stage 5 stages fit.
+template <int CG, int NH = 128>
 struct Cfg {
-  static constexpr int B_ROWS = BN_ACC / CG;        // B rows loaded per CTA
+  static constexpr int B_ROWS = NH == 128 ? BN_ACC / CG : 2 * NH;  // B rows per CTA
   static constexpr int B_STAGE = B_ROWS * BK * 2;
-  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int STAGES = CG == 2 ? 6 : (NH == 128 ? 4 : 5);
+  static constexpr int N_MMA = NH == 128 ? BN_ACC : 2 * NH;         // MMA N
 };
 
 struct Ctl {
@@ -96,6 +101,7 @@ struct KParams {
   const float* w;               // modes 2, 3
   int64_t T;                    // modes 2, 3
   int k, S;                     // modes 2, 3
+  int a_sh_x;                   // shared groups' A rows come from tmAs (x)
 };
 
 // A work unit is (group g, block of CG m-tiles, n-tile); units are ordered
@@ -112,11 +118,11 @@ struct Tile {
   bool valid;    // this CTA's m-tile lies inside the group's segment
 };
 
-template <int MODE, int CG>
+template <int MODE, int CG, int NH = 128>
 __device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs,
                                          const int64_t* ub, int G, int NT,
                                          uint32_t rank) {
-  constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
+  constexpr int BN_OUT = MODE == 0 ? NH : BN_ACC;
   int lo = 0, hi = G - 1;  // last g with ub[g] <= i
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -145,12 +151,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int NH = 128>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmAs,
                     const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmBs, const KParams p) {
-  using C = Cfg<CG>;
+  static_assert(NH == 128 || (MODE == 0 && CG == 1 && NH % 8 == 0 && NH < 128),
+                "narrow gate tiles are a mode-0, single-CTA form");
+  using C = Cfg<CG, NH>;
   constexpr int STAGES = C::STAGES;
   constexpr int B_STAGE = C::B_STAGE;
   extern __shared__ uint8_t smem_raw[];
@@ -183,6 +192,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     ctl->abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmAs);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmBs);
   }
@@ -236,9 +246,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int s = 0; s < STAGES; ++s) last_fill[s] = -1;
       bool ok = true;
       for (int64_t t = unit0; ok && t < total; t += unit_step) {
-        const Tile tl = map_tile<MODE, CG>(t, offs, ub, p.G, p.NT, rank);
+        const Tile tl = map_tile<MODE, CG, NH>(t, offs, ub, p.G, p.NT, rank);
         const bool routed = tl.g < p.E;
         const CUtensorMap* mb = routed ? &tmB : &tmBs;
+        // a shared expert's segment holds tokens 0..T-1 in order: with
+        // a_sh_x its A rows are read from the token rows themselves
+        const bool ax = !routed && p.a_sh_x;
+        const CUtensorMap* ma = ax ? &tmAs : &tmA;
+        const int32_t arow = (int32_t)(ax ? tl.row0 - offs[tl.g] : tl.row0);
         const int32_t gl = routed ? tl.g : tl.g - p.E;
         // B rows this CTA loads: mode 0 -- gate rows then up rows (CG = 1),
         // or CTA 0 the gate rows and CTA 1 the up rows (CG = 2); otherwise
@@ -254,7 +269,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           if (CG == 1) {
             mbar_expect_tx(fb, A_STAGE + B_STAGE);
-            tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0, fb);
+            tma_load_2d(sA + stage * A_STAGE, ma, kb * BK, arow, fb);
             if (MODE == 0) {
               tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
               tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * BK,
@@ -266,8 +281,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             // both CTAs' bytes complete on CTA 0's full barrier
             if (rank == 0) mbar_expect_tx(fb, 2 * (A_STAGE + B_STAGE));
             const uint32_t fb0 = fb & kPeerBitMask;
-            tma_load_2d_pair(sA + stage * A_STAGE, &tmA, kb * BK, (int32_t)tl.row0,
-                             fb0);
+            tma_load_2d_pair(sA + stage * A_STAGE, ma, kb * BK, arow, fb0);
             tma_load_2d_pair(sB + stage * B_STAGE, mb, kb * BK, brow, fb0);
           }
           last_fill[stage] = (int32_t)phase;
@@ -288,7 +302,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // --------------------------------------------------------- MMA issuer
     // (CTA 0 of the pair issues for both when CG = 2)
     if (lane == 0 && (CG == 1 || rank == 0)) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN_ACC);
+      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, C::N_MMA);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int64_t t = unit0; ok && t < total; t += unit_step) {
@@ -358,7 +372,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t empty1 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[1]), 0) : 0u;
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = unit0; t < total; t += unit_step) {
-      const Tile tl = map_tile<MODE, CG>(t, offs, ub, p.G, p.NT, rank);
+      const Tile tl = map_tile<MODE, CG, NH>(t, offs, ub, p.G, p.NT, rank);
       if (MODE <= 1) {
         // 1: a real row.  Padding rows (only in a segment's last tile) feed
         // nothing: mode 0 leaves them as they are (-1), mode 1 writes zeros
@@ -398,12 +412,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
       const int64_t wrow0 = tl.row0 + q * 32;  // first tile row of this warp
-      constexpr int CHUNKS = MODE == 0 ? 4 : 8;
+      constexpr int CHUNKS = MODE == 0 ? (NH + 31) / 32 : 8;
 #pragma unroll 1
       for (int c = 0; c < CHUNKS; ++c) {
         const int col0 = tl.n0 + c * 32;
         if (col0 >= p.N) break;
-        if (MODE == 0) {
+        if (MODE == 0 && NH == 128) {
           uint32_t g[32], u[32];
           tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
           if (!tl.valid) continue;  // the pair's empty half: nothing to store
@@ -411,6 +425,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int j = 0; j < 32; ++j)
             tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) *
                             __uint_as_float(u[j]);
+        } else if (MODE == 0) {
+          // gate columns [32c, 32c + 32); the matching up column NH + 32c + j
+          // lies in the 32-column chunk starting at 32 (NH / 32 + c) or in
+          // the next one, so every TMEM load starts at a multiple of 32
+          // columns (all of them inside this accumulator's 256)
+          constexpr int UQ = NH / 32, UR = NH % 32;
+          uint32_t g[32], u0[32], u1[32];
+          tmem_ld32x2(tb + c * 32, tb + (UQ + c) * 32, g, u0);
+          tmem_ld32(tb + (UQ + c + 1) * 32, u1);
+          if (!tl.valid) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t uj = j + UR < 32 ? u0[j + UR] : u1[j + UR - 32];
+            tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) * __uint_as_float(uj);
+          }
         } else {
           uint32_t y[32];
           tmem_ld32(tb + c * 32, y);
@@ -427,7 +456,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int i = 0; i < 4; ++i) {
             const int r = i * 8 + (lane >> 2);
             const int64_t rd = epi->rdst[q][r];
-            if (col0 + cc < p.N && rd > 0) {
+            if (col0 + cc < p.N && c * 32 + cc < NH && rd > 0) {
               uint4 o;
               o.x = pack_bf16x2(tbuf[r][cc + 0], tbuf[r][cc + 1]);
               o.y = pack_bf16x2(tbuf[r][cc + 2], tbuf[r][cc + 3]);
@@ -547,17 +576,24 @@ int num_sms() {
   return n;
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int NH = 128>
 cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
-  using C = Cfg<CG>;
-  constexpr int BN_OUT = MODE == 0 ? BN_ACC / 2 : BN_ACC;
-  CUtensorMap mA, mB, mBs;
+  using C = Cfg<CG, NH>;
+  constexpr int BN_OUT = MODE == 0 ? NH : BN_ACC;
+  CUtensorMap mA, mAs, mB, mBs;
   cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM);
   if (e != cudaSuccess) return e;
+  const bool a_sh_x = a.A_sh != nullptr && a.G > a.E && a.T > 0;
+  if (a_sh_x) {
+    e = make_map(&mAs, a.A_sh, (uint64_t)a.K, (uint64_t)a.T, BM);
+    if (e != cudaSuccess) return e;
+  } else {
+    mAs = mA;
+  }
   const uint64_t rows_per_group = MODE == 0 ? 2ull * a.N : (uint64_t)a.N;
-  // per-CTA B box: mode 0 loads 128 gate (and 128 up) rows; the others 256
+  // per-CTA B box: mode 0 loads NH gate (and NH up) rows; the others 256
   // rows, or 128 per CTA of a pair
-  const uint32_t box_rows = MODE == 0 ? BN_ACC / 2 : (uint32_t)C::B_ROWS;
+  const uint32_t box_rows = MODE == 0 ? NH : (uint32_t)C::B_ROWS;
   e = make_map(&mB, a.B, (uint64_t)a.K, rows_per_group * (uint64_t)a.E, box_rows);
   if (e != cudaSuccess) return e;
   if (a.B_sh && a.G > a.E) {
@@ -586,13 +622,14 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   p.T = a.T;
   p.k = a.k;
   p.S = a.G - a.E;
+  p.a_sh_x = a_sh_x ? 1 : 0;
 
   const size_t smem = 1024 + (size_t)C::STAGES * (A_STAGE + C::B_STAGE) +
                       sizeof(EpiSmem) + sizeof(Ctl) +
                       (sizeof(int64_t) + sizeof(int32_t)) * (size_t)(a.G + 1);
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG>,
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, NH>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024);
     if (e != cudaSuccess) return e;
@@ -623,7 +660,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG>, mA, mB, mBs, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, NH>, mA, mAs, mB, mBs, p);
 }
 
 __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
@@ -645,8 +682,18 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool 
   // CTA pairs when the experts' segments are large enough that most m-blocks
   // hold two full m-tiles; single CTAs for few rows per expert (decode-sized)
   const bool pair = a.pair;
+  // w13 with I a multiple of 88 but not of 128 (I = 704): 176-row B tiles
+  // cover the gate and up halves exactly, so no weight row is streamed for
+  // nothing.  Only below the ridge point (under 256 rows per expert, where
+  // the product is bound by streaming the weights): measured on B200, an
+  // N = 176 MMA costs the tensor-bound many-small batch 10 % on w13, and
+  // saves 5-7 % of the step at 16-256 tokens.
+  const int64_t rows = a.T * a.k + a.T * (int64_t)(a.G - a.E);
+  const bool narrow = a.N % 128 != 0 && a.N % 88 == 0 && rows < 256 * (int64_t)a.G;
   switch (a.mode) {
-    case 0: return pair ? launch_mode<0, 2>(a, st, pdl) : launch_mode<0, 1>(a, st, pdl);
+    case 0:
+      return pair ? launch_mode<0, 2>(a, st, pdl)
+                  : narrow ? launch_mode<0, 1, 88>(a, st, pdl) : launch_mode<0, 1>(a, st, pdl);
     case 1: return pair ? launch_mode<1, 2>(a, st, pdl) : launch_mode<1, 1>(a, st, pdl);
     case 2: return pair ? launch_mode<2, 2>(a, st, pdl) : launch_mode<2, 1>(a, st, pdl);
     case 3: return pair ? launch_mode<3, 2>(a, st, pdl) : launch_mode<3, 1>(a, st, pdl);

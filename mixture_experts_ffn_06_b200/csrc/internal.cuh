@@ -69,8 +69,9 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
                           cudaStream_t st, bool pdl = false);
 
-// Gathers x rows into x_perm (padding rows are left as they are); when acc
-// is given it also zeroes acc[0, n_acc) (n_acc % 4 == 0).
+// Gathers x rows into x_perm for the rows of groups [0, G) (padding rows are
+// left as they are); when acc is given it also zeroes acc[0, n_acc)
+// (n_acc % 4 == 0).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
                           int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
@@ -126,6 +127,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
 struct GroupedGemmArgs {
   int mode;
   const __nv_bfloat16* A;       // [cap, K]
+  const __nv_bfloat16* A_sh;    // [T, K] A rows of the shared groups (segment row
+                                // i is token i), or nullptr: those rows are in A
   const __nv_bfloat16* B;       // routed experts' weights
   const __nv_bfloat16* B_sh;    // shared experts' weights (or nullptr)
   const int32_t* offsets;       // [G+1]

@@ -117,7 +117,9 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   auto* h = reinterpret_cast<__nv_bfloat16*>(at(ws, m.h));
   auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
   if (!mark(ev, 2, st)) return MOE_ERR_CUDA;
-  cudaError_t e = launch_gather(x, sorted_slots, offsets, G, s.T, s.k, s.H, m.cap,
+  // the shared experts' segments hold tokens 0..T-1 in order: the w13 GEMM
+  // reads their A rows from x itself, so only the routed rows are gathered
+  cudaError_t e = launch_gather(x, sorted_slots, offsets, s.E, s.T, s.k, s.H, m.cap,
                                 x_perm, combine == 2 ? y_perm : nullptr,
                                 s.T * (int64_t)s.H, st, pdl);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -125,6 +127,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   GroupedGemmArgs a{};
   a.mode = 0;
   a.A = x_perm;
+  a.A_sh = x;
   a.B = w13;
   a.B_sh = w13_sh;
   a.offsets = offsets;
@@ -152,6 +155,7 @@ static moe_status run_expert_ffn(const moe_shape& s, const __nv_bfloat16* x,
   a.mode = combine == 0 ? 1 : combine;
   a.pair = cta_pairs == 2 || (cta_pairs == 0 && big && s.I >= 1024);
   a.A = h;
+  a.A_sh = nullptr;  // h holds the shared groups' rows too
   a.B = w2;
   a.B_sh = w2_sh;
   a.N = s.H;

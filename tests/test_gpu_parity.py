@@ -47,6 +47,10 @@ SMALL = {
                                 I_shared=88), "zero", "ones"),
     "gemma_shapes_T130": (inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),
                           "zero", "uniform"),
+    # I a multiple of 88 but not of 128: the w13 GEMM runs its 176-row
+    # (88 gate + 88 up) B tiles, here with a K tail (H = 72)
+    "narrow_w13": (inputs.Shape(T=90, H=72, E=3, k=2, I=264), "normal0.5",
+                   "uniform"),
     "wide_tiles": (inputs.Shape(T=300, H=520, E=3, k=2, I=392), "normal0.5", "uniform"),
     # T*k >= 256*E: the grouped GEMMs run on CTA pairs (M = 256), with odd
     # m-tile counts per expert, K and N tails, and shared experts
