@@ -549,7 +549,8 @@ def run_ours(args):
             achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
             peak = float(peaks["hbm_gbs"])
             roof = {"bound": "hbm",
-                    "kernel": "decode_w13_kernel (w13 + act)" if decode
+                    "kernel": ("decode_w13_few_kernel (w13 + act)" if shp.T <= 8
+                               else "decode_w13_kernel (w13 + act)") if decode
                     else "grouped_gemm_kernel<0> (w13 + activation)",
                     "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak,
@@ -569,7 +570,7 @@ def run_ours(args):
                     "layer_frac": shp.flops() / (ms_per_step / 1e3) / 1e12 / peak}
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
         # our kernels per step: prefill route, layout x4, gather, 2 GEMMs,
-        # row sum; decode route, w13, w2, row sum
+        # rounding; decode route, w13, w2, row sum
         launches_per_step = 4 if decode else 9
         cpu = None
         if world == 1 and not args.profile:

@@ -32,8 +32,7 @@
 // in flight without holding them in registers (the register-prefetch form
 // holds one or two and is bound by DRAM latency at this size).  Each lane
 // reads back only the bytes it copied itself, so the ring needs no barrier.
-// decode_w13 also asks L2 for the w2 rows of its expert when the touched
-// w2 set is small, and decode_w2 starts its ring before it waits for h.
+// decode_w2 starts its ring before it waits for h.
 #include <algorithm>
 
 #include "route_impl.cuh"
@@ -447,17 +446,14 @@ __host__ __device__ constexpr size_t w2_ring_bytes() { return 4u * kW2Ring * 2 *
 // gate and up rows streamed through the warp's ring: slot j holds the four
 // 16-byte pieces (gate rows g, g+8; up rows g, g+8) of a lane at
 // [(j * 4 + part) * 32 + lane], so a warp's reads of one part are
-// contiguous.  w2_l2 != 0: ask L2 for each touched group's w2 block, split
-// over the CTAs of the group (set only when those blocks fit in L2 together).
+// contiguous.
 template <int D>
 __global__ void __launch_bounds__(kDecThreads)
 decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
                       const __nv_bfloat16* __restrict__ w13,
                       const __nv_bfloat16* __restrict__ w13_sh,
-                      const __nv_bfloat16* __restrict__ w2,
-                      const __nv_bfloat16* __restrict__ w2_sh,
                       const int32_t* __restrict__ meta, const int32_t* __restrict__ slots,
-                      int T, int H, int I, int E, int k, int S, int act, int w2_l2,
+                      int T, int H, int I, int E, int k, int S, int act,
                       __nv_bfloat16* __restrict__ h_dec) {
   __shared__ int32_t tok_s[8];
   __shared__ int32_t slot_s[8];
@@ -469,17 +465,6 @@ decode_w13_few_kernel(const __nv_bfloat16* __restrict__ x,
   if (!load_group(meta, E + S, blockIdx.x, &grp)) return;
   const int R = T * k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (w2_l2 > 0 && warp == 0) {
-    // this CTA's share of the group's w2 block, in pieces of <= 32 KB
-    const __nv_bfloat16* W2 = grp.g < E ? w2 + (int64_t)grp.g * H * I
-                                        : w2_sh + (int64_t)(grp.g - E) * H * I;
-    const uint32_t total = (uint32_t)H * I * 2;
-    const uint32_t per = ((total + gridDim.y - 1) / gridDim.y + 15) & ~15u;
-    const uint32_t b0 = blockIdx.y * per;
-    const uint32_t b1 = min(total, b0 + per);
-    for (uint32_t o = b0 + lane * 32768u; o < b1; o += 32u * 32768u)
-      prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(W2) + o, min(32768u, b1 - o));
-  }
   const __nv_bfloat16* W = grp.g < E ? w13 + (int64_t)grp.g * 2 * I * H
                                      : w13_sh + (int64_t)(grp.g - E) * 2 * I * H;
   const int i0 = blockIdx.y * kDecRows;
@@ -699,14 +684,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
     if ((e = cudaFuncSetAttribute(w2k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)w2_smem)) != cudaSuccess)
       return e;
-    // the w2 blocks of the touched groups are asked for early when they fit
-    // in a third of L2 together (32 MB: 8 experts at H=2816, I=704)
-    const double w2_set = (double)max_groups * a.H * a.I * 2;
-    const int w2_l2 = w2_set <= 32.0 * (1 << 20) ? 1 : 0;
     e = launch_ex(w13k, dim3(max_groups, (a.I + kDecRows - 1) / kDecRows),
-                  dim3(kDecThreads), w13_smem, st, true, a.x, a.w13, a.w13_sh, a.w2,
-                  a.w2_sh, (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H,
-                  a.I, a.E, a.k, a.S, a.act, w2_l2, a.h_dec);
+                  dim3(kDecThreads), w13_smem, st, true, a.x, a.w13, a.w13_sh,
+                  (const int32_t*)a.meta, (const int32_t*)a.slots, a.T, a.H, a.I, a.E,
+                  a.k, a.S, a.act, a.h_dec);
     if (e != cudaSuccess) return e;
     if (!mark(4)) return cudaErrorUnknown;
     e = launch_ex(w2k, dim3(max_groups, (a.H + kW2Rows - 1) / kW2Rows),
