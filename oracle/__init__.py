@@ -65,9 +65,12 @@ def _load():
                                        P, P, P]
         lib.oracle_router_logits.argtypes = [i64, i32, i32, ctypes.c_double, P, P,
                                              P, P]
+        lib.oracle_route_ex.argtypes = [i64, i32, i32, P, P, i32, i32, i32, P, P]
+        lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [i32, i32, i32]
         for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
                   lib.oracle_expert_rows, lib.oracle_forward,
-                  lib.oracle_router_logits):
+                  lib.oracle_router_logits, lib.oracle_route_ex,
+                  lib.oracle_forward_ex):
             f.restype = i32
         _lib = lib
     return _lib
@@ -126,6 +129,23 @@ def route(logits, k: int, scale=None, want_probs: bool = False):
     return (ids, w, probs) if want_probs else (ids, w)
 
 
+SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
+
+
+def route_ex(logits, k: int, scale=None, scoring: int = SCORE_SOFTMAX,
+             n_group: int = 1, topk_group: int = 1):
+    """Routing variants (sigmoid scoring, expert groups) -> ids [T,k] int32,
+    w [T,k] float64."""
+    z = _f32(logits)
+    T, E = z.shape
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    sc = _f32(scale)
+    _check(_load().oracle_route_ex(T, E, k, _ptr(z), _ptr(sc), scoring, n_group,
+                                   topk_group, _ptr(ids), _ptr(w)), "route_ex")
+    return ids, w
+
+
 def layout_capacity(T: int, E: int, k: int, S: int = 0, P: int = 128) -> int:
     return int(_load().oracle_layout_capacity(T, E, k, S, P))
 
@@ -177,8 +197,10 @@ def router_logits(x, w_router, scale, eps: float) -> np.ndarray:
 
 def forward(x, logits, w13, w2, k: int, act_kind: int, scale=None,
             w13_sh=None, w2_sh=None, tokens=None, round_h: bool = False,
-            nthreads: int = 0):
-    """Whole layer in fp64 -> (out [n,H] float64, ids [T,k], w [T,k])."""
+            nthreads: int = 0, scoring: int = SCORE_SOFTMAX, n_group: int = 1,
+            topk_group: int = 1):
+    """Whole layer in fp64 -> (out [n,H] float64, ids [T,k], w [T,k]).
+    scoring / n_group / topk_group select the routing of route_ex."""
     xu, w13u, w2u = _u16(x), _u16(w13), _u16(w2)
     z = _f32(logits)
     T, H = xu.shape
@@ -193,9 +215,10 @@ def forward(x, logits, w13, w2, k: int, act_kind: int, scale=None,
     ids = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
     sc = _f32(scale)
-    _check(_load().oracle_forward(T, H, E, k, I, act_kind, S, Is, _ptr(xu),
-                                  _ptr(z), _ptr(sc), _ptr(w13u), _ptr(w2u),
-                                  _ptr(sh13), _ptr(sh2), _ptr(tok), n,
-                                  int(round_h), nthreads, _ptr(out),
-                                  _ptr(ids), _ptr(w)), "forward")
+    _check(_load().oracle_forward_ex(T, H, E, k, I, act_kind, S, Is, _ptr(xu),
+                                     _ptr(z), _ptr(sc), _ptr(w13u), _ptr(w2u),
+                                     _ptr(sh13), _ptr(sh2), _ptr(tok), n,
+                                     int(round_h), nthreads, _ptr(out),
+                                     _ptr(ids), _ptr(w), scoring, n_group,
+                                     topk_group), "forward")
     return out, ids, w

@@ -30,6 +30,8 @@
  *              page).  Act is SiLU, v/(1+e^-v), or the tanh GELU,
  *              0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))) (walkthrough
  *              section 6).
+ *   route_ex -- llama-cpp-visual-guide lesson 35: sigmoid scoring and expert
+ *              groups (see oracle_route_ex).
  *   combine -- walkthrough section 7 step 4: the k expert outputs of a token
  *              are summed weighted by its (scale-folded) gate weights; shared
  *              experts (llama-cpp-visual-guide lesson 35, "shared expert")
@@ -208,6 +210,110 @@ int oracle_route(int64_t T, int E, int k, const float* logits,
   return rc;
 }
 
+/* Descending group score; equal scores go to the lower group id first. */
+typedef struct {
+  float v;
+  int g;
+} group_score;
+
+static int cmp_group_desc(const void* a, const void* b) {
+  const group_score* x = (const group_score*)a;
+  const group_score* y = (const group_score*)b;
+  if (x->v > y->v) return -1;
+  if (x->v < y->v) return 1;
+  return (x->g > y->g) - (x->g < y->g);
+}
+
+/*
+ * Routing variants of llama-cpp-visual-guide lesson 35 (routing section and
+ * the shared-expert / expert-group fold):
+ *   scoring 0 -- probabilities are the softmax over all E logits (the
+ *                listing's ggml_soft_max), exactly oracle_route;
+ *   scoring 1 -- probabilities are sigmoid(logit) per expert (the listing's
+ *                "some models use sigmoid");
+ *   n_group > 1 -- the E experts form n_group groups of E / n_group
+ *                consecutive ids; a token first picks its topk_group best
+ *                groups, then its k experts among the experts of those
+ *                groups ("pick a group first, then experts within it").
+ *                A group's score is the best probability among its experts
+ *                (reading: the page does not say how a group is scored).
+ * Then, as in the listing: top-k of the probabilities (ties to the lower
+ * id), the k probabilities gathered and normalised to sum 1, and (section 5
+ * of the Gemma 4 walkthrough) times per_expert_scale[id].  Sigmoid and
+ * softmax are increasing in the logit, so the probabilities are ranked by
+ * comparing the fp32 logits themselves (exact).
+ * Returns -1 on bad sizes (E % n_group, topk_group out of range, fewer than
+ * k experts in topk_group groups) or a non-finite logit.
+ */
+int oracle_route_ex(int64_t T, int E, int k, const float* logits,
+                    const float* scale, int scoring, int n_group,
+                    int topk_group, int32_t* ids, double* w) {
+  if (n_group < 1) n_group = 1;
+  if (n_group == 1) topk_group = 1;
+  if (T < 0 || E < 1 || k < 1 || k > E || (scoring != 0 && scoring != 1))
+    return EINVAL_ARG;
+  if (E % n_group != 0 || topk_group < 1 || topk_group > n_group ||
+      k > topk_group * (E / n_group))
+    return EINVAL_ARG;
+  const int gs = E / n_group;
+  logit_id* pairs = (logit_id*)malloc(sizeof(logit_id) * E);
+  group_score* gsc = (group_score*)malloc(sizeof(group_score) * n_group);
+  int* keep = (int*)malloc(sizeof(int) * n_group);
+  double* p = (double*)malloc(sizeof(double) * E);
+  if (!pairs || !gsc || !keep || !p) {
+    free(pairs); free(gsc); free(keep); free(p);
+    return ENOMEM_ARG;
+  }
+  int rc = OK;
+  for (int64_t t = 0; t < T && rc == OK; ++t) {
+    const float* z = logits + t * E;
+    for (int e = 0; e < E; ++e)
+      if (!isfinite(z[e])) { rc = EINVAL_ARG; break; }
+    if (rc != OK) break;
+    /* probabilities of every expert */
+    if (scoring == 0) {
+      double zmax = (double)z[0], den = 0.0;
+      for (int e = 1; e < E; ++e) if ((double)z[e] > zmax) zmax = (double)z[e];
+      for (int e = 0; e < E; ++e) { p[e] = exp((double)z[e] - zmax); den += p[e]; }
+      for (int e = 0; e < E; ++e) p[e] /= den;
+    } else {
+      for (int e = 0; e < E; ++e) p[e] = 1.0 / (1.0 + exp(-(double)z[e]));
+    }
+    /* groups: each scored by its best member, the topk_group best kept */
+    for (int g = 0; g < n_group; ++g) {
+      float best = z[g * gs];
+      for (int i = 1; i < gs; ++i) if (z[g * gs + i] > best) best = z[g * gs + i];
+      gsc[g].v = best;
+      gsc[g].g = g;
+      keep[g] = 0;
+    }
+    qsort(gsc, (size_t)n_group, sizeof(group_score), cmp_group_desc);
+    for (int i = 0; i < topk_group; ++i) keep[gsc[i].g] = 1;
+    /* top-k among the experts of the kept groups */
+    int n = 0;
+    for (int e = 0; e < E; ++e) {
+      if (!keep[e / gs]) continue;
+      pairs[n].v = z[e];
+      pairs[n].id = e;
+      ++n;
+    }
+    qsort(pairs, (size_t)n, sizeof(logit_id), cmp_logit_desc);
+    /* gather the k probabilities and normalise them to sum 1 */
+    double sum = 0.0;
+    for (int j = 0; j < k; ++j) sum += p[pairs[j].id];
+    if (!(sum > 0.0)) sum = 1.0;
+    for (int j = 0; j < k; ++j) {
+      const int id = pairs[j].id;
+      double wt = p[id] / sum;
+      if (scale) wt *= (double)scale[id];
+      ids[t * k + j] = id;
+      w[t * k + j] = wt;
+    }
+  }
+  free(pairs); free(gsc); free(keep); free(p);
+  return rc;
+}
+
 /* ---------------------------------------------------------------- layout */
 
 /* Rows the permuted buffers need in the worst case:
@@ -379,19 +485,25 @@ static void fwd_worker(void* p, int64_t b, int64_t e) {
  *   out[r,:] = sum_j w[t,j] * FFN_{ids[t,j]}(x_t) + sum_s FFN_shared_s(x_t)
  * Routing is done for all T tokens; ids_out/w_out (NULL ok) receive it.
  */
-int oracle_forward(int64_t T, int H, int E, int k, int I, int act, int S,
-                   int Is, const uint16_t* x, const float* logits,
-                   const float* scale, const uint16_t* w13,
-                   const uint16_t* w2, const uint16_t* w13_sh,
-                   const uint16_t* w2_sh, const int64_t* tokens,
-                   int64_t n_tokens, int round_h, int nthreads, double* out,
-                   int32_t* ids_out, double* w_out) {
+/* oracle_forward with the routing of oracle_route_ex (scoring, expert
+ * groups); scoring 0 with one group is oracle_forward itself. */
+int oracle_forward_ex(int64_t T, int H, int E, int k, int I, int act, int S,
+                      int Is, const uint16_t* x, const float* logits,
+                      const float* scale, const uint16_t* w13,
+                      const uint16_t* w2, const uint16_t* w13_sh,
+                      const uint16_t* w2_sh, const int64_t* tokens,
+                      int64_t n_tokens, int round_h, int nthreads, double* out,
+                      int32_t* ids_out, double* w_out, int scoring, int n_group,
+                      int topk_group) {
   if (T < 0 || H < 1 || I < 1 || S < 0 || (S > 0 && (Is < 1 || !w13_sh || !w2_sh)))
     return EINVAL_ARG;
   int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (T * k + 1));
   double* w = w_out ? w_out : (double*)malloc(sizeof(double) * (T * k + 1));
   if (!ids || !w) return ENOMEM_ARG;
-  int rc = oracle_route(T, E, k, logits, scale, ids, w, NULL);
+  int rc = (scoring == 0 && n_group <= 1)
+               ? oracle_route(T, E, k, logits, scale, ids, w, NULL)
+               : oracle_route_ex(T, E, k, logits, scale, scoring, n_group, topk_group,
+                                 ids, w);
   if (rc == OK) {
     if (!tokens) n_tokens = T;
     for (int64_t r = 0; tokens && r < n_tokens; ++r)
@@ -405,6 +517,18 @@ int oracle_forward(int64_t T, int H, int E, int k, int I, int act, int S,
   if (!ids_out) free(ids);
   if (!w_out) free(w);
   return rc;
+}
+
+int oracle_forward(int64_t T, int H, int E, int k, int I, int act, int S,
+                   int Is, const uint16_t* x, const float* logits,
+                   const float* scale, const uint16_t* w13,
+                   const uint16_t* w2, const uint16_t* w13_sh,
+                   const uint16_t* w2_sh, const int64_t* tokens,
+                   int64_t n_tokens, int round_h, int nthreads, double* out,
+                   int32_t* ids_out, double* w_out) {
+  return oracle_forward_ex(T, H, E, k, I, act, S, Is, x, logits, scale, w13, w2,
+                           w13_sh, w2_sh, tokens, n_tokens, round_h, nthreads, out,
+                           ids_out, w_out, 0, 1, 1);
 }
 
 /* ----------------------------------------------------------------- router */

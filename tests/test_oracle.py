@@ -355,3 +355,127 @@ def test_router_zero_row_stays_finite():
     x[1] = 0.0
     z = oracle.router_logits(x, w, s, 1e-6)
     assert np.all(z[1] == 0.0) and np.all(np.isfinite(z))
+
+
+# ------------------------------------------------ routing variants (lesson 35)
+# llama-cpp-visual-guide lesson 35: the probabilities are a softmax or, for
+# some models, a sigmoid of the logits; with expert groups a token picks its
+# best groups first, then its experts inside them.  A group is scored by its
+# best expert (the reading this oracle takes).
+
+def _brute_route_ex(z, k, scoring, n_group, topk_group, scale=None):
+    """Numpy restatement by enumeration: rank groups, mask, full sort."""
+    T, E = z.shape
+    gs = E // n_group
+    ids = np.zeros((T, k), np.int64)
+    w = np.zeros((T, k))
+    for t in range(T):
+        zt = z[t].astype(np.float64)
+        if scoring == 0:
+            p = np.exp(zt - zt.max())
+            p /= p.sum()
+        else:
+            p = 1.0 / (1.0 + np.exp(-zt))
+        gmax = [zt[g * gs:(g + 1) * gs].max() for g in range(n_group)]
+        groups = sorted(range(n_group), key=lambda g: (-gmax[g], g))[:topk_group]
+        allowed = [e for e in range(E) if e // gs in groups]
+        chosen = sorted(allowed, key=lambda e: (-zt[e], e))[:k]
+        ids[t] = chosen
+        w[t] = p[chosen] / p[chosen].sum()
+        if scale is not None:
+            w[t] *= scale[chosen].astype(np.float64)
+    return ids, w
+
+
+def test_route_ex_softmax_one_group_is_route():
+    gen = torch.Generator().manual_seed(21)
+    z = inputs.router_logits(50, 64, 6, gen, "cpu").numpy()
+    ids0, w0 = oracle.route(z, 6)
+    ids1, w1 = oracle.route_ex(z, 6)
+    assert (ids0 == ids1).all()
+    np.testing.assert_allclose(w1, w0, rtol=1e-14, atol=0)
+
+
+def test_route_ex_groups_are_picked_before_experts():
+    # groups of two: {0,1} max 10, {2,3} max 9, {4,5} max 9.5, {6,7} max 0.
+    # The two best groups are {0,1} and {4,5}; their top-3 experts are 0, 4
+    # and 1 -- while the ungrouped top-3 would be 0, 4, 2.
+    z = np.array([[10, -10, 9, 8.9, 9.5, -20, 0, 0]], np.float32)
+    ids, _ = oracle.route_ex(z, 3, n_group=4, topk_group=2)
+    assert ids[0].tolist() == [0, 4, 1]
+    ids_flat, _ = oracle.route_ex(z, 3)
+    assert ids_flat[0].tolist() == [0, 4, 2]
+
+
+def test_route_ex_sigmoid_closed_form():
+    # sigmoid(0) = 1/2 and sigmoid(ln 3) = 3/4, so the normalised weights of
+    # the top-2 are 3/5 and 2/5 (ln 3 is rounded to fp32: error ~ 1e-8)
+    z = np.array([[0.0, math.log(3.0), -5.0]], np.float32)
+    ids, w = oracle.route_ex(z, 2, scoring=oracle.SCORE_SIGMOID)
+    assert ids[0].tolist() == [1, 0]
+    np.testing.assert_allclose(w[0], [0.6, 0.4], rtol=0, atol=1e-7)
+    assert math.fsum(w[0]) == pytest.approx(1.0, abs=1e-15)
+
+
+@pytest.mark.parametrize("E,k,n_group,topk_group,scoring", [
+    (8, 2, 4, 2, 0), (16, 4, 4, 1, 1), (64, 6, 8, 3, 1), (256, 8, 8, 4, 1),
+    (24, 5, 3, 2, 0)])
+def test_route_ex_matches_enumeration(E, k, n_group, topk_group, scoring):
+    gen = torch.Generator().manual_seed(E + k)
+    z = inputs.router_logits(40, E, k, gen, "cpu").numpy()
+    sc = (0.5 + np.arange(E) / E).astype(np.float32)
+    ids, w = oracle.route_ex(z, k, scale=sc, scoring=scoring, n_group=n_group,
+                             topk_group=topk_group)
+    bi, bw = _brute_route_ex(z, k, scoring, n_group, topk_group, scale=sc)
+    assert (ids == bi).all()
+    np.testing.assert_allclose(w, bw, rtol=1e-13, atol=0)
+    # at most topk_group distinct groups per token
+    gs = E // n_group
+    assert max(len(set((ids[t] // gs).tolist())) for t in range(40)) <= topk_group
+
+
+def test_route_ex_sigmoid_and_softmax_pick_the_same_ids():
+    gen = torch.Generator().manual_seed(5)
+    z = inputs.router_logits(60, 32, 4, gen, "cpu").numpy()
+    a, _ = oracle.route_ex(z, 4, scoring=oracle.SCORE_SOFTMAX, n_group=4, topk_group=2)
+    b, wb = oracle.route_ex(z, 4, scoring=oracle.SCORE_SIGMOID, n_group=4, topk_group=2)
+    assert (a == b).all()  # both are increasing in the logit
+    np.testing.assert_allclose(wb.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+
+
+def test_route_ex_one_expert_per_group_is_ungrouped():
+    gen = torch.Generator().manual_seed(9)
+    z = inputs.router_logits(30, 16, 3, gen, "cpu").numpy()
+    a, wa = oracle.route_ex(z, 3, scoring=1)
+    b, wb = oracle.route_ex(z, 3, scoring=1, n_group=16, topk_group=16)
+    assert (a == b).all() and (wa == wb).all()
+
+
+@pytest.mark.parametrize("n_group,topk_group,k", [(3, 1, 1), (4, 0, 1), (4, 5, 1),
+                                                 (4, 1, 3)])
+def test_route_ex_rejects_impossible_groups(n_group, topk_group, k):
+    z = np.zeros((2, 8), np.float32)  # E = 8: 3 does not divide it; 4 groups
+    with pytest.raises(Exception):  # of 2 cannot give k = 3 from one group
+        oracle.route_ex(z, k, n_group=n_group, topk_group=topk_group)
+
+
+def test_forward_ex_equals_dense_compute_all_then_mask():
+    shp = inputs.Shape(T=9, H=16, E=8, k=3, I=12, act=0, n_shared=1, I_shared=12)
+    inp = inputs.make_inputs(shp, seed=13, scale="uniform")
+    z = inp.logits.numpy()
+    out, ids, w = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, shp.k, shp.act,
+                                 scale=inp.scale, w13_sh=inp.w13_sh, w2_sh=inp.w2_sh,
+                                 scoring=oracle.SCORE_SIGMOID, n_group=4,
+                                 topk_group=2)
+    bi, bw = _brute_route_ex(z, shp.k, 1, 4, 2, scale=inp.scale.numpy())
+    assert (ids == bi).all()
+    x = _bf16_to_f64(inp.x)
+    D = np.zeros((shp.T, shp.E))
+    for t in range(shp.T):
+        D[t, bi[t]] = bw[t]
+    dense = np.zeros((shp.T, shp.H))
+    for e in range(shp.E):
+        dense += D[:, e:e + 1] * _ffn_dense_torch(x, inp.w13[e], inp.w2[e],
+                                                  shp.act).numpy()
+    dense += _ffn_dense_torch(x, inp.w13_sh[0], inp.w2_sh[0], shp.act).numpy()
+    np.testing.assert_allclose(out, dense, rtol=1e-12, atol=1e-14)
