@@ -118,6 +118,44 @@ MOE_API moe_status moe_route(const moe_shape* shape, const float* logits,
                      cudaStream_t stream);
 
 /*
+ * moe_route_ex -- the routing variants of llama-cpp-visual-guide lesson 35
+ * (routing section: "some models use sigmoid"; the expert-group fold: pick a
+ * group first, then experts within it, as n_expert_groups / n_group_used;
+ * the DeepSeek-V3 row of its table: 256 routed experts, top-8).
+ *   opts NULL, or:
+ *     scoring     MOE_SCORE_SOFTMAX: exactly moe_route;
+ *                 MOE_SCORE_SIGMOID: each chosen expert's weight is
+ *                 sigmoid(z_id) / (sum of sigmoid over the chosen k), times
+ *                 scale[id] (fp64, rounded once to fp32)
+ *     n_group     0 or 1: no groups.  Else the E experts form n_group groups
+ *                 of E / n_group consecutive ids (E % n_group == 0,
+ *                 n_group <= 32); each token keeps its topk_group best
+ *                 groups -- a group is scored by its largest logit, equal
+ *                 scores to the lower group id -- and picks its k experts
+ *                 among the experts of those groups only
+ *     topk_group  1..n_group, with k <= topk_group * (E / n_group)
+ *   Selection always compares the fp32 logits themselves (both scores are
+ *   increasing in the logit), so ids and their order are bit-exact with the
+ *   oracle.  Other arguments as moe_route.  Bad options return
+ *   MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for n_group > 32) before any
+ *   launch.
+ */
+typedef enum {
+  MOE_SCORE_SOFTMAX = 0,
+  MOE_SCORE_SIGMOID = 1
+} moe_scoring;
+#define MOE_MAX_GROUPS 32
+typedef struct {
+  int32_t scoring;     /* moe_scoring */
+  int32_t n_group;
+  int32_t topk_group;
+} moe_route_opts;
+
+MOE_API moe_status moe_route_ex(const moe_shape* shape, const float* logits,
+                                const float* scale, const moe_route_opts* opts,
+                                int32_t* ids, float* w, cudaStream_t stream);
+
+/*
  * moe_permute -- the dispatch permutation (walkthrough sections 6-7: the
  * "permutation map" turning token picks into per-expert token lists).
  *   ids          [T,k] int32 in (each in [0,E))
@@ -216,6 +254,8 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
  *                 workspace with RMSNorm epsilon router_eps, and ``logits``
  *                 may be NULL.  On the prefill path this is part of stage 0;
  *                 on the decode path it runs before stage 0.
+ *   route         NULL, or the routing variant of moe_route_ex (sigmoid
+ *                 scoring, expert groups) used by stage 0 on both paths.
  */
 #define MOE_NUM_STAGES 6
 typedef enum {
@@ -235,6 +275,7 @@ typedef struct {
   const moe_bf16* router_w;
   const moe_bf16* router_scale;
   float router_eps;
+  const moe_route_opts* route;   /* NULL, or the routing variant (moe_route_ex) */
 } moe_forward_opts;
 
 MOE_API moe_status moe_forward_ex(

@@ -28,7 +28,7 @@ EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_router_logits",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_ex",
            "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string",
-           "moe_permute_noalloc")
+           "moe_permute_noalloc", "moe_route_ex")
 
 
 class MoEError(RuntimeError):
@@ -41,6 +41,15 @@ PATH_AUTO, PATH_PREFILL, PATH_DECODE = 0, 1, 2
 DECODE_MAX_T = 8
 
 
+SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
+MAX_GROUPS = 32
+
+
+class moe_route_opts(ctypes.Structure):
+    _fields_ = [("scoring", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32)]
+
+
 class moe_forward_opts(ctypes.Structure):
     _fields_ = [("stage_events", ctypes.c_void_p),
                 ("out_f32", ctypes.c_void_p),
@@ -50,7 +59,8 @@ class moe_forward_opts(ctypes.Structure):
                 ("router_x", ctypes.c_void_p),
                 ("router_w", ctypes.c_void_p),
                 ("router_scale", ctypes.c_void_p),
-                ("router_eps", ctypes.c_float)]
+                ("router_eps", ctypes.c_float),
+                ("route", ctypes.POINTER(moe_route_opts))]
 
 
 class moe_shape(ctypes.Structure):
@@ -75,6 +85,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_workspace_size.restype = ctypes.c_size_t
     lib.moe_router_logits.argtypes = [S, P, P, P, ctypes.c_float, P, P]
     lib.moe_route.argtypes = [S, P, P, P, P, P]
+    lib.moe_route_ex.argtypes = [S, P, P, ctypes.POINTER(moe_route_opts), P, P, P]
     lib.moe_permute.argtypes = [S, P, P, P, P, P, ctypes.c_size_t, P]
     lib.moe_expert_ffn.argtypes = [S, P, P, P, P, P, P, P, P, P,
                                    ctypes.c_size_t, P]
@@ -91,7 +102,8 @@ def _load() -> ctypes.CDLL:
                                               ctypes.c_uint32, P]
     lib.moe_status_string.argtypes = [st]
     lib.moe_status_string.restype = ctypes.c_char_p
-    for name in ("moe_router_logits", "moe_route", "moe_permute", "moe_expert_ffn",
+    for name in ("moe_router_logits", "moe_route", "moe_route_ex", "moe_permute",
+                 "moe_expert_ffn",
                  "moe_combine",
                  "moe_forward", "moe_forward_ex", "moe_read_error",
                  "moe_selftest_wait_timeout"):
@@ -168,6 +180,22 @@ def moe_route(shape, logits, scale, ids, w, stream=None):
                          _p(w), _stream(stream)), "moe_route")
 
 
+def route_opts(route):
+    """(scoring, n_group, topk_group) -> moe_route_opts, or None."""
+    if route is None:
+        return None
+    scoring, n_group, topk_group = route
+    return moe_route_opts(scoring, n_group, topk_group)
+
+
+def moe_route_ex(shape, logits, scale, ids, w, route=None, stream=None):
+    """Routing variants: ``route`` = (scoring, n_group, topk_group)."""
+    ro = route_opts(route)
+    _check(lib.moe_route_ex(ctypes.byref(shape), _p(logits), _p(scale),
+                            ctypes.byref(ro) if ro is not None else None, _p(ids),
+                            _p(w), _stream(stream)), "moe_route_ex")
+
+
 def moe_permute(shape, ids, offsets, sorted_slots, slot_row, ws, stream=None):
     _check(lib.moe_permute(ctypes.byref(shape), _p(ids), _p(offsets),
                            _p(sorted_slots), _p(slot_row), _p(ws), ws.numel(),
@@ -208,7 +236,7 @@ def moe_forward(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
 def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
                    ids_out=None, w_out=None, events=None, out_f32=None,
                    path=PATH_AUTO, deterministic=False, cta_pairs=0,
-                   router=None, stream=None):
+                   router=None, route=None, stream=None):
     """moe_forward with options: ``events`` (NUM_STAGES + 1 torch.cuda.Event
     created with enable_timing=True, or None to skip one) recorded around
     the stages, ``out_f32``
@@ -217,7 +245,8 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
     fixed-order combine on the prefill path; ``cta_pairs`` picks the GEMM
     form (0 auto, 1 single CTAs, 2 CTA pairs); ``router`` = (router_x [T,H],
     router_w [E,H], router_scale [H], eps) computes the logits first
-    (``logits`` may then be None)."""
+    (``logits`` may then be None); ``route`` = (scoring, n_group,
+    topk_group) selects a routing variant (moe_route_ex)."""
     arr = None
     if events is not None:
         if len(events) != NUM_STAGES + 1:
@@ -230,10 +259,12 @@ def moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out, ws,
             *[ctypes.c_void_p(e.cuda_event if e is not None else 0)
               for e in events])
     rx, rw, rs, reps = router if router is not None else (None, None, None, 0.0)
+    ro = route_opts(route)
     opts = moe_forward_opts(
         ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
         _p(out_f32), path, int(bool(deterministic)), cta_pairs,
-        _p(rx), _p(rw), _p(rs), float(reps))
+        _p(rx), _p(rw), _p(rs), float(reps),
+        ctypes.pointer(ro) if ro is not None else None)
     _check(lib.moe_forward_ex(ctypes.byref(shape), _p(x), _p(logits), _p(w13),
                               _p(w2), _p(scale), _p(w13_sh), _p(w2_sh), _p(out),
                               _p(ids_out), _p(w_out), _p(ws), ws.numel(),

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(1024)
 decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
                     int T, int E, int k, int S, int32_t* __restrict__ ids,
                     float* __restrict__ w, int32_t* __restrict__ meta,
-                    int32_t* __restrict__ slots) {
+                    int32_t* __restrict__ slots, RouteOpt opt) {
   extern __shared__ int32_t dsm[];
   const int G = E + S, R = T * k;
   int32_t* cnt = dsm;            // [G] tokens, then first slot-list entry
@@ -134,7 +134,7 @@ decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ 
   for (int t = warp; t < T; t += nwarps) {
     int id;
     float wt;
-    route_token_warp<PER>(logits + (int64_t)t * E, scale, E, k, &id, &wt);
+    route_token_warp<PER>(logits + (int64_t)t * E, scale, E, k, &id, &wt, opt);
     if (lane < k) {
       ids[t * k + lane] = id;
       w[t * k + lane] = wt;
@@ -663,7 +663,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
             : a.E <= 128 ? decode_route_kernel<4> : a.E <= 256 ? decode_route_kernel<8>
             : decode_route_kernel<16>;
   cudaError_t e = launch_ex(rk, dim3(1), dim3(rthreads), smem, st, false, a.logits, a.scale,
-                            a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots);
+                            a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots, a.route);
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   const int max_groups = (R < a.E ? R : a.E) + a.S;

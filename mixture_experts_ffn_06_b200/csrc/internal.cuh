@@ -49,9 +49,18 @@ moe_status validate_shape(const moe_shape* s);
 // cudaEventRecord of a caller's stage event; an event node under capture.
 bool record_stage_event(void* ev, cudaStream_t st);
 
+// Routing variant (moe_route_opts, checked): scoring, and with n_group > 1
+// the expert groups (route_impl.cuh).
+struct RouteOpt {
+  int scoring;     // MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID
+  int n_group;     // <= 1: no groups; else <= MOE_MAX_GROUPS and E % n_group == 0
+  int topk_group;  // groups kept per token (1..n_group)
+};
+
 // ---- launch wrappers (return cudaGetLastError of the launch) ----
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
-                         int E, int k, int32_t* ids, float* w, cudaStream_t st);
+                         int E, int k, int32_t* ids, float* w, cudaStream_t st,
+                         RouteOpt opt = RouteOpt{0, 1, 1});
 
 // Router logits [T,E] fp32 from the bf16 residual [T,H], the GateLinear
 // weight [E,H] and the per-dimension scale [H] (router.cu).
@@ -101,6 +110,7 @@ struct DecodeArgs {
   const float* scale;
   const __nv_bfloat16 *w13, *w2, *w13_sh, *w2_sh;
   int T, H, E, k, I, S, act;
+  RouteOpt route;
   int32_t* ids;          // [T,k] out
   float* w;              // [T,k] out
   int32_t* meta;         // [decode_meta_ints(E+S)] scratch

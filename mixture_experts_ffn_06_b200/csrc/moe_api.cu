@@ -198,15 +198,44 @@ moe_status moe_router_logits(const moe_shape* shape, const moe_bf16* x,
                                         shape->T, shape->H, shape->E, eps, logits, stream));
 }
 
+// Checks a routing variant against the shape; NULL is the plain routing.
+static moe_status check_route_opts(const moe_shape& s, const moe_route_opts* o,
+                                   RouteOpt* out) {
+  *out = RouteOpt{MOE_SCORE_SOFTMAX, 1, 1};
+  if (!o) return MOE_OK;
+  if (o->scoring != MOE_SCORE_SOFTMAX && o->scoring != MOE_SCORE_SIGMOID)
+    return MOE_ERR_INVALID_ARG;
+  out->scoring = o->scoring;
+  if (o->n_group <= 1) {
+    if (o->n_group < 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+  }
+  if (o->n_group > MOE_MAX_GROUPS) return MOE_ERR_UNSUPPORTED;
+  if (s.E % o->n_group != 0 || o->topk_group < 1 || o->topk_group > o->n_group ||
+      s.k > o->topk_group * (s.E / o->n_group))
+    return MOE_ERR_INVALID_ARG;
+  out->n_group = o->n_group;
+  out->topk_group = o->topk_group;
+  return MOE_OK;
+}
+
 moe_status moe_route(const moe_shape* shape, const float* logits,
                      const float* scale, int32_t* ids, float* w,
                      cudaStream_t stream) {
+  return moe_route_ex(shape, logits, scale, nullptr, ids, w, stream);
+}
+
+moe_status moe_route_ex(const moe_shape* shape, const float* logits,
+                        const float* scale, const moe_route_opts* opts, int32_t* ids,
+                        float* w, cudaStream_t stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
+  RouteOpt ro;
+  if ((st = check_route_opts(*shape, opts, &ro)) != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   if (!logits || !ids || !w) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_route(logits, scale, shape->T, shape->E, shape->k, ids,
-                                w, stream));
+                                w, stream, ro));
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
@@ -281,6 +310,9 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
       return MOE_ERR_INVALID_ARG;
   }
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
+  RouteOpt ro;
+  if ((st = check_route_opts(*shape, opts ? opts->route : nullptr, &ro)) != MOE_OK)
+    return st;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   void* const* ev = opts ? opts->stage_events : nullptr;
   if (shape->T == 0) {
@@ -329,6 +361,7 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
     d.I = s.I;
     d.S = s.n_shared;
     d.act = s.act;
+    d.route = ro;
     d.ids = ids;
     d.w = w;
     d.meta = reinterpret_cast<int32_t*>(at(ws, m.dec_meta));
@@ -347,7 +380,7 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
   }
   if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
   if (!run_router()) return MOE_ERR_CUDA;
-  if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream) != cudaSuccess)
+  if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream, ro) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (!mark(ev, 1, stream)) return MOE_ERR_CUDA;
   if (launch_layout(s, ids, offsets, sorted_slots, slot_row, m.cap,

@@ -1,7 +1,8 @@
-// route.cu -- warp-per-token routing kernel (moe_route and the prefill path
-// of moe_forward).  The per-token arithmetic is route_token_warp
-// (route_impl.cuh): top-k on the fp32 logits, closed-form renormalised
-// softmax over the chosen k in fp64, times per_expert_scale.
+// route.cu -- warp-per-token routing kernel (moe_route, moe_route_ex and the
+// prefill path of moe_forward).  The per-token arithmetic is route_token_warp
+// (route_impl.cuh): optional expert-group selection, top-k on the fp32
+// logits, closed-form renormalised softmax (or normalised sigmoids) over the
+// chosen k in fp64, times per_expert_scale.
 #include "route_impl.cuh"
 
 namespace moe {
@@ -11,7 +12,7 @@ template <int PER>
 __global__ void __launch_bounds__(256)
 route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
              int64_t T, int E, int k, int32_t* __restrict__ ids,
-             float* __restrict__ w) {
+             float* __restrict__ w, RouteOpt opt) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   pdl_wait();
@@ -19,7 +20,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
   if (t >= T) return;
   int id;
   float wt;
-  route_token_warp<PER>(logits + t * E, scale, E, k, &id, &wt);
+  route_token_warp<PER>(logits + t * E, scale, E, k, &id, &wt, opt);
   if (lane < k) {
     ids[t * k + lane] = id;
     w[t * k + lane] = wt;
@@ -30,7 +31,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
 
 cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
                          int E, int k, int32_t* ids, float* w,
-                         cudaStream_t st) {
+                         cudaStream_t st, RouteOpt opt) {
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
@@ -38,7 +39,7 @@ cudaError_t launch_route(const float* logits, const float* scale, int64_t T,
   auto kern = E <= 32 ? route_kernel<1> : E <= 64 ? route_kernel<2> : E <= 128 ? route_kernel<4>
               : E <= 256 ? route_kernel<8> : route_kernel<16>;
   return launch_ex(kern, dim3((unsigned)blocks), dim3(warps * 32), 0, st, false, logits, scale,
-                   T, E, k, ids, w);
+                   T, E, k, ids, w, opt);
 }
 
 }  // namespace moe

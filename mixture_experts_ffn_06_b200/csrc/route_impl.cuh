@@ -33,17 +33,28 @@ __device__ __forceinline__ uint32_t route_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Routing variants of llama-cpp-visual-guide lesson 35 (routing section and
+// the expert-group fold): scoring 0 is the softmax over all E logits,
+// scoring 1 a sigmoid per expert; with n_group > 1 the experts form n_group
+// groups of E / n_group consecutive ids, and a token first keeps its
+// topk_group best groups (a group scored by its best expert; ties to the
+// lower group id), then picks its k experts among theirs.  Both scores are
+// increasing in the logit, so everything is ranked on the fp32 logits.
+// (RouteOpt: internal.cuh)
+
 // Routes token row z[0..E) with the calling warp (E <= 32 PER).  Lane j < k
 // returns the j-th choice in (*id, *wt); the other lanes return id 0,
 // weight 0.
 //
 // Each round, every lane takes its best untaken entry, and two warp
 // reductions (redux.sync) pick the winner: the largest key, then the lowest
-// id among the lanes holding it.
+// id among the lanes holding it.  The kept groups are picked the same way,
+// lane g holding group g's best key.
 template <int PER = kMaxExperts / 32>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
                                                  const float* __restrict__ scale,
-                                                 int E, int k, int* id, float* wt) {
+                                                 int E, int k, int* id, float* wt,
+                                                 RouteOpt opt = RouteOpt{0, 1, 1}) {
   constexpr int kPerLane = PER;
   const int lane = threadIdx.x & 31;
   float v[kPerLane];
@@ -59,6 +70,35 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i)
     if (lane + 32 * i >= E) gone |= 1u << i;
+  if (opt.n_group > 1) {
+    const int gs = E / opt.n_group;
+    int grp[kPerLane];
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) grp[i] = (lane + 32 * i) / gs;
+    // lane g < n_group gets group g's best key
+    uint32_t my_g = 0;
+    for (int g = 0; g < opt.n_group; ++g) {
+      uint32_t part = 0;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if (!((gone >> i) & 1u) && grp[i] == g && key[i] > part) part = key[i];
+      const uint32_t m = __reduce_max_sync(0xffffffffu, part);
+      if (lane == g) my_g = m;
+    }
+    // keep the topk_group best groups (larger key, then lower group id)
+    uint32_t keep = 0;
+    bool open = lane < opt.n_group;
+    for (int r = 0; r < opt.topk_group; ++r) {
+      const uint32_t gmax = __reduce_max_sync(0xffffffffu, open ? my_g : 0u);
+      const uint32_t cand = (open && my_g == gmax) ? (uint32_t)lane : 0xffffffffu;
+      const uint32_t gw = __reduce_min_sync(0xffffffffu, cand);
+      keep |= 1u << gw;
+      if (lane == (int)gw) open = false;
+    }
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)  // (grp < n_group <= 32 for e < E)
+      if (lane + 32 * i < E && !((keep >> grp[i]) & 1u)) gone |= 1u << i;
+  }
   float my_v = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
@@ -83,7 +123,11 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
     }
   }
   const float zmax = __shfl_sync(0xffffffffu, my_v, 0);
-  const double ex = (lane < k) ? exp((double)my_v - (double)zmax) : 0.0;
+  // softmax: the closed form over the k chosen logits; sigmoid: each
+  // chosen expert's sigmoid, normalised over the k
+  const double ex = (lane >= k) ? 0.0
+                    : opt.scoring == MOE_SCORE_SIGMOID ? 1.0 / (1.0 + exp(-(double)my_v))
+                                                       : exp((double)my_v - (double)zmax);
   double den = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);

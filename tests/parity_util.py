@@ -20,7 +20,7 @@ def to_device(inp: inputs.MoEInputs, device="cuda") -> inputs.MoEInputs:
 
 
 def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
-                deterministic=False, cta_pairs=0, ws_fill=None):
+                deterministic=False, cta_pairs=0, ws_fill=None, route=None):
     """moe_forward_ex through the C ABI -> (out bf16, out_f32, ids, w).
     Checks that the bf16 output is exactly the round-to-nearest-even of the
     fp32 layer output.  ws_fill: byte written over the workspace past its
@@ -38,17 +38,19 @@ def gpu_forward(api, inp: inputs.MoEInputs, with_routing=True, path=0,
     api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale,
                        inp.w13_sh, inp.w2_sh, out, ws, ids_out=ids, w_out=w,
                        out_f32=out_f32, path=path, deterministic=deterministic,
-                       cta_pairs=cta_pairs)
+                       cta_pairs=cta_pairs, route=route)
     torch.cuda.synchronize()
     assert api.moe_read_error(ws) == 0
     assert torch.equal(out, out_f32.to(torch.bfloat16)), "bf16 rounding step"
     return out, out_f32, ids, w
 
 
-def oracle_forward(inp: inputs.MoEInputs, tokens=None):
+def oracle_forward(inp: inputs.MoEInputs, tokens=None, route=None):
+    scoring, n_group, topk_group = route if route is not None else (0, 1, 1)
     return oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, inp.shape.k,
                           inp.shape.act, scale=inp.scale, w13_sh=inp.w13_sh,
-                          w2_sh=inp.w2_sh, tokens=tokens)
+                          w2_sh=inp.w2_sh, tokens=tokens, scoring=scoring,
+                          n_group=n_group, topk_group=topk_group)
 
 
 def assert_out_close(got_t: torch.Tensor, want: np.ndarray, what=""):

@@ -143,3 +143,30 @@ def test_router_logits_refuses_bad_arguments(api):
     assert f(ctypes.byref(s), null, fake, fake, ctypes.c_float(1e-6), fake, null) == 1
     empty = api.make_shape(T=0, H=64, E=8, k=1, I=8)
     assert f(ctypes.byref(empty), null, null, null, ctypes.c_float(1e-6), null, null) == 0
+
+
+@pytest.mark.parametrize("opts,status", [
+    ((2, 1, 1), 1),      # unknown scoring
+    ((0, -1, 1), 1),     # negative group count
+    ((1, 3, 1), 1),      # E = 8 is not a multiple of 3 groups
+    ((1, 4, 0), 1),      # no group kept
+    ((1, 4, 5), 1),      # more groups kept than there are
+    ((0, 8, 1), 1),      # one kept group of one expert cannot give k = 2
+    ((1, 33, 1), 2),     # above MOE_MAX_GROUPS
+])
+def test_route_ex_refuses_bad_options(api, opts, status):
+    # rejected on the host before any launch: no GPU needed
+    s = api.make_shape(T=4, H=64, E=8, k=2, I=8)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced
+    ro = api.moe_route_opts(*opts)
+    rc = api.lib.moe_route_ex(ctypes.byref(s), fake, fake, ctypes.byref(ro), fake,
+                              fake, None)
+    assert rc == status
+    # the same options reach moe_forward_ex's checks
+    fo = api.moe_forward_opts()
+    fo.route = ctypes.pointer(ro)
+    ws = ctypes.c_void_p(1 << 21)
+    rc = api.lib.moe_forward_ex(ctypes.byref(s), fake, fake, fake, fake, fake, None,
+                                None, fake, None, None, ws,
+                                api.moe_workspace_size(s), ctypes.byref(fo), None)
+    assert rc == status
