@@ -63,47 +63,45 @@ combine_kernel(const float4* __restrict__ y_perm,
 
 // Sum of the k+S weighted rows of a token, which the fused w2 epilogue has
 // stored contiguously, in order j = 0..k+S-1; one bf16 rounding.  Each thread
-// owns 8 columns (two float4) of one token at a time.
+// owns 4 columns (one float4) of one token at a time, and requests the rows
+// of a batch of 8 before it adds the first, so a token with k + S = 8 waits
+// for one round trip instead of eight; the additions stay in order j.
 __global__ void __launch_bounds__(256)
 sum_rows_kernel(const float4* __restrict__ stage, int64_t T, int ks, int H,
-                uint4* __restrict__ out, float4* __restrict__ out_f32) {
+                uint2* __restrict__ out, float4* __restrict__ out_f32) {
   pdl_wait();
   pdl_trigger();
-  const int c8 = H >> 3;
-  const int64_t n = T * c8;
+  const int c4 = H >> 2;
+  const int64_t n = T * c4;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += stride) {
-    const int64_t t = i / c8;
-    const int c = (int)(i - t * c8);
-    const float4* src = stage + (t * ks) * (int64_t)(H >> 2) + 2 * c;
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < ks; ++j) {
-      const float4 u = __ldg(src + (int64_t)j * (H >> 2));
-      const float4 v = __ldg(src + (int64_t)j * (H >> 2) + 1);
-      a[0] = __fadd_rn(a[0], u.x);
-      a[1] = __fadd_rn(a[1], u.y);
-      a[2] = __fadd_rn(a[2], u.z);
-      a[3] = __fadd_rn(a[3], u.w);
-      a[4] = __fadd_rn(a[4], v.x);
-      a[5] = __fadd_rn(a[5], v.y);
-      a[6] = __fadd_rn(a[6], v.z);
-      a[7] = __fadd_rn(a[7], v.w);
+    const int64_t t = i / c4;
+    const int c = (int)(i - t * c4);
+    const float4* src = stage + (t * ks) * (int64_t)c4 + c;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](const float4& u) {
+      a.x = __fadd_rn(a.x, u.x);
+      a.y = __fadd_rn(a.y, u.y);
+      a.z = __fadd_rn(a.z, u.z);
+      a.w = __fadd_rn(a.w, u.w);
+    };
+    int j = 0;
+    for (; j + 8 <= ks; j += 8) {
+      float4 u[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) u[q] = __ldg(src + (int64_t)(j + q) * c4);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) add(u[q]);
     }
-    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a[0], a[1]);
-    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a[2], a[3]);
-    const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[4], a[5]);
-    const __nv_bfloat162 p3 = __floats2bfloat162_rn(a[6], a[7]);
-    uint4 o;
+    for (; j < ks; ++j) add(__ldg(src + (int64_t)j * c4));
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+    uint2 o;
     o.x = *reinterpret_cast<const uint32_t*>(&p0);
     o.y = *reinterpret_cast<const uint32_t*>(&p1);
-    o.z = *reinterpret_cast<const uint32_t*>(&p2);
-    o.w = *reinterpret_cast<const uint32_t*>(&p3);
     out[i] = o;
-    if (out_f32) {
-      out_f32[2 * i] = make_float4(a[0], a[1], a[2], a[3]);
-      out_f32[2 * i + 1] = make_float4(a[4], a[5], a[6], a[7]);
-    }
+    if (out_f32) out_f32[i] = a;
   }
 }
 
@@ -165,13 +163,13 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* slot_row,
 cudaError_t launch_sum_rows(const float* stage, int64_t T, int ks, int H,
                             __nv_bfloat16* out, float* out_f32, cudaStream_t st,
                             bool pdl) {
-  const int64_t n = T * (H / 8);
+  const int64_t n = T * (H / 4);
   if (n == 0) return cudaSuccess;
   const int64_t want = (n + 255) / 256;
   const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
   return launch_ex(sum_rows_kernel, dim3(blocks), dim3(256), 0, st, pdl,
                    reinterpret_cast<const float4*>(stage), T, ks, H,
-                   reinterpret_cast<uint4*>(out), reinterpret_cast<float4*>(out_f32));
+                   reinterpret_cast<uint2*>(out), reinterpret_cast<float4*>(out_f32));
 }
 
 }  // namespace moe
