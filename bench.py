@@ -93,6 +93,28 @@ def workload_name(cfg_name, shp):
     return s
 
 
+def max_over_ranks_fn(world: int, device):
+    """The slowest rank's value of a per-rank time (all-reduce MAX); every
+    rank takes the same collective step."""
+    import torch
+    import torch.distributed as dist
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return max_over_ranks
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens/s of the whole job: every replica processes its own batch of
+    tokens_per_rank tokens per step, and the step takes the slowest rank's
+    time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -376,12 +398,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = max_over_ranks_fn(world, dev)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -530,7 +547,7 @@ def run_ours(args):
     result = None
     if rank == 0:
         peaks, peak_src = load_peaks()
-        value = world * shp.T / (ms_per_step / 1e3)
+        value = whole_job_rate(shp.T, world, ms_per_step)
         # dominant kernel: the w13 product with the fused activation (2/3 of
         # the layer's FLOPs and of its weight bytes); FLOPs count real rows
         # only, bytes count each touched expert once

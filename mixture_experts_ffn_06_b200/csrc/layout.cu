@@ -70,11 +70,23 @@ layout_scan(const int32_t* __restrict__ lt_count, int64_t n_lt, int E, int S,
   pdl_wait();
   pdl_trigger();
   const int G = E + S;
-  // per-expert running sum over layout blocks
+  // per-expert running sum over layout blocks; the counts of 8 blocks are
+  // requested before the first is added (one round trip per 8 blocks)
   for (int e = tid; e < G; e += blockDim.x) {
     int64_t total = 0;
     if (e < E) {
-      for (int64_t b = 0; b < n_lt; ++b) {
+      int64_t b = 0;
+      for (; b + 8 <= n_lt; b += 8) {
+        int32_t c[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c[q] = lt_count[(b + q) * E + e];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          lt_base[(b + q) * E + e] = (int32_t)total;
+          total += c[q];
+        }
+      }
+      for (; b < n_lt; ++b) {
         lt_base[b * E + e] = (int32_t)total;
         total += lt_count[b * E + e];
       }

@@ -124,10 +124,14 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ z,
   }
   const float zmax = __shfl_sync(0xffffffffu, my_v, 0);
   // softmax: the closed form over the k chosen logits; sigmoid: each
-  // chosen expert's sigmoid, normalised over the k
-  const double ex = (lane >= k) ? 0.0
-                    : opt.scoring == MOE_SCORE_SIGMOID ? 1.0 / (1.0 + exp(-(double)my_v))
-                                                       : exp((double)my_v - (double)zmax);
+  // chosen expert's sigmoid, normalised over the k (one exp either way)
+  double ex = 0.0;
+  if (lane < k) {
+    if (opt.scoring == MOE_SCORE_SIGMOID)
+      ex = 1.0 / (1.0 + exp(-(double)my_v));
+    else
+      ex = exp((double)my_v - (double)zmax);
+  }
   double den = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
