@@ -209,3 +209,37 @@ def zipf_weights(E: int, s: float) -> list:
     w = [(e + 1.0) ** (-s) for e in range(E)]
     tot = math.fsum(w)
     return [v / tot for v in w]
+
+
+@dataclasses.dataclass
+class Gemma4BlockInputs:
+    """Inputs of the Gemma 4 MoE block beyond the experts (``MoEInputs``):
+    the residual rows, the five gamma vectors, the dense MLP and the router."""
+    x: torch.Tensor            # [T,H] bf16 residual (the MoE experts' weights come
+                               # from MoEInputs; its x and logits are not used)
+    norms: tuple               # 5 x [H] bf16: pre_ff, post_ff_1, pre_ff_2, post_ff_2, post_ff
+    mlp_w13: torch.Tensor      # [2*I_dense, H] bf16, gate rows first
+    mlp_w2: torch.Tensor       # [H, I_dense] bf16
+    router_w: torch.Tensor     # [E,H] bf16
+    router_scale: torch.Tensor  # [H] bf16
+
+
+def gemma4_block_inputs(T: int, H: int, E: int, I_dense: int, seed: int = 0,
+                        device="cpu") -> Gemma4BlockInputs:
+    """Recipe (one generator seeded with ``seed``, in this order): residual
+    rows N(0,1) -> bf16; the five gammas 1 + N(0, 0.1) -> bf16; the dense
+    MLP's w13 [2*I_dense, H] and w2 [H, I_dense] N(0, 0.02) -> bf16; the
+    router's GateLinear weight N(0,1) -> bf16 (logits near unit scale, as in
+    ``router_inputs``); the router scale U[0.5, 1.5] -> bf16."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = _normal_bf16((T, H), 1.0, gen, device)
+    norms = tuple((1.0 + 0.1 * torch.randn(H, generator=gen, device=device))
+                  .to(torch.bfloat16) for _ in range(5))
+    mlp_w13 = _normal_bf16((2 * I_dense, H), 0.02, gen, device)
+    mlp_w2 = _normal_bf16((H, I_dense), 0.02, gen, device)
+    rw = torch.randn(E, H, generator=gen, device=device).to(torch.bfloat16)
+    rs = (0.5 + torch.rand(H, generator=gen, device=device)).to(torch.bfloat16)
+    return Gemma4BlockInputs(x=x, norms=norms, mlp_w13=mlp_w13, mlp_w2=mlp_w2,
+                             router_w=rw, router_scale=rs)

@@ -66,11 +66,15 @@ def _load():
         lib.oracle_router_logits.argtypes = [i64, i32, i32, ctypes.c_double, P, P,
                                              P, P]
         lib.oracle_route_ex.argtypes = [i64, i32, i32, P, P, i32, i32, i32, P, P]
+        dbl = ctypes.c_double
+        lib.oracle_gemma4_block.argtypes = [i64, i32, i32, i32, i32, i32, i32, P, P, P,
+                                            P, P, P, dbl, P, P, dbl, P, P, P, P, P,
+                                            i32, P]
         lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [i32, i32, i32]
         for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
                   lib.oracle_expert_rows, lib.oracle_forward,
                   lib.oracle_router_logits, lib.oracle_route_ex,
-                  lib.oracle_forward_ex):
+                  lib.oracle_forward_ex, lib.oracle_gemma4_block):
             f.restype = i32
         _lib = lib
     return _lib
@@ -222,3 +226,26 @@ def forward(x, logits, w13, w2, k: int, act_kind: int, scale=None,
                                      _ptr(ids), _ptr(w), scoring, n_group,
                                      topk_group), "forward")
     return out, ids, w
+
+
+def gemma4_block(x, norms, eps: float, router_w, router_scale, router_eps: float,
+                 w13, w2, scale, mlp_w13, mlp_w2, k: int, act_kind: int,
+                 nthreads: int = 0) -> np.ndarray:
+    """The MoE block of a Gemma 4 decoder layer from the residual x [T,H]
+    bf16 -> the output before its final bf16 rounding, [T,H] float64.
+    norms = (pre_ff, post_ff_1, pre_ff_2, post_ff_2, post_ff) gammas [H]
+    bf16; mlp_w13 [2*I_dense, H], mlp_w2 [H, I_dense] bf16."""
+    xu = _u16(x)
+    T, H = xu.shape
+    gs = [_u16(g) for g in norms]
+    w13u, w2u = _u16(w13), _u16(w2)
+    E, I = w13u.shape[0], w2u.shape[-1]
+    m13, m2 = _u16(mlp_w13), _u16(mlp_w2)
+    Id = m2.shape[-1]
+    out = np.empty((T, H), np.float64)
+    _check(_load().oracle_gemma4_block(
+        T, H, E, k, I, act_kind, Id, _ptr(xu), *[_ptr(g) for g in gs], float(eps),
+        _ptr(_u16(router_w)), _ptr(_u16(router_scale)), float(router_eps), _ptr(w13u),
+        _ptr(w2u), _ptr(_f32(scale)), _ptr(m13), _ptr(m2), nthreads, _ptr(out)),
+        "gemma4_block")
+    return out

@@ -32,6 +32,10 @@
  *              section 6).
  *   route_ex -- llama-cpp-visual-guide lesson 35: sigmoid scoring and expert
  *              groups (see oracle_route_ex).
+ *   gemma4 block -- section 1 of the Gemma 4 walkthrough: the dense MLP and
+ *              the MoE in parallel from the same residual, each between its
+ *              own gamma RMSNorms, summed unweighted, then a last norm and
+ *              the residual add (see oracle_gemma4_block).
  *   combine -- walkthrough section 7 step 4: the k expert outputs of a token
  *              are summed weighted by its (scale-folded) gate weights; shared
  *              experts (llama-cpp-visual-guide lesson 35, "shared expert")
@@ -583,4 +587,107 @@ int oracle_router_logits(int64_t T, int H, int E, double eps, const uint16_t* x,
   }
   free(b);
   return OK;
+}
+
+/* ------------------------------------------------------- gemma 4 block */
+
+/*
+ * Gamma RMSNorm of one row of bf16 values (walkthrough section 3: the
+ * standard RMSNorm is y = x / RMS(x) * gamma; the Gemma 4 norms compute in
+ * fp32 and return the activation dtype).  Reading of the fp32 steps, as for
+ * the router's norm: v = fp32(mean of the squares, taken in double),
+ * inv = 1 / sqrt(v + eps) in fp32, y_h = bf16( fp32( fp32(x_h * inv) * g_h ) ).
+ *   x [H] bf16 values held in double, g [H] bf16, y [H] out (bf16 values)
+ */
+static void gamma_rms_norm_row(const double* x, int H, double eps, const uint16_t* g,
+                               double* y) {
+  double ss = 0.0;
+  for (int h = 0; h < H; ++h) ss += x[h] * x[h];
+  const float var = (float)(ss / (double)H);
+  const float inv = 1.0f / sqrtf(var + (float)eps);
+  for (int h = 0; h < H; ++h) {
+    const float n = (float)x[h] * inv;
+    const float p = n * (float)bf16_to_double(g[h]);
+    y[h] = round_to_bf16((double)p);
+  }
+}
+
+static uint16_t double_to_bf16_bits(double v) {
+  /* v already holds a bf16 value: its float bits' upper half */
+  float f = (float)v;
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return (uint16_t)(u >> 16);
+}
+
+/*
+ * The MoE block of a Gemma 4 decoder layer (walkthrough section 1, the
+ * DecoderLayer forward; section 7 for the tensor flow), from the residual x
+ * [T,H] bf16 that the attention half hands over:
+ *   h1 = post_ff_norm_1( mlp( pre_ff_norm(x) ) )        dense GeGLU MLP
+ *   h2 = post_ff_norm_2( moe( pre_ff_norm_2(x), router(x) ) )
+ *   out = post_ff_norm( h1 + h2 ) + x                    unweighted sum
+ * Every module returns bf16 (the activation dtype): the two norm outputs,
+ * the MLP and MoE outputs (each computed in fp64 here, then rounded), h1,
+ * h2, their sum (one fp32 add, rounded), and the last norm.  out receives
+ * the final residual add in fp32, fl(z + x), before its bf16 rounding.
+ * The MLP is the E = 1 case of the expert FFN (oracle_forward with one
+ * expert and weight 1); the MoE is oracle_forward on the router's logits
+ * (oracle_router_logits) with per_expert_scale.
+ */
+int oracle_gemma4_block(int64_t T, int H, int E, int k, int I, int act, int I_dense,
+                        const uint16_t* x, const uint16_t* g_pre, const uint16_t* g_post1,
+                        const uint16_t* g_pre2, const uint16_t* g_post2,
+                        const uint16_t* g_post, double eps, const uint16_t* router_w,
+                        const uint16_t* router_scale, double router_eps,
+                        const uint16_t* w13, const uint16_t* w2, const float* scale,
+                        const uint16_t* mlp_w13, const uint16_t* mlp_w2, int nthreads,
+                        double* out) {
+  if (T < 0 || H < 1 || I_dense < 1 || !(eps >= 0.0) || !x || !g_pre || !g_post1 ||
+      !g_pre2 || !g_post2 || !g_post || !mlp_w13 || !mlp_w2 || !out)
+    return EINVAL_ARG;
+  const size_t TH = (size_t)T * (size_t)H;
+  uint16_t* a1 = (uint16_t*)malloc(sizeof(uint16_t) * (TH + 1));
+  uint16_t* a2 = (uint16_t*)malloc(sizeof(uint16_t) * (TH + 1));
+  double* y1 = (double*)malloc(sizeof(double) * (TH + 1));
+  double* y2 = (double*)malloc(sizeof(double) * (TH + 1));
+  float* z1 = (float*)calloc((size_t)T + 1, sizeof(float));   /* the MLP's logits */
+  float* lg = (float*)malloc(sizeof(float) * ((size_t)T * E + 1));
+  double* row = (double*)malloc(sizeof(double) * (size_t)H);
+  double* r1 = (double*)malloc(sizeof(double) * (size_t)H);
+  double* r2 = (double*)malloc(sizeof(double) * (size_t)H);
+  int rc = OK;
+  if (!a1 || !a2 || !y1 || !y2 || !z1 || !lg || !row || !r1 || !r2) rc = ENOMEM_ARG;
+  /* the two input norms */
+  for (int64_t t = 0; t < T && rc == OK; ++t) {
+    for (int h = 0; h < H; ++h) row[h] = bf16_to_double(x[t * H + h]);
+    gamma_rms_norm_row(row, H, eps, g_pre, r1);
+    gamma_rms_norm_row(row, H, eps, g_pre2, r2);
+    for (int h = 0; h < H; ++h) {
+      a1[t * H + h] = double_to_bf16_bits(r1[h]);
+      a2[t * H + h] = double_to_bf16_bits(r2[h]);
+    }
+  }
+  /* dense MLP: one expert, weight 1 */
+  if (rc == OK)
+    rc = oracle_forward(T, H, 1, 1, I_dense, act, 0, 0, a1, z1, NULL, mlp_w13, mlp_w2,
+                        NULL, NULL, NULL, T, 0, nthreads, y1, NULL, NULL);
+  /* router on the raw residual, MoE on the normalised one */
+  if (rc == OK) rc = oracle_router_logits(T, H, E, router_eps, x, router_w, router_scale, lg);
+  if (rc == OK)
+    rc = oracle_forward(T, H, E, k, I, act, 0, 0, a2, lg, scale, w13, w2, NULL, NULL,
+                        NULL, T, 0, nthreads, y2, NULL, NULL);
+  for (int64_t t = 0; t < T && rc == OK; ++t) {
+    double* o = out + t * H;
+    for (int h = 0; h < H; ++h) row[h] = round_to_bf16(y1[t * H + h]);
+    gamma_rms_norm_row(row, H, eps, g_post1, r1);                  /* h1 */
+    for (int h = 0; h < H; ++h) row[h] = round_to_bf16(y2[t * H + h]);
+    gamma_rms_norm_row(row, H, eps, g_post2, r2);                  /* h2 */
+    for (int h = 0; h < H; ++h) row[h] = round_to_bf16((double)(float)(r1[h] + r2[h]));
+    gamma_rms_norm_row(row, H, eps, g_post, r1);                   /* z */
+    for (int h = 0; h < H; ++h)
+      o[h] = (double)(float)(r1[h] + bf16_to_double(x[t * H + h]));  /* fl(z + x) */
+  }
+  free(a1); free(a2); free(y1); free(y2); free(z1); free(lg); free(row); free(r1); free(r2);
+  return rc;
 }

@@ -479,3 +479,77 @@ def test_forward_ex_equals_dense_compute_all_then_mask():
                                                   shp.act).numpy()
     dense += _ffn_dense_torch(x, inp.w13_sh[0], inp.w2_sh[0], shp.act).numpy()
     np.testing.assert_allclose(out, dense, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------- Gemma 4 MoE block (section 1)
+
+def _block_case(T=6, H=64, E=8, k=2, I=32, Id=48, seed=2, act=1):
+    shp = inputs.Shape(T=T, H=H, E=E, k=k, I=I, act=act)
+    moe = inputs.make_inputs(shp, seed=seed, scale="uniform")
+    blk = inputs.gemma4_block_inputs(T, H, E, Id, seed=seed + 100)
+    return shp, moe, blk
+
+
+def _run_block(shp, moe, blk, **over):
+    kw = dict(norms=blk.norms, eps=1e-6, router_w=blk.router_w,
+              router_scale=blk.router_scale, router_eps=1e-6, w13=moe.w13,
+              w2=moe.w2, scale=moe.scale, mlp_w13=blk.mlp_w13, mlp_w2=blk.mlp_w2,
+              k=shp.k, act_kind=shp.act)
+    kw.update(over)
+    return oracle.gemma4_block(blk.x, **kw)
+
+
+def _norm_torch(x64, g, eps=1e-6):
+    """The standard gamma RMSNorm in float64 (walkthrough section 3), no
+    intermediate rounding: used where the pins need only its shape."""
+    return x64 / torch.sqrt((x64 ** 2).mean(-1, keepdim=True) + eps) * _bf16_to_f64(g)
+
+
+def test_block_with_both_branches_zero_returns_the_residual():
+    # zero weights: both branch outputs are 0, each post-norm of a zero row
+    # is 0 (the eps guard), so out = fl(0 + x) = x exactly
+    shp, moe, blk = _block_case()
+    out = _run_block(shp, moe, blk, w13=torch.zeros_like(moe.w13),
+                     mlp_w13=torch.zeros_like(blk.mlp_w13))
+    np.testing.assert_array_equal(out, _bf16_to_f64(blk.x).numpy())
+
+
+def test_block_with_zero_last_gamma_returns_the_residual():
+    shp, moe, blk = _block_case(seed=4)
+    norms = blk.norms[:4] + (torch.zeros_like(blk.norms[4]),)
+    out = _run_block(shp, moe, blk, norms=norms)
+    np.testing.assert_array_equal(out, _bf16_to_f64(blk.x).numpy())
+
+
+def test_block_last_norm_sets_the_scale_of_the_update():
+    # out - x is the last norm's output: divided by its gamma it has RMS 1
+    # per token (up to bf16 rounding and the eps term), whatever the branches
+    shp, moe, blk = _block_case(E=4, k=2, I=48, Id=48, seed=6)
+    z = _run_block(shp, moe, blk) - _bf16_to_f64(blk.x).numpy()
+    gam = _bf16_to_f64(blk.norms[4]).numpy()
+    rms = np.sqrt(np.mean((z / gam) ** 2, axis=1))
+    np.testing.assert_allclose(rms, 1.0, rtol=2e-2)
+
+
+def test_block_matches_a_float64_restatement():
+    # the same block written with torch float64 ops (no intermediate
+    # rounding at all): the oracle's bf16 module boundaries stay within a
+    # few bf16 ulps of it
+    shp, moe, blk = _block_case(T=5, H=64, E=8, k=2, I=32, Id=40, seed=8)
+    out = _run_block(shp, moe, blk)
+    x = _bf16_to_f64(blk.x)
+    a1 = _norm_torch(x, blk.norms[0])
+    a2 = _norm_torch(x, blk.norms[2])
+    y1 = _ffn_dense_torch(a1, blk.mlp_w13, blk.mlp_w2, shp.act)
+    z = oracle.router_logits(blk.x, blk.router_w, blk.router_scale, 1e-6)
+    ids, w = oracle.route(z, shp.k, scale=moe.scale)
+    y2 = torch.zeros_like(x)
+    for t in range(shp.T):
+        for j in range(shp.k):
+            e = int(ids[t, j])
+            y2[t] += w[t, j] * _ffn_dense_torch(a2[t:t + 1], moe.w13[e], moe.w2[e],
+                                                shp.act)[0]
+    h = _norm_torch(y1, blk.norms[1]) + _norm_torch(y2, blk.norms[3])
+    want = (_norm_torch(h, blk.norms[4]) + x).numpy()
+    d = out - want
+    assert np.abs(d).max() <= 0.05 * np.sqrt(np.mean((want - x.numpy()) ** 2))
