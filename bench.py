@@ -61,6 +61,10 @@ def parse():
                     help="time plain stream launches instead of one CUDA graph")
     ap.add_argument("--profile", action="store_true",
                     help="device timing only: skip the e2e and CPU legs")
+    ap.add_argument("--block", type=int, default=0, metavar="I_DENSE",
+                    help="time the Gemma 4 MoE block (dense MLP of this "
+                         "intermediate size in parallel with the MoE, gamma "
+                         "norms, router on the residual) instead of the layer")
     ap.add_argument("--router", action="store_true",
                     help="start from hidden states: the router (RMSNorm, scale, "
                          "GateLinear) computes the logits inside every step")
@@ -698,10 +702,78 @@ def run_reference(args):
     return result
 
 
+def run_block(args):
+    """The Gemma 4 MoE block (moe_gemma4_block) on the config's MoE shape
+    with a dense MLP of intermediate size args.block: K steps in one CUDA
+    graph, device-timed, the L2 flushed before every step when the touched
+    weights would fit in it.  One GPU; prints one JSON line."""
+    import torch
+
+    from mixture_experts_ffn_06_b200 import api, inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_workload(args, dev, args.seed)
+    shp = inp.shape
+    Id = args.block
+    blk = inputs.gemma4_block_inputs(shp.T, shp.H, shp.E, Id, seed=args.seed + 7,
+                                     device=dev)
+    s = api.shape_from(shp)
+    ws = api.alloc_gemma4_workspace(s, Id, dev)
+    out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+
+    def step():
+        api.moe_gemma4_block(s, blk.x, blk.norms, 1e-6, blk.mlp_w13, blk.mlp_w2,
+                             blk.router_w, blk.router_scale, 1e-6, inp.w13, inp.w2,
+                             inp.scale, out, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    weights = 3.0 * shp.H * (shp.I * min(shp.E, shp.T * shp.k) + Id) * 2
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if weights < 4 * l2 else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+    g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    g.replay()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = shp.flops() + 6.0 * shp.T * shp.H * Id
+    peaks, src = load_peaks()
+    print(json.dumps({
+        "metric": "Gemma 4 MoE block tokens/s (dense MLP + MoE + norms, 1 B200)",
+        "value": shp.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_name(args.config, shp) + f" + dense I={Id}",
+                   "l2": "flushed before every step" if flush is not None
+                   else "weights far larger than L2"},
+        "tflops": flops / (ms / 1e3) / 1e12,
+        "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
+        "peak_source": src, "clocks": clk}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.block:
+        run_block(args)
     else:
         run_ours(args)
 

@@ -315,6 +315,47 @@ MOE_API moe_status moe_permute_noalloc(const moe_shape* shape,
                                        int32_t* slot_row, cudaStream_t stream);
 
 /*
+ * moe_gemma4_block -- the MoE block of a Gemma 4 decoder layer (Gemma 4
+ * walkthrough, yeyulingfeng.com/587419.html, section 1: the DecoderLayer
+ * forward; section 7: its tensor flow).  From the residual x [T,H] bf16 (the
+ * state after the attention half):
+ *   h1  = post_ff_norm_1( mlp( pre_ff_norm(x) ) )      dense GeGLU MLP
+ *   h2  = post_ff_norm_2( moe( pre_ff_norm_2(x), router(x) ) )
+ *   out = post_ff_norm( h1 + h2 ) + x                  unweighted sum
+ * The dense MLP is a gated FFN with the experts' activation (shape->act)
+ * and intermediate size I_dense; the router is moe_router_logits on the raw
+ * residual; the MoE is moe_forward_ex on the normalised one (no shared
+ * experts: shape->n_shared must be 0).  Each norm is the standard RMSNorm
+ * with a gamma (section 3), in fp32: y = bf16(fl(fl(x / sqrt(fl(mean x^2) +
+ * eps)) * gamma)); every module returns bf16, h1 + h2 is one fp32 add
+ * rounded to bf16, and the residual add is fp32, rounded once to bf16.
+ *   x        [T,H] bf16; w13 [E,2I,H], w2 [E,H,I] bf16; scale [E] fp32 or NULL
+ *   out      [T,H] bf16 out; out_f32 NULL or [T,H] fp32 out: the output
+ *            before its final rounding
+ *   ws       moe_gemma4_workspace_size(shape, I_dense) bytes, 256-byte
+ *            aligned, owned by the caller
+ * Bad shapes or arguments return before any launch.
+ */
+typedef struct {
+  int32_t I_dense;                /* dense MLP intermediate size (multiple of 8) */
+  const moe_bf16* mlp_w13;        /* [2*I_dense, H], gate rows first */
+  const moe_bf16* mlp_w2;         /* [H, I_dense] */
+  const moe_bf16* norm_w[5];      /* [H] gammas: pre_ff, post_ff_1, pre_ff_2,
+                                     post_ff_2, post_ff (16-byte aligned) */
+  float eps;                      /* epsilon of those five norms */
+  const moe_bf16* router_w;       /* [E,H] GateLinear weight */
+  const moe_bf16* router_scale;   /* [H] */
+  float router_eps;
+} moe_gemma4_block_params;
+
+MOE_API size_t moe_gemma4_workspace_size(const moe_shape* shape, int32_t I_dense);
+MOE_API moe_status moe_gemma4_block(const moe_shape* shape, const moe_bf16* x,
+                                    const moe_gemma4_block_params* params,
+                                    const moe_bf16* w13, const moe_bf16* w2,
+                                    const float* scale, moe_bf16* out, float* out_f32,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * moe_read_error -- SYNCHRONISES ``stream``, then returns the status recorded
  * in the workspace error word by earlier calls on it (MOE_OK if none) and
  * clears the word.  ws is the device workspace used by those calls.

@@ -28,7 +28,8 @@ EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_router_logits",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_ex",
            "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string",
-           "moe_permute_noalloc", "moe_route_ex")
+           "moe_permute_noalloc", "moe_route_ex", "moe_gemma4_workspace_size",
+           "moe_gemma4_block")
 
 
 class MoEError(RuntimeError):
@@ -61,6 +62,13 @@ class moe_forward_opts(ctypes.Structure):
                 ("router_scale", ctypes.c_void_p),
                 ("router_eps", ctypes.c_float),
                 ("route", ctypes.POINTER(moe_route_opts))]
+
+
+class moe_gemma4_block_params(ctypes.Structure):
+    _fields_ = [("I_dense", ctypes.c_int32), ("mlp_w13", ctypes.c_void_p),
+                ("mlp_w2", ctypes.c_void_p), ("norm_w", ctypes.c_void_p * 5),
+                ("eps", ctypes.c_float), ("router_w", ctypes.c_void_p),
+                ("router_scale", ctypes.c_void_p), ("router_eps", ctypes.c_float)]
 
 
 class moe_shape(ctypes.Structure):
@@ -96,6 +104,10 @@ def _load() -> ctypes.CDLL:
                                    ctypes.c_size_t,
                                    ctypes.POINTER(moe_forward_opts), P]
     lib.moe_read_error.argtypes = [P, ctypes.c_size_t, P]
+    lib.moe_gemma4_workspace_size.argtypes = [S, ctypes.c_int32]
+    lib.moe_gemma4_workspace_size.restype = ctypes.c_size_t
+    lib.moe_gemma4_block.argtypes = [S, P, ctypes.POINTER(moe_gemma4_block_params), P, P,
+                                     P, P, P, P, ctypes.c_size_t, P]
     lib.moe_permute_noalloc.argtypes = [S, P, P, P, P, P]
     lib.moe_permute_noalloc.restype = st
     lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t,
@@ -105,7 +117,7 @@ def _load() -> ctypes.CDLL:
     for name in ("moe_router_logits", "moe_route", "moe_route_ex", "moe_permute",
                  "moe_expert_ffn",
                  "moe_combine",
-                 "moe_forward", "moe_forward_ex", "moe_read_error",
+                 "moe_forward", "moe_forward_ex", "moe_read_error", "moe_gemma4_block",
                  "moe_selftest_wait_timeout"):
         getattr(lib, name).restype = st
     return lib
@@ -281,3 +293,29 @@ def moe_selftest_wait_timeout(ws, timeout_us: int, stream=None):
     _check(lib.moe_selftest_wait_timeout(_p(ws), ws.numel(), timeout_us,
                                          _stream(stream)),
            "moe_selftest_wait_timeout")
+
+
+def moe_gemma4_workspace_size(shape, I_dense: int) -> int:
+    return int(lib.moe_gemma4_workspace_size(ctypes.byref(shape), I_dense))
+
+
+def moe_gemma4_block(shape, x, norms, eps, mlp_w13, mlp_w2, router_w, router_scale,
+                     router_eps, w13, w2, scale, out, ws, out_f32=None, stream=None):
+    """The Gemma 4 MoE block from the residual x [T,H]: norms = the five
+    gammas (pre_ff, post_ff_1, pre_ff_2, post_ff_2, post_ff); mlp_w13
+    [2*I_dense, H], mlp_w2 [H, I_dense]; ws of moe_gemma4_workspace_size
+    bytes (alloc_gemma4_workspace)."""
+    I_dense = int(mlp_w2.shape[-1])
+    prm = moe_gemma4_block_params(
+        I_dense, _p(mlp_w13), _p(mlp_w2), (ctypes.c_void_p * 5)(*[_p(g) for g in norms]),
+        float(eps), _p(router_w), _p(router_scale), float(router_eps))
+    _check(lib.moe_gemma4_block(ctypes.byref(shape), _p(x), ctypes.byref(prm), _p(w13),
+                                _p(w2), _p(scale), _p(out), _p(out_f32), _p(ws),
+                                ws.numel(), _stream(stream)), "moe_gemma4_block")
+
+
+def alloc_gemma4_workspace(shape, I_dense: int, device="cuda") -> torch.Tensor:
+    n = moe_gemma4_workspace_size(shape, I_dense)
+    if n == 0:
+        raise MoEError(2, "moe_gemma4_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)  # error words zeroed

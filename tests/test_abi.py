@@ -170,3 +170,28 @@ def test_route_ex_refuses_bad_options(api, opts, status):
                                 None, fake, None, None, ws,
                                 api.moe_workspace_size(s), ctypes.byref(fo), None)
     assert rc == status
+
+
+def test_gemma4_block_refuses_bad_arguments(api):
+    # rejected on the host before any launch: no GPU needed
+    s = api.make_shape(T=4, H=64, E=8, k=2, I=32)
+    assert api.moe_gemma4_workspace_size(s, 48) > api.moe_workspace_size(s)
+    assert api.moe_gemma4_workspace_size(s, 44) == 0        # I_dense % 8
+    sh = api.make_shape(T=4, H=64, E=8, k=2, I=32, n_shared=1, I_shared=32)
+    assert api.moe_gemma4_workspace_size(sh, 48) == 0       # no shared experts
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced
+    ws = ctypes.c_void_p(1 << 21)
+    need = api.moe_gemma4_workspace_size(s, 48)
+    prm = api.moe_gemma4_block_params(48, fake.value, fake.value,
+                                      (ctypes.c_void_p * 5)(*[1 << 20] * 5), 1e-6,
+                                      fake.value, fake.value, 1e-6)
+    f = api.lib.moe_gemma4_block
+    assert f(ctypes.byref(s), fake, None, fake, fake, None, fake, None, ws, need,
+             None) == 1                                      # no params
+    assert f(ctypes.byref(s), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
+             need - 1, None) == 3                            # workspace too small
+    prm.norm_w[2] = None
+    assert f(ctypes.byref(s), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
+             need, None) == 1                                # a gamma missing
+    assert f(ctypes.byref(sh), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
+             need, None) == 2                                # shared experts
