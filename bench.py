@@ -734,7 +734,10 @@ def run_block(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     weights = 3.0 * shp.H * (shp.I * min(shp.E, shp.T * shp.k) + Id) * 2
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if weights < 4 * l2 else None
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # external events: captured as event-record nodes that stay timeable
+    # after the replay
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True))
           for _ in range(args.steps)]
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
