@@ -32,7 +32,9 @@
 // in flight without holding them in registers (the register-prefetch form
 // holds one or two and is bound by DRAM latency at this size).  Each lane
 // reads back only the bytes it copied itself, so the ring needs no barrier.
-// decode_w2 starts its ring before it waits for h.
+// In decode_w13_few the four warps take K chunks round-robin, so a CTA reads
+// 256 contiguous bytes of each weight row at a time; decode_w2_few starts its
+// ring before it waits for h.
 #include <algorithm>
 
 #include "route_impl.cuh"
