@@ -30,6 +30,7 @@
 //     epilogue of tile i overlap the MMAs of tile i+1.
 // Every wait is bounded (tc_ptx.cuh: mbar_wait); on a timeout the block
 // records MOE_ERR_TIMEOUT, drains what it issued and frees its TMEM.
+#include <atomic>
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -46,6 +47,7 @@ constexpr uint32_t TMEM_COLS = 2 * BN_ACC;
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kMaxStages = 6;
 constexpr int kPanel = 16;  // m-blocks per panel of the tile order
+constexpr int kMaxDevices = 64;  // per-device caches of launch attributes
 
 // CG = CTAs per MMA: 1 (M=128 per CTA, B tile 256 rows per CTA, 4 stages) or
 // 2 (a CTA pair computes M=256: each CTA loads its own 128 A rows and half of
@@ -565,13 +567,18 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, uint64_t inner,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// SMs of the current device (cached per device)
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  int n = cached ? cache[dev].load() : 0;
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+      n = 148;
+    if (cached) cache[dev].store(n);
   }
   return n;
 }
@@ -627,13 +634,17 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   const size_t smem = 1024 + (size_t)C::STAGES * (A_STAGE + C::B_STAGE) +
                       sizeof(EpiSmem) + sizeof(Ctl) +
                       (sizeof(int64_t) + sizeof(int32_t)) * (size_t)(a.G + 1);
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory opt-in is a per-device attribute: set it once on
+  // every device this process launches on
+  static std::atomic<bool> attr_set[kMaxDevices];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices || !attr_set[dev].load()) {
     e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, NH>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(true);
   }
   // units: at most (cap / BM) m-tiles, grouped CG at a time, per n-tile
   const int64_t max_units = ((a.cap / BM) / CG + a.G) * p.NT;
