@@ -13,6 +13,11 @@
  *            W13 = [W1; W3] packs the gate rows first, then the up rows;
  *   combine  out[t] = sum_j w[t,j] y[t,j] + sum_s y_shared[t,s]  (bf16 out).
  *
+ * Around it: the router ahead of the routing (moe_router_logits), routing
+ * variants (moe_route_ex: sigmoid scoring, expert groups), the Gemma 4 MoE
+ * block with its parallel dense MLP and gamma norms (moe_gemma4_block), and
+ * a permutation that needs no workspace (moe_permute_noalloc).
+ *
  * Conventions (every entry point):
  *   - All pointers are DEVICE pointers unless a parameter says otherwise.
  *     The caller owns every buffer.  The library never allocates, frees or
