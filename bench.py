@@ -20,6 +20,10 @@ no collective on the data path (weak scaling).
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
 bounded token sample per step) and prints the same line with
 ``"impl": "reference"``.
+
+``--block I_DENSE`` times the Gemma 4 MoE block instead (the config's MoE
+with a parallel dense MLP of that intermediate size, the router on the
+residual and the five gamma norms; one GPU, device-timed).
 """
 from __future__ import annotations
 
