@@ -131,5 +131,5 @@ def test_forward_from_hidden_states(api, path, T):
                                           scale=inp.scale)
     assert np.array_equal(ids.cpu().numpy(), ref_ids)
     assert np.allclose(wt.cpu().numpy(), ref_w, rtol=1e-6, atol=0)
-    assert_out_close(out32, want, f"path {path}")
+    assert_out_close(out32, want, f"path {path}", bf16=out)
     assert torch.equal(out, out32.to(torch.bfloat16))

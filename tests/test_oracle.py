@@ -349,6 +349,35 @@ def test_router_activations_are_bf16_before_the_projection():
         assert np.array_equal(torch.tensor(z).to(torch.bfloat16).float().numpy(), z)
 
 
+def test_router_rounds_after_the_constant_and_again_after_the_scale():
+    # The constant multiply and the scale multiply are two bf16 operations
+    # (Gemma4Router.forward on the vLLM page: x * root_size.to(x.dtype), then
+    # x * scale, both in the activation dtype), so each product is rounded on
+    # its own.  Worked by hand, H = 100, eps = 0:
+    #   row = [1.5, 1.75, 0.25, 0.25, 0.75, 0, then 94 entries of +-1]; its
+    #   squares sum to 2.25 + 3.0625 + 0.125 + 0.5625 + 94 = 100, so the mean
+    #   square is 1, 1/sqrt(1) = 1 and the normalised row is the row itself.
+    #   c = bf16(fp32(100^-0.5)) = 205/2048 = 0.10009765625.
+    #   h = 0: 1.5 c = 615/4096; 615 = 0b1001100111 has 10 significant bits,
+    #          its 8-bit rounding is 154/1024 = 0.150390625.  Times the scale
+    #          1.375: 211.75/1024 -> 212/1024 = 0.20703125.
+    #          One rounding of 1.5 c 1.375 = 845.625/4096 gives instead
+    #          844/4096 = 0.2060546875.
+    #   h = 1: 1.75 c = 1435/8192 -> 179/1024 = 0.1748046875 (the remainder
+    #          0b011 is under half); times 1.5: 268.5/1024 -> 268/1024 =
+    #          0.26171875.  One rounding of 2152.5/8192 gives 2160/8192 =
+    #          0.263671875.
+    # One-hot GateLinear rows return b_0 and b_1 as the two logits.
+    H = 100
+    row = [1.5, 1.75, 0.25, 0.25, 0.75, 0.0] + [(-1.0) ** i for i in range(94)]
+    s = [1.375, 1.5] + [1.0] * (H - 2)
+    w = torch.zeros(2, H)
+    w[0, 0] = w[1, 1] = 1.0
+    z = oracle.router_logits(_bf([row]), w.to(torch.bfloat16), _bf(s), 0.0)
+    assert z[0, 0] == np.float32(0.20703125)
+    assert z[0, 1] == np.float32(0.26171875)
+
+
 def test_router_zero_row_stays_finite():
     # eps keeps the norm of an all-zero row finite: its logits are zero
     x, w, s = _router_case(3, 64, 4, 4)
@@ -553,3 +582,130 @@ def test_block_matches_a_float64_restatement():
     want = (_norm_torch(h, blk.norms[4]) + x).numpy()
     d = out - want
     assert np.abs(d).max() <= 0.05 * np.sqrt(np.mean((want - x.numpy()) ** 2))
+
+
+# Hand-worked witnesses of the block's bf16 module boundaries.  Each case
+# is built so that the value it checks is exact, or is decided by a
+# rounding that a missing module boundary would change.  H = 5, eps = 0,
+# one expert (E = k = 1, I = 1, per_expert_scale 1), x tiny (2^-40 scale):
+#   * a row whose squares sum to 5 has mean square 1: it normalises to
+#     itself (1/sqrt(1) = 1).  R = [1.0625, 0.03125, 1.15625, 1.09375,
+#     1.15625] is such a row (1.12890625 + 0.0009765625 + 2 * 1.3369140625 +
+#     1.1962890625 = 5);
+#   * a row of equal magnitudes +-m normalises to +-1 (up to one fp32 ulp),
+#     so its gamma norm returns +-gamma exactly;
+#   * a gate pre-activation of 64 or more passes SiLU and tanh-GELU
+#     unchanged in double (exp(-64) and 1 - tanh(...) are below 2^-53);
+#   * x is below half an fp32 ulp of every output, so the final fp32
+#     residual add returns the last norm's output itself (a double add
+#     would not).
+# 1.0625 * 1.0625 = 1.12890625 lies halfway between the bf16 values 1.125
+# and 1.1328125: round-to-nearest-even gives 1.125.
+
+_R5 = [1.0625, 0.03125, 1.15625, 1.09375, 1.15625]
+
+
+def _e5(p, c=1.0):
+    v = [0.0] * 5
+    v[p] = c
+    return v
+
+
+def _block5(x, norms, mlp13, mlp2, w13, w2, act_kind):
+    b = lambda a: torch.tensor(np.asarray(a, np.float64)).to(torch.bfloat16)  # noqa: E731
+    return oracle.gemma4_block(
+        b([x]), tuple(b(g) for g in norms), 0.0, b(np.zeros((1, 5))), b([1.0] * 5),
+        0.0, b(w13), b(w2), torch.ones(1), b(mlp13), b(mlp2), 1, act_kind)[0]
+
+
+@pytest.mark.parametrize("act_kind", [0, 1])
+def test_block_rounds_the_branch_sum_and_the_last_norm(act_kind):
+    # Both branches: gate 64 e_0, up e_0 on a normalised row of ones, and a
+    # w2 column of ones: each branch output is a row of equal magnitudes, so
+    # h1 = gamma_post1 and h2 = gamma_post2 exactly.
+    #   h1 + h2 = [1 + 0.0634765625, 0.03125, 1.15625, 1.09375, 1.15625]; its
+    #   first entry 1.0634765625 rounds to the bf16 1.0625, which gives the
+    #   row R (mean square 1).  The last norm (gamma [1.0625, 1, 1, 1, 1])
+    #   returns bf16(1.0625 * 1.0625) = 1.125 (the tie) and R elsewhere.
+    # Without the rounding of h1 + h2 the first entry would come out as
+    # 1.1328125; without the last norm's rounding as 1.12890625; with a
+    # double residual add every entry would carry x.
+    one, e0 = [1.0] * 5, _e5(0)
+    norms = (one, [1.0, *_R5[1:]], one, [0.0634765625, 0, 0, 0, 0],
+             [1.0625, 1, 1, 1, 1])
+    out = _block5([2.0 ** -40] * 5, norms, [e0, e0], np.ones((5, 1)), [[e0, e0]],
+                  np.ones((1, 5, 1)), act_kind)
+    assert out.tolist() == [1.125, *_R5[1:]]
+
+
+@pytest.mark.parametrize("act_kind", [0, 1])
+def test_block_rounds_the_post_norm_outputs(act_kind):
+    # Dense MLP: gate 64 e_0, up e_0 on a row of ones gives the hidden value
+    # 64 exactly, and its w2 column R gives y1 = 64 R (bf16, mean square
+    # 64^2), which normalises to R.  With gamma_post1 = [1.0625, 1, 1, 1, 1]:
+    #   h1 = [bf16(1.12890625) = 1.125, R[1:]].
+    # MoE branch: equal magnitudes, gamma_post2 = [-0.0615234375, 0, ...]:
+    #   h2 = [-0.0615234375, 0, 0, 0, 0].
+    # h1 + h2 = [1.0634765625, R[1:]] -> bf16 -> R, which the last norm
+    # (gamma 1) returns as it is.  Had h1 not been rounded,
+    # 1.12890625 - 0.0615234375 = 1.0673828125 would round to 1.0703125.
+    one = [1.0] * 5
+    norms = (one, [1.0625, 1, 1, 1, 1], one, [-0.0615234375, 0, 0, 0, 0], one)
+    out = _block5([2.0 ** -40] * 5, norms, [_e5(0, 64), _e5(0)],
+                  np.array(_R5).reshape(5, 1), [[_e5(0, 64), _e5(0)]],
+                  np.ones((1, 5, 1)), act_kind)
+    assert out.tolist() == _R5
+
+
+@pytest.mark.parametrize("act_kind", [0, 1])
+def test_block_rounds_the_input_norm_and_the_branch_output(act_kind):
+    # x = 2^-40 R normalises to R; gamma_pre = [1.0625, 1, 1, 1, 1] gives
+    #   a1 = [bf16(1.12890625) = 1.125, R[1:]]            (the input norm)
+    # Dense MLP, I = 2: both gates 64 e_0 (pre-activation 72, passed as it
+    # is), ups e_0 and 0.25 e_3:
+    #   hidden = [72 * 1.125, 72 * 0.2734375] = [81, 19.6875]
+    #   w2 = [e_0; e_1]: y1 = [81, 19.6875, 0, 0, 0]; 19.6875 is halfway
+    #   between the bf16 values 19.625 and 19.75 -> 19.75 (the branch
+    #   output rounds to bf16).
+    # Post norm of [81, 19.75, 0, 0, 0] (gamma 1): mean square 1390.2125,
+    #   1/sqrt in fp32 = 0.02682004, products 2.1724231 and 0.52969575 ->
+    #   bf16 2.171875 and 0.53125.  The MoE branch has gamma 0 (h2 = 0).
+    # Last norm: mean square 0.9998535, 1/sqrt = 1.0000733, products
+    #   2.1720343 and 0.5312889 -> bf16 2.171875 and 0.53125.
+    # Had the input norm not rounded (a1_0 = 1.12890625), y1 would be
+    # [81.5, 19.75] and the second entry 0.52734375; had y1 not been rounded
+    # ([81, 19.6875]), also 0.52734375.  The last three entries are x itself
+    # (zero rows of the last norm, plus the residual).
+    one, zero = [1.0] * 5, [0.0] * 5
+    x = [2.0 ** -40 * r for r in _R5]
+    norms = ([1.0625, 1, 1, 1, 1], one, one, zero, one)
+    mlp2 = np.zeros((5, 2))
+    mlp2[0, 0] = mlp2[1, 1] = 1.0
+    out = _block5(x, norms, [_e5(0, 64), _e5(0, 64), _e5(0), _e5(3, 0.25)], mlp2,
+                  [[_e5(0, 64), _e5(0)]], np.ones((1, 5, 1)), act_kind)
+    want = [2.171875, 0.53125] + [float(np.float32(v)) for v in x[2:]]
+    assert out.tolist() == want
+
+
+# -------------------------------------------- the output tolerance reading
+
+@pytest.mark.parametrize("shape,seed", [
+    (inputs.Shape(T=200, H=256, E=4, k=2, I=192, act=1), 0),
+    (inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1), 0)])
+def test_bf16_rounding_of_the_exact_output_exceeds_the_bound(shape, seed):
+    # Why the 2e-2 x RMS bound is applied to the fp32 layer output (before
+    # its bf16 rounding) and the bf16 tensor gets 2^-8 |want| on top: the
+    # exact fp64 answer rounded to bf16 already misses 2e-2 x RMS on these
+    # batches (the second is a shape the GPU parity tests run).  A bf16 value
+    # keeps 8 significant bits, so its rounding error can reach |v| 2^-8,
+    # and these outputs have heavy tails (max |out| over 5 x RMS).
+    inp = inputs.make_inputs(shape, seed=seed, scale="uniform")
+    out, _, _ = oracle.forward(inp.x, inp.logits, inp.w13, inp.w2, shape.k,
+                               shape.act, scale=inp.scale)
+    rms = float(np.sqrt(np.mean(out ** 2)))
+    rounded = torch.from_numpy(out).to(torch.bfloat16).double().numpy()
+    err = np.abs(rounded - out)
+    assert err.max() > 2e-2 * rms
+    assert np.abs(out).max() > 5 * rms
+    # ... and the rounding stays inside the half-ulp bound the bf16 check uses
+    assert (err <= 2.0 ** -8 * np.abs(out)).all()

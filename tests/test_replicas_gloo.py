@@ -31,7 +31,7 @@ def _worker(rank, world, port, times, out):
 def test_two_replicas_take_the_slowest_rank():
     port = 29500 + os.getpid() % 2000
     times = [2.5, 3.25]
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of a threaded process
         out = m.dict()
         mp.spawn(_worker, args=(2, port, times, out), nprocs=2, join=True)
         got = dict(out)
