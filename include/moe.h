@@ -174,6 +174,10 @@ MOE_API moe_status moe_route_ex(const moe_shape* shape, const float* logits,
  *   slot_row     [T,k+S] int32 out: the row of (t, j), and of (t, shared s)
  *                at column k+s
  *   ws           workspace of ws_bytes >= moe_workspace_size bytes
+ * An id outside [0,E) is a caller error that the kernels catch: its slot is
+ * given no row (no segment counts it), its slot_row entry is -1, nothing is
+ * written out of bounds, and the workspace error word records
+ * MOE_ERR_INVALID_ARG, which moe_read_error returns.
  */
 MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
                        int32_t* offsets, int32_t* sorted_slots,
@@ -206,6 +210,8 @@ MOE_API moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
  *   y_perm [cap,H] fp32, slot_row [T,k+S] int32, w [T,k] fp32
  *   out    [T,H] bf16 out: w[t,j] * y rounded, then added in fp32 in order
  *          j = 0..k-1, then the shared experts; rounded once to bf16
+ * A negative slot_row entry (a slot that moe_permute gave no row) adds
+ * nothing.
  */
 MOE_API moe_status moe_combine(const moe_shape* shape, const float* y_perm,
                        const int32_t* slot_row, const float* w, moe_bf16* out,
@@ -312,6 +318,11 @@ MOE_API moe_status moe_forward_ex(
  *     the GPU (other streams, other host threads) race and must not overlap.
  *     Every call writes the scratch it later reads, so nothing in the array
  *     has to start at zero and the previous call's leftovers do no harm.
+ *   - An id outside [0,E) gets no row and slot_row -1, as in moe_permute;
+ *     with no workspace there is no error word to record it in.
+ *   - The cached address is kept with the id of the context it belongs to;
+ *     after a device reset (a new primary context) the next call looks it
+ *     up again, so that call too should come before any stream capture.
  */
 #define MOE_NOALLOC_MAX_SLOTS 131072
 MOE_API moe_status moe_permute_noalloc(const moe_shape* shape,

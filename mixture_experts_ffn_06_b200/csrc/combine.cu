@@ -44,6 +44,7 @@ combine_kernel(const float4* __restrict__ y_perm,
       // product rounded, then added (no fma), the same arithmetic as the
       // fused path's weighted epilogue followed by sum_rows_kernel
       for (int j = 0; j < ks; ++j) {
+        if (rows[j] < 0) continue;  // a slot moe_permute gave no row
         const float4 v = __ldg(y_perm + rows[j] + c);
         const float wt = wts[j];
         a0 = __fadd_rn(a0, __fmul_rn(wt, v.x));

@@ -72,11 +72,13 @@ cudaError_t launch_router_logits(const __nv_bfloat16* x, const __nv_bfloat16* w_
 // pdl on any launch function: launch its first kernel as a programmatic
 // dependent of the previous kernel on the stream (later kernels of the same
 // function always are).
+// err (may be null): error word that records MOE_ERR_INVALID_ARG when an id
+// lies outside [0,E) (such slots get no row and slot_row -1).
 cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* offsets, int32_t* sorted_slots,
                           int32_t* slot_row, int64_t cap, int32_t* lt_count,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
-                          cudaStream_t st, bool pdl = false);
+                          uint32_t* err, cudaStream_t st, bool pdl = false);
 
 // Gathers x rows into x_perm for the rows of groups [0, G) (padding rows are
 // left as they are); when acc is given it also zeroes acc[0, n_acc)

@@ -124,13 +124,17 @@ layout_scan(const int32_t* __restrict__ lt_count, int64_t n_lt, int E, int S,
 }
 
 // Index space: [0,R) routed slots, then [R, R+T*S) shared-expert slots.
+// A routed slot whose id lies outside [0,E) (a caller's bad input to
+// moe_permute) is given no row: layout_count did not count it, its slot_row
+// entry is set to -1, and the error word (when given) records
+// MOE_ERR_INVALID_ARG.
 __global__ void __launch_bounds__(256)
 layout_scatter(const int32_t* __restrict__ ids, int64_t T, int k, int E, int S,
                const int32_t* __restrict__ offsets,
                const int32_t* __restrict__ lt_base,
                const int32_t* __restrict__ lt_rank,
                int32_t* __restrict__ sorted_slots,
-               int32_t* __restrict__ slot_row) {
+               int32_t* __restrict__ slot_row, uint32_t* err) {
   const int64_t R = T * k, RS = T * S;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   pdl_wait();
@@ -139,6 +143,12 @@ layout_scatter(const int32_t* __restrict__ ids, int64_t T, int k, int E, int S,
        i += stride) {
     if (i < R) {
       const int e = ids[i];
+      if (e < 0 || e >= E) {
+        const int64_t t = i / k;
+        slot_row[t * (k + S) + (i - t * k)] = -1;
+        record_error(err, MOE_ERR_INVALID_ARG);
+        continue;
+      }
       const int64_t b = i / kLayoutTile;
       const int64_t row = (int64_t)offsets[e] + lt_base[b * E + e] + lt_rank[i];
       sorted_slots[row] = (int32_t)i;
@@ -233,7 +243,7 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                           int32_t* offsets, int32_t* sorted_slots,
                           int32_t* slot_row, int64_t cap, int32_t* lt_count,
                           int32_t* lt_base, int32_t* lt_rank, int64_t n_lt,
-                          cudaStream_t st, bool pdl) {
+                          uint32_t* err, cudaStream_t st, bool pdl) {
   const int64_t R = s.T * s.k;
   const int E = s.E, S = s.n_shared, G = E + S;
   const int P = s.pad ? s.pad : kSegPad;
@@ -262,7 +272,7 @@ cudaError_t launch_layout(const moe_shape& s, const int32_t* ids,
                   dim3((unsigned)(blocks < 65535 * 16 ? blocks : 65535 * 16)),
                   dim3(256), 0, st, true, ids, s.T, s.k, E, S,
                   (const int32_t*)offsets, (const int32_t*)lt_base,
-                  (const int32_t*)lt_rank, sorted_slots, slot_row);
+                  (const int32_t*)lt_rank, sorted_slots, slot_row, err);
     if (e != cudaSuccess) return e;
   }
   e = launch_ex(layout_pad, dim3((unsigned)(G + 148)), dim3(256), 0, st, true,

@@ -252,7 +252,8 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
       *shape, ids, offsets, sorted_slots, slot_row, m.cap,
       reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
       reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
-      reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt, stream));
+      reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt,
+      reinterpret_cast<uint32_t*>(at(ws, m.err)), stream));
 }
 
 moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
@@ -387,7 +388,8 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
                     reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
                     reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
                     reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt,
-                    stream, /*pdl=*/true) != cudaSuccess)
+                    reinterpret_cast<uint32_t*>(at(ws, m.err)), stream,
+                    /*pdl=*/true) != cudaSuccess)
     return MOE_ERR_CUDA;
   const bool det = opts && opts->deterministic;
   float* acc = reinterpret_cast<float*>(at(ws, m.acc));

@@ -10,8 +10,10 @@
 // only the scratch pointers differ.
 //
 // Host code must not hand the symbol itself to a kernel: on the host it is a
-// stand-in, not a device address.  The device address is looked up once per
-// device with cudaGetSymbolAddress (with that device current) and cached.
+// stand-in, not a device address.  The device address is looked up with
+// cudaGetSymbolAddress (with that device current) and cached per device,
+// together with the id of the context it belongs to; when the context has
+// changed (after a device reset) it is looked up again.
 #include <mutex>
 
 #include "internal.cuh"
@@ -30,21 +32,56 @@ static __device__ __align__(256) int32_t g_permute_scratch[kScratchInts];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int32_t* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context id of each entry
 
-// Device address of g_permute_scratch on the current device (cached).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (0 when there is none or the driver
+// cannot say).  A device reset gives the device a new primary context with a
+// new id, so an address cached under the old id is never reused.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_permute_scratch on the current device, cached per
+// device and context.
 cudaError_t scratch_address(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (dev >= 0 && dev < kMaxDevices && g_scratch_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (slot && g_scratch_ptr[dev] && ctx != 0 && g_scratch_ctx[dev] == ctx) {
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
   }
   void* p = nullptr;
   e = cudaGetSymbolAddress(&p, g_permute_scratch);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kMaxDevices) g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  if (slot) {
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    g_scratch_ctx[dev] = current_context_id();  // the lookup made it current
+  }
   *out = static_cast<int32_t*>(p);
   return cudaSuccess;
 }
@@ -74,6 +111,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* shape,
   if (n_lt < 1) n_lt = 1;
   const int64_t cap = workspace_map(*shape).cap;
   const cudaError_t e = launch_layout(*shape, ids, offsets, sorted_slots, slot_row,
-                                      cap, lt_count, lt_base, lt_rank, n_lt, stream);
+                                      cap, lt_count, lt_base, lt_rank, n_lt,
+                                      /*err=*/nullptr, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

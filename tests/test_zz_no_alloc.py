@@ -79,3 +79,61 @@ def test_noalloc_refuses_batches_over_its_limit(api):
     rc = api.lib.moe_permute_noalloc(ctypes.byref(bad), fake, fake, fake,
                                      fake, null)
     assert rc == 1  # MOE_ERR_INVALID_ARG
+
+
+def _distinct_ids(T, E, k, seed):
+    # k distinct experts per token, uniformly random (no margin needed: the
+    # permutation takes ids, not logits)
+    g = torch.Generator().manual_seed(seed)
+    return torch.rand(T, E, generator=g).argsort(dim=1)[:, :k].to(torch.int32)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_its_limit_with_512_experts(api):
+    # T*k == MOE_NOALLOC_MAX_SLOTS and E = 512: every layout block's counts
+    # use the full 512-expert stride of the scratch, and layout_count needs
+    # its shared-memory opt-in (32 warps x 512 counters)
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    T, E, k = 16384, 512, 8
+    assert T * k == 131072
+    ids = _distinct_ids(T, E, k, seed=11).cuda()
+    s = api.make_shape(T=T, H=64, E=E, k=k, I=64)
+    ref = _outputs(api, s, E, 0, T, k)
+    ws = api.alloc_workspace(s)
+    api.moe_permute(s, ids, *ref, ws)
+    got = _outputs(api, s, E, 0, T, k)
+    api.moe_permute_noalloc(s, ids, *got)
+    torch.cuda.synchronize()
+    for r, g, what in zip(ref, got, ("offsets", "sorted_slots", "slot_row")):
+        assert torch.equal(r, g), what
+
+
+@pytest.mark.gpu
+def test_noalloc_call_captured_in_a_cuda_graph(api):
+    # the use case of the entry point: one call before capture (it looks up
+    # the scratch address), then a call recorded into a CUDA graph and
+    # replayed, with new ids copied into the captured input buffer
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    T, E, k = 5000, 128, 8
+    s = api.make_shape(T=T, H=64, E=E, k=k, I=64)
+    ids = _distinct_ids(T, E, k, seed=12).cuda()
+    outs = _outputs(api, s, E, 0, T, k)
+    api.moe_permute_noalloc(s, ids, *outs)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        api.moe_permute_noalloc(s, ids, *outs, stream=stream)
+    for seed in (13, 14):
+        ids.copy_(_distinct_ids(T, E, k, seed=seed).cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = _outputs(api, s, E, 0, T, k)
+        ws = api.alloc_workspace(s)
+        api.moe_permute(s, ids, *ref, ws)
+        torch.cuda.synchronize()
+        for r, g, what in zip(ref, outs, ("offsets", "sorted_slots", "slot_row")):
+            assert torch.equal(r, g), f"replay {seed}: {what}"
+    del graph
