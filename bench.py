@@ -17,6 +17,16 @@ With N > 1 (torchrun, one rank per GPU) every rank runs its own replica of
 the layer on its own batch: the layer has no cross-GPU exchange, so there is
 no collective on the data path (weak scaling).
 
+The default run (the Mixtral-shaped headline, one GPU) adds a ``configs``
+key with one entry for each other workload of the benchmark -- the
+many-small-experts and skewed prefills and the decode sweep T = 1, 4, 16,
+64, 256 -- each device-timed the same way, with its roofline fraction, its
+CPU baseline and ``parity``: the layer outputs the oracle computed for the
+baseline's token sample set beside the GPU's (max |err| / RMS of the fp32
+and bf16 outputs), and the routing ids, gate weights and layout of the whole
+batch compared with the oracle's.  The headline carries the same ``parity``.
+``--headline-only`` leaves the other workloads out.
+
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
 bounded token sample per step) and prints the same line with
 ``"impl": "reference"``.
@@ -69,6 +79,8 @@ def parse():
                     help="time the Gemma 4 MoE block (dense MLP of this "
                          "intermediate size in parallel with the MoE, gamma "
                          "norms, router on the residual) instead of the layer")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other workloads' lines (the configs key)")
     ap.add_argument("--router", action="store_true",
                     help="start from hidden states: the router (RMSNorm, scale, "
                          "GateLinear) computes the logits inside every step")
@@ -220,38 +232,80 @@ def traffic_for(kernel_src: str, config: str, shape_override):
 
 # ----------------------------------------------------------- CPU baseline
 
-def cpu_oracle_rate(inp, budget_s: float = 12.0, max_rounds: int = 64):
-    """Time the oracle as it stands on the host cores, on rounds of
-    ``cores`` tokens until ``budget_s`` has passed.  Returns
-    (tokens/s, cores used, tokens, seconds)."""
+def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int = 1):
+    """The CPU baseline: the oracle as it stands, timed on the host cores, on
+    rounds of ``cores`` tokens drawn from the batch until ``budget_s`` has
+    passed.  The layer outputs it computes for those tokens are then set
+    beside the GPU's for the same tokens, and the routing and the layout of
+    the whole batch beside the library's (``gpu``: host copies of one call's
+    out, out_f32, ids, w and moe_permute's offsets / sorted_slots /
+    slot_row).  Returns (baseline, parity) dicts."""
     import numpy as np
     import oracle
     cores = oracle.num_threads()
-    T = inp.shape.T
+    shp = inp.shape
+    T = shp.T
     host = {k: (None if v is None else v.cpu()) for k, v in
             dict(x=inp.x, logits=inp.logits, w13=inp.w13, w2=inp.w2,
                  scale=inp.scale, w13_sh=inp.w13_sh, w2_sh=inp.w2_sh).items()}
     xu = oracle._u16(host["x"])
     w13u, w2u = oracle._u16(host["w13"]), oracle._u16(host["w2"])
     sh13, sh2 = oracle._u16(host["w13_sh"]), oracle._u16(host["w2_sh"])
-    rng = np.random.default_rng(1)
+    rng = np.random.default_rng(seed)
     per_round = min(cores, T)
     done, elapsed, rounds = 0, 0.0, 0
+    toks, outs = [], []
     while rounds < max_rounds and (elapsed < budget_s or rounds == 0):
-        tok = rng.choice(T, per_round, replace=False)
+        tok = np.sort(rng.choice(T, per_round, replace=False))
         t0 = time.perf_counter()
-        oracle.forward(xu, host["logits"], w13u, w2u, inp.shape.k,
-                       inp.shape.act, scale=host["scale"], w13_sh=sh13,
-                       w2_sh=sh2, tokens=tok, nthreads=per_round)
+        o, _, _ = oracle.forward(xu, host["logits"], w13u, w2u, shp.k, shp.act,
+                                 scale=host["scale"], w13_sh=sh13, w2_sh=sh2,
+                                 tokens=tok, nthreads=per_round)
         elapsed += time.perf_counter() - t0
+        toks.append(tok)
+        outs.append(o)
         done += per_round
         rounds += 1
-    return done / elapsed, per_round, done, elapsed
+    baseline = {"value": done / elapsed, "unit": UNIT, "cores": per_round,
+                "kind": "oracle",
+                "sample": f"{done} tokens drawn from the same {T}-token batch in "
+                          f"rounds of {per_round}, full layer per token (fp64), "
+                          f"{elapsed:.1f} s"}
+
+    tok = np.concatenate(toks)
+    want = np.concatenate(outs)
+    got32 = gpu["out_f32"][tok].astype(np.float64)
+    gotbf = gpu["out"][tok].astype(np.float64)
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    bound = 2e-2 * rms + 2.0 ** -8 * np.abs(want)
+    ids_ref, w_ref = oracle.route(host["logits"], shp.k, scale=host["scale"])
+    lay = oracle.layout(ids_ref, shp.E, shp.n_shared, 128)
+    lay_bad = sum(int((np.asarray(g) != np.asarray(w)).sum())
+                  for g, w in zip(gpu["layout"], lay))
+    parity = {
+        "tokens_compared": int(np.unique(tok).size),
+        "out_f32_max_err_over_rms": float(np.abs(got32 - want).max() / rms),
+        "out_bf16_max_err_over_rms": float(np.abs(gotbf - want).max() / rms),
+        "bf16_within_bound": bool((np.abs(gotbf - want) <= bound).all()),
+        "ids_mismatched": int((gpu["ids"] != ids_ref).sum()),
+        "weights_max_rel_err": float((np.abs(gpu["w"].astype(np.float64) - w_ref)
+                                      / np.abs(w_ref)).max()),
+        "layout_entries_mismatched": lay_bad,
+        "tolerance": "out_f32 max|err| <= 2e-2 x RMS(oracle); bf16 within "
+                     "2e-2 x RMS + 2^-8 |oracle|; ids and layout bit-exact; "
+                     "weights 1e-6 relative",
+    }
+    parity["pass"] = (parity["out_f32_max_err_over_rms"] <= 2e-2
+                      and parity["bf16_within_bound"]
+                      and parity["ids_mismatched"] == 0
+                      and parity["layout_entries_mismatched"] == 0
+                      and parity["weights_max_rel_err"] <= 1e-6)
+    return baseline, parity
 
 
 # ---------------------------------------------------------------- our arm
 
-def touched_experts(api, s, inp, ws) -> int:
+def touched_experts(api, s, inp) -> int:
     """Distinct experts the batch routes to (+ shared experts), from one call
     of the library's own routing."""
     import torch
@@ -260,6 +314,210 @@ def touched_experts(api, s, inp, ws) -> int:
     w = torch.empty(shp.T, shp.k, dtype=torch.float32, device=inp.x.device)
     api.moe_route(s, inp.logits, inp.scale, ids, w)
     return int(torch.unique(ids).numel()) + shp.n_shared
+
+
+def gpu_result(api, inp, s, path, args):
+    """One call of the layer with every optional output, copied to the host
+    (for the parity comparison of the CPU-baseline leg)."""
+    import torch
+    shp = inp.shape
+    dev = inp.x.device
+    ws = api.alloc_workspace(s, dev)
+    out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty(shp.T, shp.H, dtype=torch.float32, device=dev)
+    ids = torch.empty(shp.T, shp.k, dtype=torch.int32, device=dev)
+    w = torch.empty(shp.T, shp.k, dtype=torch.float32, device=dev)
+    api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                       inp.w2_sh, out, ws, ids_out=ids, w_out=w, out_f32=out32,
+                       path=path, deterministic=args.deterministic,
+                       cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs])
+    cap = api.moe_layout_capacity(s)
+    G = shp.E + shp.n_shared
+    lay = (torch.empty(G + 1, dtype=torch.int32, device=dev),
+           torch.empty(cap, dtype=torch.int32, device=dev),
+           torch.empty(shp.T, shp.k + shp.n_shared, dtype=torch.int32, device=dev))
+    api.moe_permute(s, ids, *lay, ws)
+    torch.cuda.synchronize()
+    if api.moe_read_error(ws) != 0:
+        raise RuntimeError("device error in the parity call")
+    return {"out": out.float().cpu().numpy(), "out_f32": out32.cpu().numpy(),
+            "ids": ids.cpu().numpy(), "w": w.cpu().numpy(),
+            "layout": tuple(t.cpu().numpy() for t in lay)}
+
+
+def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
+                max_over_ranks, sample_clocks_gpu=None):
+    """Device time of K steps of one workload.  By default the K steps are
+    captured once into a CUDA graph and the timed region is one replay of
+    it, so that host launch overhead does not pace small batches (the
+    library makes no allocation or synchronisation, so its calls capture as
+    they are); a second graph with an event between the stages gives the
+    per-stage times.  A step whose expert weights (the distinct experts it
+    routes to) fit a few times over in L2 would find them there on the next
+    step: then every step is preceded by a write of twice the L2 size,
+    outside that step's events, and the step time is the mean of the
+    per-step event pairs; larger working sets stream from HBM by themselves.
+    Returns a dict (ms_per_step, stage_ms, touched, weight_set, flush, ...)."""
+    import torch
+    shp = inp.shape
+    dev = inp.x.device
+
+    def step(events=None):
+        api.moe_forward_ex(s, inp.x, inp.logits if router is None else None, inp.w13,
+                           inp.w2, inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
+                           events=events, path=path, deterministic=args.deterministic,
+                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs],
+                           router=router)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    status = api.moe_read_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device error during warm-up: {status}")
+
+    touched = touched_experts(api, s, inp)
+    weight_set = touched * 3.0 * shp.H * shp.I * 2
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = None
+    if weight_set < 4 * l2_bytes:
+        flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+
+    def flush(i):
+        if flush_buf is not None:
+            with torch.cuda.stream(stream):  # ordered before the step's kernels
+                flush_buf.fill_(i & 0xFF)
+
+    nst = api.NUM_STAGES
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+                for _ in range(args.steps)]
+    # with the flush: only the first and last event of each step, so that no
+    # event node sits between the step's kernels
+    step_ev = [[e[0]] + [None] * (nst - 1) + [e[nst]] for e in
+               [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+                for _ in range(args.steps)]]
+    for evs in stage_ev + step_ev:  # create the events before the timed region
+        for e in evs:
+            if e is not None:
+                e.record(stream)
+
+    def plain_step(i):
+        flush(i)
+        step(step_ev[i] if flush_buf is not None else None)
+
+    def staged_step(i):
+        flush(i)
+        step(stage_ev[i])
+
+    graph = staged = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(args.steps):
+                plain_step(i)
+        staged = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(staged, stream=stream):
+            for i in range(args.steps):
+                staged_step(i)
+        graph.replay()  # untimed first replays
+        staged.replay()
+        torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(sample_clocks_gpu) if sample_clocks_gpu is not None else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)  # let the sampler start before the timed work
+    t_start.record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            plain_step(i)
+    t_end.record(stream)
+    if staged is not None:
+        staged.replay()
+    else:
+        for i in range(args.steps):
+            staged_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks is not None else None
+    if graph is not None:
+        del graph, staged
+    if flush_buf is None:
+        ms_total = t_start.elapsed_time(t_end)
+    else:
+        ms_total = sum(e[0].elapsed_time(e[nst]) for e in step_ev)
+    ms_per_step = max_over_ranks(ms_total) / args.steps
+    try:
+        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
+                                    for ev in stage_ev) for j in range(nst)]
+    except RuntimeError:
+        # events inside the graph could not be timed: take the stage times
+        # from the same K steps launched on the stream instead
+        for i in range(args.steps):
+            staged_step(i)
+        torch.cuda.synchronize()
+        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
+                                    for ev in stage_ev) for j in range(nst)]
+    status = api.moe_read_error(ws)
+    if status != 0:
+        raise RuntimeError(f"device error in the timed region: {status}")
+    return {"ms_per_step": ms_per_step, "stage_ms": stage_ms, "touched": touched,
+            "weight_set": weight_set, "flush": flush if flush_buf is not None else None,
+            "flush_bytes": 2 * l2_bytes if flush_buf is not None else 0,
+            "clocks": clk}
+
+
+def w13_kernel_name(decode: bool, T: int) -> str:
+    if not decode:
+        return "grouped_gemm_kernel<0> (w13 + activation)"
+    if T <= 8:
+        return "decode_w13_few_kernel (w13 + act, cp.async rings, mma.sync)"
+    if T <= 64:
+        return "decode_tc_kernel<N,0> (w13 + act, tcgen05, split over all SMs)"
+    return "decode_w13_kernel (w13 + act)"
+
+
+def roofline_of(args, shp, m, decode, peaks, peak_src, config_name):
+    """Roofline of the dominant kernel, the w13 product with the fused
+    activation (2/3 of the layer's FLOPs and of its weight bytes), and the
+    whole layer's fraction.  FLOPs count real rows only, bytes count each
+    touched expert once.  The w13 product does 2 FLOP per weight byte per
+    token routed to the expert; below the ridge point (peak FLOP/s / peak
+    B/s) it is bound by streaming the touched experts' weights from HBM."""
+    touched = m["touched"]
+    w13_ms = m["stage_ms"][3]
+    rows = shp.T * shp.k + shp.T * shp.n_shared
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    if rows / max(touched, 1) < ridge:
+        achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        return {"bound": "hbm", "kernel": w13_kernel_name(decode, shp.T),
+                "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
+                "traffic": traffic_for(("decode.cu" if shp.T <= 8 else "decode_tc.cu")
+                                       if decode else "gemm_tc.cu",
+                                       config_name, args.shape),
+                "layer_frac": m["weight_set"] / (m["ms_per_step"] / 1e3) / 1e9 / peak,
+                "touched_experts": touched}
+    w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) * shp.H * 2
+    achieved = w13_flops / (w13_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"bound": "tensor", "kernel": w13_kernel_name(decode, shp.T),
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "traffic": traffic_for("gemm_tc.cu", config_name, args.shape),
+            "layer_frac": shp.flops() / (m["ms_per_step"] / 1e3) / 1e12 / peak}
+
+
+def launches_per_step(decode: bool, router: bool) -> int:
+    # prefill: route, layout x4, gather, two GEMMs, rounding; decode: route,
+    # w13, w2, row sum
+    return (4 if decode else 9) + (1 if router else 0)
 
 
 def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
@@ -362,6 +620,42 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
     return max_over_ranks(t0.elapsed_time(t1)) / args.steps, h2d, d2h
 
 
+def other_config_entry(args, api, inputs, name, dev, stream, peaks, peak_src):
+    """One line of the ``configs`` key: the same device-timed measurement,
+    roofline and CPU-baseline leg (with its parity comparison) for another
+    workload, one GPU."""
+    import torch
+    inp = inputs.make_inputs(name, seed=args.seed, device=dev)
+    shp = inp.shape
+    s = api.shape_from(shp)
+    ws = api.alloc_workspace(s, dev)
+    out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
+    path = api.PATH_AUTO
+    decode = shp.T <= api.DECODE_MAX_T
+    m = timed_steps(args, api, inp, s, ws, out, stream, path, None, lambda: None,
+                    lambda v: v, sample_clocks_gpu=dev.index or 0)
+    roof = roofline_of(args, shp, m, decode, peaks, peak_src, name)
+    gpu = gpu_result(api, inp, s, path, args)
+    base, parity = cpu_baseline_leg(inp, gpu, budget_s=1.5)
+    entry = {"workload": workload_name(name, shp),
+             "path": "decode" if decode else "prefill",
+             "ms_per_step": m["ms_per_step"],
+             "value": shp.T / (m["ms_per_step"] / 1e3), "unit": UNIT,
+             "roofline": roof, "layer_frac": roof["layer_frac"],
+             "stage_ms": dict(zip(api.STAGE_NAMES, m["stage_ms"])),
+             "l2": "flushed before every step" if m["flush"] is not None
+                   else "weights far larger than L2",
+             "parity": parity, "cpu_baseline": base, "clocks": m["clocks"],
+             "gpu_launches": launches_per_step(decode, False) * args.steps}
+    del inp, ws, out
+    torch.cuda.empty_cache()
+    return entry
+
+
+OTHER_CONFIGS = ("many_small_prefill", "skewed_shared_prefill", "decode_t1",
+                 "decode_t4", "decode_t16", "decode_t64", "decode_t256")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -395,136 +689,22 @@ def run_ours(args):
         rg = torch.Generator(device=dev).manual_seed(args.seed + 1000 + rank)
         router = (*inputs.router_inputs(shp.T, shp.H, shp.E, rg, dev), 1e-6)
 
-    def step(events=None):
-        api.moe_forward_ex(s, inp.x, inp.logits if router is None else None, inp.w13,
-                           inp.w2, inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
-                           events=events, path=path, deterministic=args.deterministic,
-                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs],
-                           router=router)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
     max_over_ranks = max_over_ranks_fn(world, dev)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    status = api.moe_read_error(ws)
-    if status != 0:
-        raise RuntimeError(f"device error during warm-up: {status}")
-
-    # ---- L2.  A step whose expert weights (the distinct experts it routes
-    # to) fit a few times over in L2 would find them there on the next step:
-    # then every step is preceded by a write of twice the L2 size, outside
-    # that step's events, and the step time is the mean of the per-step
-    # event pairs.  Larger working sets stream from HBM by themselves.
-    touched = touched_experts(api, s, inp, ws)
-    expert_bytes = 3.0 * shp.H * shp.I * 2
-    weight_set = touched * expert_bytes
-    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_buf = None
-    if weight_set < 4 * l2_bytes:
-        flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
-
-    def flush(i):
-        if flush_buf is not None:
-            with torch.cuda.stream(stream):  # ordered before the step's kernels
-                flush_buf.fill_(i & 0xFF)
-
-    # ---- device-resident timed region (per-stage events on the stream).
-    # By default the K steps are captured once into a CUDA graph and the
-    # timed region is one replay of it, so that host launch overhead does
-    # not pace small batches; the library makes no allocation or
-    # synchronisation, so its calls capture as they are.
-    nst = api.NUM_STAGES
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
-                for _ in range(args.steps)]
-    # with the flush: only the first and last event of each step, so that no
-    # event node sits between the step's kernels
-    step_ev = [[e[0]] + [None] * (nst - 1) + [e[nst]] for e in
-               [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
-                for _ in range(args.steps)]]
-    for evs in stage_ev + step_ev:  # create the events before the timed region
-        for e in evs:
-            if e is not None:
-                e.record(stream)
-
-    def plain_step(i):
-        flush(i)
-        step(step_ev[i] if flush_buf is not None else None)
-
-    def staged_step(i):
-        flush(i)
-        step(stage_ev[i])
-
-    graph = staged = None
-    if not args.no_graph:
-        # one graph of K plain steps (the timed region) and one of K steps
-        # with stage events (per-kernel times: an event node adds a few
-        # microseconds, so it stays out of the step time)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(args.steps):
-                plain_step(i)
-        staged = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(staged, stream=stream):
-            for i in range(args.steps):
-                staged_step(i)
-        graph.replay()  # untimed first replays
-        staged.replay()
-        torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)  # let the sampler start before the timed work
-    t_start.record(stream)
-    if graph is not None:
-        graph.replay()
-    else:
-        for i in range(args.steps):
-            plain_step(i)
-    t_end.record(stream)
-    if staged is not None:
-        staged.replay()
-    else:
-        for i in range(args.steps):
-            staged_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    if graph is not None:
-        del graph, staged
-    if flush_buf is None:
-        ms_total = t_start.elapsed_time(t_end)
-    else:
-        ms_total = sum(e[0].elapsed_time(e[nst]) for e in step_ev)
-    ms_per_step = max_over_ranks(ms_total) / args.steps
-    try:
-        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
-                                    for ev in stage_ev) for j in range(nst)]
-    except RuntimeError:
-        # events inside the graph could not be timed: take the stage times
-        # from the same K steps launched on the stream instead
-        for i in range(args.steps):
-            staged_step(i)
-        torch.cuda.synchronize()
-        stage_ms = [statistics.mean(ev[j].elapsed_time(ev[j + 1])
-                                    for ev in stage_ev) for j in range(nst)]
-    status = api.moe_read_error(ws)
-    if status != 0:
-        raise RuntimeError(f"device error in the timed region: {status}")
+    m = timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
+                    max_over_ranks, sample_clocks_gpu=local)
+    ms_per_step, stage_ms = m["ms_per_step"], m["stage_ms"]
+    flush = m["flush"]
 
     # ---- the router kernel alone (--router): L2 flushed before each launch
     router_stats = None
     if router is not None:
+        l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
         rz = torch.empty(shp.T, shp.E, dtype=torch.float32, device=dev)
-        fl = flush_buf if flush_buf is not None else \
-            torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+        fl = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
         for _ in range(3):
             api.moe_router_logits(s, *router, rz, stream=stream)
         rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -548,62 +728,20 @@ def run_ours(args):
 
     # ---- end to end: pinned host inputs in, host output back, every step
     e2e_ms, h2d, d2h = run_e2e(
-        args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
-        flush if flush_buf is not None else None) \
+        args, api, inp, s, ws, out, stream, barrier, max_over_ranks, flush) \
         if not (args.profile or args.router) else (None, 0, 0)
 
     result = None
     if rank == 0:
         peaks, peak_src = load_peaks()
         value = whole_job_rate(shp.T, world, ms_per_step)
-        # dominant kernel: the w13 product with the fused activation (2/3 of
-        # the layer's FLOPs and of its weight bytes); FLOPs count real rows
-        # only, bytes count each touched expert once
-        w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) \
-            * shp.H * 2
-        w13_ms = stage_ms[3]
-        layer_bytes = weight_set
-        # the w13 product does 2 FLOP per weight byte per token routed to the
-        # expert; below the ridge point (peak FLOP/s / peak B/s) it is bound
-        # by streaming the touched experts' weights from HBM
-        rows = shp.T * shp.k + shp.T * shp.n_shared
-        tokens_per_expert = rows / max(touched, 1)
-        ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
-        hbm_bound = tokens_per_expert < ridge
-        if hbm_bound:
-            achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
-            peak = float(peaks["hbm_gbs"])
-            roof = {"bound": "hbm",
-                    "kernel": ("decode_w13_few_kernel (w13 + act)" if shp.T <= 8
-                               else "decode_w13_kernel (w13 + act)") if decode
-                    else "grouped_gemm_kernel<0> (w13 + activation)",
-                    "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak,
-                    "peak_source": f"{peak_src} hbm_gbs",
-                    "traffic": traffic_for("decode.cu" if decode else "gemm_tc.cu",
-                                           args.config, args.shape),
-                    "layer_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peak,
-                    "touched_experts": touched}
-        else:
-            achieved = w13_flops / (w13_ms / 1e3) / 1e12
-            peak = float(peaks["bf16_tflops"])
-            roof = {"bound": "tensor", "kernel": "grouped_gemm_kernel<0> "
-                    "(w13 + activation)", "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": f"{peak_src} bf16_tflops (burst)",
-                    "traffic": traffic_for("gemm_tc.cu", args.config, args.shape),
-                    "layer_frac": shp.flops() / (ms_per_step / 1e3) / 1e12 / peak}
+        roof = roofline_of(args, shp, m, decode, peaks, peak_src, args.config)
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
-        # our kernels per step: prefill route, layout x4, gather, 2 GEMMs,
-        # rounding; decode route, w13, w2, row sum
-        launches_per_step = 4 if decode else 9
-        cpu = None
+        cpu = parity = None
         if world == 1 and not args.profile:
-            rate, cores, ntok, secs = cpu_oracle_rate(inp)
-            cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                   "sample": f"{ntok} tokens drawn from the same {shp.T}-token "
-                             f"batch in rounds of {cores}, full layer per token "
-                             f"(fp64), {secs:.1f} s"}
+            gpu = gpu_result(api, inp, s, path, args)
+            cpu, parity = cpu_baseline_leg(inp, gpu, budget_s=12.0)
+        weight_set = m["weight_set"]
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -618,35 +756,47 @@ def run_ours(args):
                        "timing": ("one CUDA-graph replay of the K steps"
                                   if not args.no_graph else "stream launches")
                                  + ("; step time = mean of per-step event pairs"
-                                    if flush_buf is not None else ""),
+                                    if flush is not None else ""),
                        "global_batch": world * shp.T, "seq_len": shp.T,
                        "parallelism": "replicas" if world > 1 else "single",
-                       "l2": (f"L2 flushed before every step ({2 * l2_bytes / 1e6:.0f}"
+                       "l2": (f"L2 flushed before every step ({m['flush_bytes'] / 1e6:.0f}"
                               " MB write outside the step's events): the step "
                               f"touches {weight_set / 1e6:.0f} MB of expert weights"
-                              if flush_buf is not None else
+                              if flush is not None else
                               "inputs larger than L2: the step streams the "
-                              f"{weight_set / 1e9:.2f} GB of the {touched} experts "
-                              "it routes to")},
+                              f"{weight_set / 1e9:.2f} GB of the {m['touched']} "
+                              "experts it routes to")},
             "roofline": roof,
             "layer_tflops": layer_tflops,
             "stage_ms": dict(zip(api.STAGE_NAMES, stage_ms)),
             "cpu_baseline": cpu,
+            "parity": parity,
             "e2e": None if e2e_ms is None else
                    {"value": world * shp.T / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "timing": "steps one after another, L2 flushed before each"
-                              if flush_buf is not None else
+                              if flush is not None else
                               "pipelined: input copies, moe_forward and output "
                               "copies on three streams, two buffers each"},
-            "gpu_launches": (launches_per_step + (1 if router is not None else 0))
-                            * args.steps,
-            "clocks": clk,
+            "gpu_launches": launches_per_step(decode, router is not None) * args.steps,
+            "clocks": m["clocks"],
         }
         if router_stats is not None:
             router_stats["frac_hbm"] = router_stats["achieved_gbs"] / float(peaks["hbm_gbs"])
             result["router"] = router_stats
             result["config"]["workload"] += " + router (from hidden states)"
+        if world == 1 and not args.profile and not args.router and not args.shape \
+                and args.config == "mixtral_prefill" and not args.headline_only:
+            # the other workloads of the benchmark, one GPU each, after the
+            # headline: device time, roofline, parity against the oracle
+            del inp, ws, out
+            torch.cuda.empty_cache()
+            result["configs"] = {
+                name: other_config_entry(args, api, inputs, name, dev, stream, peaks,
+                                         peak_src)
+                for name in OTHER_CONFIGS}
+            result["gpu_launches"] += sum(c["gpu_launches"]
+                                          for c in result["configs"].values())
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.barrier()

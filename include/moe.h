@@ -254,10 +254,13 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
  *                 its rounding to bf16.
  *   path          which kernels run (moe_path).  The decode path (T small)
  *                 routes in one block and streams each touched expert's
- *                 weights once through skinny tensor-core kernels; its
- *                 stages 1 and 2 are empty (folded into stage 0).  Both
- *                 paths compute the same function; they differ in the order
- *                 of fp32 additions inside the products.
+ *                 weights once: for T <= 8 through skinny mma.sync kernels,
+ *                 for 8 < T <= 64 through tcgen05 kernels that split the
+ *                 weight stream evenly over all SMs, above that through the
+ *                 skinny kernels' many-token form.  Its stages 1 and 2 are
+ *                 empty (folded into stage 0).  Both paths compute the same
+ *                 function; they differ in the order of fp32 additions
+ *                 inside the products.
  *   router_w      NULL, or the router ahead of the routing (see
  *                 moe_router_logits): with router_w [E,H], router_x [T,H]
  *                 (the residual rows the router reads) and router_scale [H]
@@ -274,7 +277,7 @@ typedef enum {
   MOE_PATH_PREFILL = 1,  /* tcgen05 grouped GEMMs over padded expert segments */
   MOE_PATH_DECODE = 2    /* touched experts streamed by skinny kernels; T <= 1024 */
 } moe_path;
-#define MOE_DECODE_MAX_T 8
+#define MOE_DECODE_MAX_T 16
 typedef struct {
   void* const* stage_events;
   float* out_f32;

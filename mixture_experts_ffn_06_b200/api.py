@@ -39,7 +39,7 @@ class MoEError(RuntimeError):
 
 
 PATH_AUTO, PATH_PREFILL, PATH_DECODE = 0, 1, 2
-DECODE_MAX_T = 8
+DECODE_MAX_T = 16
 
 
 SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1

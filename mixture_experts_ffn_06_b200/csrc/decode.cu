@@ -14,6 +14,8 @@
 //   decode_w2     one CTA per (touched expert, 64 rows of H): y = h W2^T,
 //                 times the gate weight, stored at the (token, choice) row;
 //   sum_rows      (combine.cu) adds each token's k+S rows in order, bf16 out.
+// For 8 < T <= 64 the two products run as tcgen05 kernels instead
+// (decode_tc.cu); the routing and the row sum stay the same.
 //
 // The skinny products use mma.sync m16n8k16 (bf16 in, fp32 accumulate) with
 // weight rows as the 16-row A operand and up to 8 tokens per B tile.  The K
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(1024)
 decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ scale,
                     int T, int E, int k, int S, int32_t* __restrict__ ids,
                     float* __restrict__ w, int32_t* __restrict__ meta,
-                    int32_t* __restrict__ slots, RouteOpt opt) {
+                    int32_t* __restrict__ slots, RouteOpt opt,
+                    int32_t* __restrict__ zero, int n_zero) {
   extern __shared__ int32_t dsm[];
   const int G = E + S, R = T * k;
   int32_t* cnt = dsm;            // [G] tokens, then first slot-list entry
@@ -131,6 +134,8 @@ decode_route_kernel(const float* __restrict__ logits, const float* __restrict__ 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
   pdl_trigger();
+  // the arrival counters of the tensor-core products start at zero
+  for (int i = tid; i < n_zero; i += blockDim.x) zero[i] = 0;
   for (int i = tid; i < G; i += blockDim.x) cnt[i] = (i < E) ? 0 : T;
   __syncthreads();
   for (int t = warp; t < T; t += nwarps) {
@@ -659,15 +664,33 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   auto mark = [&](int i) -> bool { return !ev || !ev[i] || record_stage_event(ev[i], st); };
   const int G = a.E + a.S, R = a.T * a.k;
   if (!mark(0)) return cudaErrorUnknown;
+
   const size_t smem = sizeof(int32_t) * ((size_t)G + R);
   const int rthreads = 32 * std::min(32, std::max((G + 31) / 32, std::min(a.T, 32)));
   auto rk = a.E <= 32 ? decode_route_kernel<1> : a.E <= 64 ? decode_route_kernel<2>
             : a.E <= 128 ? decode_route_kernel<4> : a.E <= 256 ? decode_route_kernel<8>
             : decode_route_kernel<16>;
+  // the tensor-core form counts its (unit, k-block) iterations in 32 bits
+  const int64_t dt_iters = (int64_t)(std::min(R, a.E) + a.S) *
+                           dt_row_blocks(a.H, a.I) * ((std::max(a.H, a.I) + 63) / 64);
+  const bool tc = a.tc && dt_iters < (int64_t(1) << 30);
+  const int n_zero = tc ? 2 * G * dt_row_blocks(a.H, a.I) : 0;
   cudaError_t e = launch_ex(rk, dim3(1), dim3(rthreads), smem, st, false, a.logits, a.scale,
-                            a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots, a.route);
+                            a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots, a.route,
+                            tc ? a.dt_cnt : (int32_t*)nullptr, n_zero);
   if (e != cudaSuccess) return e;
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
+  if (tc) {
+    // tensor-core products (decode_tc.cu): h in [touched, N, I] order
+    if ((e = launch_decode_tc_w13(a, a.h_dec, st)) != cudaSuccess) return e;
+    if (!mark(4)) return cudaErrorUnknown;
+    if ((e = launch_decode_tc_w2(a, a.h_dec, st)) != cudaSuccess) return e;
+    if (!mark(5)) return cudaErrorUnknown;
+    e = launch_sum_rows(a.stage, a.T, a.k + a.S, a.H, a.out, a.out_f32, st,
+                        /*pdl=*/true);
+    if (e != cudaSuccess) return e;
+    return mark(6) ? cudaSuccess : cudaErrorUnknown;
+  }
   const int max_groups = (R < a.E ? R : a.E) + a.S;
   // every expert (and shared expert) has at most T tokens: with T <= 8 one
   // B tile holds them all, and the ring kernels keep those token rows in
@@ -675,7 +698,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
   const int nx = a.T < 8 ? a.T : 8;
   const size_t w13_smem = w13_ring_bytes() + (size_t)nx * a.H * 2;
   const size_t w2_smem = w2_ring_bytes() + (size_t)nx * a.I * 2;
-  const bool few = a.T <= 8 && w13_smem <= 200 * 1024 && w2_smem <= 200 * 1024;
+  const bool few = a.T <= kDecodeFewMaxT && w13_smem <= 200 * 1024 &&
+                   w2_smem <= 200 * 1024;
   if (few) {
     auto w13k = decode_w13_few_kernel<kW13Ring>;
     auto w2k = decode_w2_few_kernel<kW2Ring>;

@@ -712,6 +712,13 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool 
   return cudaErrorInvalidValue;
 }
 
+cudaError_t make_tma_map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner,
+                              uint64_t outer, uint32_t box_rows) {
+  return make_map(m, ptr, inner, outer, box_rows);
+}
+
+int device_sm_count() { return num_sms(); }
+
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
                                  cudaStream_t st) {
   return launch_ex(wait_selftest_kernel, dim3(1), dim3(32), 0, st, false, err,

@@ -35,6 +35,8 @@ struct WsMap {
   size_t stage;        // [T,k+S,H] fp32 weighted expert rows (moe_forward)
   size_t acc;          // [T,H] fp32 accumulator (moe_forward, fast combine)
   size_t dec_meta;     // decode path: touched-expert lists
+  size_t dt_part;      // decode path, tensor-core form: [2*kDtMaxCtas,128,T] fp32
+  size_t dt_cnt;       // decode path, tensor-core form: [2, G*row blocks] int32
   size_t logits;       // [T,E] fp32 router logits (moe_forward_ex with a router)
   size_t total;
   int64_t cap;
@@ -121,8 +123,26 @@ struct DecodeArgs {
   float* stage;          // [T*(k+S), H] scratch
   __nv_bfloat16* out;    // [T,H]
   float* out_f32;        // [T,H] or nullptr
+  // the tensor-core form (decode_tc.cu), T <= kDecodeTcMaxT
+  bool tc;
+  float* dt_part;        // [2 * kDtMaxCtas, 128, T] fp32 partial sums
+  int32_t* dt_cnt;       // [2, G * dt_row_blocks] arrival counters
+  uint32_t* err;         // error word
 };
 size_t decode_meta_ints(int G);
+
+// Tensor-core decode products (decode_tc.cu).
+constexpr int kDecodeTcMaxT = 64;
+constexpr int kDecodeFewMaxT = 8;   // the skinny kernels' one-B-tile form
+constexpr int kDtMaxCtas = 2 * 160;  // persistent CTAs: up to 2 per SM
+// row blocks of one group: max(ceil(I / 64), ceil(H / 128))
+int dt_row_blocks(int H, int I);
+// kernels of the tensor-core form: w13 (+ act) -> h, w2 (x gate weight) -> stage.
+// meta / slots come from decode_route; h_dense [touched groups * N, I] bf16.
+cudaError_t launch_decode_tc_w13(const DecodeArgs& a, __nv_bfloat16* h_dense,
+                                 cudaStream_t st);
+cudaError_t launch_decode_tc_w2(const DecodeArgs& a, const __nv_bfloat16* h_dense,
+                                cudaStream_t st);
 // ev: nullptr or MOE_NUM_STAGES + 1 events (see moe_forward_ex)
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev);
 
@@ -162,6 +182,13 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st,
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
                                  cudaStream_t st);
+
+// TMA map of a row-major bf16 [outer, inner] tensor: box {64, box_rows},
+// 128-byte swizzle, out-of-range elements read as zero (gemm_tc.cu).
+cudaError_t make_tma_map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner,
+                              uint64_t outer, uint32_t box_rows);
+// SMs of the current device (cached per device).
+int device_sm_count();
 
 // ---------------------------------------------------------------- device
 #ifdef __CUDACC__

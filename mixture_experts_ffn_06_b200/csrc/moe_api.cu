@@ -40,6 +40,10 @@ WsMap workspace_map(const moe_shape& s) {
   m.stage = take(4ull * T * (k + S) * s.H);
   m.acc = take(4ull * T * s.H);
   m.dec_meta = take(sizeof(int32_t) * decode_meta_ints((int)G));
+  // the tensor-core decode form: partial sums of split units and counters
+  const bool dt = T >= 1 && T <= kDecodeTcMaxT;
+  m.dt_part = take(dt ? sizeof(float) * 2 * kDtMaxCtas * 128 * T : 0);
+  m.dt_cnt = take(dt ? sizeof(int32_t) * 2 * G * dt_row_blocks(s.H, s.I) : 0);
   m.logits = take(sizeof(float) * T * s.E);
   m.total = o;
   return m;
@@ -371,6 +375,13 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
     d.stage = stage;
     d.out = reinterpret_cast<__nv_bfloat16*>(out);
     d.out_f32 = opts ? opts->out_f32 : nullptr;
+    // tensor-core products above the few-token form's 8 tokens (measured on
+    // B200: the skinny kernels are faster up to 8 tokens, the tcgen05 form
+    // from 16 on)
+    d.tc = s.T > kDecodeFewMaxT && s.T <= kDecodeTcMaxT;
+    d.dt_part = reinterpret_cast<float*>(at(ws, m.dt_part));
+    d.dt_cnt = reinterpret_cast<int32_t*>(at(ws, m.dt_cnt));
+    d.err = reinterpret_cast<uint32_t*>(at(ws, m.err));
     if (!use_router) return from_cuda(launch_decode(d, stream, ev));
     // the router counts in the first stage: event 0 goes ahead of it
     void* dev[MOE_NUM_STAGES + 1] = {};

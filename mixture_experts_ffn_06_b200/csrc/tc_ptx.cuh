@@ -43,7 +43,7 @@ __device__ __forceinline__ uint32_t mbar_test(uint32_t bar, uint32_t parity) {
 // Bounded: gives up after ``timeout_ns`` of wall time (recording
 // MOE_ERR_TIMEOUT and raising the block's abort flag), or as soon as another
 // role of the block has raised the abort flag.  Returns false when it gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                        volatile int32_t* abort_flag,
                                        uint64_t timeout_ns, uint32_t* err) {
   if (mbar_test(bar, parity)) return true;
@@ -183,7 +183,7 @@ __device__ __forceinline__ uint32_t mbar_test_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok;
 }
-__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
                                                volatile int32_t* abort_flag,
                                                uint64_t timeout_ns, uint32_t* err) {
   if (mbar_test_cluster(bar, parity)) return true;
