@@ -243,3 +243,56 @@ def gemma4_block_inputs(T: int, H: int, E: int, I_dense: int, seed: int = 0,
     rs = (0.5 + torch.rand(H, generator=gen, device=device)).to(torch.bfloat16)
     return Gemma4BlockInputs(x=x, norms=norms, mlp_w13=mlp_w13, mlp_w2=mlp_w2,
                              router_w=rw, router_scale=rs)
+
+
+@dataclasses.dataclass
+class FP8Experts:
+    """Expert weights as e4m3 codes (uint8) with one fp32 scale per output
+    row: the per-expert FP8 checkpoints' weight / weight_scale pairs, packed
+    as w13 (gate rows first) and w2."""
+    w13_q: torch.Tensor                     # [E,2I,H] uint8
+    w13_s: torch.Tensor                     # [E,2I] fp32
+    w2_q: torch.Tensor                      # [E,H,I] uint8
+    w2_s: torch.Tensor                      # [E,H] fp32
+    sh13_q: Optional[torch.Tensor] = None   # [S,2I,H] uint8
+    sh13_s: Optional[torch.Tensor] = None   # [S,2I] fp32
+    sh2_q: Optional[torch.Tensor] = None    # [S,H,I] uint8
+    sh2_s: Optional[torch.Tensor] = None    # [S,H] fp32
+
+
+def _e4m3_codes(shape, gen: torch.Generator, device) -> torch.Tensor:
+    """N(0, 64^2) draws clamped to the e4m3 range and rounded to e4m3 (torch's
+    float8_e4m3fn cast), as uint8 codes; 3-d tensors expert by expert."""
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    parts = [out[e] for e in range(shape[0])] if len(shape) == 3 else [out]
+    for o in parts:
+        t = torch.randn(o.shape, generator=gen, device=device, dtype=torch.float32)
+        o.copy_((64.0 * t).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn)
+                .view(torch.uint8))
+    return out
+
+
+def _row_scales(shape, gen: torch.Generator, device) -> torch.Tensor:
+    return ((0.5 + torch.rand(shape, generator=gen, device=device,
+                              dtype=torch.float32)) * (0.02 / 64.0)).contiguous()
+
+
+def fp8_experts(shp: Shape, seed: int = 0, device="cpu") -> FP8Experts:
+    """Recipe (one generator seeded with ``seed``, draws in this order): w13
+    codes, w13 row scales, w2 codes, w2 row scales, then the shared experts'
+    in the same order.  Codes are e4m3 roundings of N(0, 64^2) draws, scales
+    (0.5 + U[0,1]) * 0.02 / 64, so the weights they stand for spread like the
+    bf16 recipe's N(0, 0.02^2)."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    E, H, I, S = shp.E, shp.H, shp.I, shp.n_shared
+    w13_q = _e4m3_codes((E, 2 * I, H), gen, device)
+    w13_s = _row_scales((E, 2 * I), gen, device)
+    w2_q = _e4m3_codes((E, H, I), gen, device)
+    w2_s = _row_scales((E, H), gen, device)
+    sh = [None] * 4
+    if S:
+        sh = [_e4m3_codes((S, 2 * I, H), gen, device), _row_scales((S, 2 * I), gen, device),
+              _e4m3_codes((S, H, I), gen, device), _row_scales((S, H), gen, device)]
+    return FP8Experts(w13_q, w13_s, w2_q, w2_s, *sh)

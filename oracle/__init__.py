@@ -16,7 +16,10 @@ and tanh-GELU in float64.  The router ahead of the routing (walkthrough
 section 3, Gemma4Router) is pinned by the closed form of a constant row, the
 unit RMS of the normalised row, exact invariance under power-of-two row
 scaling, exact linearity in the scale and the weight, bf16-valued
-activations, and a finite zero row.
+activations, and a finite zero row.  The FP8 forms (e4m3 codec, per-row
+dynamic quantisation, the layer with FP8 experts) are pinned against torch's
+float8_e4m3fn conversion, the reconstruction bound of a quantised row, exact
+linearity in the w2 scales and a dense float64 restatement.
 """
 from __future__ import annotations
 
@@ -71,10 +74,17 @@ def _load():
                                             P, P, P, dbl, P, P, dbl, P, P, P, P, P,
                                             i32, P]
         lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [i32, i32, i32]
+        lib.oracle_e4m3_values.argtypes = [i64, P, P]
+        lib.oracle_e4m3_codes.argtypes = [i64, P, P]
+        lib.oracle_quantize_rows_e4m3.argtypes = [i64, i32, P, P, P]
+        lib.oracle_forward_fp8.argtypes = [i64, i32, i32, i32, i32, i32, i32, P, P, P,
+                                           P, P, P, P, P, P, P, P, P, i64, i32, P, P, P]
         for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
                   lib.oracle_expert_rows, lib.oracle_forward,
                   lib.oracle_router_logits, lib.oracle_route_ex,
-                  lib.oracle_forward_ex, lib.oracle_gemma4_block):
+                  lib.oracle_forward_ex, lib.oracle_gemma4_block,
+                  lib.oracle_e4m3_values, lib.oracle_e4m3_codes,
+                  lib.oracle_quantize_rows_e4m3, lib.oracle_forward_fp8):
             f.restype = i32
         _lib = lib
     return _lib
@@ -249,3 +259,75 @@ def gemma4_block(x, norms, eps: float, router_w, router_scale, router_eps: float
         _ptr(w2u), _ptr(_f32(scale)), _ptr(m13), _ptr(m2), nthreads, _ptr(out)),
         "gemma4_block")
     return out
+
+
+# ------------------------------------------------------------ FP8 experts
+
+def _u8(a) -> Optional[np.ndarray]:
+    """uint8 codes (torch uint8 / float8 tensor or ndarray) -> contiguous uint8."""
+    if a is None:
+        return None
+    if not isinstance(a, np.ndarray):
+        import torch
+        t = a.detach().to("cpu").contiguous()
+        if t.dtype != torch.uint8:
+            t = t.view(torch.uint8)
+        a = t.numpy()
+    return np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def e4m3_values(codes) -> np.ndarray:
+    """Value of every e4m3 code (float64; NaN for 0x7F / 0xFF)."""
+    c = _u8(codes)
+    out = np.empty(c.shape, np.float64)
+    _check(_load().oracle_e4m3_values(c.size, _ptr(c), _ptr(out)), "e4m3_values")
+    return out
+
+
+def e4m3_codes(v) -> np.ndarray:
+    """Nearest e4m3 code of each float32 value (ties to even, saturating)."""
+    f = _f32(v)
+    out = np.empty(f.shape, np.uint8)
+    _check(_load().oracle_e4m3_codes(f.size, _ptr(f), _ptr(out)), "e4m3_codes")
+    return out
+
+
+def quantize_rows_e4m3(src):
+    """Per-row dynamic e4m3 quantisation of bf16 rows [R, C] -> (codes uint8
+    [R, C], scales float32 [R])."""
+    su = _u16(src)
+    R, C = su.shape
+    codes = np.empty((R, C), np.uint8)
+    scales = np.empty(R, np.float32)
+    _check(_load().oracle_quantize_rows_e4m3(R, C, _ptr(su), _ptr(codes), _ptr(scales)),
+           "quantize_rows_e4m3")
+    return codes, scales
+
+
+def forward_fp8(x, logits, w13_q, w13_s, w2_q, w2_s, k: int, act_kind: int, scale=None,
+                sh13_q=None, sh13_s=None, sh2_q=None, sh2_s=None, tokens=None,
+                nthreads: int = 0):
+    """The layer with FP8 experts in fp64 -> (out [n,H] float64, ids, w).
+    w13_q [E,2I,H] / w2_q [E,H,I] e4m3 codes with per-row fp32 scales
+    w13_s [E,2I] / w2_s [E,H]; shared experts likewise."""
+    xu = _u16(x)
+    z = _f32(logits)
+    T, H = xu.shape
+    E = z.shape[1]
+    c13, c2 = _u8(w13_q), _u8(w2_q)
+    I = c2.shape[-1]
+    s13, s2 = _f32(w13_s), _f32(w2_s)
+    h13, h2 = _u8(sh13_q), _u8(sh2_q)
+    hs13, hs2 = _f32(sh13_s), _f32(sh2_s)
+    S = 0 if h13 is None else h13.shape[0]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, np.int64)
+    n = T if tok is None else tok.size
+    out = np.empty((n, H), np.float64)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    _check(_load().oracle_forward_fp8(T, H, E, k, I, act_kind, S, _ptr(xu), _ptr(z),
+                                      _ptr(_f32(scale)), _ptr(c13), _ptr(s13), _ptr(c2),
+                                      _ptr(s2), _ptr(h13), _ptr(hs13), _ptr(h2),
+                                      _ptr(hs2), _ptr(tok), n, nthreads, _ptr(out),
+                                      _ptr(ids), _ptr(w)), "forward_fp8")
+    return out, ids, w

@@ -691,3 +691,218 @@ int oracle_gemma4_block(int64_t T, int H, int E, int k, int I, int act, int I_de
   free(a1); free(a2); free(y1); free(y2); free(z1); free(lg); free(row); free(r1); free(r2);
   return rc;
 }
+
+/* ------------------------------------------------------------ FP8 experts */
+
+/*
+ * FP8 expert weights.  The sglang PR on Gemma 4 (prhub.com.cn, PR #24696,
+ * "FP8 per-expert MoE weight-loader fix") loads per-expert FP8 checkpoints
+ * whose gate / up / down weights each come with a weight_scale, into
+ * FusedMoE's w13_weight / w2_weight and their _scale parameters; the vLLM API
+ * page (load_weights) names the same parameters.  The pages fix neither the
+ * number format nor the granularity of the scales.  The reading taken here
+ * (the checkpoint is an "FP8-Dynamic" one):
+ *   - a weight is an e4m3 code (E4M3FN: 1 sign bit, 4 exponent bits with
+ *     bias 7, 3 mantissa bits, no infinities, 0x7F / 0xFF are NaN, largest
+ *     finite 448) times one fp32 scale per output row;
+ *   - activations are quantised per row when the layer runs: with amax the
+ *     largest |v| of the row, s = fl32(amax / 448) (an all-zero row gets
+ *     s = 1), and code(v) = e4m3(fl32(v / s)), rounded to the nearest e4m3
+ *     value (ties to the even code), saturating at +-448;
+ *   - the layer on the dequantised values, in fp64: per routed (t, e),
+ *       g_i = sum_h x'_h w1'_ih,  u_i = sum_h x'_h w3'_ih,  a_i = Act(g_i) u_i,
+ *     x' the quantised token row (code times s_x), w' code times row scale;
+ *     the row a is then quantised the same way (the exact a, not a rounded
+ *     copy), and y_h = sum_i a'_i w2'_hi; the combine is the one of
+ *     oracle_forward.  A code times an fp32 scale is exact in double.
+ */
+
+static double e4m3_table[256];
+static pthread_once_t e4m3_once = PTHREAD_ONCE_INIT;
+
+/* value of an e4m3 code: (8 + m) 2^(e-10) for e > 0, m 2^-9 for e = 0 */
+static void e4m3_init(void) {
+  for (int b = 0; b < 256; ++b) {
+    const int e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+      v = NAN;
+    else
+      v = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    e4m3_table[b] = (b & 0x80) ? -v : v;
+  }
+}
+
+static double e4m3_value(uint8_t b) { return e4m3_table[b]; }
+
+/* nearest e4m3 code of v (ties to the even code), saturating at 448 */
+static uint8_t e4m3_code(float v) {
+  if (v != v) return 0x7F;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs((double)v);
+  if (a >= 448.0) return sign | 0x7E;
+  int lo = 0, hi = 126;  /* largest code whose value is <= a */
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (e4m3_table[mid] <= a) lo = mid; else hi = mid - 1;
+  }
+  const double below = e4m3_table[lo], above = e4m3_table[lo + 1];
+  int c;
+  if (a - below < above - a) c = lo;
+  else if (a - below > above - a) c = lo + 1;
+  else c = (lo & 1) ? lo + 1 : lo;
+  return sign | (uint8_t)c;
+}
+
+int oracle_e4m3_values(int64_t n, const uint8_t* codes, double* out) {
+  pthread_once(&e4m3_once, e4m3_init);
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+  return OK;
+}
+
+int oracle_e4m3_codes(int64_t n, const float* v, uint8_t* out) {
+  pthread_once(&e4m3_once, e4m3_init);
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(v[i]);
+  return OK;
+}
+
+/* per-row scale and codes of n values held as floats */
+static float quantize_row(int n, const float* v, uint8_t* codes) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    const float a = fabsf(v[i]);
+    if (a > amax) amax = a;
+  }
+  const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+  for (int i = 0; i < n; ++i) codes[i] = e4m3_code(v[i] / s);
+  return s;
+}
+
+/* per-row dynamic quantisation of bf16 rows: codes [rows, cols], scales [rows] */
+int oracle_quantize_rows_e4m3(int64_t rows, int cols, const uint16_t* src,
+                              uint8_t* codes, float* scales) {
+  if (rows < 0 || cols < 1 || !src || !codes || !scales) return EINVAL_ARG;
+  pthread_once(&e4m3_once, e4m3_init);
+  float* v = (float*)malloc(sizeof(float) * (size_t)cols);
+  if (!v) return ENOMEM_ARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int c = 0; c < cols; ++c) v[c] = (float)bf16_to_double(src[r * cols + c]);
+    scales[r] = quantize_row(cols, v, codes + r * cols);
+  }
+  free(v);
+  return OK;
+}
+
+/* one expert (or shared expert) on one quantised token row, added to y
+ * with the given weight */
+static void ffn_row_fp8(int H, int I, int act, const double* xq, const uint8_t* w13c,
+                        const float* w13s, const uint8_t* w2c, const float* w2s,
+                        double weight, double* a, float* af, uint8_t* ac, double* y) {
+  for (int i = 0; i < I; ++i) {
+    const uint8_t* r1 = w13c + (int64_t)i * H;
+    const uint8_t* r3 = w13c + (int64_t)(I + i) * H;
+    double g = 0.0, u = 0.0;
+    for (int h = 0; h < H; ++h) {
+      g += xq[h] * (e4m3_value(r1[h]) * (double)w13s[i]);
+      u += xq[h] * (e4m3_value(r3[h]) * (double)w13s[I + i]);
+    }
+    a[i] = act_fn(act, g) * u;
+  }
+  /* quantise the intermediate row: amax of the exact values, then the
+   * float steps of quantize_row */
+  double amax = 0.0;
+  for (int i = 0; i < I; ++i)
+    if (fabs(a[i]) > amax) amax = fabs(a[i]);
+  const float famax = (float)amax;
+  const float s = famax > 0.0f ? famax / 448.0f : 1.0f;
+  for (int i = 0; i < I; ++i) {
+    af[i] = (float)a[i];
+    ac[i] = e4m3_code(af[i] / s);
+    a[i] = e4m3_value(ac[i]) * (double)s;
+  }
+  for (int h = 0; h < H; ++h) {
+    const uint8_t* r2 = w2c + (int64_t)h * I;
+    double acc = 0.0;
+    for (int i = 0; i < I; ++i) acc += a[i] * (e4m3_value(r2[i]) * (double)w2s[h]);
+    y[h] += weight * acc;
+  }
+}
+
+typedef struct {
+  int64_t T;
+  int H, E, k, I, act, S;
+  const uint16_t* x;
+  const uint8_t *w13c, *w2c, *sh13c, *sh2c;
+  const float *w13s, *w2s, *sh13s, *sh2s;
+  const int32_t* ids;
+  const double* w;
+  const int64_t* tokens;
+  double* out;
+} fwd8_ctx;
+
+static void fwd8_worker(void* p, int64_t b, int64_t e) {
+  fwd8_ctx* c = (fwd8_ctx*)p;
+  const int H = c->H, I = c->I;
+  float* xf = (float*)malloc(sizeof(float) * H);
+  uint8_t* xc = (uint8_t*)malloc(H);
+  double* xq = (double*)malloc(sizeof(double) * H);
+  double* a = (double*)malloc(sizeof(double) * I);
+  float* af = (float*)malloc(sizeof(float) * I);
+  uint8_t* ac = (uint8_t*)malloc(I);
+  for (int64_t r = b; r < e; ++r) {
+    const int64_t t = c->tokens ? c->tokens[r] : r;
+    double* y = c->out + r * H;
+    for (int h = 0; h < H; ++h) y[h] = 0.0;
+    /* the token row, quantised once */
+    for (int h = 0; h < H; ++h) xf[h] = (float)bf16_to_double(c->x[t * H + h]);
+    const float sx = quantize_row(H, xf, xc);
+    for (int h = 0; h < H; ++h) xq[h] = e4m3_value(xc[h]) * (double)sx;
+    for (int j = 0; j < c->k; ++j) {
+      const int64_t ex = c->ids[t * c->k + j];
+      ffn_row_fp8(H, I, c->act, xq, c->w13c + ex * 2 * (int64_t)I * H,
+                  c->w13s + ex * 2 * (int64_t)I, c->w2c + ex * (int64_t)H * I,
+                  c->w2s + ex * (int64_t)H, c->w[t * c->k + j], a, af, ac, y);
+    }
+    for (int s = 0; s < c->S; ++s)
+      ffn_row_fp8(H, I, c->act, xq, c->sh13c + (int64_t)s * 2 * I * H,
+                  c->sh13s + (int64_t)s * 2 * I, c->sh2c + (int64_t)s * H * I,
+                  c->sh2s + (int64_t)s * H, 1.0, a, af, ac, y);
+  }
+  free(xf); free(xc); free(xq); free(a); free(af); free(ac);
+}
+
+/*
+ * The layer with FP8 experts, for the tokens listed in ``tokens`` (NULL =
+ * all T): routing as oracle_forward; w13 codes [E,2I,H] with scales [E,2I]
+ * (gate rows first), w2 codes [E,H,I] with scales [E,H]; shared experts
+ * likewise ([S,...], the same I).
+ */
+int oracle_forward_fp8(int64_t T, int H, int E, int k, int I, int act, int S,
+                       const uint16_t* x, const float* logits, const float* scale,
+                       const uint8_t* w13c, const float* w13s, const uint8_t* w2c,
+                       const float* w2s, const uint8_t* sh13c, const float* sh13s,
+                       const uint8_t* sh2c, const float* sh2s, const int64_t* tokens,
+                       int64_t n_tokens, int nthreads, double* out, int32_t* ids_out,
+                       double* w_out) {
+  if (T < 0 || H < 1 || I < 1 || S < 0 || !x || !w13c || !w13s || !w2c || !w2s ||
+      (S > 0 && (!sh13c || !sh13s || !sh2c || !sh2s)))
+    return EINVAL_ARG;
+  pthread_once(&e4m3_once, e4m3_init);
+  int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (T * k + 1));
+  double* w = w_out ? w_out : (double*)malloc(sizeof(double) * (T * k + 1));
+  if (!ids || !w) return ENOMEM_ARG;
+  int rc = oracle_route(T, E, k, logits, scale, ids, w, NULL);
+  if (rc == OK) {
+    if (!tokens) n_tokens = T;
+    for (int64_t r = 0; tokens && r < n_tokens; ++r)
+      if (tokens[r] < 0 || tokens[r] >= T) rc = EINVAL_ARG;
+  }
+  if (rc == OK) {
+    fwd8_ctx c = {T, H, E, k, I, act, S, x, w13c, w2c, sh13c, sh2c,
+                  w13s, w2s, sh13s, sh2s, ids, w, tokens, out};
+    parallel_for(n_tokens, nthreads, fwd8_worker, &c);
+  }
+  if (!ids_out) free(ids);
+  if (!w_out) free(w);
+  return rc;
+}

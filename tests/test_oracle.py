@@ -709,3 +709,140 @@ def test_bf16_rounding_of_the_exact_output_exceeds_the_bound(shape, seed):
     assert np.abs(out).max() > 5 * rms
     # ... and the rounding stays inside the half-ulp bound the bf16 check uses
     assert (err <= 2.0 ** -8 * np.abs(out)).all()
+
+
+# ------------------------------------------------------------ FP8 experts
+# Per-expert FP8 checkpoints (the sglang PR on Gemma 4 FP8 per-expert
+# loading; load_weights on the vLLM API page): e4m3 weights with a
+# weight_scale.  Reading: one fp32 scale per output row, activations
+# quantised per row when the layer runs (scale fl32(amax / 448)).
+
+def _fp8(codes) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(codes)).view(torch.float8_e4m3fn)
+
+
+def test_e4m3_values_match_torch():
+    c = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_values(c)
+    t = _fp8(c).double().numpy()
+    assert (np.isnan(v) == np.isnan(t)).all()
+    assert np.array_equal(v[~np.isnan(v)], t[~np.isnan(t)])
+    assert v[0x7E] == 448.0 and v[0x38] == 1.0 and v[0x01] == 2.0 ** -9
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+
+
+def test_e4m3_rounding_matches_torch_and_saturates():
+    vals = oracle.e4m3_values(np.arange(127, dtype=np.uint8))  # 0 .. 448
+    mids = (vals[:-1] + vals[1:]) / 2                          # exact ties
+    probe = np.concatenate([vals, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20),
+                            [2.0 ** -10, 2.0 ** -11, 3 * 2.0 ** -11, 1e-30]])
+    probe = np.concatenate([probe, -probe]).astype(np.float32)
+    want = torch.from_numpy(probe).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_codes(probe)
+    assert np.array_equal(got, want)
+    # above the largest value: saturation, not NaN
+    big = np.array([448.0, 450.0, 480.0, 1e6, -500.0], np.float32)
+    assert oracle.e4m3_codes(big).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_quantize_rows_reconstruct_within_half_a_step():
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(6, 200, generator=g)
+    x[1] *= 1e-3
+    x[2, 7] = 50.0          # one large value sets the scale
+    x[3] = 0.0              # zero row: scale 1, all codes 0
+    x[4, ::3] = 0.0
+    xb = x.to(torch.bfloat16)
+    codes, s = oracle.quantize_rows_e4m3(xb)
+    xv = xb.double().numpy()
+    deq = oracle.e4m3_values(codes) * s.astype(np.float64)[:, None]
+    # half an e4m3 step: 2^-4 relative above 2^-6 s, 2^-10 s below
+    tol = np.maximum(np.abs(xv) * 2.0 ** -4, 2.0 ** -10 * s.astype(np.float64)[:, None])
+    assert (np.abs(deq - xv) <= tol * (1 + 1e-12)).all()
+    assert s[3] == 1.0 and (codes[3] == 0).all()
+    for r in (0, 1, 2, 4, 5):  # the largest |value| of a row maps to +-448
+        j = np.argmax(np.abs(xv[r]))
+        assert codes[r, j] in (0x7E, 0xFE)
+    # a power-of-two row scaling moves only the scale
+    c2, s2 = oracle.quantize_rows_e4m3((x * 8).to(torch.bfloat16))
+    assert np.array_equal(c2[[0, 1, 2, 4, 5]], codes[[0, 1, 2, 4, 5]])
+    assert np.array_equal(s2[[0, 1, 2, 4, 5]], 8 * s[[0, 1, 2, 4, 5]])
+
+
+def _dense_fp8_torch(inp, fp, ids, w, act_kind):
+    """The FP8 layer restated with torch float64 ops and torch's e4m3 cast as
+    the quantiser: every expert on every token, then masked by the dispatch
+    weights (compute all, then discard)."""
+    def quant(v64):
+        v = v64.float()
+        amax = v.abs().amax(-1, keepdim=True)
+        s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        return (v / s).to(torch.float8_e4m3fn).double() * s.double()
+
+    def ffn(xq, c13, s13, c2, s2):
+        I = c2.shape[-1]
+        w13 = _fp8(c13).double() * torch.as_tensor(s13).double()[:, None]
+        w2 = _fp8(c2).double() * torch.as_tensor(s2).double()[:, None]
+        g, u = xq @ w13[:I].T, xq @ w13[I:].T
+        a = (F.silu(g) if act_kind == 0 else F.gelu(g, approximate="tanh")) * u
+        return quant(a) @ w2.T
+
+    shp = inp.shape
+    xq = quant(inp.x.double())
+    D = torch.zeros(shp.T, shp.E, dtype=torch.float64)
+    for t in range(shp.T):
+        D[t, torch.as_tensor(ids[t]).long()] = torch.as_tensor(w[t])
+    out = torch.zeros(shp.T, shp.H, dtype=torch.float64)
+    for e in range(shp.E):
+        out += D[:, e:e + 1] * ffn(xq, fp.w13_q[e], fp.w13_s[e], fp.w2_q[e], fp.w2_s[e])
+    for s in range(shp.n_shared):
+        out += ffn(xq, fp.sh13_q[s], fp.sh13_s[s], fp.sh2_q[s], fp.sh2_s[s])
+    return out.numpy()
+
+
+def _fp8_case(S=1, act_kind=1, seed=3, T=9, E=5):
+    shp = inputs.Shape(T=T, H=48, E=E, k=2, I=24, act=act_kind, n_shared=S,
+                       I_shared=24 if S else 0)
+    inp = inputs.make_inputs(shp, seed=seed, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=seed + 100)
+    return shp, inp, fp
+
+
+def _fwd8(inp, fp, shp, **over):
+    kw = dict(w13_q=fp.w13_q, w13_s=fp.w13_s, w2_q=fp.w2_q, w2_s=fp.w2_s,
+              sh13_q=fp.sh13_q, sh13_s=fp.sh13_s, sh2_q=fp.sh2_q, sh2_s=fp.sh2_s)
+    kw.update(over)
+    return oracle.forward_fp8(inp.x, inp.logits, k=shp.k, act_kind=shp.act,
+                              scale=inp.scale, **kw)
+
+
+@pytest.mark.parametrize("S,act_kind", [(0, 0), (1, 1), (2, 0)])
+def test_forward_fp8_equals_dense_restatement(S, act_kind):
+    shp, inp, fp = _fp8_case(S, act_kind)
+    out, ids, w = _fwd8(inp, fp, shp)
+    ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
+    assert (ids == ids_ref).all() and np.array_equal(w, w_ref)
+    want = _dense_fp8_torch(inp, fp, ids, w, act_kind)
+    rms = np.sqrt(np.mean(want ** 2))
+    assert np.abs(out - want).max() <= 1e-10 * rms
+
+
+def test_forward_fp8_is_linear_in_the_w2_scales():
+    shp, inp, fp = _fp8_case()
+    out, _, _ = _fwd8(inp, fp, shp)
+    out2, _, _ = _fwd8(inp, fp, shp, w2_s=fp.w2_s * 2, sh2_s=fp.sh2_s * 2)
+    assert np.array_equal(out2, 2 * out)
+
+
+def test_forward_fp8_never_reads_unselected_experts():
+    shp, inp, fp = _fp8_case(T=3, E=8)
+    out, ids, _ = _fwd8(inp, fp, shp)
+    unused = sorted(set(range(shp.E)) - set(ids.ravel().tolist()))
+    if not unused:
+        pytest.skip("every expert is selected")
+    w13 = fp.w13_q.clone()
+    w2 = fp.w2_q.clone()
+    w13[unused] = 0x7F  # NaN codes
+    w2[unused] = 0x7F
+    out2, _, _ = _fwd8(inp, fp, shp, w13_q=w13, w2_q=w2)
+    assert np.array_equal(out2, out)
