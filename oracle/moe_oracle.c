@@ -65,7 +65,8 @@ static double bf16_to_double(uint16_t b) {
 }
 
 /* Round a double to the nearest bf16 value (8 significant bits, ties to
- * even), returned as a double.  Used only by the diagnostic "round h" flag. */
+ * even), returned as a double.  Used by the diagnostic "round h" flag and
+ * by the FP8 layer's bf16 intermediate. */
 static double round_to_bf16(double v) {
   if (v == 0.0 || !isfinite(v)) return v;
   int e;
@@ -712,8 +713,10 @@ int oracle_gemma4_block(int64_t T, int H, int E, int k, int I, int act, int I_de
  *   - the layer on the dequantised values, in fp64: per routed (t, e),
  *       g_i = sum_h x'_h w1'_ih,  u_i = sum_h x'_h w3'_ih,  a_i = Act(g_i) u_i,
  *     x' the quantised token row (code times s_x), w' code times row scale;
- *     the row a is then quantised the same way (the exact a, not a rounded
- *     copy), and y_h = sum_i a'_i w2'_hi; the combine is the one of
+ *     the intermediate is a bf16 tensor between the two products, as in the
+ *     bf16 layer (FusedMoE's activation output in the activation dtype), so
+ *     the row a is rounded to bf16 and that bf16 row quantised the same way
+ *     as x; then y_h = sum_i a'_i w2'_hi, and the combine is the one of
  *     oracle_forward.  A code times an fp32 scale is exact in double.
  */
 
@@ -808,18 +811,10 @@ static void ffn_row_fp8(int H, int I, int act, const double* xq, const uint8_t* 
     }
     a[i] = act_fn(act, g) * u;
   }
-  /* quantise the intermediate row: amax of the exact values, then the
-   * float steps of quantize_row */
-  double amax = 0.0;
-  for (int i = 0; i < I; ++i)
-    if (fabs(a[i]) > amax) amax = fabs(a[i]);
-  const float famax = (float)amax;
-  const float s = famax > 0.0f ? famax / 448.0f : 1.0f;
-  for (int i = 0; i < I; ++i) {
-    af[i] = (float)a[i];
-    ac[i] = e4m3_code(af[i] / s);
-    a[i] = e4m3_value(ac[i]) * (double)s;
-  }
+  /* the intermediate row in bf16, quantised by the steps of quantize_row */
+  for (int i = 0; i < I; ++i) af[i] = (float)round_to_bf16(a[i]);
+  const float s = quantize_row(I, af, ac);
+  for (int i = 0; i < I; ++i) a[i] = e4m3_value(ac[i]) * (double)s;
   for (int h = 0; h < H; ++h) {
     const uint8_t* r2 = w2c + (int64_t)h * I;
     double acc = 0.0;

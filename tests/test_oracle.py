@@ -785,7 +785,7 @@ def _dense_fp8_torch(inp, fp, ids, w, act_kind):
         w2 = _fp8(c2).double() * torch.as_tensor(s2).double()[:, None]
         g, u = xq @ w13[:I].T, xq @ w13[I:].T
         a = (F.silu(g) if act_kind == 0 else F.gelu(g, approximate="tanh")) * u
-        return quant(a) @ w2.T
+        return quant(a.to(torch.bfloat16).double()) @ w2.T  # h is bf16, then quantised
 
     shp = inp.shape
     xq = quant(inp.x.double())
