@@ -15,8 +15,10 @@
  *
  * Around it: the router ahead of the routing (moe_router_logits), routing
  * variants (moe_route_ex: sigmoid scoring, expert groups), the Gemma 4 MoE
- * block with its parallel dense MLP and gamma norms (moe_gemma4_block), and
- * a permutation that needs no workspace (moe_permute_noalloc).
+ * block with its parallel dense MLP and gamma norms (moe_gemma4_block), the
+ * layer with FP8 (e4m3) experts and per-row scales (moe_forward_fp8, with
+ * its row quantiser moe_quantize_rows_e4m3), and a permutation that needs
+ * no workspace (moe_permute_noalloc).
  *
  * Conventions (every entry point):
  *   - All pointers are DEVICE pointers unless a parameter says otherwise.
@@ -373,6 +375,66 @@ MOE_API moe_status moe_gemma4_block(const moe_shape* shape, const moe_bf16* x,
                                     const moe_bf16* w13, const moe_bf16* w2,
                                     const float* scale, moe_bf16* out, float* out_f32,
                                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * FP8 experts.  Per-expert FP8 checkpoints store each expert's gate, up and
+ * down weights with a weight_scale, which FusedMoE packs as w13_weight /
+ * w2_weight and their _scale parameters (prhub.com.cn, sglang PR #24696,
+ * the per-expert FP8 loader fix; vLLM API page, load_weights).  The pages fix
+ * neither the format nor the scale granularity; this library reads them as:
+ *   - a weight is an e4m3 (E4M3FN) code times one fp32 scale per output row;
+ *   - activations are quantised per row when the layer runs: with amax the
+ *     row's largest |value|, s = fl32(amax / 448) (1 for an all-zero row) and
+ *     code = the nearest e4m3 value of fl32(v / s), ties to even, saturating
+ *     at +-448 ("FP8-Dynamic").  The intermediate h is quantised the same
+ *     way, per (token, expert) row.
+ * The products run on the tensor cores as e4m3 x e4m3 with fp32
+ * accumulation (tcgen05 kind::f8f6f4); both scales are applied to the fp32
+ * result.
+ */
+typedef struct {
+  const uint8_t* w13;          /* [E,2I,H] e4m3 codes, gate rows first */
+  const float* w13_scale;      /* [E,2I] */
+  const uint8_t* w2;           /* [E,H,I] */
+  const float* w2_scale;       /* [E,H] */
+  const uint8_t* w13_sh;       /* [S,2I,H], or NULL when S == 0 */
+  const float* w13_sh_scale;   /* [S,2I] */
+  const uint8_t* w2_sh;        /* [S,H,I] */
+  const float* w2_sh_scale;    /* [S,H] */
+} moe_fp8_experts;
+
+/*
+ * moe_quantize_rows_e4m3 -- the per-row dynamic quantisation above, of bf16
+ * rows src [rows, cols] (cols % 8 == 0, src 16-byte aligned) into codes
+ * [rows, cols] (8-byte aligned) and scales [rows].  It turns bf16 expert
+ * weights into the FP8 form (rows = output channels) as well.  Each code and
+ * scale is fixed by IEEE fp32 arithmetic, so it is reproducible bit for bit.
+ * Argument errors return MOE_ERR_INVALID_ARG before any launch.
+ */
+MOE_API moe_status moe_quantize_rows_e4m3(const moe_bf16* src, int64_t rows, int cols,
+                                          uint8_t* codes, float* scales,
+                                          cudaStream_t stream);
+
+/* Workspace bytes of moe_forward_fp8 (0 for an invalid shape). */
+MOE_API size_t moe_workspace_size_fp8(const moe_shape* shape);
+
+/*
+ * moe_forward_fp8 -- the layer of moe_forward_ex with FP8 experts:
+ * routing, permutation, x quantised per token and gathered, the w13
+ * product (+ activation, h in bf16), h quantised per row, the w2 product
+ * with the gate weights and the combine, one bf16 rounding.  Requires
+ * H % 16 == 0 and I % 16 == 0 (MOE_ERR_UNSUPPORTED otherwise), a workspace
+ * of moe_workspace_size_fp8 bytes (MOE_ERR_WORKSPACE) and the prefill path:
+ * opts->path MOE_PATH_DECODE returns MOE_ERR_UNSUPPORTED, the others run
+ * the tcgen05 grouped GEMMs at every T.  The other options (stage events,
+ * out_f32, deterministic, cta_pairs, router, route) mean what they mean for
+ * moe_forward_ex.
+ */
+MOE_API moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x,
+                                   const float* logits, const moe_fp8_experts* weights,
+                                   const float* scale, moe_bf16* out, int32_t* ids_out,
+                                   float* w_out, void* ws, size_t ws_bytes,
+                                   const moe_forward_opts* opts, cudaStream_t stream);
 
 /*
  * moe_read_error -- SYNCHRONISES ``stream``, then returns the status recorded

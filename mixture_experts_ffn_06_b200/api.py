@@ -29,7 +29,8 @@ EXPORTS = ("moe_layout_capacity", "moe_workspace_size", "moe_router_logits",
            "moe_forward_ex",
            "moe_read_error", "moe_selftest_wait_timeout", "moe_status_string",
            "moe_permute_noalloc", "moe_route_ex", "moe_gemma4_workspace_size",
-           "moe_gemma4_block")
+           "moe_gemma4_block", "moe_quantize_rows_e4m3", "moe_workspace_size_fp8",
+           "moe_forward_fp8")
 
 
 class MoEError(RuntimeError):
@@ -49,6 +50,13 @@ MAX_GROUPS = 32
 class moe_route_opts(ctypes.Structure):
     _fields_ = [("scoring", ctypes.c_int32), ("n_group", ctypes.c_int32),
                 ("topk_group", ctypes.c_int32)]
+
+
+class moe_fp8_experts(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("w13_scale", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p),
+                ("w13_sh", ctypes.c_void_p), ("w13_sh_scale", ctypes.c_void_p),
+                ("w2_sh", ctypes.c_void_p), ("w2_sh_scale", ctypes.c_void_p)]
 
 
 class moe_forward_opts(ctypes.Structure):
@@ -109,6 +117,11 @@ def _load() -> ctypes.CDLL:
     lib.moe_gemma4_block.argtypes = [S, P, ctypes.POINTER(moe_gemma4_block_params), P, P,
                                      P, P, P, P, ctypes.c_size_t, P]
     lib.moe_permute_noalloc.argtypes = [S, P, P, P, P, P]
+    lib.moe_quantize_rows_e4m3.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P]
+    lib.moe_workspace_size_fp8.argtypes = [S]
+    lib.moe_workspace_size_fp8.restype = ctypes.c_size_t
+    lib.moe_forward_fp8.argtypes = [S, P, P, ctypes.POINTER(moe_fp8_experts), P, P, P, P,
+                                    P, ctypes.c_size_t, ctypes.POINTER(moe_forward_opts), P]
     lib.moe_permute_noalloc.restype = st
     lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t,
                                               ctypes.c_uint32, P]
@@ -118,7 +131,7 @@ def _load() -> ctypes.CDLL:
                  "moe_expert_ffn",
                  "moe_combine",
                  "moe_forward", "moe_forward_ex", "moe_read_error", "moe_gemma4_block",
-                 "moe_selftest_wait_timeout"):
+                 "moe_selftest_wait_timeout", "moe_quantize_rows_e4m3", "moe_forward_fp8"):
         getattr(lib, name).restype = st
     return lib
 
@@ -319,3 +332,63 @@ def alloc_gemma4_workspace(shape, I_dense: int, device="cuda") -> torch.Tensor:
     if n == 0:
         raise MoEError(2, "moe_gemma4_workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)  # error words zeroed
+
+
+# ------------------------------------------------------------ FP8 experts
+
+def moe_quantize_rows_e4m3(src, codes, scales, stream=None):
+    """Per-row dynamic e4m3 quantisation of bf16 rows src [R, C] into codes
+    (uint8 [R, C]) and scales (fp32 [R])."""
+    R, C = src.shape
+    _check(lib.moe_quantize_rows_e4m3(_p(src), R, C, _p(codes), _p(scales),
+                                      _stream(stream)), "moe_quantize_rows_e4m3")
+
+
+def moe_workspace_size_fp8(shape: moe_shape) -> int:
+    return int(lib.moe_workspace_size_fp8(ctypes.byref(shape)))
+
+
+def alloc_workspace_fp8(shape: moe_shape, device="cuda") -> torch.Tensor:
+    n = moe_workspace_size_fp8(shape)
+    if n == 0:
+        raise MoEError(1, "moe_workspace_size_fp8")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def fp8_experts(w13, w13_scale, w2, w2_scale, w13_sh=None, w13_sh_scale=None, w2_sh=None,
+                w2_sh_scale=None) -> moe_fp8_experts:
+    """The weights argument of moe_forward_fp8 (uint8 code tensors, fp32
+    row scales)."""
+    return moe_fp8_experts(_p(w13), _p(w13_scale), _p(w2), _p(w2_scale), _p(w13_sh),
+                           _p(w13_sh_scale), _p(w2_sh), _p(w2_sh_scale))
+
+
+def moe_forward_fp8(shape, x, logits, weights: moe_fp8_experts, scale, out, ws,
+                    ids_out=None, w_out=None, events=None, out_f32=None,
+                    path=PATH_AUTO, deterministic=False, cta_pairs=0, router=None,
+                    route=None, stream=None):
+    """The layer with FP8 experts; ``weights`` from fp8_experts(); the
+    options as for moe_forward_ex."""
+    arr = None
+    if events is not None:
+        if len(events) != NUM_STAGES + 1:
+            raise ValueError("need NUM_STAGES + 1 events")
+        st = stream if stream is not None else torch.cuda.current_stream()
+        for e in events:
+            if e is not None and not e.cuda_event:
+                e.record(st)
+        arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
+            *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in events])
+    rx, rw, rs, reps = router if router is not None else (None, None, None, 0.0)
+    ro = route_opts(route)
+    opts = moe_forward_opts(
+        ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None,
+        _p(out_f32), path, int(bool(deterministic)), cta_pairs,
+        _p(rx), _p(rw), _p(rs), float(reps),
+        ctypes.pointer(ro) if ro is not None else None)
+    _check(lib.moe_forward_fp8(ctypes.byref(shape), _p(x), _p(logits), ctypes.byref(weights),
+                               _p(scale), _p(out), _p(ids_out), _p(w_out), _p(ws),
+                               ws.numel(), ctypes.byref(opts), _stream(stream)),
+           "moe_forward_fp8")

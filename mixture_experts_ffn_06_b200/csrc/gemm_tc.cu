@@ -104,6 +104,11 @@ struct KParams {
   int64_t T;                    // modes 2, 3
   int k, S;                     // modes 2, 3
   int a_sh_x;                   // shared groups' A rows come from tmAs (x)
+  // FP8 operands: the product of row r and column n is scaled by
+  // a_scale[r] * b_scale[group row of n] (b_scale_sh for shared groups)
+  const float* a_scale;
+  const float* b_scale;
+  const float* b_scale_sh;
 };
 
 // A work unit is (group g, block of CG m-tiles, n-tile); units are ordered
@@ -153,7 +158,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int MODE, int CG, int NH = 128>
+// F8: e4m3 operands (tcgen05.mma kind::f8f6f4): a k-block is 128 values of
+// one byte, so the shared-memory tiles keep their 128-byte rows.
+template <int MODE, int CG, int NH = 128, bool F8 = false>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmAs,
@@ -164,6 +171,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   using C = Cfg<CG, NH>;
   constexpr int STAGES = C::STAGES;
   constexpr int B_STAGE = C::B_STAGE;
+  constexpr int KBE = F8 ? 2 * BK : BK;  // elements of one k-block (128 bytes)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -271,20 +279,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           if (CG == 1) {
             mbar_expect_tx(fb, A_STAGE + B_STAGE);
-            tma_load_2d(sA + stage * A_STAGE, ma, kb * BK, arow, fb);
+            tma_load_2d(sA + stage * A_STAGE, ma, kb * KBE, arow, fb);
             if (MODE == 0) {
-              tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
-              tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * BK,
+              tma_load_2d(sB + stage * B_STAGE, mb, kb * KBE, brow, fb);
+              tma_load_2d(sB + stage * B_STAGE + B_STAGE / 2, mb, kb * KBE,
                           brow + p.up_off, fb);
             } else {
-              tma_load_2d(sB + stage * B_STAGE, mb, kb * BK, brow, fb);
+              tma_load_2d(sB + stage * B_STAGE, mb, kb * KBE, brow, fb);
             }
           } else {
             // both CTAs' bytes complete on CTA 0's full barrier
             if (rank == 0) mbar_expect_tx(fb, 2 * (A_STAGE + B_STAGE));
             const uint32_t fb0 = fb & kPeerBitMask;
-            tma_load_2d_pair(sA + stage * A_STAGE, ma, kb * BK, arow, fb0);
-            tma_load_2d_pair(sB + stage * B_STAGE, mb, kb * BK, brow, fb0);
+            tma_load_2d_pair(sA + stage * A_STAGE, ma, kb * KBE, arow, fb0);
+            tma_load_2d_pair(sB + stage * B_STAGE, mb, kb * KBE, brow, fb0);
           }
           last_fill[stage] = (int32_t)phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -304,7 +312,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // --------------------------------------------------------- MMA issuer
     // (CTA 0 of the pair issues for both when CG = 2)
     if (lane == 0 && (CG == 1 || rank == 0)) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, C::N_MMA);
+      constexpr uint32_t idesc =
+          F8 ? idesc_e4m3_f32(BM * CG, C::N_MMA) : idesc_bf16_f32(BM * CG, C::N_MMA);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int64_t t = unit0; ok && t < total; t += unit_step) {
@@ -327,14 +336,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(sA + stage * A_STAGE);
           const uint64_t bd = sw128_kmajor_desc(sB + stage * B_STAGE);
+          // four MMAs of 32 bytes of K each (16 bf16 or 32 e4m3 values)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {
             if (CG == 2)
-              umma_bf16_pair(d, ad + 2u * kk, bd + 2u * kk, idesc,
-                             (kb | kk) != 0 ? 1u : 0u);
+              umma_pair<F8>(d, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
             else
-              umma_bf16(d, ad + 2u * kk, bd + 2u * kk, idesc,
-                        (kb | kk) != 0 ? 1u : 0u);
+              umma<F8>(d, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if (CG == 2)
             umma_commit_pair_mc(smem_u32(&ctl->empty[stage]), 0x3);
@@ -415,6 +423,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
       const int64_t wrow0 = tl.row0 + q * 32;  // first tile row of this warp
       constexpr int CHUNKS = MODE == 0 ? (NH + 31) / 32 : 8;
+      // FP8: this lane's row scale, and the column scales of the group's
+      // B rows (mode 0: gate row n at n, up row n at N + n)
+      float sa = 1.0f;
+      const float* sb = nullptr;
+      if (F8 && tl.valid) {
+        sa = __ldg(p.a_scale + wrow0 + lane);
+        const bool routed = tl.g < p.E;
+        sb = (routed ? p.b_scale : p.b_scale_sh) +
+             (int64_t)(routed ? tl.g : tl.g - p.E) * (MODE == 0 ? 2 * p.N : p.N);
+      }
+      // value of accumulator column j of B row `brow` (for a column past N
+      // the scale is not read: nothing of it is stored)
+      auto scaled = [&](uint32_t bits, int brow, bool in) -> float {
+        const float v = __uint_as_float(bits);
+        if (!F8) return v;
+        return in ? v * (sa * __ldg(sb + brow)) : 0.0f;
+      };
 #pragma unroll 1
       for (int c = 0; c < CHUNKS; ++c) {
         const int col0 = tl.n0 + c * 32;
@@ -424,9 +449,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
           if (!tl.valid) continue;  // the pair's empty half: nothing to store
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) *
-                            __uint_as_float(u[j]);
+          for (int j = 0; j < 32; ++j) {
+            const bool in = col0 + j < p.N;
+            tbuf[lane][j] = act_apply(p.act, scaled(g[j], col0 + j, in)) *
+                            scaled(u[j], p.N + col0 + j, in);
+          }
         } else if (MODE == 0) {
           // gate columns [32c, 32c + 32); the matching up column NH + 32c + j
           // lies in the 32-column chunk starting at 32 (NH / 32 + c) or in
@@ -440,14 +467,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const uint32_t uj = j + UR < 32 ? u0[j + UR] : u1[j + UR - 32];
-            tbuf[lane][j] = act_apply(p.act, __uint_as_float(g[j])) * __uint_as_float(uj);
+            const bool in = col0 + j < p.N && c * 32 + j < NH;
+            tbuf[lane][j] = act_apply(p.act, scaled(g[j], col0 + j, in)) *
+                            scaled(uj, p.N + col0 + j, in);
           }
         } else {
           uint32_t y[32];
           tmem_ld32(tb + c * 32, y);
           if (!tl.valid) continue;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tbuf[lane][j] = __uint_as_float(y[j]);
+          for (int j = 0; j < 32; ++j) tbuf[lane][j] = scaled(y[j], col0 + j, col0 + j < p.N);
         }
         __syncwarp();
         if (MODE == 0) {
@@ -550,16 +579,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [outer, inner] row-major bf16 tensor, box {64, box_rows}, 128-byte swizzle.
+// [outer, inner] row-major tensor of bf16 (box {64, box_rows}) or of e4m3
+// bytes (f8: box {128, box_rows}); rows of 128 bytes, 128-byte swizzle.
 cudaError_t make_map(CUtensorMap* m, const void* ptr, uint64_t inner,
-                     uint64_t outer, uint32_t box_rows) {
+                     uint64_t outer, uint32_t box_rows, bool f8 = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint64_t strides[1] = {inner * (f8 ? 1 : 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)(f8 ? 2 * BK : BK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUresult r = enc(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                          const_cast<void*>(ptr), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -583,16 +613,17 @@ int num_sms() {
   return n;
 }
 
-template <int MODE, int CG, int NH = 128>
+template <int MODE, int CG, int NH = 128, bool F8 = false>
 cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   using C = Cfg<CG, NH>;
   constexpr int BN_OUT = MODE == 0 ? NH : BN_ACC;
+  constexpr int KBE = F8 ? 2 * BK : BK;
   CUtensorMap mA, mAs, mB, mBs;
-  cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM);
+  cudaError_t e = make_map(&mA, a.A, (uint64_t)a.K, (uint64_t)a.cap, BM, F8);
   if (e != cudaSuccess) return e;
   const bool a_sh_x = a.A_sh != nullptr && a.G > a.E && a.T > 0;
   if (a_sh_x) {
-    e = make_map(&mAs, a.A_sh, (uint64_t)a.K, (uint64_t)a.T, BM);
+    e = make_map(&mAs, a.A_sh, (uint64_t)a.K, (uint64_t)a.T, BM, F8);
     if (e != cudaSuccess) return e;
   } else {
     mAs = mA;
@@ -601,11 +632,11 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   // per-CTA B box: mode 0 loads NH gate (and NH up) rows; the others 256
   // rows, or 128 per CTA of a pair
   const uint32_t box_rows = MODE == 0 ? NH : (uint32_t)C::B_ROWS;
-  e = make_map(&mB, a.B, (uint64_t)a.K, rows_per_group * (uint64_t)a.E, box_rows);
+  e = make_map(&mB, a.B, (uint64_t)a.K, rows_per_group * (uint64_t)a.E, box_rows, F8);
   if (e != cudaSuccess) return e;
   if (a.B_sh && a.G > a.E) {
     e = make_map(&mBs, a.B_sh, (uint64_t)a.K,
-                 rows_per_group * (uint64_t)(a.G - a.E), box_rows);
+                 rows_per_group * (uint64_t)(a.G - a.E), box_rows, F8);
     if (e != cudaSuccess) return e;
   } else {
     mBs = mB;
@@ -617,7 +648,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   p.N = a.N;
   p.K = a.K;
   p.NT = (a.N + BN_OUT - 1) / BN_OUT;
-  p.KB = (a.K + BK - 1) / BK;
+  p.KB = (a.K + KBE - 1) / KBE;
   p.b_rows_per_group = (int32_t)rows_per_group;
   p.up_off = MODE == 0 ? a.N : 0;
   p.out = a.out;
@@ -630,6 +661,9 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   p.k = a.k;
   p.S = a.G - a.E;
   p.a_sh_x = a_sh_x ? 1 : 0;
+  p.a_scale = a.a_scale;
+  p.b_scale = a.b_scale;
+  p.b_scale_sh = a.b_scale_sh;
 
   const size_t smem = 1024 + (size_t)C::STAGES * (A_STAGE + C::B_STAGE) +
                       sizeof(EpiSmem) + sizeof(Ctl) +
@@ -640,7 +674,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices || !attr_set[dev].load()) {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, NH>,
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, NH, F8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024);
     if (e != cudaSuccess) return e;
@@ -671,7 +705,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, NH>, mA, mAs, mB, mBs, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, NH, F8>, mA, mAs, mB, mBs, p);
 }
 
 __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
@@ -701,6 +735,24 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st, bool 
   // saves 5-7 % of the step at 16-256 tokens.
   const int64_t rows = a.T * a.k + a.T * (int64_t)(a.G - a.E);
   const bool narrow = a.N % 128 != 0 && a.N % 88 == 0 && rows < 256 * (int64_t)a.G;
+  if (a.f8) {
+    switch (a.mode) {
+      case 0:
+        return pair ? launch_mode<0, 2, 128, true>(a, st, pdl)
+               : narrow ? launch_mode<0, 1, 88, true>(a, st, pdl)
+                        : launch_mode<0, 1, 128, true>(a, st, pdl);
+      case 1:
+        return pair ? launch_mode<1, 2, 128, true>(a, st, pdl)
+                    : launch_mode<1, 1, 128, true>(a, st, pdl);
+      case 2:
+        return pair ? launch_mode<2, 2, 128, true>(a, st, pdl)
+                    : launch_mode<2, 1, 128, true>(a, st, pdl);
+      case 3:
+        return pair ? launch_mode<3, 2, 128, true>(a, st, pdl)
+                    : launch_mode<3, 1, 128, true>(a, st, pdl);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (a.mode) {
     case 0:
       return pair ? launch_mode<0, 2>(a, st, pdl)

@@ -39,6 +39,13 @@ struct WsMap {
   size_t dt_cnt;       // decode path, tensor-core form: [2, G*row blocks] int32
   size_t logits;       // [T,E] fp32 router logits (moe_forward_ex with a router)
   size_t total;
+  // moe_forward_fp8, after `total` (the permuted codes of x reuse x_perm):
+  size_t x_q;          // [T,H] e4m3 codes of the token rows
+  size_t s_x;          // [T] their scales
+  size_t a_scale;      // [cap] row scales of the w13 product's A rows
+  size_t h_q;          // [cap,I] e4m3 codes of h
+  size_t s_h;          // [cap] their scales
+  size_t total_fp8;
   int64_t cap;
   int64_t n_lt;
 };
@@ -89,6 +96,21 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* sorted_slots,
                           const int32_t* offsets, int G, int64_t T, int k,
                           int H, int64_t cap, __nv_bfloat16* x_perm, float* acc,
                           int64_t n_acc, cudaStream_t st, bool pdl = false);
+
+// FP8 (fp8.cu).  Per-row dynamic e4m3 quantisation of bf16 rows [rows, cols]
+// (cols % 8 == 0): codes [rows, cols] bytes, scales [rows].  rows_used
+// (device, or null): only rows below *rows_used; slots (or null): rows whose
+// slot is negative are skipped.
+cudaError_t launch_quantize_rows(const __nv_bfloat16* src, int64_t rows, int cols,
+                                 uint8_t* codes, float* scales, const int32_t* rows_used,
+                                 const int32_t* slots, cudaStream_t st, bool pdl = false);
+// Codes of x's token rows into the routed experts' permuted rows (H % 16 ==
+// 0), the row scale of every row in use (shared experts' too), and zeroes
+// acc[0, n_acc) when given.
+cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, const int32_t* sorted_slots,
+                              const int32_t* offsets, int E, int G, int64_t T, int k, int H,
+                              int64_t cap, uint8_t* x_perm, float* a_scale, float* acc,
+                              int64_t n_acc, cudaStream_t st, bool pdl = false);
 
 // out = bf16(acc) (round to nearest even), out_f32 = acc if given; n % 8 == 0.
 cudaError_t launch_finalize(const float* acc, int64_t n, __nv_bfloat16* out,
@@ -176,6 +198,13 @@ struct GroupedGemmArgs {
   int64_t T;
   int k;
   bool pair;                    // run on CTA pairs (2-SM MMA, M = 256)
+  // FP8 operands: A and B hold e4m3 bytes (K % 16 == 0); the product of A
+  // row r and B row n is scaled by a_scale[r] * b_scale[group row n]
+  // (b_scale_sh for the shared groups) before the epilogue uses it
+  bool f8;
+  const float* a_scale;         // [cap]
+  const float* b_scale;         // [E, rows per group]
+  const float* b_scale_sh;      // [S, rows per group] or nullptr
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st,
                                 bool pdl = false);

@@ -46,6 +46,12 @@ WsMap workspace_map(const moe_shape& s) {
   m.dt_cnt = take(dt ? sizeof(int32_t) * 2 * G * dt_row_blocks(s.H, s.I) : 0);
   m.logits = take(sizeof(float) * T * s.E);
   m.total = o;
+  m.x_q = take((size_t)T * s.H);
+  m.s_x = take(sizeof(float) * T);
+  m.a_scale = take(sizeof(float) * m.cap);
+  m.h_q = take((size_t)m.cap * Imax);
+  m.s_h = take(sizeof(float) * m.cap);
+  m.total_fp8 = o;
   return m;
 }
 
@@ -433,6 +439,164 @@ moe_status moe_forward(const moe_shape* shape, const moe_bf16* x,
                        size_t ws_bytes, cudaStream_t stream) {
   return moe_forward_ex(shape, x, logits, w13, w2, scale, w13_sh, w2_sh, out,
                         ids_out, w_out, ws, ws_bytes, nullptr, stream);
+}
+
+size_t moe_workspace_size_fp8(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return workspace_map(*shape).total_fp8;
+}
+
+moe_status moe_quantize_rows_e4m3(const moe_bf16* src, int64_t rows, int cols,
+                                  uint8_t* codes, float* scales, cudaStream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!src || !codes || !scales || !aligned16(src) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7u) != 0)
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_quantize_rows(reinterpret_cast<const __nv_bfloat16*>(src), rows,
+                                        cols, codes, scales, nullptr, nullptr, stream));
+}
+
+moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x, const float* logits,
+                           const moe_fp8_experts* wq, const float* scale, moe_bf16* out,
+                           int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes,
+                           const moe_forward_opts* opts, cudaStream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const moe_shape& s = *shape;
+  // e4m3 rows are TMA tiles: their byte strides must be multiples of 16
+  if (s.H % 16 != 0 || s.I % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!wq || !wq->w13 || !wq->w13_scale || !wq->w2 || !wq->w2_scale) return MOE_ERR_INVALID_ARG;
+  if (s.n_shared > 0 && (!wq->w13_sh || !wq->w13_sh_scale || !wq->w2_sh ||
+                         !wq->w2_sh_scale))
+    return MOE_ERR_INVALID_ARG;
+  const bool use_router = opts && opts->router_w;
+  if (s.T > 0 && (!x || (!logits && !use_router) || !out)) return MOE_ERR_INVALID_ARG;
+  if (use_router) {
+    if (!(opts->router_eps >= 0.0f) || !std::isfinite(opts->router_eps))
+      return MOE_ERR_INVALID_ARG;
+    if (s.T > 0 && (!opts->router_x || !opts->router_scale || !aligned16(opts->router_x) ||
+                    !aligned16(opts->router_w) || !aligned16(opts->router_scale)))
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (opts && (opts->cta_pairs < 0 || opts->cta_pairs > 2)) return MOE_ERR_INVALID_ARG;
+  const int path = opts ? opts->path : MOE_PATH_AUTO;
+  if (path == MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+  RouteOpt ro;
+  if ((st = check_route_opts(s, opts ? opts->route : nullptr, &ro)) != MOE_OK) return st;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  const WsMap m = workspace_map(s);
+  if (ws_bytes < m.total_fp8) return MOE_ERR_WORKSPACE;
+  void* const* ev = opts ? opts->stage_events : nullptr;
+  if (s.T == 0) {
+    for (int i = 0; i <= MOE_NUM_STAGES; ++i)
+      if (!mark(ev, i, stream)) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const int G = s.E + s.n_shared;
+  int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(at(ws, m.ids));
+  float* w = w_out ? w_out : reinterpret_cast<float*>(at(ws, m.w));
+  auto* offsets = reinterpret_cast<int32_t*>(at(ws, m.offsets));
+  auto* sorted_slots = reinterpret_cast<int32_t*>(at(ws, m.sorted_slots));
+  auto* slot_row = reinterpret_cast<int32_t*>(at(ws, m.slot_row));
+  auto* err = reinterpret_cast<uint32_t*>(at(ws, m.err));
+  auto* xq = reinterpret_cast<uint8_t*>(at(ws, m.x_q));
+  auto* sx = reinterpret_cast<float*>(at(ws, m.s_x));
+  auto* x_perm = reinterpret_cast<uint8_t*>(at(ws, m.x_perm));
+  auto* a_scale = reinterpret_cast<float*>(at(ws, m.a_scale));
+  auto* h = reinterpret_cast<__nv_bfloat16*>(at(ws, m.h));
+  auto* hq = reinterpret_cast<uint8_t*>(at(ws, m.h_q));
+  auto* sh = reinterpret_cast<float*>(at(ws, m.s_h));
+  auto* stage = reinterpret_cast<float*>(at(ws, m.stage));
+  float* acc = reinterpret_cast<float*>(at(ws, m.acc));
+  const bool det = opts && opts->deterministic;
+  const int cta_pairs = opts ? opts->cta_pairs : 0;
+  if (use_router) logits = reinterpret_cast<float*>(at(ws, m.logits));
+
+  // stage 0: router (if any) and routing; 1: layout; 2: the codes of x and
+  // their gather; 3: w13 + activation; 4: the codes of h and w2 + combine;
+  // 5: the rounding
+  if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
+  if (use_router &&
+      launch_router_logits(reinterpret_cast<const __nv_bfloat16*>(opts->router_x),
+                           reinterpret_cast<const __nv_bfloat16*>(opts->router_w),
+                           reinterpret_cast<const __nv_bfloat16*>(opts->router_scale), s.T,
+                           s.H, s.E, opts->router_eps, const_cast<float*>(logits),
+                           stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_route(logits, scale, s.T, s.E, s.k, ids, w, stream, ro) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (!mark(ev, 1, stream)) return MOE_ERR_CUDA;
+  if (launch_layout(s, ids, offsets, sorted_slots, slot_row, m.cap,
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_count)),
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_base)),
+                    reinterpret_cast<int32_t*>(at(ws, m.lt_rank)), m.n_lt, err, stream,
+                    /*pdl=*/true) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (!mark(ev, 2, stream)) return MOE_ERR_CUDA;
+  if (launch_quantize_rows(reinterpret_cast<const __nv_bfloat16*>(x), s.T, s.H, xq, sx,
+                           nullptr, nullptr, stream, /*pdl=*/true) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_gather_fp8(xq, sx, sorted_slots, offsets, s.E, G, s.T, s.k, s.H, m.cap, x_perm,
+                        a_scale, det ? nullptr : acc, s.T * (int64_t)s.H, stream,
+                        /*pdl=*/true) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (!mark(ev, 3, stream)) return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.mode = 0;
+  a.A = reinterpret_cast<const __nv_bfloat16*>(x_perm);
+  a.A_sh = reinterpret_cast<const __nv_bfloat16*>(xq);
+  a.B = reinterpret_cast<const __nv_bfloat16*>(wq->w13);
+  a.B_sh = reinterpret_cast<const __nv_bfloat16*>(wq->w13_sh);
+  a.offsets = offsets;
+  a.G = G;
+  a.E = s.E;
+  a.N = s.I;
+  a.K = s.H;
+  a.cap = m.cap;
+  a.out = h;
+  a.act = s.act;
+  a.err = err;
+  a.sorted_slots = sorted_slots;
+  a.w = w;
+  a.T = s.T;
+  a.k = s.k;
+  a.pair = cta_pairs == 2;
+  a.f8 = true;
+  a.a_scale = a_scale;
+  a.b_scale = wq->w13_scale;
+  a.b_scale_sh = wq->w13_sh_scale;
+  if (launch_grouped_gemm(a, stream, true) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(ev, 4, stream)) return MOE_ERR_CUDA;
+  // h rows in use: below offsets[G]; padding rows (slot -1) are skipped
+  if (launch_quantize_rows(h, m.cap, s.I, hq, sh, offsets + G, sorted_slots, stream,
+                           /*pdl=*/true) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const bool big = s.T * (int64_t)s.k >= 2 * 128 * (int64_t)s.E;
+  a.mode = det ? 3 : 2;
+  a.pair = cta_pairs == 2 || (cta_pairs == 0 && big && s.I >= 1024);
+  a.A = reinterpret_cast<const __nv_bfloat16*>(hq);
+  a.A_sh = nullptr;
+  a.B = reinterpret_cast<const __nv_bfloat16*>(wq->w2);
+  a.B_sh = reinterpret_cast<const __nv_bfloat16*>(wq->w2_sh);
+  a.N = s.H;
+  a.K = s.I;
+  a.out = det ? stage : acc;
+  a.a_scale = sh;
+  a.b_scale = wq->w2_scale;
+  a.b_scale_sh = wq->w2_sh_scale;
+  if (launch_grouped_gemm(a, stream, true) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(ev, 5, stream)) return MOE_ERR_CUDA;
+  float* out_f32 = opts ? opts->out_f32 : nullptr;
+  const cudaError_t e =
+      det ? launch_sum_rows(stage, s.T, s.k + s.n_shared, s.H,
+                            reinterpret_cast<__nv_bfloat16*>(out), out_f32, stream, true)
+          : launch_finalize(acc, s.T * (int64_t)s.H, reinterpret_cast<__nv_bfloat16*>(out),
+                            out_f32, stream, true);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return mark(ev, 6, stream) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_read_error(void* ws, size_t ws_bytes, cudaStream_t stream) {

@@ -195,3 +195,37 @@ def test_gemma4_block_refuses_bad_arguments(api):
              need, None) == 1                                # a gamma missing
     assert f(ctypes.byref(sh), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
              need, None) == 2                                # shared experts
+
+
+def test_fp8_entry_points_refuse_bad_arguments(api):
+    # all rejected on the host before any launch: no GPU needed
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced
+    null = ctypes.c_void_p(0)
+    lib = api.lib
+    # quantiser: cols must be a positive multiple of 8
+    assert lib.moe_quantize_rows_e4m3(fake, 4, 12, fake, fake, null) == 1
+    assert lib.moe_quantize_rows_e4m3(fake, -1, 16, fake, fake, null) == 1
+    assert lib.moe_quantize_rows_e4m3(null, 4, 16, fake, fake, null) == 1
+    assert lib.moe_quantize_rows_e4m3(fake, 0, 16, fake, fake, null) == 0  # empty
+    s = api.make_shape(T=8, H=64, E=4, k=2, I=64)
+    assert api.moe_workspace_size_fp8(s) > api.moe_workspace_size(s)
+    w = api.moe_fp8_experts(fake, fake, fake, fake, None, None, None, None)
+    opts = api.moe_forward_opts()
+    ws_n = api.moe_workspace_size_fp8(s)
+    # e4m3 rows need H % 16 == 0 and I % 16 == 0
+    s8 = api.make_shape(T=8, H=72, E=4, k=2, I=64)
+    assert lib.moe_forward_fp8(ctypes.byref(s8), fake, fake, ctypes.byref(w), None, fake,
+                               None, None, fake, 1 << 40, ctypes.byref(opts), null) == 2
+    # missing weights, small workspace, the decode path
+    w_bad = api.moe_fp8_experts(fake, None, fake, fake, None, None, None, None)
+    assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w_bad), None,
+                               fake, None, None, ctypes.c_void_p(1 << 20), ws_n,
+                               ctypes.byref(opts), null) == 1
+    assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w), None, fake,
+                               None, None, ctypes.c_void_p(1 << 20), ws_n - 256,
+                               ctypes.byref(opts), null) == 3
+    dec = api.moe_forward_opts()
+    dec.path = api.PATH_DECODE
+    assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w), None, fake,
+                               None, None, ctypes.c_void_p(1 << 20), ws_n,
+                               ctypes.byref(dec), null) == 2

@@ -17,6 +17,8 @@ FIELDS = {
                          "router_x", "router_w", "router_scale", "router_eps", "route"],
     "moe_gemma4_block_params": ["I_dense", "mlp_w13", "mlp_w2", "norm_w", "eps",
                                 "router_w", "router_scale", "router_eps"],
+    "moe_fp8_experts": ["w13", "w13_scale", "w2", "w2_scale", "w13_sh", "w13_sh_scale",
+                        "w2_sh", "w2_sh_scale"],
 }
 
 

@@ -1,0 +1,148 @@
+"""Parity of the layer with FP8 (e4m3) experts on the GPU with the fp64
+oracle (through the C ABI).
+
+Per-expert FP8 checkpoints (the sglang PR on Gemma 4 FP8 per-expert
+loading; load_weights on the vLLM API page) carry a weight_scale per
+weight; the reading is one fp32 scale per output row, activations and the
+bf16 intermediate quantised per row at run time.  Bars: the row quantiser's
+codes and scales bit-exact (IEEE fp32 steps on both sides); routing ids
+bit-exact and gate weights within 1e-6 relative; the layer output within
+2e-2 x RMS(oracle) on the fp32 result, the bf16 output its exact rounding
+and within 2e-2 x RMS + 2^-8 |oracle|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_ffn_06_b200 import inputs
+from parity_util import assert_out_close, assert_routing_exact
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixture_experts_ffn_06_b200 import api as a
+    return a
+
+
+@pytest.mark.parametrize("R,C", [(1, 8), (37, 104), (300, 2816), (64, 4096)])
+def test_quantize_rows_bit_exact(api, R, C):
+    g = torch.Generator().manual_seed(R + C)
+    x = torch.randn(R, C, generator=g) * torch.exp(torch.randn(R, 1, generator=g) * 3)
+    if R > 2:
+        x[1] = 0.0                      # all-zero row: scale 1
+        x[2, 5] = 3e4                   # one large value sets the scale
+        x[2, 6] = -2e-30                # tiny values flush to (signed) zero
+    xb = x.to(torch.bfloat16)
+    codes = torch.empty(R, C, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(R, dtype=torch.float32, device="cuda")
+    api.moe_quantize_rows_e4m3(xb.cuda(), codes, scales)
+    torch.cuda.synchronize()
+    want_c, want_s = oracle.quantize_rows_e4m3(xb)
+    assert np.array_equal(scales.cpu().numpy(), want_s)
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+
+
+def _to(t):
+    return None if t is None else t.cuda().contiguous()
+
+
+def _gpu_fp8(api, inp, fp, det=False, pairs=0, path=0):
+    shp = inp.shape
+    s = api.shape_from(shp)
+    T, H, k = shp.T, shp.H, shp.k
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty(T, H, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ws = api.alloc_workspace_fp8(s)
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
+                            fp.sh2_q, fp.sh2_s)]
+    weights = api.fp8_experts(*wts)
+    api.moe_forward_fp8(s, _to(inp.x), _to(inp.logits), weights, _to(inp.scale), out, ws,
+                        ids_out=ids, w_out=w, out_f32=out32, deterministic=det,
+                        cta_pairs=pairs, path=path)
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    assert torch.equal(out, out32.to(torch.bfloat16)), "bf16 rounding step"
+    return out, out32, ids, w
+
+
+def _oracle_fp8(inp, fp, tokens=None):
+    return oracle.forward_fp8(inp.x, inp.logits, fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s,
+                              k=inp.shape.k, act_kind=inp.shape.act, scale=inp.scale,
+                              sh13_q=fp.sh13_q, sh13_s=fp.sh13_s, sh2_q=fp.sh2_q,
+                              sh2_s=fp.sh2_s, tokens=tokens)
+
+
+SHAPES = {
+    "tiny": inputs.Shape(T=64, H=256, E=8, k=2, I=512),
+    "ragged": inputs.Shape(T=37, H=208, E=5, k=3, I=112, act=1),  # K, N tails
+    "shared": inputs.Shape(T=40, H=128, E=6, k=2, I=96, n_shared=2, I_shared=96),
+    "one_token": inputs.Shape(T=1, H=128, E=8, k=2, I=128),
+    "gemma_T130": inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),  # narrow tiles
+    "pairs": inputs.Shape(T=700, H=208, E=3, k=2, I=112, act=1),
+    "pairs_wide_I": inputs.Shape(T=600, H=128, E=2, k=2, I=1024),
+}
+VARIANTS = {"fast": (False, 0), "det": (True, 0), "pairs": (False, 2)}
+
+
+@pytest.mark.parametrize("variant", list(VARIANTS))
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_forward_fp8_every_element(api, name, variant):
+    shp = SHAPES[name]
+    inp = inputs.make_inputs(shp, seed=4, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=104)
+    want, ids_ref, w_ref = _oracle_fp8(inp, fp)
+    det, pairs = VARIANTS[variant]
+    out, out32, ids, w = _gpu_fp8(api, inp, fp, det=det, pairs=pairs)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out32, want, f"{name} fp8 ({variant})", bf16=out)
+
+
+def test_forward_fp8_refuses_the_decode_path(api):
+    shp = SHAPES["one_token"]
+    inp = inputs.make_inputs(shp, seed=1)
+    fp = inputs.fp8_experts(shp, seed=2)
+    with pytest.raises(api.MoEError) as e:
+        _gpu_fp8(api, inp, fp, path=api.PATH_DECODE)
+    assert e.value.status == 2
+
+
+def test_forward_fp8_deterministic_repeats_bit_for_bit(api):
+    shp = SHAPES["gemma_T130"]
+    inp = inputs.make_inputs(shp, seed=5, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=105)
+    a = _gpu_fp8(api, inp, fp, det=True)
+    b = _gpu_fp8(api, inp, fp, det=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_forward_fp8_full_size_many_small(api):
+    """The many-small-experts prefill (T=8192, H=2816, E=128, k=8, I=704,
+    tanh-GELU) with FP8 experts: every routing decision, and the outputs of
+    one token from every 128-row (expert, m-tile) of the layout."""
+    shp = inputs.shape_of("many_small_prefill")
+    inp = inputs.make_inputs("many_small_prefill", seed=0, device="cuda")
+    fp = inputs.fp8_experts(shp, seed=1, device="cuda")
+    out, out32, ids, w = _gpu_fp8(api, inp, fp)
+    ids_ref, w_ref = oracle.route(inp.logits, shp.k, scale=inp.scale)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    offsets, sorted_slots, _ = oracle.layout(ids_ref, shp.E, 0, 128)
+    rng = np.random.default_rng(3)
+    tok = {0, shp.T - 1}
+    for g in range(shp.E):
+        for r0 in range(int(offsets[g]), int(offsets[g + 1]), 128):
+            rows = sorted_slots[r0:r0 + 128]
+            real = rows[rows >= 0]
+            if real.size:
+                tok.add(int(real[rng.integers(real.size)]) // shp.k)
+    tok = np.array(sorted(tok), np.int64)
+    want, _, _ = _oracle_fp8(inp, fp, tokens=tok)
+    sel = torch.from_numpy(tok).cuda()
+    assert_out_close(out32[sel], want, f"many-small fp8, {len(tok)} tokens",
+                     bf16=out[sel])
