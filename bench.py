@@ -19,13 +19,15 @@ no collective on the data path (weak scaling).
 
 The default run (the Mixtral-shaped headline, one GPU) adds a ``configs``
 key with one entry for each other workload of the benchmark -- the
-many-small-experts and skewed prefills and the decode sweep T = 1, 4, 16,
-64, 256 -- each device-timed the same way, with its roofline fraction, its
+many-small-experts and skewed prefills, the decode sweep T = 1, 4, 16, 64,
+256, and the Mixtral-shaped and many-small prefills with FP8 (e4m3)
+experts -- each device-timed the same way, with its roofline fraction, its
 CPU baseline and ``parity``: the layer outputs the oracle computed for the
 baseline's token sample set beside the GPU's (max |err| / RMS of the fp32
 and bf16 outputs), and the routing ids, gate weights and layout of the whole
 batch compared with the oracle's.  The headline carries the same ``parity``.
-``--headline-only`` leaves the other workloads out.
+``--headline-only`` leaves the other workloads out; ``--fp8`` runs the
+headline with FP8 experts (``moe_forward_fp8``, prefill path).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
 bounded token sample per step) and prints the same line with
@@ -79,6 +81,8 @@ def parse():
                     help="time the Gemma 4 MoE block (dense MLP of this "
                          "intermediate size in parallel with the MoE, gamma "
                          "norms, router on the residual) instead of the layer")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 experts (e4m3 weights with per-row scales, moe_forward_fp8)")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the other workloads' lines (the configs key)")
     ap.add_argument("--router", action="store_true",
@@ -232,7 +236,8 @@ def traffic_for(kernel_src: str, config: str, shape_override):
 
 # ----------------------------------------------------------- CPU baseline
 
-def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int = 1):
+def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int = 1,
+                     fp8=None):
     """The CPU baseline: the oracle as it stands, timed on the host cores, on
     rounds of ``cores`` tokens drawn from the batch until ``budget_s`` has
     passed.  The layer outputs it computes for those tokens are then set
@@ -249,8 +254,14 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
             dict(x=inp.x, logits=inp.logits, w13=inp.w13, w2=inp.w2,
                  scale=inp.scale, w13_sh=inp.w13_sh, w2_sh=inp.w2_sh).items()}
     xu = oracle._u16(host["x"])
-    w13u, w2u = oracle._u16(host["w13"]), oracle._u16(host["w2"])
-    sh13, sh2 = oracle._u16(host["w13_sh"]), oracle._u16(host["w2_sh"])
+    if fp8 is None:
+        w13u, w2u = oracle._u16(host["w13"]), oracle._u16(host["w2"])
+        sh13, sh2 = oracle._u16(host["w13_sh"]), oracle._u16(host["w2_sh"])
+    else:  # FP8Experts on the device: codes and scales on the host
+        t = fp8
+        cv = lambda a: None if a is None else a.cpu()  # noqa: E731
+        fp8 = (cv(t.w13_q), cv(t.w13_s), cv(t.w2_q), cv(t.w2_s))
+        fp8_sh = (cv(t.sh13_q), cv(t.sh13_s), cv(t.sh2_q), cv(t.sh2_s))
     rng = np.random.default_rng(seed)
     per_round = min(cores, T)
     done, elapsed, rounds = 0, 0.0, 0
@@ -258,9 +269,15 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
     while rounds < max_rounds and (elapsed < budget_s or rounds == 0):
         tok = np.sort(rng.choice(T, per_round, replace=False))
         t0 = time.perf_counter()
-        o, _, _ = oracle.forward(xu, host["logits"], w13u, w2u, shp.k, shp.act,
-                                 scale=host["scale"], w13_sh=sh13, w2_sh=sh2,
-                                 tokens=tok, nthreads=per_round)
+        if fp8 is None:
+            o, _, _ = oracle.forward(xu, host["logits"], w13u, w2u, shp.k, shp.act,
+                                     scale=host["scale"], w13_sh=sh13, w2_sh=sh2,
+                                     tokens=tok, nthreads=per_round)
+        else:
+            o, _, _ = oracle.forward_fp8(xu, host["logits"], *fp8, shp.k, shp.act,
+                                         scale=host["scale"], sh13_q=fp8_sh[0],
+                                         sh13_s=fp8_sh[1], sh2_q=fp8_sh[2],
+                                         sh2_s=fp8_sh[3], tokens=tok, nthreads=per_round)
         elapsed += time.perf_counter() - t0
         toks.append(tok)
         outs.append(o)
@@ -269,7 +286,8 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
     baseline = {"value": done / elapsed, "unit": UNIT, "cores": per_round,
                 "kind": "oracle",
                 "sample": f"{done} tokens drawn from the same {T}-token batch in "
-                          f"rounds of {per_round}, full layer per token (fp64), "
+                          f"rounds of {per_round}, full layer per token (fp64"
+                          f"{', FP8 experts' if fp8 is not None else ''}), "
                           f"{elapsed:.1f} s"}
 
     tok = np.concatenate(toks)
@@ -316,21 +334,26 @@ def touched_experts(api, s, inp) -> int:
     return int(torch.unique(ids).numel()) + shp.n_shared
 
 
-def gpu_result(api, inp, s, path, args):
+def gpu_result(api, inp, s, path, args, fp8=None):
     """One call of the layer with every optional output, copied to the host
     (for the parity comparison of the CPU-baseline leg)."""
     import torch
     shp = inp.shape
     dev = inp.x.device
-    ws = api.alloc_workspace(s, dev)
+    ws = api.alloc_workspace_fp8(s, dev) if fp8 is not None else api.alloc_workspace(s, dev)
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
     out32 = torch.empty(shp.T, shp.H, dtype=torch.float32, device=dev)
     ids = torch.empty(shp.T, shp.k, dtype=torch.int32, device=dev)
     w = torch.empty(shp.T, shp.k, dtype=torch.float32, device=dev)
-    api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale, inp.w13_sh,
-                       inp.w2_sh, out, ws, ids_out=ids, w_out=w, out_f32=out32,
-                       path=path, deterministic=args.deterministic,
-                       cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs])
+    pairs = {"auto": 0, "off": 1, "on": 2}[args.pairs]
+    if fp8 is not None:
+        api.moe_forward_fp8(s, inp.x, inp.logits, fp8_weights(api, fp8), inp.scale, out, ws,
+                            ids_out=ids, w_out=w, out_f32=out32, path=path,
+                            deterministic=args.deterministic, cta_pairs=pairs)
+    else:
+        api.moe_forward_ex(s, inp.x, inp.logits, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                           inp.w2_sh, out, ws, ids_out=ids, w_out=w, out_f32=out32,
+                           path=path, deterministic=args.deterministic, cta_pairs=pairs)
     cap = api.moe_layout_capacity(s)
     G = shp.E + shp.n_shared
     lay = (torch.empty(G + 1, dtype=torch.int32, device=dev),
@@ -345,8 +368,14 @@ def gpu_result(api, inp, s, path, args):
             "layout": tuple(t.cpu().numpy() for t in lay)}
 
 
+def fp8_weights(api, fp):
+    """moe_fp8_experts of an inputs.FP8Experts held on the device."""
+    return api.fp8_experts(fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
+                           fp.sh2_q, fp.sh2_s)
+
+
 def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
-                max_over_ranks, sample_clocks_gpu=None):
+                max_over_ranks, sample_clocks_gpu=None, fp8=None):
     """Device time of K steps of one workload.  By default the K steps are
     captured once into a CUDA graph and the timed region is one replay of
     it, so that host launch overhead does not pace small batches (the
@@ -362,12 +391,20 @@ def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
     shp = inp.shape
     dev = inp.x.device
 
+    w8 = fp8_weights(api, fp8) if fp8 is not None else None
+
     def step(events=None):
+        pairs = {"auto": 0, "off": 1, "on": 2}[args.pairs]
+        if w8 is not None:
+            api.moe_forward_fp8(s, inp.x, inp.logits if router is None else None, w8,
+                                inp.scale, out, ws, events=events, path=path,
+                                deterministic=args.deterministic, cta_pairs=pairs,
+                                router=router)
+            return
         api.moe_forward_ex(s, inp.x, inp.logits if router is None else None, inp.w13,
                            inp.w2, inp.scale, inp.w13_sh, inp.w2_sh, out, ws,
                            events=events, path=path, deterministic=args.deterministic,
-                           cta_pairs={"auto": 0, "off": 1, "on": 2}[args.pairs],
-                           router=router)
+                           cta_pairs=pairs, router=router)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -377,7 +414,7 @@ def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
         raise RuntimeError(f"device error during warm-up: {status}")
 
     touched = touched_experts(api, s, inp)
-    weight_set = touched * 3.0 * shp.H * shp.I * 2
+    weight_set = touched * 3.0 * shp.H * shp.I * (1 if fp8 is not None else 2)
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = None
     if weight_set < 4 * l2_bytes:
@@ -482,7 +519,7 @@ def w13_kernel_name(decode: bool, T: int) -> str:
     return "decode_w13_kernel (w13 + act)"
 
 
-def roofline_of(args, shp, m, decode, peaks, peak_src, config_name):
+def roofline_of(args, shp, m, decode, peaks, peak_src, config_name, fp8=False):
     """Roofline of the dominant kernel, the w13 product with the fused
     activation (2/3 of the layer's FLOPs and of its weight bytes), and the
     whole layer's fraction.  FLOPs count real rows only, bytes count each
@@ -492,25 +529,33 @@ def roofline_of(args, shp, m, decode, peaks, peak_src, config_name):
     touched = m["touched"]
     w13_ms = m["stage_ms"][3]
     rows = shp.T * shp.k + shp.T * shp.n_shared
-    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    # FP8: one byte per weight, and the e4m3 tensor peak at the nominal 2x of
+    # the measured bf16 figure
+    wbytes = 1 if fp8 else 2
+    tpeak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+    ridge = tpeak * 1e12 / (float(peaks["hbm_gbs"]) * 1e9) * (wbytes / 2.0)
     if rows / max(touched, 1) < ridge:
-        achieved = touched * (2.0 * shp.I * shp.H * 2) / (w13_ms / 1e3) / 1e9
+        achieved = touched * (2.0 * shp.I * shp.H * wbytes) / (w13_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         return {"bound": "hbm", "kernel": w13_kernel_name(decode, shp.T),
                 "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": traffic_for(("decode.cu" if shp.T <= 8 else "decode_tc.cu")
-                                       if decode else "gemm_tc.cu",
-                                       config_name, args.shape),
+                "traffic": None if fp8 else
+                traffic_for(("decode.cu" if shp.T <= 8 else "decode_tc.cu")
+                            if decode else "gemm_tc.cu", config_name, args.shape),
                 "layer_frac": m["weight_set"] / (m["ms_per_step"] / 1e3) / 1e9 / peak,
                 "touched_experts": touched}
     w13_flops = 2.0 * shp.T * (shp.k * shp.I + shp.n_shared * shp.I_shared) * shp.H * 2
     achieved = w13_flops / (w13_ms / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    return {"bound": "tensor", "kernel": w13_kernel_name(decode, shp.T),
+    peak = tpeak
+    return {"bound": "tensor",
+            "kernel": ("grouped_gemm_kernel<0, F8> (e4m3 w13 + activation)" if fp8
+                       else w13_kernel_name(decode, shp.T)),
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
-            "traffic": traffic_for("gemm_tc.cu", config_name, args.shape),
+            "frac": achieved / peak,
+            "peak_source": (f"{peak_src} bf16_tflops (burst) x 2, the nominal e4m3:bf16 "
+                            "ratio" if fp8 else f"{peak_src} bf16_tflops (burst)"),
+            "traffic": None if fp8 else traffic_for("gemm_tc.cu", config_name, args.shape),
             "layer_frac": shp.flops() / (m["ms_per_step"] / 1e3) / 1e12 / peak}
 
 
@@ -521,7 +566,7 @@ def launches_per_step(decode: bool, router: bool) -> int:
 
 
 def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
-            flush=None):
+            flush=None, fp8=None):
     """Same metric through the C ABI with every step's token inputs copied
     from pinned host memory and its output copied back, inside the timed
     region.
@@ -538,6 +583,15 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
     import torch
     shp = inp.shape
     dev = inp.x.device
+    w8 = fp8_weights(api, fp8) if fp8 is not None else None
+
+    def forward(x_d, z_d, o_d, **kw):
+        if w8 is not None:
+            api.moe_forward_fp8(s, x_d, z_d, w8, inp.scale, o_d, ws, **kw)
+        else:
+            api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
+                            inp.w2_sh, o_d, ws, **kw)
+
     x_h = inp.x.cpu().pin_memory()
     z_h = inp.logits.cpu().pin_memory()
     h2d = x_h.numel() * x_h.element_size() + z_h.numel() * z_h.element_size()
@@ -550,8 +604,7 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
         def e2e_step():
             x_d.copy_(x_h, non_blocking=True)
             z_d.copy_(z_h, non_blocking=True)
-            api.moe_forward(s, x_d, z_d, inp.w13, inp.w2, inp.scale, inp.w13_sh,
-                            inp.w2_sh, out, ws)
+            forward(x_d, z_d, out)
             out_h.copy_(out, non_blocking=True)
 
         for _ in range(max(args.warmup, 3)):
@@ -600,8 +653,7 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
                 stream.wait_event(ev_in[i])
                 if i >= 2:
                     stream.wait_event(ev_out[i - 2])  # output buffer b copied out
-                api.moe_forward(s, x_d[b], z_d[b], inp.w13, inp.w2, inp.scale,
-                                inp.w13_sh, inp.w2_sh, o_d[b], ws, stream=stream)
+                forward(x_d[b], z_d[b], o_d[b], stream=stream)
                 ev_c[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_c[i])
@@ -623,21 +675,28 @@ def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
 def other_config_entry(args, api, inputs, name, dev, stream, peaks, peak_src):
     """One line of the ``configs`` key: the same device-timed measurement,
     roofline and CPU-baseline leg (with its parity comparison) for another
-    workload, one GPU."""
+    workload, one GPU.  A name ending in +fp8 runs that workload with FP8
+    experts (moe_forward_fp8)."""
     import torch
-    inp = inputs.make_inputs(name, seed=args.seed, device=dev)
+    fp8 = name.endswith("+fp8")
+    base_name = name[:-4] if fp8 else name
+    inp = inputs.make_inputs(base_name, seed=args.seed, device=dev)
     shp = inp.shape
+    fpw = inputs.fp8_experts(shp, seed=args.seed + 1, device=dev) if fp8 else None
+    if fp8:  # the bf16 weights are not used
+        inp.w13 = inp.w2 = inp.w13_sh = inp.w2_sh = None
     s = api.shape_from(shp)
-    ws = api.alloc_workspace(s, dev)
+    ws = api.alloc_workspace_fp8(s, dev) if fp8 else api.alloc_workspace(s, dev)
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
     path = api.PATH_AUTO
-    decode = shp.T <= api.DECODE_MAX_T
+    decode = shp.T <= api.DECODE_MAX_T and not fp8
     m = timed_steps(args, api, inp, s, ws, out, stream, path, None, lambda: None,
-                    lambda v: v, sample_clocks_gpu=dev.index or 0)
-    roof = roofline_of(args, shp, m, decode, peaks, peak_src, name)
-    gpu = gpu_result(api, inp, s, path, args)
-    base, parity = cpu_baseline_leg(inp, gpu, budget_s=1.5)
-    entry = {"workload": workload_name(name, shp),
+                    lambda v: v, sample_clocks_gpu=dev.index or 0, fp8=fpw)
+    roof = roofline_of(args, shp, m, decode, peaks, peak_src, name, fp8=fp8)
+    gpu = gpu_result(api, inp, s, path, args, fp8=fpw)
+    base, parity = cpu_baseline_leg(inp, gpu, budget_s=1.5, fp8=fpw)
+    entry = {"workload": workload_name(base_name, shp) +
+                         (" with FP8 (e4m3) experts, per-row scales" if fp8 else ""),
              "path": "decode" if decode else "prefill",
              "ms_per_step": m["ms_per_step"],
              "value": shp.T / (m["ms_per_step"] / 1e3), "unit": UNIT,
@@ -647,13 +706,14 @@ def other_config_entry(args, api, inputs, name, dev, stream, peaks, peak_src):
                    else "weights far larger than L2",
              "parity": parity, "cpu_baseline": base, "clocks": m["clocks"],
              "gpu_launches": launches_per_step(decode, False) * args.steps}
-    del inp, ws, out
+    del inp, ws, out, fpw
     torch.cuda.empty_cache()
     return entry
 
 
 OTHER_CONFIGS = ("many_small_prefill", "skewed_shared_prefill", "decode_t1",
-                 "decode_t4", "decode_t16", "decode_t64", "decode_t256")
+                 "decode_t4", "decode_t16", "decode_t64", "decode_t256",
+                 "mixtral_prefill+fp8", "many_small_prefill+fp8")
 
 
 def run_ours(args):
@@ -672,7 +732,12 @@ def run_ours(args):
     inp = make_workload(args, dev, args.seed + rank)
     shp = inp.shape
     s = api.shape_from(shp)
-    ws = api.alloc_workspace(s, dev)
+    fpw = inputs.fp8_experts(shp, seed=args.seed + 1 + rank, device=dev) \
+        if args.fp8 else None
+    if fpw is not None:  # the bf16 weights are not used
+        inp.w13 = inp.w2 = inp.w13_sh = inp.w2_sh = None
+        torch.cuda.empty_cache()
+    ws = api.alloc_workspace_fp8(s, dev) if args.fp8 else api.alloc_workspace(s, dev)
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
     torch.cuda.synchronize()
     # all work on a side stream (CUDA graphs are captured off the default one)
@@ -683,6 +748,9 @@ def run_ours(args):
             "decode": api.PATH_DECODE}[args.path]
     decode = path == api.PATH_DECODE or (path == api.PATH_AUTO
                                          and shp.T <= api.DECODE_MAX_T)
+    if args.fp8 and decode:
+        raise SystemExit("--fp8: FP8 experts run on the prefill path only "
+                         "(use --path prefill)")
 
     router = None
     if args.router:
@@ -695,7 +763,7 @@ def run_ours(args):
 
     max_over_ranks = max_over_ranks_fn(world, dev)
     m = timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
-                    max_over_ranks, sample_clocks_gpu=local)
+                    max_over_ranks, sample_clocks_gpu=local, fp8=fpw)
     ms_per_step, stage_ms = m["ms_per_step"], m["stage_ms"]
     flush = m["flush"]
 
@@ -728,28 +796,32 @@ def run_ours(args):
 
     # ---- end to end: pinned host inputs in, host output back, every step
     e2e_ms, h2d, d2h = run_e2e(
-        args, api, inp, s, ws, out, stream, barrier, max_over_ranks, flush) \
+        args, api, inp, s, ws, out, stream, barrier, max_over_ranks, flush, fp8=fpw) \
         if not (args.profile or args.router) else (None, 0, 0)
 
     result = None
     if rank == 0:
         peaks, peak_src = load_peaks()
         value = whole_job_rate(shp.T, world, ms_per_step)
-        roof = roofline_of(args, shp, m, decode, peaks, peak_src, args.config)
+        roof = roofline_of(args, shp, m, decode, peaks, peak_src, args.config,
+                           fp8=args.fp8)
         layer_tflops = shp.flops() / (ms_per_step / 1e3) / 1e12
         cpu = parity = None
         if world == 1 and not args.profile:
-            gpu = gpu_result(api, inp, s, path, args)
-            cpu, parity = cpu_baseline_leg(inp, gpu, budget_s=12.0)
+            gpu = gpu_result(api, inp, s, path, args, fp8=fpw)
+            cpu, parity = cpu_baseline_leg(inp, gpu, budget_s=12.0, fp8=fpw)
         weight_set = m["weight_set"]
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 experts, bf16 activations" if args.fp8 else "bf16",
             "data": "synthetic: seeded N(0,1) tokens, N(0,0.02) bf16 random-init "
                     "expert weights, fp32 router logits with a 1e-3 top-k margin",
-            "config": {"workload": workload_name(args.config, shp),
+            "config": {"workload": workload_name(args.config, shp)
+                                   + (" with FP8 (e4m3) experts, per-row scales"
+                                      if args.fp8 else ""),
                        "path": "decode" if decode else "prefill",
                        "combine": "fixed-order" if (decode or args.deterministic)
                                   else "fp32 reductions",
@@ -786,10 +858,11 @@ def run_ours(args):
             result["router"] = router_stats
             result["config"]["workload"] += " + router (from hidden states)"
         if world == 1 and not args.profile and not args.router and not args.shape \
-                and args.config == "mixtral_prefill" and not args.headline_only:
+                and args.config == "mixtral_prefill" and not args.headline_only \
+                and not args.fp8:
             # the other workloads of the benchmark, one GPU each, after the
             # headline: device time, roofline, parity against the oracle
-            del inp, ws, out
+            del inp, ws, out, fpw
             torch.cuda.empty_cache()
             result["configs"] = {
                 name: other_config_entry(args, api, inputs, name, dev, stream, peaks,
