@@ -265,7 +265,7 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
     rng = np.random.default_rng(seed)
     per_round = min(cores, T)
     done, elapsed, rounds = 0, 0.0, 0
-    toks, outs = [], []
+    toks, outs, slacks = [], [], []
     while rounds < max_rounds and (elapsed < budget_s or rounds == 0):
         tok = np.sort(rng.choice(T, per_round, replace=False))
         t0 = time.perf_counter()
@@ -274,10 +274,13 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
                                      scale=host["scale"], w13_sh=sh13, w2_sh=sh2,
                                      tokens=tok, nthreads=per_round)
         else:
-            o, _, _ = oracle.forward_fp8(xu, host["logits"], *fp8, shp.k, shp.act,
-                                         scale=host["scale"], sh13_q=fp8_sh[0],
-                                         sh13_s=fp8_sh[1], sh2_q=fp8_sh[2],
-                                         sh2_s=fp8_sh[3], tokens=tok, nthreads=per_round)
+            # with the validity slack of the intermediate's quantisation
+            o, _, _, sl = oracle.forward_fp8(xu, host["logits"], *fp8, shp.k, shp.act,
+                                             scale=host["scale"], sh13_q=fp8_sh[0],
+                                             sh13_s=fp8_sh[1], sh2_q=fp8_sh[2],
+                                             sh2_s=fp8_sh[3], tokens=tok,
+                                             nthreads=per_round, with_slack=True)
+            slacks.append(sl)
         elapsed += time.perf_counter() - t0
         toks.append(tok)
         outs.append(o)
@@ -292,10 +295,11 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
 
     tok = np.concatenate(toks)
     want = np.concatenate(outs)
+    slack = np.concatenate(slacks) if slacks else 0.0
     got32 = gpu["out_f32"][tok].astype(np.float64)
     gotbf = gpu["out"][tok].astype(np.float64)
     rms = float(np.sqrt(np.mean(want ** 2)))
-    bound = 2e-2 * rms + 2.0 ** -8 * np.abs(want)
+    bound = 2e-2 * rms + 2.0 ** -8 * np.abs(want) + slack
     ids_ref, w_ref = oracle.route(host["logits"], shp.k, scale=host["scale"])
     lay = oracle.layout(ids_ref, shp.E, shp.n_shared, 128)
     lay_bad = sum(int((np.asarray(g) != np.asarray(w)).sum())
@@ -311,9 +315,16 @@ def cpu_baseline_leg(inp, gpu, budget_s: float, max_rounds: int = 64, seed: int 
         "layout_entries_mismatched": lay_bad,
         "tolerance": "out_f32 max|err| <= 2e-2 x RMS(oracle); bf16 within "
                      "2e-2 x RMS + 2^-8 |oracle|; ids and layout bit-exact; "
-                     "weights 1e-6 relative",
+                     "weights 1e-6 relative"
+                     + ("; FP8: both output bounds + the oracle's validity slack "
+                        "of the intermediate's quantisation decisions"
+                        if fp8 is not None else ""),
     }
-    parity["pass"] = (parity["out_f32_max_err_over_rms"] <= 2e-2
+    f32_ok = bool((np.abs(got32 - want) <= 2e-2 * rms + slack).all())
+    if fp8 is not None:
+        parity["out_f32_within_bound_with_slack"] = f32_ok
+        parity["max_slack_over_rms"] = float(np.max(slack) / rms)
+    parity["pass"] = (f32_ok
                       and parity["bf16_within_bound"]
                       and parity["ids_mismatched"] == 0
                       and parity["layout_entries_mismatched"] == 0

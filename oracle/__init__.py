@@ -78,7 +78,8 @@ def _load():
         lib.oracle_e4m3_codes.argtypes = [i64, P, P]
         lib.oracle_quantize_rows_e4m3.argtypes = [i64, i32, P, P, P]
         lib.oracle_forward_fp8.argtypes = [i64, i32, i32, i32, i32, i32, i32, P, P, P,
-                                           P, P, P, P, P, P, P, P, P, i64, i32, P, P, P]
+                                           P, P, P, P, P, P, P, P, P, i64, i32, P, P, P,
+                                           P]
         for f in (lib.oracle_act, lib.oracle_route, lib.oracle_layout,
                   lib.oracle_expert_rows, lib.oracle_forward,
                   lib.oracle_router_logits, lib.oracle_route_ex,
@@ -306,10 +307,13 @@ def quantize_rows_e4m3(src):
 
 def forward_fp8(x, logits, w13_q, w13_s, w2_q, w2_s, k: int, act_kind: int, scale=None,
                 sh13_q=None, sh13_s=None, sh2_q=None, sh2_s=None, tokens=None,
-                nthreads: int = 0):
-    """The layer with FP8 experts in fp64 -> (out [n,H] float64, ids, w).
-    w13_q [E,2I,H] / w2_q [E,H,I] e4m3 codes with per-row fp32 scales
-    w13_s [E,2I] / w2_s [E,H]; shared experts likewise."""
+                nthreads: int = 0, with_slack: bool = False):
+    """The layer with FP8 experts in fp64 -> (out [n,H] float64, ids, w),
+    and with ``with_slack`` the validity slack [n,H] of every output element
+    as a fourth result: how far the admissible other decisions of the
+    intermediate's quantisation (bf16 rounding, amax, codes) of an fp32
+    implementation can move it.  w13_q [E,2I,H] / w2_q [E,H,I] e4m3 codes with
+    per-row fp32 scales w13_s [E,2I] / w2_s [E,H]; shared experts likewise."""
     xu = _u16(x)
     z = _f32(logits)
     T, H = xu.shape
@@ -325,9 +329,10 @@ def forward_fp8(x, logits, w13_q, w13_s, w2_q, w2_s, k: int, act_kind: int, scal
     out = np.empty((n, H), np.float64)
     ids = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
+    slack = np.empty((n, H), np.float64) if with_slack else None
     _check(_load().oracle_forward_fp8(T, H, E, k, I, act_kind, S, _ptr(xu), _ptr(z),
                                       _ptr(_f32(scale)), _ptr(c13), _ptr(s13), _ptr(c2),
                                       _ptr(s2), _ptr(h13), _ptr(hs13), _ptr(h2),
                                       _ptr(hs2), _ptr(tok), n, nthreads, _ptr(out),
-                                      _ptr(ids), _ptr(w)), "forward_fp8")
-    return out, ids, w
+                                      _ptr(ids), _ptr(w), _ptr(slack)), "forward_fp8")
+    return (out, ids, w, slack) if with_slack else (out, ids, w)

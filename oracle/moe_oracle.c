@@ -796,24 +796,160 @@ int oracle_quantize_rows_e4m3(int64_t rows, int cols, const uint16_t* src,
   return OK;
 }
 
+/*
+ * Validity slack of the FP8 layer.  Quantising the intermediate takes
+ * integer decisions (its bf16 rounding, the row's amax and with it the
+ * scale, each e4m3 code) from a row that an implementation computes in
+ * fp32: a value within that arithmetic's error of a rounding boundary can
+ * go either way, and both outcomes are the layer's result.  The decisions
+ * taken here are those of the exact row; the slack of an output element is
+ * the most the other admissible decisions can move it:
+ *   - an fp32 implementation's g (and u) lies within
+ *       dg = 2^-20 sum_h |x'_h w1'_ih| + 2^-22 |g|
+ *     of the exact value (16 fp32 ulps of the sum of magnitudes for the
+ *     accumulation, and the scale products), and its a = Act(g) u within
+ *       da = dAct (|u| + du) + |Act(g)| du + 2^-21 |a|,
+ *     dAct the largest change of Act over [g - dg, g + dg];
+ *   - an element's admissible bf16 values are those of [a - da, a + da];
+ *     the row's admissible amax values follow, and with them its scales;
+ *   - under each admissible scale, d_i = the most an admissible bf16 value
+ *     of element i moves its dequantised value, and the slack of y_h adds
+ *     weight * (sum_i d_i |w2'_hi| + the largest |change of y_h| that
+ *     another admissible scale makes with the exact row's bf16 values).
+ */
+typedef struct {
+  double* g1;   /* sum of |terms| of g, then da */
+  double* u1;   /* sum of |terms| of u */
+  double* lo;   /* admissible bf16 values of each element */
+  double* hi;
+  double* d;    /* largest change of each dequantised element */
+} fp8_slack_scratch;
+
+static double act_spread(int act, double g, double dg) {
+  const double f = act_fn(act, g);
+  const double a = fabs(act_fn(act, g - dg) - f), b = fabs(act_fn(act, g + dg) - f);
+  return a > b ? a : b;
+}
+
+/* the next bf16 value above v >= 0 (8 significant bits; 2^-133 after 0) */
+static double bf16_next_up(double v) {
+  if (v <= 0.0) return ldexp(1.0, -133);
+  int ex;
+  frexp(v, &ex);  /* v in [2^(ex-1), 2^ex) */
+  const double ulp = ldexp(1.0, ex - 8 < -133 ? -133 : ex - 8);
+  return v + ulp;
+}
+
+/* dequantised value of v (a bf16 value held as a float) with scale s */
+static double deq(float v, float s) { return e4m3_value(e4m3_code(v / s)) * (double)s; }
+
+static void fp8_row_slack(int H, int I, int act, const double* gv, const double* uv,
+                          const double* a_exact, const float* af, float s,
+                          const uint8_t* w2c, const float* w2s, double weight,
+                          fp8_slack_scratch* sc, double* slack) {
+  double amax_lo = 0.0, amax_hi = 0.0;
+  for (int i = 0; i < I; ++i) {
+    const double dg = ldexp(sc->g1[i], -20) + ldexp(fabs(gv[i]), -22);
+    const double du = ldexp(sc->u1[i], -20) + ldexp(fabs(uv[i]), -22);
+    const double fa = act_fn(act, gv[i]);
+    const double da = act_spread(act, gv[i], dg) * (fabs(uv[i]) + du) + fabs(fa) * du +
+                      ldexp(fabs(a_exact[i]), -21);
+    const double b0 = round_to_bf16(a_exact[i] - da), b1 = round_to_bf16(a_exact[i] + da);
+    sc->lo[i] = b0;
+    sc->hi[i] = b1;
+    /* |values| the element can take span [min |b|, max |b|] over [b0, b1] */
+    const double mn = (b0 <= 0.0 && b1 >= 0.0) ? 0.0 : fmin(fabs(b0), fabs(b1));
+    const double mx = fmax(fabs(b0), fabs(b1));
+    if (mn > amax_lo) amax_lo = mn;
+    if (mx > amax_hi) amax_hi = mx;
+  }
+  /* admissible scales: every bf16 amax in [amax_lo, amax_hi] (a few values
+   * at most; the list is cut at 16) */
+  float scales[16];
+  int ns = 0;
+  for (double m = amax_lo; m <= amax_hi && ns < 16; m = bf16_next_up(m)) {
+    const float mf = (float)m;
+    scales[ns++] = mf > 0.0f ? mf / 448.0f : 1.0f;
+  }
+  /* element decisions: for each admissible scale, the most an admissible
+   * bf16 value of the element moves its dequantised value (monotone in the
+   * bf16 value, so the ends of [lo, hi] bound it) */
+  int any = 0;
+  for (int i = 0; i < I; ++i) {
+    sc->d[i] = 0.0;
+    if (sc->lo[i] == sc->hi[i]) continue;
+    for (int q = 0; q < ns; ++q) {
+      const double mid = deq(af[i], scales[q]);
+      const double c0 = fabs(deq((float)sc->lo[i], scales[q]) - mid);
+      const double c1 = fabs(deq((float)sc->hi[i], scales[q]) - mid);
+      if (c0 > sc->d[i]) sc->d[i] = c0;
+      if (c1 > sc->d[i]) sc->d[i] = c1;
+    }
+    if (sc->d[i] > 0.0) any = 1;
+  }
+  /* scale decisions: the row's change under every other admissible scale,
+   * computed exactly (every element moves with the scale) */
+  double* dq = NULL;
+  int nalt = 0;
+  if (ns > 1) {
+    dq = (double*)malloc(sizeof(double) * (size_t)ns * I);
+    for (int q = 0; dq && q < ns; ++q) {
+      if (scales[q] == s) continue;
+      for (int i = 0; i < I; ++i) dq[(size_t)nalt * I + i] = deq(af[i], scales[q]) - deq(af[i], s);
+      ++nalt;
+    }
+  }
+  if (!any && nalt == 0) {
+    free(dq);
+    return;
+  }
+  for (int h = 0; h < H; ++h) {
+    const uint8_t* r2 = w2c + (int64_t)h * I;
+    double acc = 0.0, worst = 0.0;
+    for (int i = 0; any && i < I; ++i)
+      if (sc->d[i] > 0.0) acc += sc->d[i] * fabs(e4m3_value(r2[i]) * (double)w2s[h]);
+    for (int q = 0; q < nalt; ++q) {
+      double y = 0.0;
+      for (int i = 0; i < I; ++i) y += dq[(size_t)q * I + i] * (e4m3_value(r2[i]) * (double)w2s[h]);
+      if (fabs(y) > worst) worst = fabs(y);
+    }
+    slack[h] += fabs(weight) * (acc + worst);
+  }
+  free(dq);
+}
+
 /* one expert (or shared expert) on one quantised token row, added to y
- * with the given weight */
+ * with the given weight (and its validity slack to ``slack``, if given) */
 static void ffn_row_fp8(int H, int I, int act, const double* xq, const uint8_t* w13c,
                         const float* w13s, const uint8_t* w2c, const float* w2s,
-                        double weight, double* a, float* af, uint8_t* ac, double* y) {
+                        double weight, double* a, float* af, uint8_t* ac, double* y,
+                        double* gv, double* uv, fp8_slack_scratch* sc, double* slack) {
   for (int i = 0; i < I; ++i) {
     const uint8_t* r1 = w13c + (int64_t)i * H;
     const uint8_t* r3 = w13c + (int64_t)(I + i) * H;
-    double g = 0.0, u = 0.0;
+    double g = 0.0, u = 0.0, g1 = 0.0, u1 = 0.0;
     for (int h = 0; h < H; ++h) {
-      g += xq[h] * (e4m3_value(r1[h]) * (double)w13s[i]);
-      u += xq[h] * (e4m3_value(r3[h]) * (double)w13s[I + i]);
+      const double tg = xq[h] * (e4m3_value(r1[h]) * (double)w13s[i]);
+      const double tu = xq[h] * (e4m3_value(r3[h]) * (double)w13s[I + i]);
+      g += tg;
+      u += tu;
+      if (slack) {
+        g1 += fabs(tg);
+        u1 += fabs(tu);
+      }
     }
     a[i] = act_fn(act, g) * u;
+    if (slack) {
+      gv[i] = g;
+      uv[i] = u;
+      sc->g1[i] = g1;
+      sc->u1[i] = u1;
+    }
   }
   /* the intermediate row in bf16, quantised by the steps of quantize_row */
   for (int i = 0; i < I; ++i) af[i] = (float)round_to_bf16(a[i]);
   const float s = quantize_row(I, af, ac);
+  if (slack) fp8_row_slack(H, I, act, gv, uv, a, af, s, w2c, w2s, weight, sc, slack);
   for (int i = 0; i < I; ++i) a[i] = e4m3_value(ac[i]) * (double)s;
   for (int h = 0; h < H; ++h) {
     const uint8_t* r2 = w2c + (int64_t)h * I;
@@ -833,6 +969,7 @@ typedef struct {
   const double* w;
   const int64_t* tokens;
   double* out;
+  double* slack;
 } fwd8_ctx;
 
 static void fwd8_worker(void* p, int64_t b, int64_t e) {
@@ -844,10 +981,15 @@ static void fwd8_worker(void* p, int64_t b, int64_t e) {
   double* a = (double*)malloc(sizeof(double) * I);
   float* af = (float*)malloc(sizeof(float) * I);
   uint8_t* ac = (uint8_t*)malloc(I);
+  double* sbuf = (double*)malloc(sizeof(double) * 7 * I);  /* g, u and the slack scratch */
+  fp8_slack_scratch sc = {sbuf + 2 * I, sbuf + 3 * I, sbuf + 4 * I, sbuf + 5 * I,
+                          sbuf + 6 * I};
   for (int64_t r = b; r < e; ++r) {
     const int64_t t = c->tokens ? c->tokens[r] : r;
     double* y = c->out + r * H;
+    double* sl = c->slack ? c->slack + r * H : NULL;
     for (int h = 0; h < H; ++h) y[h] = 0.0;
+    for (int h = 0; sl && h < H; ++h) sl[h] = 0.0;
     /* the token row, quantised once */
     for (int h = 0; h < H; ++h) xf[h] = (float)bf16_to_double(c->x[t * H + h]);
     const float sx = quantize_row(H, xf, xc);
@@ -856,21 +998,23 @@ static void fwd8_worker(void* p, int64_t b, int64_t e) {
       const int64_t ex = c->ids[t * c->k + j];
       ffn_row_fp8(H, I, c->act, xq, c->w13c + ex * 2 * (int64_t)I * H,
                   c->w13s + ex * 2 * (int64_t)I, c->w2c + ex * (int64_t)H * I,
-                  c->w2s + ex * (int64_t)H, c->w[t * c->k + j], a, af, ac, y);
+                  c->w2s + ex * (int64_t)H, c->w[t * c->k + j], a, af, ac, y, sbuf,
+                  sbuf + I, &sc, sl);
     }
     for (int s = 0; s < c->S; ++s)
       ffn_row_fp8(H, I, c->act, xq, c->sh13c + (int64_t)s * 2 * I * H,
                   c->sh13s + (int64_t)s * 2 * I, c->sh2c + (int64_t)s * H * I,
-                  c->sh2s + (int64_t)s * H, 1.0, a, af, ac, y);
+                  c->sh2s + (int64_t)s * H, 1.0, a, af, ac, y, sbuf, sbuf + I, &sc, sl);
   }
-  free(xf); free(xc); free(xq); free(a); free(af); free(ac);
+  free(xf); free(xc); free(xq); free(a); free(af); free(ac); free(sbuf);
 }
 
 /*
  * The layer with FP8 experts, for the tokens listed in ``tokens`` (NULL =
  * all T): routing as oracle_forward; w13 codes [E,2I,H] with scales [E,2I]
  * (gate rows first), w2 codes [E,H,I] with scales [E,H]; shared experts
- * likewise ([S,...], the same I).
+ * likewise ([S,...], the same I).  ``slack`` (NULL: not computed) receives
+ * the validity slack of every output element (see fp8_row_slack).
  */
 int oracle_forward_fp8(int64_t T, int H, int E, int k, int I, int act, int S,
                        const uint16_t* x, const float* logits, const float* scale,
@@ -878,7 +1022,7 @@ int oracle_forward_fp8(int64_t T, int H, int E, int k, int I, int act, int S,
                        const float* w2s, const uint8_t* sh13c, const float* sh13s,
                        const uint8_t* sh2c, const float* sh2s, const int64_t* tokens,
                        int64_t n_tokens, int nthreads, double* out, int32_t* ids_out,
-                       double* w_out) {
+                       double* w_out, double* slack) {
   if (T < 0 || H < 1 || I < 1 || S < 0 || !x || !w13c || !w13s || !w2c || !w2s ||
       (S > 0 && (!sh13c || !sh13s || !sh2c || !sh2s)))
     return EINVAL_ARG;
@@ -894,7 +1038,7 @@ int oracle_forward_fp8(int64_t T, int H, int E, int k, int I, int act, int S,
   }
   if (rc == OK) {
     fwd8_ctx c = {T, H, E, k, I, act, S, x, w13c, w2c, sh13c, sh2c,
-                  w13s, w2s, sh13s, sh2s, ids, w, tokens, out};
+                  w13s, w2s, sh13s, sh2s, ids, w, tokens, out, slack};
     parallel_for(n_tokens, nthreads, fwd8_worker, &c);
   }
   if (!ids_out) free(ids);

@@ -54,22 +54,28 @@ def oracle_forward(inp: inputs.MoEInputs, tokens=None, route=None):
 
 
 def assert_out_close(got_t: torch.Tensor, want: np.ndarray, what="",
-                     bf16: torch.Tensor = None):
+                     bf16: torch.Tensor = None, slack: np.ndarray = None):
     """Literal bound on the layer output before its final bf16 rounding:
     max|got - want| <= OUT_TOL * RMS(want).  With ``bf16`` (the rounded
     output tensor) that tensor is bounded too, element by element, by
     OUT_TOL * RMS(want) + 2^-8 |want|: the bound plus the largest error a
-    rounding to 8 significant bits can add."""
+    rounding to 8 significant bits can add.  ``slack`` (the FP8 layer's
+    validity slack from the oracle, per element) widens both bounds by how
+    far the admissible other quantisation decisions can move each element."""
     got = got_t.float().cpu().numpy().astype(np.float64)
     assert got.shape == want.shape, (got.shape, want.shape)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     rms = float(np.sqrt(np.mean(want ** 2)))
+    sl = 0.0 if slack is None else slack
     err = float(np.abs(got - want).max())
-    assert err <= OUT_TOL * rms, f"{what}: max|err| {err:.3e} > {OUT_TOL} x RMS {rms:.3e}"
+    excess = np.abs(got - want) - (OUT_TOL * rms + sl)
+    assert (excess <= 0).all(), \
+        f"{what}: max|err| {err:.3e} > {OUT_TOL} x RMS {rms:.3e}" + \
+        ("" if slack is None else f" + slack (by {excess.max():.3e})")
     if bf16 is not None:
         b = bf16.float().cpu().numpy().astype(np.float64)
         assert b.shape == want.shape
-        excess = np.abs(b - want) - (OUT_TOL * rms + 2.0 ** -8 * np.abs(want))
+        excess = np.abs(b - want) - (OUT_TOL * rms + 2.0 ** -8 * np.abs(want) + sl)
         assert (excess <= 0).all(), \
             f"{what}: bf16 output exceeds the bound by {excess.max():.3e}"
     return err / rms

@@ -7,8 +7,12 @@ weight; the reading is one fp32 scale per output row, activations and the
 bf16 intermediate quantised per row at run time.  Bars: the row quantiser's
 codes and scales bit-exact (IEEE fp32 steps on both sides); routing ids
 bit-exact and gate weights within 1e-6 relative; the layer output within
-2e-2 x RMS(oracle) on the fp32 result, the bf16 output its exact rounding
-and within 2e-2 x RMS + 2^-8 |oracle|.
+2e-2 x RMS(oracle) + slack on the fp32 result, the bf16 output its exact
+rounding and within 2e-2 x RMS + 2^-8 |oracle| + slack.  The slack (from
+the oracle, per element) is how far the quantisation decisions on the
+intermediate that an fp32 computation of it may take either way (a value
+within its rounding error of a bf16 or e4m3 boundary, or of the row's amax)
+can move the element; it is zero where no such decision exists.
 """
 import numpy as np
 import pytest
@@ -73,10 +77,11 @@ def _gpu_fp8(api, inp, fp, det=False, pairs=0, path=0):
 
 
 def _oracle_fp8(inp, fp, tokens=None):
+    """-> (out, ids, w, slack)"""
     return oracle.forward_fp8(inp.x, inp.logits, fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s,
                               k=inp.shape.k, act_kind=inp.shape.act, scale=inp.scale,
                               sh13_q=fp.sh13_q, sh13_s=fp.sh13_s, sh2_q=fp.sh2_q,
-                              sh2_s=fp.sh2_s, tokens=tokens)
+                              sh2_s=fp.sh2_s, tokens=tokens, with_slack=True)
 
 
 SHAPES = {
@@ -97,11 +102,11 @@ def test_forward_fp8_every_element(api, name, variant):
     shp = SHAPES[name]
     inp = inputs.make_inputs(shp, seed=4, scale="uniform")
     fp = inputs.fp8_experts(shp, seed=104)
-    want, ids_ref, w_ref = _oracle_fp8(inp, fp)
+    want, ids_ref, w_ref, slack = _oracle_fp8(inp, fp)
     det, pairs = VARIANTS[variant]
     out, out32, ids, w = _gpu_fp8(api, inp, fp, det=det, pairs=pairs)
     assert_routing_exact(ids, w, ids_ref, w_ref)
-    assert_out_close(out32, want, f"{name} fp8 ({variant})", bf16=out)
+    assert_out_close(out32, want, f"{name} fp8 ({variant})", bf16=out, slack=slack)
 
 
 def test_forward_fp8_refuses_the_decode_path(api):
@@ -142,7 +147,7 @@ def test_forward_fp8_full_size_many_small(api):
             if real.size:
                 tok.add(int(real[rng.integers(real.size)]) // shp.k)
     tok = np.array(sorted(tok), np.int64)
-    want, _, _ = _oracle_fp8(inp, fp, tokens=tok)
+    want, _, _, slack = _oracle_fp8(inp, fp, tokens=tok)
     sel = torch.from_numpy(tok).cuda()
     assert_out_close(out32[sel], want, f"many-small fp8, {len(tok)} tokens",
-                     bf16=out[sel])
+                     bf16=out[sel], slack=slack)

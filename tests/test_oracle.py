@@ -769,21 +769,25 @@ def test_quantize_rows_reconstruct_within_half_a_step():
     assert np.array_equal(s2[[0, 1, 2, 4, 5]], 8 * s[[0, 1, 2, 4, 5]])
 
 
-def _dense_fp8_torch(inp, fp, ids, w, act_kind):
-    """The FP8 layer restated with torch float64 ops and torch's e4m3 cast as
-    the quantiser: every expert on every token, then masked by the dispatch
-    weights (compute all, then discard)."""
-    def quant(v64):
-        v = v64.float()
+def _dense_fp8_torch(inp, fp, ids, w, act_kind, dtype=torch.float64):
+    """The FP8 layer restated with torch ops and torch's e4m3 cast as the
+    quantiser: every expert on every token, then masked by the dispatch
+    weights (compute all, then discard).  ``dtype`` float64: the exact layer;
+    float32: the intermediate computed the way an fp32 kernel does (fp32
+    products and activation, then bf16), so its quantisation decisions are
+    the ones an fp32 implementation takes."""
+    def quant(v):
+        v = v.float()
         amax = v.abs().amax(-1, keepdim=True)
         s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
         return (v / s).to(torch.float8_e4m3fn).double() * s.double()
 
     def ffn(xq, c13, s13, c2, s2):
         I = c2.shape[-1]
-        w13 = _fp8(c13).double() * torch.as_tensor(s13).double()[:, None]
+        w13 = (_fp8(c13).double() * torch.as_tensor(s13).double()[:, None]).to(dtype)
         w2 = _fp8(c2).double() * torch.as_tensor(s2).double()[:, None]
-        g, u = xq @ w13[:I].T, xq @ w13[I:].T
+        xd = xq.to(dtype)
+        g, u = xd @ w13[:I].T, xd @ w13[I:].T
         a = (F.silu(g) if act_kind == 0 else F.gelu(g, approximate="tanh")) * u
         return quant(a.to(torch.bfloat16).double()) @ w2.T  # h is bf16, then quantised
 
@@ -846,3 +850,51 @@ def test_forward_fp8_never_reads_unselected_experts():
     w2[unused] = 0x7F
     out2, _, _ = _fwd8(inp, fp, shp, w13_q=w13, w2_q=w2)
     assert np.array_equal(out2, out)
+
+
+# The validity slack: an fp32 computation of the intermediate takes the
+# quantisation decisions near a boundary either way.  These cases (seeds
+# chosen so that the fp32 restatement does flip a decision) check that it
+# differs from the oracle only where, and by no more than, the slack allows,
+# and that the slack does not hide a real mistake.
+_SLACK_CASES = [((256, 256, 8, 1, 128, 1), 7), ((128, 512, 8, 2, 256, 0), 4)]
+
+
+def _slack_case(dims, seed):
+    T, H, E, k, I, act = dims
+    shp = inputs.Shape(T=T, H=H, E=E, k=k, I=I, act=act)
+    inp = inputs.make_inputs(shp, seed=seed, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=seed + 50)
+    out, ids, w, slack = oracle.forward_fp8(inp.x, inp.logits, fp.w13_q, fp.w13_s, fp.w2_q,
+                                            fp.w2_s, k=k, act_kind=act, scale=inp.scale,
+                                            with_slack=True)
+    return shp, inp, fp, out, ids, w, slack
+
+
+@pytest.mark.parametrize("dims,seed", _SLACK_CASES)
+def test_forward_fp8_slack_explains_an_fp32_restatement(dims, seed):
+    shp, inp, fp, out, ids, w, slack = _slack_case(dims, seed)
+    got = _dense_fp8_torch(inp, fp, ids, w, shp.act, dtype=torch.float32)
+    rms = np.sqrt(np.mean(out ** 2))
+    err = np.abs(got - out)
+    assert (err > 1e-4 * rms).any(), "the case should contain a flipped decision"
+    # away from the flipped decisions the two agree to fp32 rounding
+    assert (err <= 1e-5 * rms + slack).all()
+    assert (slack >= 0).all() and slack.max() <= 0.25 * rms
+
+
+@pytest.mark.parametrize("dims,seed", _SLACK_CASES)
+def test_forward_fp8_slack_is_exact_zero_for_the_exact_decisions(dims, seed):
+    """The exact (float64) restatement takes the oracle's own decisions: it
+    matches without any slack."""
+    shp, inp, fp, out, ids, w, slack = _slack_case(dims, seed)
+    got = _dense_fp8_torch(inp, fp, ids, w, shp.act)
+    assert np.abs(got - out).max() <= 1e-10 * np.sqrt(np.mean(out ** 2))
+
+
+def test_forward_fp8_slack_does_not_hide_a_wrong_activation():
+    dims, seed = _SLACK_CASES[1]
+    shp, inp, fp, out, ids, w, slack = _slack_case(dims, seed)
+    wrong = _dense_fp8_torch(inp, fp, ids, w, 1 - shp.act, dtype=torch.float32)
+    rms = np.sqrt(np.mean(out ** 2))
+    assert (np.abs(wrong - out) > 2e-2 * rms + slack).any()
