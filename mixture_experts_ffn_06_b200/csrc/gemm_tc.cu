@@ -83,11 +83,15 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
 }
 
 // Epilogue scratch: one padded 32x33 fp32 tile per epilogue warp, and the
-// destination row / gate weight of each tile row (modes 2 and 3).
+// destination row / gate weight of each tile row (modes 2 and 3).  With FP8
+// operands each warp also keeps the tile's 256 column scales (mode 0: the
+// gate rows' at [0, 128), the up rows' at [128, 256); 0 past the tile).
+template <bool F8>
 struct EpiSmem {
   float buf[4][32][33];
   int64_t rdst[4][32];
   float rw[4][32];
+  float cs[F8 ? 4 : 1][F8 ? 256 : 1];
 };
 
 struct KParams {
@@ -147,10 +151,24 @@ __device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs,
   return Tile{lo, offs[lo] + mt * BM, (int)nt * BN_OUT, mt < mtg};
 }
 
-__device__ __forceinline__ float act_apply(int act, float g) {
-  if (act == MOE_ACT_SILU) return g / (1.0f + expf(-g));
-  const float c = 0.7978845608028654f;  // sqrt(2/pi)
-  return 0.5f * g * (1.0f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
+// The gate activation in the sigmoid form: SiLU(g) = g sigma(g), and the
+// tanh approximation of GELU, 0.5 g (1 + tanh(v)) with v = sqrt(2/pi) (g +
+// 0.044715 g^3), is g sigma(2v) since 0.5 (1 + tanh(v)) = 1 / (1 + e^-2v).
+// Both use the fast exponential and division intrinsics (a few ulp; the
+// limits g -> +-inf come out as g and 0).
+template <int ACT>
+__device__ __forceinline__ float act_fast(float g) {
+  if (ACT == MOE_ACT_SILU) return __fdividef(g, 1.0f + __expf(-g));
+  const float m2v = -1.5957691216057308f * fmaf(0.044715f * g, g * g, g);  // -2 v
+  return __fdividef(g, 1.0f + __expf(m2v));
+}
+
+// h of 32 columns of one row: Act(g_j) * u_j into a row of the transpose tile
+template <int ACT>
+__device__ __forceinline__ void act_row(const float (&g)[32], const float (&u)[32],
+                                        float* row) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) row[j] = act_fast<ACT>(g[j]) * u[j];
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -178,7 +196,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * A_STAGE;
-  EpiSmem* epi = reinterpret_cast<EpiSmem*>(gbase + STAGES * (A_STAGE + B_STAGE));
+  using Epi = EpiSmem<F8>;
+  Epi* epi = reinterpret_cast<Epi*>(gbase + STAGES * (A_STAGE + B_STAGE));
   Ctl* ctl = reinterpret_cast<Ctl*>(epi + 1);
   int64_t* ub = reinterpret_cast<int64_t*>(ctl + 1);        // [G+1]
   int32_t* offs = reinterpret_cast<int32_t*>(ub + p.G + 1);  // [G+1]
@@ -378,11 +397,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // covers whole 64/128-byte row segments instead of 32 scattered rows.
     const int q = warp & 3;
     float(*tbuf)[33] = epi->buf[q];
+    float* cs = epi->cs[F8 ? q : 0];
     const uint32_t empty0 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[0]), 0) : 0u;
     const uint32_t empty1 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[1]), 0) : 0u;
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = unit0; t < total; t += unit_step) {
       const Tile tl = map_tile<MODE, CG, NH>(t, offs, ub, p.G, p.NT, rank);
+      const int64_t wrow0 = tl.row0 + q * 32;  // first tile row of this warp
+      // FP8: this lane's row scale, and the tile's column scales (the B rows
+      // of the group; mode 0: gate row n at n, up row n at N + n)
+      float sa = 1.0f;
+      if (F8) {
+        if (tl.valid) sa = __ldg(p.a_scale + wrow0 + lane);
+        const bool routed = tl.g < p.E;
+        const float* sb = (routed ? p.b_scale : p.b_scale_sh) +
+                          (int64_t)(routed ? tl.g : tl.g - p.E) * (MODE == 0 ? 2 * p.N : p.N);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int i = lane + 32 * m;
+          float v = 0.0f;
+          if (MODE == 0) {
+            const int col = tl.n0 + (i & 127);
+            if ((i & 127) < NH && col < p.N) v = __ldg(sb + (i < 128 ? col : p.N + col));
+          } else {
+            const int col = tl.n0 + i;
+            if (col < p.N) v = __ldg(sb + col);
+          }
+          cs[i] = v;
+        }
+        __syncwarp();  // every lane reads every column's scale
+      }
       if (MODE <= 1) {
         // 1: a real row.  Padding rows (only in a segment's last tile) feed
         // nothing: mode 0 leaves them as they are (-1), mode 1 writes zeros
@@ -390,8 +434,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const bool real = tl.row0 + BM < (int64_t)offs[tl.g + 1] ||
                           (tl.valid && p.sorted_slots[tl.row0 + q * 32 + lane] >= 0);
         epi->rdst[q][lane] = real ? 1 : (MODE == 1 ? 0 : -1);
+        epi->rw[q][lane] = sa;  // mode 1 with FP8: the row's scale
       } else {
-        // destination row and gate weight of this lane's tile row
+        // destination row and gate weight of this lane's tile row (with
+        // FP8, times the row's scale)
         int64_t dst = -1;
         float wt = 1.0f;
         if (tl.valid) {
@@ -413,7 +459,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
         epi->rdst[q][lane] = dst;
-        epi->rw[q][lane] = wt;
+        epi->rw[q][lane] = F8 ? wt * sa : wt;
       }
       const bool got = mbar_wait(smem_u32(&ctl->tmem_full[acc]), acc_phase,
                                  abort_flag, p.timeout_ns, p.err);
@@ -421,62 +467,65 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
-      const int64_t wrow0 = tl.row0 + q * 32;  // first tile row of this warp
       constexpr int CHUNKS = MODE == 0 ? (NH + 31) / 32 : 8;
-      // FP8: this lane's row scale, and the column scales of the group's
-      // B rows (mode 0: gate row n at n, up row n at N + n)
-      float sa = 1.0f;
-      const float* sb = nullptr;
-      if (F8 && tl.valid) {
-        sa = __ldg(p.a_scale + wrow0 + lane);
-        const bool routed = tl.g < p.E;
-        sb = (routed ? p.b_scale : p.b_scale_sh) +
-             (int64_t)(routed ? tl.g : tl.g - p.E) * (MODE == 0 ? 2 * p.N : p.N);
-      }
-      // value of accumulator column j of B row `brow` (for a column past N
-      // the scale is not read: nothing of it is stored)
-      auto scaled = [&](uint32_t bits, int brow, bool in) -> float {
-        const float v = __uint_as_float(bits);
-        if (!F8) return v;
-        return in ? v * (sa * __ldg(sb + brow)) : 0.0f;
-      };
 #pragma unroll 1
       for (int c = 0; c < CHUNKS; ++c) {
         const int col0 = tl.n0 + c * 32;
         if (col0 >= p.N) break;
-        if (MODE == 0 && NH == 128) {
-          uint32_t g[32], u[32];
-          tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, g, u);
+        if (MODE == 0) {
+          // gate columns [32c, 32c + 32) and the matching up columns (NH + 32c
+          // + j: with NH = 128 the chunk at 128 + 32c; with a narrow tile it
+          // straddles the 32-column chunks starting at 32 (NH / 32 + c) and
+          // 32 (NH / 32 + c + 1), so every TMEM load starts at a multiple of
+          // 32 columns, all of them inside this accumulator's 256)
+          float g[32], u[32];
+          {
+            uint32_t gb[32], ub0[32];
+            if (NH == 128) {
+              tmem_ld32x2(tb + c * 32, tb + BN_ACC / 2 + c * 32, gb, ub0);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) u[j] = __uint_as_float(ub0[j]);
+            } else {
+              constexpr int UQ = NH / 32, UR = NH % 32;
+              uint32_t ub1[32];
+              tmem_ld32x2(tb + c * 32, tb + (UQ + c) * 32, gb, ub0);
+              tmem_ld32(tb + (UQ + c + 1) * 32, ub1);
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                u[j] = __uint_as_float(j + UR < 32 ? ub0[j + UR] : ub1[j + UR - 32]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) g[j] = __uint_as_float(gb[j]);
+          }
           if (!tl.valid) continue;  // the pair's empty half: nothing to store
+          if (F8) {
+            // column scales of the chunk (the same for every lane: broadcast
+            // reads), times this lane's row scale
+            const float4* cg = reinterpret_cast<const float4*>(cs + c * 32);
+            const float4* cu = reinterpret_cast<const float4*>(cs + 128 + c * 32);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const bool in = col0 + j < p.N;
-            tbuf[lane][j] = act_apply(p.act, scaled(g[j], col0 + j, in)) *
-                            scaled(u[j], p.N + col0 + j, in);
+            for (int i = 0; i < 8; ++i) {
+              const float4 a = cg[i], b = cu[i];
+              g[4 * i + 0] *= sa * a.x;
+              g[4 * i + 1] *= sa * a.y;
+              g[4 * i + 2] *= sa * a.z;
+              g[4 * i + 3] *= sa * a.w;
+              u[4 * i + 0] *= sa * b.x;
+              u[4 * i + 1] *= sa * b.y;
+              u[4 * i + 2] *= sa * b.z;
+              u[4 * i + 3] *= sa * b.w;
+            }
           }
-        } else if (MODE == 0) {
-          // gate columns [32c, 32c + 32); the matching up column NH + 32c + j
-          // lies in the 32-column chunk starting at 32 (NH / 32 + c) or in
-          // the next one, so every TMEM load starts at a multiple of 32
-          // columns (all of them inside this accumulator's 256)
-          constexpr int UQ = NH / 32, UR = NH % 32;
-          uint32_t g[32], u0[32], u1[32];
-          tmem_ld32x2(tb + c * 32, tb + (UQ + c) * 32, g, u0);
-          tmem_ld32(tb + (UQ + c + 1) * 32, u1);
-          if (!tl.valid) continue;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const uint32_t uj = j + UR < 32 ? u0[j + UR] : u1[j + UR - 32];
-            const bool in = col0 + j < p.N && c * 32 + j < NH;
-            tbuf[lane][j] = act_apply(p.act, scaled(g[j], col0 + j, in)) *
-                            scaled(uj, p.N + col0 + j, in);
-          }
+          if (p.act == MOE_ACT_SILU)
+            act_row<MOE_ACT_SILU>(g, u, tbuf[lane]);
+          else
+            act_row<MOE_ACT_GELU_TANH>(g, u, tbuf[lane]);
         } else {
           uint32_t y[32];
           tmem_ld32(tb + c * 32, y);
           if (!tl.valid) continue;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tbuf[lane][j] = scaled(y[j], col0 + j, col0 + j < p.N);
+          for (int j = 0; j < 32; ++j) tbuf[lane][j] = __uint_as_float(y[j]);
         }
         __syncwarp();
         if (MODE == 0) {
@@ -500,15 +549,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           // 4 rows x 128 bytes per instruction
           float* out = static_cast<float*>(p.out);
           const int cc = (lane & 7) * 4;
+          // FP8: the scales of this lane's four columns (the row's scale is
+          // folded into rw)
+          float4 c4 = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (F8) c4 = *reinterpret_cast<const float4*>(cs + c * 32 + cc);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = i * 4 + (lane >> 3);
             if (col0 + cc < p.N) {
-              const float a0 = tbuf[r][cc + 0], a1 = tbuf[r][cc + 1];
-              const float a2 = tbuf[r][cc + 2], a3 = tbuf[r][cc + 3];
+              float a0 = tbuf[r][cc + 0], a1 = tbuf[r][cc + 1];
+              float a2 = tbuf[r][cc + 2], a3 = tbuf[r][cc + 3];
+              if (F8) {
+                a0 *= c4.x;
+                a1 *= c4.y;
+                a2 *= c4.z;
+                a3 *= c4.w;
+              }
               if (MODE == 1) {
+                const float rs = F8 ? epi->rw[q][r] : 1.0f;
                 *reinterpret_cast<float4*>(out + (wrow0 + r) * (int64_t)p.N + col0 + cc) =
-                    epi->rdst[q][r] > 0 ? make_float4(a0, a1, a2, a3)
+                    epi->rdst[q][r] > 0 ? make_float4(a0 * rs, a1 * rs, a2 * rs, a3 * rs)
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
               } else {
                 const int64_t dst = epi->rdst[q][r];
@@ -666,7 +726,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t st, bool pdl) {
   p.b_scale_sh = a.b_scale_sh;
 
   const size_t smem = 1024 + (size_t)C::STAGES * (A_STAGE + C::B_STAGE) +
-                      sizeof(EpiSmem) + sizeof(Ctl) +
+                      sizeof(EpiSmem<F8>) + sizeof(Ctl) +
                       (sizeof(int64_t) + sizeof(int32_t)) * (size_t)(a.G + 1);
   // the shared-memory opt-in is a per-device attribute: set it once on
   // every device this process launches on
