@@ -82,13 +82,17 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                : "memory");
 }
 
-// Epilogue scratch: one padded 32x33 fp32 tile per epilogue warp, and the
-// destination row / gate weight of each tile row (modes 2 and 3).  With FP8
-// operands each warp also keeps the tile's 256 column scales (mode 0: the
-// gate rows' at [0, 128), the up rows' at [128, 256); 0 past the tile).
+// Epilogue scratch: one 32x32 fp32 transpose tile per epilogue warp, and
+// the destination row / gate weight of each tile row (modes 2 and 3).  With
+// FP8 operands each warp also keeps the tile's 256 column scales (mode 0:
+// the gate rows' at [0, 128), the up rows' at [128, 256); 0 past the tile).
+// The tile is read and written in 16-byte slots: slot q of row r (columns
+// 4q..4q+3) sits at slot q ^ (r mod 8) of the row, so that eight lanes
+// writing one slot of eight rows, or reading eight slots of one row, touch
+// all 32 banks once.
 template <bool F8>
 struct EpiSmem {
-  float buf[4][32][33];
+  float buf[4][32][32];
   int64_t rdst[4][32];
   float rw[4][32];
   float cs[F8 ? 4 : 1][F8 ? 256 : 1];
@@ -151,6 +155,11 @@ __device__ __forceinline__ Tile map_tile(int64_t i, const int32_t* offs,
   return Tile{lo, offs[lo] + mt * BM, (int)nt * BN_OUT, mt < mtg};
 }
 
+// 16-byte slot q of row r of a transpose tile (see EpiSmem)
+__device__ __forceinline__ float4* tslot(float (*t)[32], int r, int q) {
+  return reinterpret_cast<float4*>(&t[r][4 * (q ^ (r & 7))]);
+}
+
 // The gate activation in the sigmoid form: SiLU(g) = g sigma(g), and the
 // tanh approximation of GELU, 0.5 g (1 + tanh(v)) with v = sqrt(2/pi) (g +
 // 0.044715 g^3), is g sigma(2v) since 0.5 (1 + tanh(v)) = 1 / (1 + e^-2v).
@@ -163,12 +172,15 @@ __device__ __forceinline__ float act_fast(float g) {
   return __fdividef(g, 1.0f + __expf(m2v));
 }
 
-// h of 32 columns of one row: Act(g_j) * u_j into a row of the transpose tile
+// h of 32 columns of row r: Act(g_j) * u_j into the transpose tile
 template <int ACT>
 __device__ __forceinline__ void act_row(const float (&g)[32], const float (&u)[32],
-                                        float* row) {
+                                        float (*t)[32], int r) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) row[j] = act_fast<ACT>(g[j]) * u[j];
+  for (int q = 0; q < 8; ++q)
+    *tslot(t, r, q) = make_float4(
+        act_fast<ACT>(g[4 * q + 0]) * u[4 * q + 0], act_fast<ACT>(g[4 * q + 1]) * u[4 * q + 1],
+        act_fast<ACT>(g[4 * q + 2]) * u[4 * q + 2], act_fast<ACT>(g[4 * q + 3]) * u[4 * q + 3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -392,11 +404,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // ----------------------------------------------------------- epilogue
     // Each warp owns TMEM lanes [32q, 32q+32), i.e. 32 rows of this CTA's
     // m-tile.  Per 32-column chunk it loads its rows' accumulators (one row
-    // per lane), parks them in a padded 32x33 shared tile and writes them out
+    // per lane), parks them in a swizzled 32x32 shared tile and writes them out
     // transposed, so that every store (or reduction) instruction of the warp
     // covers whole 64/128-byte row segments instead of 32 scattered rows.
     const int q = warp & 3;
-    float(*tbuf)[33] = epi->buf[q];
+    float(*tbuf)[32] = epi->buf[q];
     float* cs = epi->cs[F8 ? q : 0];
     const uint32_t empty0 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[0]), 0) : 0u;
     const uint32_t empty1 = CG == 2 ? mapa_shared(smem_u32(&ctl->tmem_empty[1]), 0) : 0u;
@@ -517,15 +529,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
           }
           if (p.act == MOE_ACT_SILU)
-            act_row<MOE_ACT_SILU>(g, u, tbuf[lane]);
+            act_row<MOE_ACT_SILU>(g, u, tbuf, lane);
           else
-            act_row<MOE_ACT_GELU_TANH>(g, u, tbuf[lane]);
+            act_row<MOE_ACT_GELU_TANH>(g, u, tbuf, lane);
         } else {
           uint32_t y[32];
           tmem_ld32(tb + c * 32, y);
           if (!tl.valid) continue;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tbuf[lane][j] = __uint_as_float(y[j]);
+          for (int j = 0; j < 8; ++j)
+            *tslot(tbuf, lane, j) =
+                make_float4(__uint_as_float(y[4 * j]), __uint_as_float(y[4 * j + 1]),
+                            __uint_as_float(y[4 * j + 2]), __uint_as_float(y[4 * j + 3]));
         }
         __syncwarp();
         if (MODE == 0) {
@@ -537,11 +552,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             const int r = i * 8 + (lane >> 2);
             const int64_t rd = epi->rdst[q][r];
             if (col0 + cc < p.N && c * 32 + cc < NH && rd > 0) {
+              const float4 v0 = *tslot(tbuf, r, cc / 4), v1 = *tslot(tbuf, r, cc / 4 + 1);
               uint4 o;
-              o.x = pack_bf16x2(tbuf[r][cc + 0], tbuf[r][cc + 1]);
-              o.y = pack_bf16x2(tbuf[r][cc + 2], tbuf[r][cc + 3]);
-              o.z = pack_bf16x2(tbuf[r][cc + 4], tbuf[r][cc + 5]);
-              o.w = pack_bf16x2(tbuf[r][cc + 6], tbuf[r][cc + 7]);
+              o.x = pack_bf16x2(v0.x, v0.y);
+              o.y = pack_bf16x2(v0.z, v0.w);
+              o.z = pack_bf16x2(v1.x, v1.y);
+              o.w = pack_bf16x2(v1.z, v1.w);
               *reinterpret_cast<uint4*>(out + (wrow0 + r) * (int64_t)p.N + col0 + cc) = o;
             }
           }
@@ -557,8 +573,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int i = 0; i < 8; ++i) {
             const int r = i * 4 + (lane >> 3);
             if (col0 + cc < p.N) {
-              float a0 = tbuf[r][cc + 0], a1 = tbuf[r][cc + 1];
-              float a2 = tbuf[r][cc + 2], a3 = tbuf[r][cc + 3];
+              const float4 v = *tslot(tbuf, r, lane & 7);
+              float a0 = v.x, a1 = v.y, a2 = v.z, a3 = v.w;
               if (F8) {
                 a0 *= c4.x;
                 a1 *= c4.y;
