@@ -194,8 +194,9 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const int32_t* ids,
  *   w13       [E,2I,H] bf16: rows [0,I) gate (w1), rows [I,2I) up (w3)
  *   w2        [E,H,I] bf16
  *   w13_sh    [S,2I,H] bf16 or NULL when S == 0;  w2_sh [S,H,I] likewise
- *   y_perm    [cap,H] fp32 out: unweighted expert output of every row in use;
- *             padding rows get 0, rows past offsets[E+S] are not written
+ *   y_perm    [cap,H] fp32 out, 16-byte aligned (else MOE_ERR_INVALID_ARG):
+ *             unweighted expert output of every row in use; padding rows
+ *             get 0, rows past offsets[E+S] are not written
  * h = Act(g) (*) u is rounded to bf16 (the second GEMM's operand); every
  * product accumulates in fp32 on the tensor cores.
  */

@@ -278,6 +278,8 @@ moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
       (shape->T > 0 && !x))
     return MOE_ERR_INVALID_ARG;
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
+  // y_perm rows are written by 16-byte bulk copies
+  if (!aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   return run_expert_ffn(*shape, reinterpret_cast<const __nv_bfloat16*>(x), offsets,

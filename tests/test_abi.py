@@ -114,6 +114,11 @@ def test_null_pointers_and_small_workspace(api):
                                 null, null, fake, fake,
                                 api.moe_workspace_size(sh), null)
     assert rc == 1  # shared weights missing
+    s1 = _shape(api)
+    rc = api.lib.moe_expert_ffn(ctypes.byref(s1), fake, fake, fake, fake, fake,
+                                null, null, ctypes.c_void_p((1 << 20) + 8), fake,
+                                api.moe_workspace_size(s1), null)
+    assert rc == 1  # y_perm not 16-byte aligned
 
 
 def test_empty_batch_is_a_no_op(api):
