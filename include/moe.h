@@ -22,8 +22,10 @@
  *
  * Conventions (every entry point):
  *   - All pointers are DEVICE pointers unless a parameter says otherwise.
- *     The caller owns every buffer.  The library never allocates, frees or
- *     synchronises (except moe_read_error, which says so).
+ *     The caller owns every buffer.  The library never allocates device
+ *     memory, frees or synchronises (except moe_read_error, which says so);
+ *     moe_gemma4_block creates one CUDA stream and two events per device on
+ *     its first call there and keeps them.
  *   - Buffers are dense, row-major and 16-byte aligned.
  *   - bf16 data is passed as uint16_t bit patterns (moe_bf16).
  *   - Work is enqueued on ``stream`` and runs asynchronously.
@@ -355,7 +357,15 @@ MOE_API moe_status moe_permute_noalloc(const moe_shape* shape,
  *   out      [T,H] bf16 out; out_f32 NULL or [T,H] fp32 out: the output
  *            before its final rounding
  *   ws       moe_gemma4_workspace_size(shape, I_dense) bytes, 256-byte
- *            aligned, owned by the caller
+ *            aligned, owned by the caller, first 256 bytes zeroed once (its
+ *            error word: moe_read_error covers both branches)
+ * The two branches run side by side: after the input norms on ``stream``
+ * the dense MLP is forked onto a second stream of the library's own (one per
+ * device, made on the first call) and joined back by an event before the
+ * output norms, so ``stream`` alone orders the call with the caller's work,
+ * and the call can be captured into a CUDA graph (make the first call on a
+ * device outside a capture: it creates that stream).  Calls from several
+ * host threads are serialised while they enqueue.
  * Bad shapes or arguments return before any launch.
  */
 typedef struct {

@@ -7,14 +7,26 @@
 // Each norm is the standard RMSNorm with a gamma (section 3), computed in
 // fp32 and returned in bf16; every module hands bf16 to the next.
 //
-// Four steps on one stream:
+// The two branches read the same residual and meet only in the last step,
+// so they run side by side (section 1: the dense MLP and the MoE in
+// parallel):
 //   pre_norm_kernel    one block per token: both input norms from one read
 //                      of x (and zeroes the dense MLP's one-expert logits);
-//   moe_forward_ex     the dense MLP as the one-expert, weight-1 case of the
+//   then, forked onto a second stream of the library's own:
+//     moe_forward_ex   the dense MLP as the one-expert, weight-1 case of the
 //                      layer (E = 1, k = 1, I = I_dense) -> y1;
-//   moe_forward_ex     the router on x, then the MoE on pre_ff_norm_2(x) -> y2;
+//   while the caller's stream runs
+//     moe_forward_ex   the router on x, then the MoE on pre_ff_norm_2(x) -> y2;
+//   joined back:
 //   post_norm_kernel   one block per token: the two output norms, their
 //                      bf16 sum, the last norm and the residual add.
+// The fork and the join are an event each, so the pattern holds under CUDA
+// graph capture as well (the second stream joins the capture).  Each branch
+// has its own layer workspace; the MoE branch's sits at offset 0, so its
+// error word is the block's, and post_norm moves the dense branch's error
+// code (if any) into it.
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace moe {
@@ -53,7 +65,7 @@ __global__ void __launch_bounds__(kNormThreads)
 pre_norm_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ g1,
                 const __nv_bfloat16* __restrict__ g2, int H, float eps,
                 __nv_bfloat16* __restrict__ a1, __nv_bfloat16* __restrict__ a2,
-                float* __restrict__ zero_logits) {
+                float* __restrict__ zero_logits, uint32_t* __restrict__ dense_err) {
   __shared__ double red[kNormThreads / 32];
   const int64_t t = blockIdx.x;
   const __nv_bfloat16* xr = x + t * H;
@@ -69,6 +81,9 @@ pre_norm_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
     a2[t * H + h] = norm_elem(v, inv, g2[h]);
   }
   if (threadIdx.x == 0) zero_logits[t] = 0.0f;
+  // the dense branch's error word starts clear (post_norm moved out what
+  // the previous call left)
+  if (t == 0 && threadIdx.x == 0) *dense_err = 0u;
 }
 
 __global__ void __launch_bounds__(kNormThreads)
@@ -76,9 +91,14 @@ post_norm_kernel(const __nv_bfloat16* __restrict__ y1, const __nv_bfloat16* __re
                  const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ g1,
                  const __nv_bfloat16* __restrict__ g2, const __nv_bfloat16* __restrict__ g,
                  int H, float eps, __nv_bfloat16* __restrict__ out,
-                 float* __restrict__ out_f32) {
+                 float* __restrict__ out_f32, uint32_t* __restrict__ dense_err,
+                 uint32_t* __restrict__ block_err) {
   __shared__ double red[kNormThreads / 32];
   const int64_t t = blockIdx.x;
+  if (t == 0 && threadIdx.x == 0) {
+    const uint32_t e = atomicExch(dense_err, 0u);
+    if (e) atomicCAS(block_err, 0u, e);
+  }
   const __nv_bfloat16* r1 = y1 + t * H;
   const __nv_bfloat16* r2 = y2 + t * H;
   double s1 = 0.0, s2 = 0.0;
@@ -119,15 +139,19 @@ moe_shape dense_shape(const moe_shape& s, int I_dense) {
   return d;
 }
 
+// [MoE layer workspace | a1 | a2 | y1 | y2 | zl | dense layer workspace]
 struct BlockWs {
-  size_t a1, a2, y1, y2, zl, inner, total;
+  size_t moe, a1, a2, y1, y2, zl, dense, total;
 };
 
 BlockWs block_ws(const moe_shape& s, int I_dense) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t th = (size_t)s.T * (size_t)s.H * 2;
+  const moe_shape d = dense_shape(s, I_dense);
   BlockWs w{};
   size_t o = 0;
+  w.moe = o;
+  o += up(moe_workspace_size(&s));
   w.a1 = o;
   o += up(th);
   w.a2 = o;
@@ -138,12 +162,29 @@ BlockWs block_ws(const moe_shape& s, int I_dense) {
   o += up(th);
   w.zl = o;
   o += up(sizeof(float) * (size_t)s.T + 4);
-  w.inner = o;
-  const moe_shape d = dense_shape(s, I_dense);
-  const size_t a = moe_workspace_size(&s), b = moe_workspace_size(&d);
-  o += a > b ? a : b;
+  w.dense = o;
+  o += up(moe_workspace_size(&d));
   w.total = o;
   return w;
+}
+
+// The second stream and the fork / join events, one set per device, made on
+// the first call and kept for the life of the process.  The mutex covers the
+// enqueueing from the fork to the join, so that calls from several host
+// threads do not interleave their event records.
+struct SideStream {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+constexpr int kMaxBlockDevices = 64;
+SideStream g_side[kMaxBlockDevices];
+
+SideStream* side_stream(int dev) {
+  if (dev < 0 || dev >= kMaxBlockDevices) return nullptr;
+  return &g_side[dev];
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -193,33 +234,57 @@ moe_status moe_gemma4_block(const moe_shape* shape, const moe_bf16* x,
   auto* y1 = reinterpret_cast<__nv_bfloat16*>(base + m.y1);
   auto* y2 = reinterpret_cast<__nv_bfloat16*>(base + m.y2);
   auto* zl = reinterpret_cast<float*>(base + m.zl);
-  void* inner = base + m.inner;
-  const size_t inner_bytes = ws_bytes - m.inner;
+  void* ws_moe = base + m.moe;
+  void* ws_dense = base + m.dense;
+  auto* block_err = reinterpret_cast<uint32_t*>(ws_moe);     // the block's error word
+  auto* dense_err = reinterpret_cast<uint32_t*>(ws_dense);
+  const size_t moe_bytes = m.a1 - m.moe, dense_bytes = m.total - m.dense;
   const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   auto nw = [&](int i) { return reinterpret_cast<const __nv_bfloat16*>(p->norm_w[i]); };
 
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  SideStream* side = side_stream(dev);
+  if (!side) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(side->mu);
+  if (!side->ready) {
+    if (cudaStreamCreateWithFlags(&side->s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&side->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&side->join, cudaEventDisableTiming) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    side->ready = true;
+  }
+
   if (launch_ex(pre_norm_kernel, dim3((unsigned)s.T), dim3(kNormThreads), 0, stream, false,
-                xb, nw(0), nw(2), s.H, p->eps, a1, a2, zl) != cudaSuccess)
+                xb, nw(0), nw(2), s.H, p->eps, a1, a2, zl, dense_err) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // the dense MLP: one expert, every token with weight 1
+  // fork: the dense MLP (one expert, every token with weight 1) on the
+  // second stream, once the input norms are written
+  if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
+      cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
   auto mb = [](void* q) { return reinterpret_cast<moe_bf16*>(q); };
-  if ((st = moe_forward_ex(&d, mb(a1), zl, p->mlp_w13, p->mlp_w2, nullptr, nullptr,
-                           nullptr, mb(y1), nullptr, nullptr, inner, inner_bytes, nullptr,
-                           stream)) !=
-      MOE_OK)
-    return st;
+  moe_status sd = moe_forward_ex(&d, mb(a1), zl, p->mlp_w13, p->mlp_w2, nullptr, nullptr,
+                                 nullptr, mb(y1), nullptr, nullptr, ws_dense, dense_bytes,
+                                 nullptr, side->s);
+  // the join is recorded whatever the dense branch returned, so that the
+  // caller's stream (or its capture) is never left forked
+  if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
   // the router reads the raw residual, the experts its pre_ff_norm_2
   moe_forward_opts o{};
   o.router_x = x;
   o.router_w = p->router_w;
   o.router_scale = p->router_scale;
   o.router_eps = p->router_eps;
-  if ((st = moe_forward_ex(&s, mb(a2), nullptr, w13, w2, scale, nullptr, nullptr, mb(y2),
-                           nullptr, nullptr, inner, inner_bytes, &o, stream)) != MOE_OK)
-    return st;
+  st = moe_forward_ex(&s, mb(a2), nullptr, w13, w2, scale, nullptr, nullptr, mb(y2),
+                      nullptr, nullptr, ws_moe, moe_bytes, &o, stream);
+  if (cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (sd != MOE_OK) return sd;
+  if (st != MOE_OK) return st;
   if (launch_ex(post_norm_kernel, dim3((unsigned)s.T), dim3(kNormThreads), 0, stream, false,
                 (const __nv_bfloat16*)y1, (const __nv_bfloat16*)y2, xb, nw(1), nw(3), nw(4),
-                s.H, p->eps, reinterpret_cast<__nv_bfloat16*>(out), out_f32) != cudaSuccess)
+                s.H, p->eps, reinterpret_cast<__nv_bfloat16*>(out), out_f32, dense_err,
+                block_err) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

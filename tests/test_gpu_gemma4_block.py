@@ -66,3 +66,68 @@ def test_block_matches_oracle(api, name):
     excess = np.abs(got - want) - bound
     assert excess.max() <= 0, (f"max|err| {np.abs(got - want).max():.3e}, update RMS "
                                f"{upd:.3e}, worst excess {excess.max():.3e}")
+
+
+def _block_args(api, shp, moe, blk):
+    """moe_gemma4_block's arguments up to ``out``, on the device."""
+    c = lambda t: t.cuda().contiguous()  # noqa: E731
+    s = api.shape_from(shp)
+    args = (s, c(blk.x), [c(g) for g in blk.norms], 1e-6, c(blk.mlp_w13), c(blk.mlp_w2),
+            c(blk.router_w), c(blk.router_scale), 1e-6, c(moe.w13), c(moe.w2),
+            c(moe.scale))
+    return args
+
+
+def test_block_branches_join_on_the_callers_stream(api):
+    """The dense MLP runs on a second stream; the call must still be
+    complete once the caller's stream alone is synchronised, and the
+    block's error word (moe_read_error on its workspace) is clear."""
+    shp, Id = CASES["gemma4_26b_shapes"]
+    moe = inputs.make_inputs(shp, seed=3, scale="uniform")
+    blk = inputs.gemma4_block_inputs(shp.T, shp.H, shp.E, Id, seed=4)
+    args = _block_args(api, shp, moe, blk)
+    s = args[0]
+    ws = api.alloc_gemma4_workspace(s, Id)
+    ref = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device="cuda")
+    api.moe_gemma4_block(*args, ref, ws)
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream()
+    for _ in range(3):
+        out = torch.full((shp.T, shp.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        torch.cuda.current_stream().synchronize()
+        with torch.cuda.stream(st):
+            api.moe_gemma4_block(*args, out, ws, stream=st)
+        st.synchronize()  # the caller's stream only
+        assert torch.equal(out, ref)
+    assert api.moe_read_error(ws) == 0
+
+
+def test_block_captured_in_a_cuda_graph(api):
+    """The fork onto the second stream and the join back are events, so the
+    call captures into one graph; replays give the eager result bit for bit
+    (both inner layers take the deterministic decode path here)."""
+    shp, Id = CASES["few_tokens"]
+    moe = inputs.make_inputs(shp, seed=5, scale="uniform")
+    blk = inputs.gemma4_block_inputs(shp.T, shp.H, shp.E, Id, seed=6)
+    args = _block_args(api, shp, moe, blk)
+    s = args[0]
+    ws = api.alloc_gemma4_workspace(s, Id)
+    ref = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device="cuda")
+    api.moe_gemma4_block(*args, ref, ws)
+    torch.cuda.synchronize()
+    out = torch.zeros(shp.T, shp.H, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        api.moe_gemma4_block(*args, out, ws, stream=st)  # warm-up outside capture
+    st.synchronize()
+    out.zero_()
+    with torch.cuda.graph(g, stream=st):
+        api.moe_gemma4_block(*args, out, ws, stream=st)
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    del g
+    assert api.moe_read_error(ws) == 0
