@@ -55,6 +55,12 @@ def _gpu_logits(api, x, w, s, eps):
     (37, 200, 5),       # H not a multiple of 32: a partial 32-column chunk
     (16, 64, 130),      # E > 128: two expert blocks, the second ragged
     (1, 4096, 8),       # one token
+    (65, 256, 8),       # two token tiles, the second with one token
+    (300, 200, 40),     # a ragged token tile and a partial 32-column chunk
+    (257, 128, 300),    # many expert blocks, the last one ragged
+    (1000, 2048, 64),   # the skewed batch's H and E
+    (129, 1024, 256),   # E = 256
+    (4096, 4096, 8),    # the Mixtral-shaped batch
 ])
 def test_router_logits_match_oracle(api, T, H, E):
     x, w, s = _case(T, H, E, seed=T + H + E)
@@ -66,9 +72,10 @@ def test_router_logits_match_oracle(api, T, H, E):
     assert err <= TOL * rms, f"max|err| {err:.3e} > {TOL} x RMS {rms:.3e}"
 
 
-def test_zero_and_constant_rows(api):
+@pytest.mark.parametrize("T,E", [(20, 8), (150, 32)])
+def test_zero_and_constant_rows(api, T, E):
     # all-zero rows stay finite (eps); constant rows normalise to +-1
-    x, w, s = _case(20, 128, 8, seed=7)
+    x, w, s = _case(T, 128, E, seed=7)
     x[3] = 0.0
     x[5] = 1.5
     want = oracle.router_logits(x, w, s, 1e-6)
