@@ -55,6 +55,9 @@ def _gpu_logits(api, x, w, s, eps):
     (37, 200, 5),       # H not a multiple of 32: a partial 32-column chunk
     (16, 64, 130),      # E > 128: two expert blocks, the second ragged
     (1, 4096, 8),       # one token
+    (4, 2816, 128),     # a decode step of the many-small shape
+    (13, 200, 5),       # 13 tokens, H = 200
+    (16, 1024, 300),    # many expert blocks for one token tile
     (65, 256, 8),       # two token tiles, the second with one token
     (300, 200, 40),     # a ragged token tile and a partial 32-column chunk
     (257, 128, 300),    # many expert blocks, the last one ragged
@@ -72,7 +75,7 @@ def test_router_logits_match_oracle(api, T, H, E):
     assert err <= TOL * rms, f"max|err| {err:.3e} > {TOL} x RMS {rms:.3e}"
 
 
-@pytest.mark.parametrize("T,E", [(20, 8), (150, 32)])
+@pytest.mark.parametrize("T,E", [(8, 8), (20, 8), (150, 32)])
 def test_zero_and_constant_rows(api, T, E):
     # all-zero rows stay finite (eps); constant rows normalise to +-1
     x, w, s = _case(T, 128, E, seed=7)
