@@ -215,19 +215,18 @@ gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_slot
     if (s < 0) continue;
     const int64_t t = (s < R) ? (int64_t)s / k : ((int64_t)s - R) % T;
     const uint4* src = x + t * chunks;
-    // four 16-byte loads in flight per lane before the stores; the copies
-    // are written with the streaming hint so they do not push x (read k
-    // times) out of L2
-    int c = lane;
-    for (; c + 96 < chunks; c += 128) {
-      const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32);
-      const uint4 v2 = __ldg(src + c + 64), v3 = __ldg(src + c + 96);
-      __stcs(dst + c, v0);
-      __stcs(dst + c + 32, v1);
-      __stcs(dst + c + 64, v2);
-      __stcs(dst + c + 96, v3);
+    // up to eight 16-byte loads in flight per lane before the stores (a
+    // 5.6 KB row in two rounds); the copies are written with the streaming
+    // hint so they do not push x (read k times) out of L2
+    for (int c0 = 0; c0 < chunks; c0 += 256) {
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c0 + lane + 32 * j < chunks) v[j] = __ldg(src + c0 + lane + 32 * j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c0 + lane + 32 * j < chunks) __stcs(dst + c0 + lane + 32 * j, v[j]);
     }
-    for (; c < chunks; c += 32) __stcs(dst + c, __ldg(src + c));
   }
   // zero the fp32 accumulator the w2 epilogue adds into (fast combine)
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
