@@ -43,6 +43,7 @@ import argparse
 import hashlib
 import json
 import os
+import select
 import statistics
 import subprocess
 import sys
@@ -150,46 +151,148 @@ def load_peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+_NVML_POLL = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+try:
+    h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+except Exception:
+    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+           or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    print(time.monotonic(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+          reasons(h), flush=True)
+    time.sleep(0.001)
+"""
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """SM clock and throttle-reason sampling while the timed region runs.
+    A child process polls NVML every millisecond and stamps each sample
+    with the monotonic clock (the device found by its UUID, so that a
+    CUDA_VISIBLE_DEVICES mapping is followed); the caller marks the timed
+    region (begin / end) and only the samples inside it are reported (at
+    least the first one after its start).  Without NVML, nvidia-smi every
+    100 ms.  Reads only; changes no setting."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,"
              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (hw_slowdown with the power brake)
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8 | 0x80,
+                   "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
         self._t = None
+        self.nvml = False
+        self.sm_max = None
+        self.t_begin = self.t_end = None
+
+    def _uuid(self):
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return ""
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                [sys.executable, "-c", _NVML_POLL, self._uuid(), str(self.gpu)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
+            # the child is sampling once it has printed the maximum clock
+            # (bounded wait: a child stuck in NVML falls back to nvidia-smi)
+            ready, _, _ = select.select([self.proc.stdout], [], [], 10.0)
+            first = self.proc.stdout.readline().split() if ready else []
+            if len(first) == 2 and first[0] == "max":
+                self.sm_max = float(first[1])
+                self.nvml = True
+            else:
+                self._kill()
+        except (OSError, ValueError):
+            self._kill()
+        if not self.nvml:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+                return
+            time.sleep(0.3)  # let nvidia-smi start
         self._t = threading.Thread(target=self._read, daemon=True)
         self._t.start()
+
+    def begin(self):
+        self.t_begin = time.monotonic()
+
+    def end(self):
+        self.t_end = time.monotonic()
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    def _kill(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+
+    def _stamp(self, ln):
+        try:
+            return float(ln.split()[0])
+        except (ValueError, IndexError):
+            return None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        if self.nvml and self.t_begin is not None:
+            # a timed region shorter than a sampling period: wait (briefly)
+            # for the first sample taken after its start
+            deadline = time.monotonic() + 0.2
+            while time.monotonic() < deadline and not any(
+                    (self._stamp(ln) or 0.0) >= self.t_begin for ln in self.lines[-4:]):
+                time.sleep(0.002)
+        self._kill()
         if self._t:
-            self._t.join(timeout=2)
+            self._t.join(timeout=5)
+        if self.nvml:
+            rows = []
+            for ln in self.lines:
+                parts = ln.split()
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), int(parts[2])))
+                except (ValueError, IndexError):
+                    continue
+            b = self.t_begin if self.t_begin is not None else float("-inf")
+            e = self.t_end if self.t_end is not None else float("inf")
+            inside = [r for r in rows if b <= r[0] <= e]
+            if not inside:
+                inside = [r for r in rows if r[0] >= b][:1]
+            if not inside:
+                return None
+            bits = 0
+            for r in inside:
+                bits |= r[2]
+            return {"sm_mhz": statistics.median(r[1] for r in inside),
+                    "sm_max_mhz": self.sm_max,
+                    "reasons": sorted(n for n, m in self.REASON_BITS.items() if bits & m),
+                    "samples": len(inside),
+                    "source": "nvml every 1 ms, samples inside the timed region"}
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
@@ -208,7 +311,8 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvidia-smi every 100 ms"}
 
 
 def traffic_for(kernel_src: str, config: str, shape_override):
@@ -477,7 +581,7 @@ def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
     torch.cuda.synchronize()
     if clocks is not None:
         clocks.start()
-        time.sleep(0.3)  # let the sampler start before the timed work
+        clocks.begin()
     t_start.record(stream)
     if graph is not None:
         graph.replay()
@@ -485,6 +589,9 @@ def timed_steps(args, api, inp, s, ws, out, stream, path, router, barrier,
         for i in range(args.steps):
             plain_step(i)
     t_end.record(stream)
+    if clocks is not None:
+        torch.cuda.synchronize()
+        clocks.end()  # the clock samples cover the timed steps only
     if staged is not None:
         staged.replay()
     else:
@@ -995,9 +1102,10 @@ def run_block(args):
     torch.cuda.synchronize()
     clocks = ClockSampler(0)
     clocks.start()
-    time.sleep(0.3)
+    clocks.begin()
     g.replay()
     torch.cuda.synchronize()
+    clocks.end()
     clk = clocks.stop()
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     flops = shp.flops() + 6.0 * shp.T * shp.H * Id
