@@ -151,3 +151,142 @@ def test_forward_fp8_full_size_many_small(api):
     sel = torch.from_numpy(tok).cuda()
     assert_out_close(out32[sel], want, f"many-small fp8, {len(tok)} tokens",
                      bf16=out[sel], slack=slack)
+
+
+# ---------------------------------------------------------------- integrity
+
+BAND = 4096      # guard bytes on each side of a buffer
+PATTERN = 0xA5
+
+
+class _Guarded:
+    """A buffer inside an allocation whose BAND bytes on either side hold
+    PATTERN."""
+
+    def __init__(self, shape, dtype):
+        n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+        self.n = n
+        self.raw = torch.full((BAND + n + BAND,), PATTERN, dtype=torch.uint8,
+                              device="cuda")
+        self.t = self.raw[BAND:BAND + n].view(dtype).view(*shape)
+
+    def intact(self) -> bool:
+        torch.cuda.synchronize()
+        return bool((self.raw[:BAND] == PATTERN).all()) and \
+            bool((self.raw[BAND + self.n:] == PATTERN).all())
+
+
+@pytest.mark.parametrize("variant", list(VARIANTS))
+@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_T130", "pairs"])
+def test_forward_fp8_writes_only_its_buffers(api, name, variant):
+    shp = SHAPES[name]
+    inp = inputs.make_inputs(shp, seed=6, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=106)
+    s = api.shape_from(shp)
+    T, H, k = shp.T, shp.H, shp.k
+    out = _Guarded((T, H), torch.bfloat16)
+    out32 = _Guarded((T, H), torch.float32)
+    ids = _Guarded((T, k), torch.int32)
+    w = _Guarded((T, k), torch.float32)
+    ws = _Guarded((api.moe_workspace_size_fp8(s),), torch.uint8)
+    ws.t[:256].zero_()
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
+                            fp.sh2_q, fp.sh2_s)]
+    det, pairs = VARIANTS[variant]
+    for _ in range(2):  # the second call finds the first call's workspace
+        api.moe_forward_fp8(s, _to(inp.x), _to(inp.logits), api.fp8_experts(*wts),
+                            _to(inp.scale), out.t, ws.t, ids_out=ids.t, w_out=w.t,
+                            out_f32=out32.t, deterministic=det, cta_pairs=pairs)
+    assert api.moe_read_error(ws.t) == 0
+    assert torch.isfinite(out32.t).all()
+    for nm, g in (("out", out), ("out_f32", out32), ("ids", ids), ("w", w),
+                  ("workspace", ws)):
+        assert g.intact(), f"{nm}: a guard band was overwritten"
+
+
+def test_forward_fp8_stale_workspace_changes_nothing(api):
+    """A workspace full of 0xFF bytes (NaN in bf16 and fp32, -1 as an index)
+    past its zeroed header gives the same bits as a clean one (fixed-order
+    combine)."""
+    shp = SHAPES["gemma_T130"]
+    inp = inputs.make_inputs(shp, seed=7, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=107)
+    s = api.shape_from(shp)
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s)]
+    outs = []
+    for fill in (None, 0xFF):
+        ws = api.alloc_workspace_fp8(s)
+        if fill is not None:
+            ws[256:].fill_(fill)
+        out32 = torch.empty(shp.T, shp.H, dtype=torch.float32, device="cuda")
+        out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device="cuda")
+        api.moe_forward_fp8(s, _to(inp.x), _to(inp.logits), api.fp8_experts(*wts),
+                            _to(inp.scale), out, ws, out_f32=out32, deterministic=True)
+        torch.cuda.synchronize()
+        assert api.moe_read_error(ws) == 0
+        outs.append(out32)
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_forward_fp8_captured_in_a_cuda_graph(api):
+    """One graph of the FP8 layer (fixed-order combine) replays the eager
+    result bit for bit."""
+    shp = SHAPES["shared"]
+    inp = inputs.make_inputs(shp, seed=8, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=108)
+    s = api.shape_from(shp)
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
+                            fp.sh2_q, fp.sh2_s)]
+    weights = api.fp8_experts(*wts)
+    x, z, sc = _to(inp.x), _to(inp.logits), _to(inp.scale)
+    ws = api.alloc_workspace_fp8(s)
+    ref = torch.empty(shp.T, shp.H, dtype=torch.float32, device="cuda")
+    out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device="cuda")
+    api.moe_forward_fp8(s, x, z, weights, sc, out, ws, out_f32=ref, deterministic=True)
+    torch.cuda.synchronize()
+    got = torch.zeros_like(ref)
+    st = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        api.moe_forward_fp8(s, x, z, weights, sc, out, ws, out_f32=got, deterministic=True,
+                            stream=st)
+    for _ in range(2):
+        got.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
+    del g
+    assert api.moe_read_error(ws) == 0
+
+
+def test_forward_fp8_from_hidden_states(api):
+    """moe_forward_fp8 with the router options: the logits come from the
+    residual first.  The oracle runs the FP8 layer on the GPU router's own
+    logits (moe_router_logits, checked against the oracle's router in the
+    router tests), so both take the same routing decisions."""
+    from parity_util import assert_routing_exact
+    shp = SHAPES["ragged"]
+    T, H, E = shp.T, shp.H, shp.E
+    inp = inputs.make_inputs(shp, seed=9, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=109)
+    g = torch.Generator().manual_seed(19)
+    rx, rw, rs = (t.cuda() for t in inputs.router_inputs(T, H, E, g, "cpu"))
+    s = api.shape_from(shp)
+    ws = api.alloc_workspace_fp8(s)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty(T, H, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, shp.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, shp.k, dtype=torch.float32, device="cuda")
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s)]
+    api.moe_forward_fp8(s, _to(inp.x), None, api.fp8_experts(*wts), _to(inp.scale), out,
+                        ws, ids_out=ids, w_out=w, out_f32=out32, router=(rx, rw, rs, 1e-6))
+    zg = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    api.moe_router_logits(s, rx, rw, rs, 1e-6, zg)
+    torch.cuda.synchronize()
+    assert api.moe_read_error(ws) == 0
+    zg = zg.cpu().numpy()
+    want, ids_ref, w_ref, slack = oracle.forward_fp8(
+        inp.x, zg, fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, k=shp.k, act_kind=shp.act,
+        scale=inp.scale, with_slack=True)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out32, want, "fp8 from hidden states", bf16=out, slack=slack)
