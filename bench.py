@@ -20,8 +20,8 @@ no collective on the data path (weak scaling).
 The default run (the Mixtral-shaped headline, one GPU) adds a ``configs``
 key with one entry for each other workload of the benchmark -- the
 many-small-experts and skewed prefills, the decode sweep T = 1, 4, 16, 64,
-256, and the Mixtral-shaped and many-small prefills and decode T = 16, 64
-with FP8 (e4m3) experts -- each device-timed the same way, with its roofline fraction, its
+256, and the Mixtral-shaped and many-small prefills and decode T = 4, 16,
+64 with FP8 (e4m3) experts -- each device-timed the same way, with its roofline fraction, its
 CPU baseline and ``parity``: the layer outputs the oracle computed for the
 baseline's token sample set beside the GPU's (max |err| / RMS of the fp32
 and bf16 outputs), and the routing ids, gate weights and layout of the whole
@@ -656,8 +656,9 @@ def roofline_of(args, shp, m, decode, peaks, peak_src, config_name, fp8=False):
         achieved = touched * (2.0 * shp.I * shp.H * wbytes) / (w13_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         return {"bound": "hbm",
-                "kernel": ("grouped_gemm_kernel<0, F8> (e4m3 w13 + activation)" if fp8
-                           else w13_kernel_name(decode, shp.T)),
+                "kernel": (("decode_tc_kernel<N,0,F8> (e4m3 w13 + act, tcgen05)" if decode
+                            else "grouped_gemm_kernel<0, F8> (e4m3 w13 + activation)")
+                           if fp8 else w13_kernel_name(decode, shp.T)),
                 "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": None if fp8 else
@@ -680,9 +681,9 @@ def roofline_of(args, shp, m, decode, peaks, peak_src, config_name, fp8=False):
 
 
 def launches_per_step(decode: bool, router: bool, fp8: bool = False) -> int:
-    # prefill: route, layout x4, gather, two GEMMs, rounding (FP8: and the
-    # two row quantisers); decode: route, w13, w2, row sum
-    return (4 if decode else 9) + (2 if fp8 and not decode else 0) + (1 if router else 0)
+    # prefill: route, layout x4, gather, two GEMMs, rounding; decode: route,
+    # w13, w2, row sum; FP8 adds the two row quantisers on either path
+    return (4 if decode else 9) + (2 if fp8 else 0) + (1 if router else 0)
 
 
 def run_e2e(args, api, inp, s, ws, out, stream, barrier, max_over_ranks,
@@ -809,7 +810,7 @@ def other_config_entry(args, api, inputs, name, dev, stream, peaks, peak_src):
     ws = api.alloc_workspace_fp8(s, dev) if fp8 else api.alloc_workspace(s, dev)
     out = torch.empty(shp.T, shp.H, dtype=torch.bfloat16, device=dev)
     path = api.PATH_AUTO
-    decode = shp.T <= api.DECODE_MAX_T and not fp8
+    decode = shp.T <= api.DECODE_MAX_T
     m = timed_steps(args, api, inp, s, ws, out, stream, path, None, lambda: None,
                     lambda v: v, sample_clocks_gpu=dev.index or 0, fp8=fpw)
     roof = roofline_of(args, shp, m, decode, peaks, peak_src, name, fp8=fp8)
@@ -833,8 +834,8 @@ def other_config_entry(args, api, inputs, name, dev, stream, peaks, peak_src):
 
 OTHER_CONFIGS = ("many_small_prefill", "skewed_shared_prefill", "decode_t1",
                  "decode_t4", "decode_t16", "decode_t64", "decode_t256",
-                 "mixtral_prefill+fp8", "many_small_prefill+fp8", "decode_t16+fp8",
-                 "decode_t64+fp8")
+                 "mixtral_prefill+fp8", "many_small_prefill+fp8", "decode_t4+fp8",
+                 "decode_t16+fp8", "decode_t64+fp8")
 
 
 def run_ours(args):
@@ -869,11 +870,8 @@ def run_ours(args):
             "decode": api.PATH_DECODE}[args.path]
     decode = path == api.PATH_DECODE or (path == api.PATH_AUTO
                                          and shp.T <= api.DECODE_MAX_T)
-    if args.fp8:
-        # the library runs FP8 experts on the prefill path at any T
-        if path == api.PATH_DECODE:
-            raise SystemExit("--fp8: the decode path takes bf16 experts only")
-        decode = False
+    if args.fp8 and decode and shp.T > 64:
+        raise SystemExit("--fp8: the decode path takes FP8 experts up to 64 tokens")
 
     router = None
     if args.router:

@@ -434,10 +434,12 @@ MOE_API size_t moe_workspace_size_fp8(const moe_shape* shape);
  * routing, permutation, x quantised per token and gathered, the w13
  * product (+ activation, h in bf16), h quantised per row, the w2 product
  * with the gate weights and the combine, one bf16 rounding.  Requires
- * H % 16 == 0 and I % 16 == 0 (MOE_ERR_UNSUPPORTED otherwise), a workspace
- * of moe_workspace_size_fp8 bytes (MOE_ERR_WORKSPACE) and the prefill path:
- * opts->path MOE_PATH_DECODE returns MOE_ERR_UNSUPPORTED, the others run
- * the tcgen05 grouped GEMMs at every T.  The other options (stage events,
+ * H % 16 == 0 and I % 16 == 0 (MOE_ERR_UNSUPPORTED otherwise) and a
+ * workspace of moe_workspace_size_fp8 bytes (MOE_ERR_WORKSPACE).  The decode
+ * path (MOE_PATH_DECODE, or MOE_PATH_AUTO with T <= MOE_DECODE_MAX_T) runs
+ * the decode path's tcgen05 form on the codes of the touched experts (up to
+ * 64 tokens: MOE_ERR_UNSUPPORTED beyond) and is deterministic; the prefill
+ * path runs the tcgen05 grouped GEMMs.  The other options (stage events,
  * out_f32, deterministic, cta_pairs, router, route) mean what they mean for
  * moe_forward_ex.
  */

@@ -679,6 +679,28 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, void* const* ev)
                             a.T, a.E, a.k, a.S, a.ids, a.w, a.meta, a.slots, a.route,
                             tc ? a.dt_cnt : (int32_t*)nullptr, n_zero);
   if (e != cudaSuccess) return e;
+  if (a.f8) {
+    // FP8 experts, on the tensor-core form only: the codes of x, w13 (+ act)
+    // -> h, the codes of each (group, token column) row of h, w2 -> stage
+    if (!tc) return cudaErrorInvalidValue;
+    if (!mark(1) || !mark(2)) return cudaErrorUnknown;
+    if ((e = launch_quantize_rows(a.x, a.T, a.H, a.xq, a.sx, nullptr, nullptr, st,
+                                  /*pdl=*/true)) != cudaSuccess)
+      return e;
+    if (!mark(3)) return cudaErrorUnknown;
+    if ((e = launch_decode_tc_w13(a, a.h_dec, st)) != cudaSuccess) return e;
+    const int64_t h_rows = (int64_t)(std::min(R, a.E) + a.S) * dt_columns(a.T);
+    if ((e = launch_quantize_rows(a.h_dec, h_rows, a.I, a.hq, a.sh, nullptr, nullptr, st,
+                                  /*pdl=*/true)) != cudaSuccess)
+      return e;
+    if (!mark(4)) return cudaErrorUnknown;
+    if ((e = launch_decode_tc_w2(a, a.h_dec, st)) != cudaSuccess) return e;
+    if (!mark(5)) return cudaErrorUnknown;
+    e = launch_sum_rows(a.stage, a.T, a.k + a.S, a.H, a.out, a.out_f32, st,
+                        /*pdl=*/true);
+    if (e != cudaSuccess) return e;
+    return mark(6) ? cudaSuccess : cudaErrorUnknown;
+  }
   if (!mark(1) || !mark(2) || !mark(3)) return cudaErrorUnknown;
   if (tc) {
     // tensor-core products (decode_tc.cu): h in [touched, N, I] order

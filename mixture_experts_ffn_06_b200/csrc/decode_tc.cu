@@ -67,6 +67,11 @@ struct DtParams {
   float* stage;          // MODE 1 out: [T*(k+S)][H]
   float* part;           // [2 * gridDim.x][128][T] partial sums
   int32_t* cnt;          // [touched * RB] arrival counters, zero on entry
+  // FP8: weight row scales (routed, shared) and the B rows' scales (x's per
+  // token, or h's per group and token column)
+  const float* ascale;
+  const float* ascale_sh;
+  const float* bscale;
   uint32_t* err;
   uint64_t timeout_ns;
 };
@@ -146,13 +151,15 @@ __device__ __forceinline__ DtRange dt_range(int n_groups, int RB, int KB) {
   return r;
 }
 
-template <int N, int MODE>
+template <int N, int MODE, bool F8>
 __global__ void __launch_bounds__(kDtThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                  const __grid_constant__ CUtensorMap tmAs,
                  const __grid_constant__ CUtensorMap tmB, const DtParams p) {
   using C = DtCfg<N>;
   constexpr int ST = C::STAGES;
+  // a k-block is 128 bytes of each row: 64 bf16 values or 128 e4m3 codes
+  constexpr int KBE = F8 ? 128 : 64;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -201,7 +208,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool routed = g < p.E;
       const uint32_t fb = smem_u32(&ctl->full[j]);
       mbar_expect_tx(fb, C::A_STAGE + C::B_STAGE);
-      tma_load_2d(sA + j * C::A_STAGE, routed ? &tmA : &tmAs, kb * 64,
+      tma_load_2d(sA + j * C::A_STAGE, routed ? &tmA : &tmAs, kb * KBE,
                   (routed ? g : g - p.E) * p.H + rb * 128, fb);
     }
   }
@@ -241,7 +248,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t fb = smem_u32(&ctl->full[stage]);
           if (it0 + (kb - kb0) - s0 < pre) {
             // weights already requested before the wait: only h is left
-            tma_load_2d(sB + stage * C::B_STAGE, &tmB, kb * 64, br, fb);
+            tma_load_2d(sB + stage * C::B_STAGE, &tmB, kb * KBE, br, fb);
           } else {
             if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
                            p.timeout_ns, p.err)) {
@@ -250,11 +257,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             mbar_expect_tx(fb, C::A_STAGE + C::B_STAGE);
             const uint32_t a_dst = sA + stage * C::A_STAGE;
-            tma_load_2d(a_dst, ma, kb * 64, ar, fb);
+            tma_load_2d(a_dst, ma, kb * KBE, ar, fb);
             // w13: the up rows matching the gate rows, I rows further on
             if (MODE == 0)
-              tma_load_2d(a_dst + C::A_STAGE / 2, ma, kb * 64, ar + p.I, fb);
-            tma_load_2d(sB + stage * C::B_STAGE, &tmB, kb * 64, br, fb);
+              tma_load_2d(a_dst + C::A_STAGE / 2, ma, kb * KBE, ar + p.I, fb);
+            tma_load_2d(sB + stage * C::B_STAGE, &tmB, kb * KBE, br, fb);
           }
           last_fill[stage] = (int32_t)phase;
           if (++stage == ST) { stage = 0; phase ^= 1u; }
@@ -273,7 +280,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, N);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int it = s0; ok && it < s1;) {
@@ -299,7 +306,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint64_t bd = sw128_kmajor_desc(sB + stage * C::B_STAGE);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(d, ad + 2u * kk, bd + 2u * kk, idesc,
+            umma<F8>(d, ad + 2u * kk, bd + 2u * kk, idesc,
                       (kb != kb0 || kk != 0) ? 1u : 0u);
           umma_commit(smem_u32(&ctl->empty[stage]));
           if (++stage == ST) { stage = 0; phase ^= 1u; }
@@ -420,6 +427,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
 
+      if (F8) {
+        // the accumulator of codes times this row's weight scale and each
+        // column's scale (x: per token; h: per group and token column)
+        const int g = __ldg(p.meta + 1 + i);
+        const bool routed = g < p.E;
+        const int gl = routed ? g : g - p.E;
+        const float* as = routed ? p.ascale : p.ascale_sh;
+        float sa = 0.0f;
+        if (MODE == 0) {
+          const int r = rb * 64 + (row & 63);  // row of I (gate or up half)
+          if (r < p.I) sa = __ldg(as + (int64_t)gl * 2 * p.I + (row >= 64 ? p.I : 0) + r);
+        } else {
+          const int r = rb * 128 + row;  // row of H
+          if (r < p.H) sa = __ldg(as + (int64_t)gl * p.H + r);
+        }
+#pragma unroll
+        for (int c = 0; c < N; ++c) {
+          float sb = 0.0f;
+          if (MODE == 0) {
+            if (c < p.T) sb = __ldg(p.bscale + c);
+          } else {
+            sb = __ldg(p.bscale + (int64_t)i * N + c);
+          }
+          v[c] *= sa * sb;
+        }
+      }
       if (MODE == 0 && row >= 64) {
 #pragma unroll
         for (int c = 0; c < N; ++c) xch[row - 64][c] = v[c];
@@ -463,25 +496,29 @@ constexpr size_t dt_smem_bytes() {
          64 * (N + 1) * sizeof(float) + sizeof(DtCtl);
 }
 
-template <int N, int MODE>
+template <int N, int MODE, bool F8>
 cudaError_t launch_dt(const DecodeArgs& a, const void* b_ptr, void* out,
                       cudaStream_t st) {
   const int G = a.E + a.S;
   const int n_max = std::min(a.T * a.k, a.E) + a.S;  // touched groups, at most
+  constexpr int KBE = F8 ? 128 : 64;
+  auto map = F8 ? make_tma_map_e4m3 : make_tma_map_bf16;
+  const void* wa = MODE == 0 ? (F8 ? (const void*)a.w13q : (const void*)a.w13)
+                             : (F8 ? (const void*)a.w2q : (const void*)a.w2);
+  const void* wa_sh = MODE == 0 ? (F8 ? (const void*)a.w13q_sh : (const void*)a.w13_sh)
+                                : (F8 ? (const void*)a.w2q_sh : (const void*)a.w2_sh);
   CUtensorMap mA, mAs, mB;
   cudaError_t e;
   if (MODE == 0) {
-    e = make_tma_map_bf16(&mA, a.w13, a.H, 2ull * a.I * a.E, 64);
+    e = map(&mA, wa, a.H, 2ull * a.I * a.E, 64);
     if (e == cudaSuccess)
-      e = a.S ? make_tma_map_bf16(&mAs, a.w13_sh, a.H, 2ull * a.I * a.S, 64)
-              : (mAs = mA, cudaSuccess);
-    if (e == cudaSuccess) e = make_tma_map_bf16(&mB, b_ptr, a.H, a.T, N);
+      e = a.S ? map(&mAs, wa_sh, a.H, 2ull * a.I * a.S, 64) : (mAs = mA, cudaSuccess);
+    if (e == cudaSuccess) e = map(&mB, b_ptr, a.H, a.T, N);
   } else {
-    e = make_tma_map_bf16(&mA, a.w2, a.I, (uint64_t)a.H * a.E, 128);
+    e = map(&mA, wa, a.I, (uint64_t)a.H * a.E, 128);
     if (e == cudaSuccess)
-      e = a.S ? make_tma_map_bf16(&mAs, a.w2_sh, a.I, (uint64_t)a.H * a.S, 128)
-              : (mAs = mA, cudaSuccess);
-    if (e == cudaSuccess) e = make_tma_map_bf16(&mB, b_ptr, a.I, (uint64_t)n_max * N, N);
+      e = a.S ? map(&mAs, wa_sh, a.I, (uint64_t)a.H * a.S, 128) : (mAs = mA, cudaSuccess);
+    if (e == cudaSuccess) e = map(&mB, b_ptr, a.I, (uint64_t)n_max * N, N);
   }
   if (e != cudaSuccess) return e;
   DtParams p;
@@ -495,7 +532,7 @@ cudaError_t launch_dt(const DecodeArgs& a, const void* b_ptr, void* out,
   p.G = G;
   p.H = a.H;
   p.I = a.I;
-  p.KB = MODE == 0 ? (a.H + 63) / 64 : (a.I + 63) / 64;
+  p.KB = MODE == 0 ? (a.H + KBE - 1) / KBE : (a.I + KBE - 1) / KBE;
   p.RB = MODE == 0 ? (a.I + 63) / 64 : (a.H + 127) / 128;
   p.act = a.act;
   p.h = MODE == 0 ? static_cast<__nv_bfloat16*>(out) : nullptr;
@@ -504,17 +541,20 @@ cudaError_t launch_dt(const DecodeArgs& a, const void* b_ptr, void* out,
   p.cnt = a.dt_cnt + (MODE == 0 ? 0 : (size_t)G * dt_row_blocks(a.H, a.I));
   p.err = a.err;
   p.timeout_ns = kDtTimeoutNs;
+  p.ascale = F8 ? (MODE == 0 ? a.w13s : a.w2s) : nullptr;
+  p.ascale_sh = F8 ? (MODE == 0 ? a.w13s_sh : a.w2s_sh) : nullptr;
+  p.bscale = F8 ? (MODE == 0 ? a.sx : a.sh) : nullptr;
   constexpr size_t smem = dt_smem_bytes<N>();
-  e = cudaFuncSetAttribute(decode_tc_kernel<N, MODE>,
+  e = cudaFuncSetAttribute(decode_tc_kernel<N, MODE, F8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   static_assert(2 * (smem + 1024) <= 228 * 1024, "two CTAs per SM");
-  e = cudaFuncSetAttribute(decode_tc_kernel<N, MODE>,
+  e = cudaFuncSetAttribute(decode_tc_kernel<N, MODE, F8>,
                            cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int grid = std::min(kDtMaxCtas, 2 * device_sm_count());
-  return launch_ex(decode_tc_kernel<N, MODE>, dim3(grid), dim3(kDtThreads), smem, st,
+  return launch_ex(decode_tc_kernel<N, MODE, F8>, dim3(grid), dim3(kDtThreads), smem, st,
                    true, mA, mAs, mB, p);
 }
 
@@ -522,18 +562,32 @@ cudaError_t launch_dt(const DecodeArgs& a, const void* b_ptr, void* out,
 
 int dt_row_blocks(int H, int I) { return std::max((I + 63) / 64, (H + 127) / 128); }
 
+int dt_columns(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : 64; }
+
 cudaError_t launch_decode_tc_w13(const DecodeArgs& a, __nv_bfloat16* h_dense,
                                  cudaStream_t st) {
-  if (a.T <= 16) return launch_dt<16, 0>(a, a.x, h_dense, st);
-  if (a.T <= 32) return launch_dt<32, 0>(a, a.x, h_dense, st);
-  return launch_dt<64, 0>(a, a.x, h_dense, st);
+  // B: the token rows of x (bf16), or their e4m3 codes
+  if (a.f8) {
+    if (a.T <= 16) return launch_dt<16, 0, true>(a, a.xq, h_dense, st);
+    if (a.T <= 32) return launch_dt<32, 0, true>(a, a.xq, h_dense, st);
+    return launch_dt<64, 0, true>(a, a.xq, h_dense, st);
+  }
+  if (a.T <= 16) return launch_dt<16, 0, false>(a, a.x, h_dense, st);
+  if (a.T <= 32) return launch_dt<32, 0, false>(a, a.x, h_dense, st);
+  return launch_dt<64, 0, false>(a, a.x, h_dense, st);
 }
 
 cudaError_t launch_decode_tc_w2(const DecodeArgs& a, const __nv_bfloat16* h_dense,
                                 cudaStream_t st) {
-  if (a.T <= 16) return launch_dt<16, 1>(a, h_dense, a.stage, st);
-  if (a.T <= 32) return launch_dt<32, 1>(a, h_dense, a.stage, st);
-  return launch_dt<64, 1>(a, h_dense, a.stage, st);
+  // B: h [touched * N, I] (bf16), or its e4m3 codes
+  if (a.f8) {
+    if (a.T <= 16) return launch_dt<16, 1, true>(a, a.hq, a.stage, st);
+    if (a.T <= 32) return launch_dt<32, 1, true>(a, a.hq, a.stage, st);
+    return launch_dt<64, 1, true>(a, a.hq, a.stage, st);
+  }
+  if (a.T <= 16) return launch_dt<16, 1, false>(a, h_dense, a.stage, st);
+  if (a.T <= 32) return launch_dt<32, 1, false>(a, h_dense, a.stage, st);
+  return launch_dt<64, 1, false>(a, h_dense, a.stage, st);
 }
 
 }  // namespace moe

@@ -845,6 +845,11 @@ cudaError_t make_tma_map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner,
   return make_map(m, ptr, inner, outer, box_rows);
 }
 
+cudaError_t make_tma_map_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner,
+                              uint64_t outer, uint32_t box_rows) {
+  return make_map(m, ptr, inner, outer, box_rows, /*f8=*/true);
+}
+
 int device_sm_count() { return num_sms(); }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,

@@ -150,6 +150,15 @@ struct DecodeArgs {
   float* dt_part;        // [2 * kDtMaxCtas, 128, T] fp32 partial sums
   int32_t* dt_cnt;       // [2, G * dt_row_blocks] arrival counters
   uint32_t* err;         // error word
+  // FP8 experts (the tensor-core form only): e4m3 codes with one fp32 scale
+  // per output row, x and h quantised per row on the way
+  bool f8;
+  const uint8_t *w13q, *w2q, *w13q_sh, *w2q_sh;
+  const float *w13s, *w2s, *w13s_sh, *w2s_sh;
+  uint8_t* xq;           // [T,H] codes of x, scales sx [T]
+  float* sx;
+  uint8_t* hq;           // [touched * N, I] codes of h, scales sh [touched * N]
+  float* sh;
 };
 size_t decode_meta_ints(int G);
 
@@ -159,6 +168,8 @@ constexpr int kDecodeFewMaxT = 8;   // the skinny kernels' one-B-tile form
 constexpr int kDtMaxCtas = 2 * 160;  // persistent CTAs: up to 2 per SM
 // row blocks of one group: max(ceil(I / 64), ceil(H / 128))
 int dt_row_blocks(int H, int I);
+// token columns N of the tensor-core form for T tokens: 16, 32 or 64
+int dt_columns(int T);
 // kernels of the tensor-core form: w13 (+ act) -> h, w2 (x gate weight) -> stage.
 // meta / slots come from decode_route; h_dense [touched groups * N, I] bf16.
 cudaError_t launch_decode_tc_w13(const DecodeArgs& a, __nv_bfloat16* h_dense,
@@ -215,6 +226,9 @@ cudaError_t launch_wait_selftest(uint32_t* err, uint32_t timeout_us,
 // TMA map of a row-major bf16 [outer, inner] tensor: box {64, box_rows},
 // 128-byte swizzle, out-of-range elements read as zero (gemm_tc.cu).
 cudaError_t make_tma_map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner,
+                              uint64_t outer, uint32_t box_rows);
+// The same for a row-major tensor of e4m3 bytes: box {128, box_rows}.
+cudaError_t make_tma_map_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner,
                               uint64_t outer, uint32_t box_rows);
 // SMs of the current device (cached per device).
 int device_sm_count();

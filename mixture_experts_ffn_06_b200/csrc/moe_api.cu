@@ -483,8 +483,10 @@ moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x, const floa
   }
   if (opts && (opts->cta_pairs < 0 || opts->cta_pairs > 2)) return MOE_ERR_INVALID_ARG;
   const int path = opts ? opts->path : MOE_PATH_AUTO;
-  if (path == MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_PREFILL && path != MOE_PATH_DECODE)
+    return MOE_ERR_INVALID_ARG;
+  // the decode path takes FP8 experts on its tensor-core form: up to 64 tokens
+  if (path == MOE_PATH_DECODE && s.T > kDecodeTcMaxT) return MOE_ERR_UNSUPPORTED;
   RouteOpt ro;
   if ((st = check_route_opts(s, opts ? opts->route : nullptr, &ro)) != MOE_OK) return st;
   if (!ws) return MOE_ERR_INVALID_ARG;
@@ -516,6 +518,60 @@ moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x, const floa
   const bool det = opts && opts->deterministic;
   const int cta_pairs = opts ? opts->cta_pairs : 0;
   if (use_router) logits = reinterpret_cast<float*>(at(ws, m.logits));
+
+  if (path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && s.T <= kDecodeMaxT)) {
+    // few tokens: stream only the touched experts' codes (decode.cu,
+    // decode_tc.cu).  Stage 0: router and routing; 2: the codes of x;
+    // 3: w13 + activation and the codes of h; 4: w2; 5: the row sum.
+    DecodeArgs d{};
+    d.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    d.logits = logits;
+    d.scale = scale;
+    d.T = (int)s.T;
+    d.H = s.H;
+    d.E = s.E;
+    d.k = s.k;
+    d.I = s.I;
+    d.S = s.n_shared;
+    d.act = s.act;
+    d.route = ro;
+    d.ids = ids;
+    d.w = w;
+    d.meta = reinterpret_cast<int32_t*>(at(ws, m.dec_meta));
+    d.slots = sorted_slots;
+    d.h_dec = h;
+    d.stage = stage;
+    d.out = reinterpret_cast<__nv_bfloat16*>(out);
+    d.out_f32 = opts ? opts->out_f32 : nullptr;
+    d.tc = true;
+    d.dt_part = reinterpret_cast<float*>(at(ws, m.dt_part));
+    d.dt_cnt = reinterpret_cast<int32_t*>(at(ws, m.dt_cnt));
+    d.err = err;
+    d.f8 = true;
+    d.w13q = wq->w13;
+    d.w2q = wq->w2;
+    d.w13q_sh = wq->w13_sh;
+    d.w2q_sh = wq->w2_sh;
+    d.w13s = wq->w13_scale;
+    d.w2s = wq->w2_scale;
+    d.w13s_sh = wq->w13_sh_scale;
+    d.w2s_sh = wq->w2_sh_scale;
+    d.xq = xq;
+    d.sx = sx;
+    d.hq = hq;
+    d.sh = sh;
+    if (!use_router) return from_cuda(launch_decode(d, stream, ev));
+    void* dev[MOE_NUM_STAGES + 1] = {};
+    for (int i = 1; ev && i <= MOE_NUM_STAGES; ++i) dev[i] = ev[i];
+    if (!mark(ev, 0, stream)) return MOE_ERR_CUDA;
+    if (launch_router_logits(reinterpret_cast<const __nv_bfloat16*>(opts->router_x),
+                             reinterpret_cast<const __nv_bfloat16*>(opts->router_w),
+                             reinterpret_cast<const __nv_bfloat16*>(opts->router_scale),
+                             s.T, s.H, s.E, opts->router_eps, const_cast<float*>(logits),
+                             stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return from_cuda(launch_decode(d, stream, ev ? dev : nullptr));
+  }
 
   // stage 0: router (if any) and routing; 1: layout; 2: the codes of x and
   // their gather; 3: w13 + activation; 4: the codes of h and w2 + combine;

@@ -221,7 +221,7 @@ def test_fp8_entry_points_refuse_bad_arguments(api):
     s8 = api.make_shape(T=8, H=72, E=4, k=2, I=64)
     assert lib.moe_forward_fp8(ctypes.byref(s8), fake, fake, ctypes.byref(w), None, fake,
                                None, None, fake, 1 << 40, ctypes.byref(opts), null) == 2
-    # missing weights, small workspace, the decode path
+    # missing weights, small workspace, the decode path past 64 tokens
     w_bad = api.moe_fp8_experts(fake, None, fake, fake, None, None, None, None)
     assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w_bad), None,
                                fake, None, None, ctypes.c_void_p(1 << 20), ws_n,
@@ -231,6 +231,7 @@ def test_fp8_entry_points_refuse_bad_arguments(api):
                                ctypes.byref(opts), null) == 3
     dec = api.moe_forward_opts()
     dec.path = api.PATH_DECODE
-    assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w), None, fake,
-                               None, None, ctypes.c_void_p(1 << 20), ws_n,
-                               ctypes.byref(dec), null) == 2
+    s65 = api.make_shape(T=65, H=64, E=4, k=2, I=64)
+    assert lib.moe_forward_fp8(ctypes.byref(s65), fake, fake, ctypes.byref(w), None, fake,
+                               None, None, ctypes.c_void_p(1 << 20),
+                               api.moe_workspace_size_fp8(s65), ctypes.byref(dec), null) == 2

@@ -114,3 +114,4 @@ def test_launches_per_step_follows_the_path():
     assert bench.launches_per_step(False, False) == 9
     assert bench.launches_per_step(False, True) == 10
     assert bench.launches_per_step(False, False, fp8=True) == 11
+    assert bench.launches_per_step(True, False, fp8=True) == 6

@@ -109,8 +109,41 @@ def test_forward_fp8_every_element(api, name, variant):
     assert_out_close(out32, want, f"{name} fp8 ({variant})", bf16=out, slack=slack)
 
 
-def test_forward_fp8_refuses_the_decode_path(api):
-    shp = SHAPES["one_token"]
+DECODE_SHAPES = {
+    "one_token": SHAPES["one_token"],                        # N = 16
+    "few": inputs.Shape(T=5, H=208, E=5, k=3, I=112, act=1),  # K and row tails
+    "gemma_T16": inputs.Shape(T=16, H=2816, E=128, k=8, I=704, act=1),
+    "ragged": SHAPES["ragged"],                              # N = 64, T = 37
+    "shared": SHAPES["shared"],                              # 2 shared experts
+    "T64": inputs.Shape(T=64, H=256, E=8, k=2, I=128),       # N = 64, split units
+}
+
+
+@pytest.mark.parametrize("name", list(DECODE_SHAPES))
+def test_forward_fp8_decode_path_every_element(api, name):
+    """The decode path's tensor-core form with e4m3 weights: x and each
+    (expert, token) row of h quantised per row, the scales applied after the
+    split units' fixed-order reduction."""
+    shp = DECODE_SHAPES[name]
+    inp = inputs.make_inputs(shp, seed=10, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=110)
+    want, ids_ref, w_ref, slack = _oracle_fp8(inp, fp)
+    out, out32, ids, w = _gpu_fp8(api, inp, fp, path=api.PATH_DECODE)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out32, want, f"{name} fp8 decode", bf16=out, slack=slack)
+
+
+def test_forward_fp8_decode_path_is_deterministic(api):
+    shp = DECODE_SHAPES["gemma_T16"]
+    inp = inputs.make_inputs(shp, seed=11, scale="uniform")
+    fp = inputs.fp8_experts(shp, seed=111)
+    a = _gpu_fp8(api, inp, fp, path=api.PATH_DECODE)
+    b = _gpu_fp8(api, inp, fp, path=api.PATH_DECODE)
+    assert torch.equal(a[1], b[1])
+
+
+def test_forward_fp8_refuses_the_decode_path_past_64_tokens(api):
+    shp = inputs.Shape(T=65, H=128, E=8, k=2, I=128)
     inp = inputs.make_inputs(shp, seed=1)
     fp = inputs.fp8_experts(shp, seed=2)
     with pytest.raises(api.MoEError) as e:
@@ -176,7 +209,7 @@ class _Guarded:
             bool((self.raw[BAND + self.n:] == PATTERN).all())
 
 
-@pytest.mark.parametrize("variant", list(VARIANTS))
+@pytest.mark.parametrize("variant", list(VARIANTS) + ["decode"])
 @pytest.mark.parametrize("name", ["ragged", "shared", "gemma_T130", "pairs"])
 def test_forward_fp8_writes_only_its_buffers(api, name, variant):
     shp = SHAPES[name]
@@ -192,11 +225,15 @@ def test_forward_fp8_writes_only_its_buffers(api, name, variant):
     ws.t[:256].zero_()
     wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
                             fp.sh2_q, fp.sh2_s)]
-    det, pairs = VARIANTS[variant]
+    if variant == "decode" and T > 64:
+        pytest.skip("the decode path takes FP8 experts up to 64 tokens")
+    det, pairs = VARIANTS.get(variant, (False, 0))
+    path = api.PATH_DECODE if variant == "decode" else 0
     for _ in range(2):  # the second call finds the first call's workspace
         api.moe_forward_fp8(s, _to(inp.x), _to(inp.logits), api.fp8_experts(*wts),
                             _to(inp.scale), out.t, ws.t, ids_out=ids.t, w_out=w.t,
-                            out_f32=out32.t, deterministic=det, cta_pairs=pairs)
+                            out_f32=out32.t, deterministic=det, cta_pairs=pairs,
+                            path=path)
     assert api.moe_read_error(ws.t) == 0
     assert torch.isfinite(out32.t).all()
     for nm, g in (("out", out), ("out_f32", out32), ("ids", ids), ("w", w),
