@@ -472,8 +472,14 @@ moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x, const floa
   if (s.n_shared > 0 && (!wq->w13_sh || !wq->w13_sh_scale || !wq->w2_sh ||
                          !wq->w2_sh_scale))
     return MOE_ERR_INVALID_ARG;
+  // the codes are TMA tiles and x is read in 16-byte vectors: both need
+  // 16-byte aligned bases
+  if (!aligned16(wq->w13) || !aligned16(wq->w2) ||
+      (s.n_shared > 0 && (!aligned16(wq->w13_sh) || !aligned16(wq->w2_sh))))
+    return MOE_ERR_INVALID_ARG;
   const bool use_router = opts && opts->router_w;
   if (s.T > 0 && (!x || (!logits && !use_router) || !out)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !aligned16(x)) return MOE_ERR_INVALID_ARG;
   if (use_router) {
     if (!(opts->router_eps >= 0.0f) || !std::isfinite(opts->router_eps))
       return MOE_ERR_INVALID_ARG;

@@ -229,6 +229,15 @@ def test_fp8_entry_points_refuse_bad_arguments(api):
     assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w), None, fake,
                                None, None, ctypes.c_void_p(1 << 20), ws_n - 256,
                                ctypes.byref(opts), null) == 3
+    # codes and x not 16-byte aligned
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    w_odd = api.moe_fp8_experts(fake, fake, odd, fake, None, None, None, None)
+    assert lib.moe_forward_fp8(ctypes.byref(s), fake, fake, ctypes.byref(w_odd), None,
+                               fake, None, None, ctypes.c_void_p(1 << 20), ws_n,
+                               ctypes.byref(opts), null) == 1
+    assert lib.moe_forward_fp8(ctypes.byref(s), odd, fake, ctypes.byref(w), None, fake,
+                               None, None, ctypes.c_void_p(1 << 20), ws_n,
+                               ctypes.byref(opts), null) == 1
     dec = api.moe_forward_opts()
     dec.path = api.PATH_DECODE
     s65 = api.make_shape(T=65, H=64, E=4, k=2, I=64)

@@ -92,6 +92,7 @@ SHAPES = {
     "gemma_T130": inputs.Shape(T=130, H=2816, E=128, k=8, I=704, act=1),  # narrow tiles
     "pairs": inputs.Shape(T=700, H=208, E=3, k=2, I=112, act=1),
     "pairs_wide_I": inputs.Shape(T=600, H=128, E=2, k=2, I=1024),
+    "few_shared": inputs.Shape(T=3, H=208, E=6, k=2, I=96, n_shared=2, I_shared=96),
 }
 VARIANTS = {"fast": (False, 0), "det": (True, 0), "pairs": (False, 2)}
 
@@ -112,6 +113,9 @@ def test_forward_fp8_every_element(api, name, variant):
 DECODE_SHAPES = {
     "one_token": SHAPES["one_token"],                        # N = 16
     "few": inputs.Shape(T=5, H=208, E=5, k=3, I=112, act=1),  # K and row tails
+    "few_shared": SHAPES["few_shared"],                      # 2 shared experts, T = 3
+    "eight": inputs.Shape(T=8, H=1024, E=16, k=4, I=320),    # N = 16
+    "nine": inputs.Shape(T=9, H=1024, E=16, k=4, I=320),     # N = 16
     "gemma_T16": inputs.Shape(T=16, H=2816, E=128, k=8, I=704, act=1),
     "ragged": SHAPES["ragged"],                              # N = 64, T = 37
     "shared": SHAPES["shared"],                              # 2 shared experts
@@ -133,8 +137,24 @@ def test_forward_fp8_decode_path_every_element(api, name):
     assert_out_close(out32, want, f"{name} fp8 decode", bf16=out, slack=slack)
 
 
-def test_forward_fp8_decode_path_is_deterministic(api):
-    shp = DECODE_SHAPES["gemma_T16"]
+@pytest.mark.parametrize("name", ["decode_t1", "decode_t4", "decode_t16", "decode_t64"])
+def test_forward_fp8_decode_sweep_every_element(api, name):
+    """The decode sweep's shapes (H=2816, E=128, k=8, I=704, tanh-GELU) with
+    FP8 experts, on the path the layer picks by itself: the tensor-core
+    decode form up to 16 tokens, the prefill GEMMs above.  Every output
+    element against the oracle."""
+    shp = inputs.shape_of(name)
+    inp = inputs.make_inputs(name, seed=0, device="cuda")
+    fp = inputs.fp8_experts(shp, seed=1, device="cuda")
+    out, out32, ids, w = _gpu_fp8(api, inp, fp)
+    want, ids_ref, w_ref, slack = _oracle_fp8(inp, fp)
+    assert_routing_exact(ids, w, ids_ref, w_ref)
+    assert_out_close(out32, want, f"{name} fp8", bf16=out, slack=slack)
+
+
+@pytest.mark.parametrize("name", ["gemma_T16", "eight"])
+def test_forward_fp8_decode_path_is_deterministic(api, name):
+    shp = DECODE_SHAPES[name]
     inp = inputs.make_inputs(shp, seed=11, scale="uniform")
     fp = inputs.fp8_experts(shp, seed=111)
     a = _gpu_fp8(api, inp, fp, path=api.PATH_DECODE)
@@ -210,7 +230,7 @@ class _Guarded:
 
 
 @pytest.mark.parametrize("variant", list(VARIANTS) + ["decode"])
-@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_T130", "pairs"])
+@pytest.mark.parametrize("name", ["ragged", "shared", "gemma_T130", "pairs", "few_shared"])
 def test_forward_fp8_writes_only_its_buffers(api, name, variant):
     shp = SHAPES[name]
     inp = inputs.make_inputs(shp, seed=6, scale="uniform")
@@ -241,15 +261,17 @@ def test_forward_fp8_writes_only_its_buffers(api, name, variant):
         assert g.intact(), f"{nm}: a guard band was overwritten"
 
 
-def test_forward_fp8_stale_workspace_changes_nothing(api):
+@pytest.mark.parametrize("name", ["gemma_T130", "few_shared"])
+def test_forward_fp8_stale_workspace_changes_nothing(api, name):
     """A workspace full of 0xFF bytes (NaN in bf16 and fp32, -1 as an index)
     past its zeroed header gives the same bits as a clean one (fixed-order
-    combine)."""
-    shp = SHAPES["gemma_T130"]
+    combine; the decode path at 3 tokens)."""
+    shp = SHAPES[name]
     inp = inputs.make_inputs(shp, seed=7, scale="uniform")
     fp = inputs.fp8_experts(shp, seed=107)
     s = api.shape_from(shp)
-    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s)]
+    wts = [_to(t) for t in (fp.w13_q, fp.w13_s, fp.w2_q, fp.w2_s, fp.sh13_q, fp.sh13_s,
+                            fp.sh2_q, fp.sh2_s)]
     outs = []
     for fill in (None, 0xFF):
         ws = api.alloc_workspace_fp8(s)
@@ -265,10 +287,11 @@ def test_forward_fp8_stale_workspace_changes_nothing(api):
     assert torch.equal(outs[0], outs[1])
 
 
-def test_forward_fp8_captured_in_a_cuda_graph(api):
-    """One graph of the FP8 layer (fixed-order combine) replays the eager
-    result bit for bit."""
-    shp = SHAPES["shared"]
+@pytest.mark.parametrize("name", ["shared", "few_shared"])
+def test_forward_fp8_captured_in_a_cuda_graph(api, name):
+    """One graph of the FP8 layer (fixed-order combine; the decode path at 3
+    tokens) replays the eager result bit for bit."""
+    shp = SHAPES[name]
     inp = inputs.make_inputs(shp, seed=8, scale="uniform")
     fp = inputs.fp8_experts(shp, seed=108)
     s = api.shape_from(shp)
