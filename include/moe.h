@@ -26,7 +26,10 @@
  *     memory, frees or synchronises (except moe_read_error, which says so);
  *     moe_gemma4_block creates one CUDA stream and two events per device on
  *     its first call there and keeps them.
- *   - Buffers are dense, row-major and 16-byte aligned.
+ *   - Buffers are dense, row-major and 16-byte aligned.  The layer entry
+ *     points (moe_expert_ffn, moe_forward, moe_forward_ex, moe_forward_fp8,
+ *     moe_gemma4_block) check it for the token rows and the weights and
+ *     return MOE_ERR_INVALID_ARG otherwise.
  *   - bf16 data is passed as uint16_t bit patterns (moe_bf16).
  *   - Work is enqueued on ``stream`` and runs asynchronously.
  *   - Argument and shape errors are returned before anything is launched.

@@ -227,6 +227,11 @@ moe_status moe_gemma4_block(const moe_shape* shape, const moe_bf16* x,
     return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < 5; ++i)
     if (!p->norm_w[i] || !aligned16(p->norm_w[i])) return MOE_ERR_INVALID_ARG;
+  // what the two layer calls below would refuse, refused before anything is
+  // launched: rows and weights read in 16-byte vectors or TMA tiles
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(p->mlp_w13) ||
+      !aligned16(p->mlp_w2) || !aligned16(p->router_w) || !aligned16(p->router_scale))
+    return MOE_ERR_INVALID_ARG;
   const BlockWs m = block_ws(s, p->I_dense);
   uint8_t* base = static_cast<uint8_t*>(ws);
   auto* a1 = reinterpret_cast<__nv_bfloat16*>(base + m.a1);

@@ -191,6 +191,11 @@ size_t moe_workspace_size(const moe_shape* shape) {
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool weights_aligned(const moe_shape& s, const void* w13, const void* w2,
+                            const void* w13_sh, const void* w2_sh) {
+  return aligned16(w13) && aligned16(w2) &&
+         (s.n_shared == 0 || (aligned16(w13_sh) && aligned16(w2_sh)));
+}
 
 moe_status moe_router_logits(const moe_shape* shape, const moe_bf16* x,
                              const moe_bf16* w_router, const moe_bf16* scale, float eps,
@@ -278,8 +283,11 @@ moe_status moe_expert_ffn(const moe_shape* shape, const moe_bf16* x,
       (shape->T > 0 && !x))
     return MOE_ERR_INVALID_ARG;
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
-  // y_perm rows are written by 16-byte bulk copies
-  if (!aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  // y_perm rows are written by 16-byte bulk copies; the weights are TMA
+  // tiles and x is read in 16-byte vectors
+  if (!aligned16(y_perm) || !weights_aligned(*shape, w13, w2, w13_sh, w2_sh) ||
+      (shape->T > 0 && !aligned16(x)))
+    return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   return run_expert_ffn(*shape, reinterpret_cast<const __nv_bfloat16*>(x), offsets,
@@ -323,6 +331,9 @@ moe_status moe_forward_ex(const moe_shape* shape, const moe_bf16* x,
       return MOE_ERR_INVALID_ARG;
   }
   if (shape->n_shared > 0 && (!w13_sh || !w2_sh)) return MOE_ERR_INVALID_ARG;
+  // the weights are TMA tiles or 16-byte copies, x is read in 16-byte vectors
+  if (!weights_aligned(*shape, w13, w2, w13_sh, w2_sh) || (shape->T > 0 && !aligned16(x)))
+    return MOE_ERR_INVALID_ARG;
   RouteOpt ro;
   if ((st = check_route_opts(*shape, opts ? opts->route : nullptr, &ro)) != MOE_OK)
     return st;
@@ -474,9 +485,7 @@ moe_status moe_forward_fp8(const moe_shape* shape, const moe_bf16* x, const floa
     return MOE_ERR_INVALID_ARG;
   // the codes are TMA tiles and x is read in 16-byte vectors: both need
   // 16-byte aligned bases
-  if (!aligned16(wq->w13) || !aligned16(wq->w2) ||
-      (s.n_shared > 0 && (!aligned16(wq->w13_sh) || !aligned16(wq->w2_sh))))
-    return MOE_ERR_INVALID_ARG;
+  if (!weights_aligned(s, wq->w13, wq->w2, wq->w13_sh, wq->w2_sh)) return MOE_ERR_INVALID_ARG;
   const bool use_router = opts && opts->router_w;
   if (s.T > 0 && (!x || (!logits && !use_router) || !out)) return MOE_ERR_INVALID_ARG;
   if (s.T > 0 && !aligned16(x)) return MOE_ERR_INVALID_ARG;

@@ -200,6 +200,40 @@ def test_gemma4_block_refuses_bad_arguments(api):
              need, None) == 1                                # a gamma missing
     assert f(ctypes.byref(sh), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
              need, None) == 2                                # shared experts
+    prm.norm_w[2] = 1 << 20
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert f(ctypes.byref(s), odd, ctypes.byref(prm), fake, fake, None, fake, None, ws,
+             need, None) == 1                                # x not 16-byte aligned
+    prm.mlp_w13 = odd.value
+    assert f(ctypes.byref(s), fake, ctypes.byref(prm), fake, fake, None, fake, None, ws,
+             need, None) == 1                                # a weight not aligned
+
+
+def test_layer_refuses_unaligned_rows_and_weights(api):
+    # rejected on the host before any launch: no GPU needed
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    null = ctypes.c_void_p(0)
+    lib = api.lib
+    s = _shape(api)
+    need = api.moe_workspace_size(s)
+    ws = ctypes.c_void_p(1 << 21)
+    fwd = lib.moe_forward_ex
+    assert fwd(ctypes.byref(s), fake, fake, odd, fake, null, null, null, fake, null, null,
+               ws, need, None, None) == 1                    # w13
+    assert fwd(ctypes.byref(s), fake, fake, fake, odd, null, null, null, fake, null, null,
+               ws, need, None, None) == 1                    # w2
+    assert fwd(ctypes.byref(s), odd, fake, fake, fake, null, null, null, fake, null, null,
+               ws, need, None, None) == 1                    # x
+    sh = _shape(api, n_shared=1, I_shared=512)
+    need_sh = api.moe_workspace_size(sh)
+    assert fwd(ctypes.byref(sh), fake, fake, fake, fake, null, odd, fake, fake, null, null,
+               ws, need_sh, None, None) == 1                 # a shared expert's w13
+    ffn = lib.moe_expert_ffn
+    assert ffn(ctypes.byref(s), fake, fake, fake, fake, odd, null, null, fake, ws, need,
+               null) == 1                                    # w2
+    assert ffn(ctypes.byref(s), odd, fake, fake, fake, fake, null, null, fake, ws, need,
+               null) == 1                                    # x
 
 
 def test_fp8_entry_points_refuse_bad_arguments(api):
